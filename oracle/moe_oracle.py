@@ -1,0 +1,228 @@
+"""CPU oracle for the MoE-layer forward: plain, slow, fp64.
+
+TEST INFRASTRUCTURE ONLY. Only the tests, the package's ``smoke()`` check and
+the CPU-baseline leg of the benchmark may import this module. The CUDA library
+never imports it and shares no code, table or constant generator with it.
+
+What it computes is the plain dropless top-k mixture-of-experts layer, the
+operation that the pages fuse into one kernel:
+
+* "FlashMoE Kernel", opening paragraph: the layer is gate -> dispatch ->
+  expert FFN -> combine, in that order.
+* "FlashMoE Kernel", section "架构" (unified task abstraction t=(M,*,phi)): the
+  two FFN matmuls and the combine's Hadamard weighting are the tasks.
+* "FlashMoE Kernel", section "通信" (in-place padding): tokens are padded to the
+  tile only for local compute.
+* "MegaMoE 在 MoE 系统谱系中的位置", section 2.4 (TokenSrcMetadata): each pool
+  slot records the (token, top-k position) it came from; the combine writes
+  through that record.
+* "MegaMoE 在 MoE 系统谱系中的位置", sections 2.5/2.6: BLOCK_M is chosen from
+  the expected tokens per expert T*k/E, and the pool is dropless with at most
+  BLOCK_M-1 padding rows per expert.
+
+Readings where the pages are silent (each is also listed in the design notes):
+
+* Gate: softmax over all E logits, keep the k largest, renormalise over the k
+  kept. This equals a softmax over the k selected logits, which is what is
+  computed here.
+* Ties in the top-k go to the lower expert id. Within a token the k selected
+  experts are listed in ascending expert id.
+* W1 is the gated branch (SiLU applied), W3 the linear branch, W2 the down
+  projection: a = silu(x W1) * (x W3), o = a W2.
+* The SwiGLU activation a is rounded to bf16 (round to nearest, ties to even)
+  before the down projection, because the GPU path stores it as bf16.
+* The gate bias, when present, is added to the logits before both the
+  selection and the softmax.
+* BLOCK_M rule for one GPU: with n = T*k/E expected tokens per expert,
+  BLOCK_M = 16 if n <= 16, 32 if n <= 32, 64 if n <= 64, else 128.
+* Padding slots of the per-expert blocks hold the record (-1, -1).
+
+Everything is fp64 on inputs given as fp64 arrays holding bf16 values.
+"""
+from __future__ import annotations
+
+from typing import Callable, Optional, Sequence
+
+import numpy as np
+
+# --------------------------------------------------------------------------
+# Rounding
+
+
+def bf16_round(a) -> np.ndarray:
+    """Round fp64 values to the nearest bf16 value (ties to even), as fp64.
+
+    bf16 keeps 8 significant bits (1 implicit + 7 stored) and fp32's exponent
+    range. Written from that definition: split a = m * 2**e with m in
+    [0.5, 1), round m * 2**8 to the nearest integer (numpy's rint rounds half
+    to even), scale back. Values below the smallest normal bf16 (2**-126) are
+    rounded on the fixed subnormal grid 2**-133. Overflow rounds to +-inf.
+    """
+    a = np.asarray(a, dtype=np.float64)
+    out = np.empty_like(a)
+    finite = np.isfinite(a)
+    m, e = np.frexp(a[finite])
+    r = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)
+    tiny = np.abs(a[finite]) < 2.0 ** -126
+    if np.any(tiny):
+        r[tiny] = np.rint(a[finite][tiny] * 2.0 ** 133) * 2.0 ** -133
+    # largest finite bf16 is (2 - 2**-7) * 2**127
+    big = np.abs(r) > (2.0 - 2.0 ** -7) * 2.0 ** 127
+    r[big] = np.copysign(np.inf, r[big])
+    out[finite] = r
+    out[~finite] = a[~finite]
+    return out
+
+
+# --------------------------------------------------------------------------
+# Gate
+
+
+def gate_logits(x: np.ndarray, Wg: np.ndarray, bias: Optional[np.ndarray]) -> np.ndarray:
+    """l[t,e] = sum_h x[t,h] Wg[h,e] (+ b[e]), fp64. x [T,H], Wg [H,E]."""
+    l = np.asarray(x, np.float64) @ np.asarray(Wg, np.float64)
+    if bias is not None:
+        l = l + np.asarray(bias, np.float64)[None, :]
+    return l
+
+
+def top_k_select(l: np.ndarray, k: int) -> np.ndarray:
+    """For each token the k largest logits, ties to the lower expert id.
+
+    Returns expert ids [T,k] listed in ascending expert id.
+    """
+    T, E = l.shape
+    idx = np.empty((T, k), dtype=np.int64)
+    experts = np.arange(E)
+    for t in range(T):
+        # lexsort sorts by the last key first: descending logit, then ascending id
+        order = np.lexsort((experts, -l[t]))
+        idx[t] = np.sort(order[:k])
+    return idx
+
+
+def renormalised_softmax(l: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    """w[t,j] = exp(l[t,idx_j] - m) / sum_i exp(l[t,idx_i] - m), m = max over the k kept."""
+    sel = np.take_along_axis(l, idx, axis=1)
+    m = sel.max(axis=1, keepdims=True)
+    p = np.exp(sel - m)
+    return p / p.sum(axis=1, keepdims=True)
+
+
+def route(x, Wg, bias, k: int):
+    """Gate step: (topk_idx [T,k] int64 ascending, topk_w [T,k] fp64, logits [T,E])."""
+    l = gate_logits(x, Wg, bias)
+    idx = top_k_select(l, k)
+    w = renormalised_softmax(l, idx)
+    return idx, w, l
+
+
+# --------------------------------------------------------------------------
+# Dispatch
+
+
+def block_m_rule(T: int, k: int, E: int) -> int:
+    """BLOCK_M from the expected tokens per expert n = T*k/E (one GPU).
+
+    The pages' candidate table steps BLOCK_M up with n; on one GPU with a
+    128-row MMA tile the candidates kept are 16, 32, 64 and 128.
+    """
+    n = T * k / E
+    if n <= 16:
+        return 16
+    if n <= 32:
+        return 32
+    if n <= 64:
+        return 64
+    return 128
+
+
+def dispatch(idx: np.ndarray, E: int, block_m: int) -> dict:
+    """Histogram, padded exclusive scan and stable slot permutation.
+
+    count[e]   = number of (t, j) with idx[t,j] == e
+    padded[e]  = ceil(count[e] / block_m) * block_m
+    offset[e]  = sum of padded[e'] over e' < e  (offset has E+1 entries)
+    Slot offset[e] + r holds the r-th token, in ascending token order, routed
+    to e, with its top-k position j; the remaining slots of the expert's
+    blocks hold (-1, -1).
+    """
+    T, k = idx.shape
+    count = np.zeros(E, dtype=np.int64)
+    for t in range(T):
+        for j in range(k):
+            count[idx[t, j]] += 1
+    padded = (count + block_m - 1) // block_m * block_m
+    offset = np.zeros(E + 1, dtype=np.int64)
+    for e in range(E):
+        offset[e + 1] = offset[e] + padded[e]
+    P = int(offset[E])
+    slot_token = np.full(P, -1, dtype=np.int64)
+    slot_topk = np.full(P, -1, dtype=np.int64)
+    fill = offset[:E].copy()
+    for t in range(T):              # ascending t makes the permutation stable
+        for j in range(k):
+            e = idx[t, j]
+            slot_token[fill[e]] = t
+            slot_topk[fill[e]] = j
+            fill[e] += 1
+    return dict(count=count, padded=padded, offset=offset, num_padded=P,
+                slot_token=slot_token, slot_topk=slot_topk, block_m=block_m)
+
+
+def pool_capacity(T: int, k: int, E: int, block_m: int) -> int:
+    """Worst-case number of slots: every routed pair plus BLOCK_M-1 padding per expert."""
+    return T * k + E * (block_m - 1)
+
+
+# --------------------------------------------------------------------------
+# Expert FFN and combine
+
+
+def silu(g: np.ndarray) -> np.ndarray:
+    return g / (1.0 + np.exp(-g))
+
+
+def expert_ffn(xr: np.ndarray, W1e: np.ndarray, W3e: np.ndarray, W2e: np.ndarray) -> np.ndarray:
+    """o = bf16(silu(xr W1e) * (xr W3e)) W2e for rows xr [n,H]; W1e,W3e [H,I]; W2e [I,H]."""
+    g = xr @ W1e
+    u = xr @ W3e
+    a = bf16_round(silu(g) * u)
+    return a @ W2e
+
+
+def stacked_expert_weights(W1, W3, W2) -> Callable[[int], tuple]:
+    """Expert loader over stacked arrays W1,W3 [E,H,I], W2 [E,I,H] (any float dtype)."""
+    def load(e):
+        return (np.asarray(W1[e], np.float64), np.asarray(W3[e], np.float64),
+                np.asarray(W2[e], np.float64))
+    return load
+
+
+def moe_forward(x, Wg, bias, expert_weights: Callable[[int], tuple], k: int,
+                block_m: Optional[int] = None, tokens: Optional[Sequence[int]] = None) -> dict:
+    """The whole layer: gate, dispatch, expert FFN, gate-weighted combine.
+
+    x [T,H] fp64; Wg [H,E] fp64; bias [E] or None; ``expert_weights(e)``
+    returns (W1[e], W3[e], W2[e]) as fp64. If ``tokens`` is given, y is
+    computed only for those token rows (routing and dispatch always cover all
+    T tokens). y[t] = sum_j w[t,j] * FFN_{idx[t,j]}(x[t]).
+    """
+    x = np.asarray(x, np.float64)
+    T, H = x.shape
+    E = np.asarray(Wg).shape[1]
+    idx, w, logits = route(x, Wg, bias, k)
+    bm = block_m_rule(T, k, E) if block_m is None else block_m
+    disp = dispatch(idx, E, bm)
+    rows = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    y = np.zeros((len(rows), H), dtype=np.float64)
+    for e in range(E):
+        # (row position in `rows`, top-k position) of every selected pair routed to e
+        hit = np.nonzero(idx[rows] == e)
+        if hit[0].size == 0:
+            continue
+        W1e, W3e, W2e = expert_weights(e)
+        o = expert_ffn(x[rows[hit[0]]], W1e, W3e, W2e)
+        wt = w[rows[hit[0]], hit[1]]
+        np.add.at(y, hit[0], wt[:, None] * o)
+    return dict(topk_idx=idx, topk_w=w, logits=logits, y=y, tokens=rows, **disp)

@@ -1,0 +1,182 @@
+/*
+ * moe_b200.h - C ABI of the single-GPU MoE-layer forward for B200 (sm_100a).
+ *
+ * The library computes one dropless top-k mixture-of-experts layer forward on
+ * one GPU:
+ *
+ *   gate      l = x Wg (+ b); keep the k largest logits per token; weights are
+ *             the softmax over the k kept logits.
+ *   dispatch  per-expert histogram, exclusive scan of the counts padded to
+ *             BLOCK_M, stable token -> slot permutation with a (token, top-k
+ *             position) record per slot.
+ *   expert    h = bf16(silu(x W1[e]) * (x W3[e])) for every slot of expert e,
+ *             then o = h W2[e].
+ *   combine   y[t] = sum_j w[t,j] * o(t,j), scatter-added from the down
+ *             projection's epilogue.
+ *
+ * Sources: "FlashMoE Kernel" (opening paragraph: the layer is gate -> dispatch
+ * -> expert FFN -> combine; section "架构": the FFN matmuls and the combine's
+ * weighting are fused tile tasks; section "通信": in-place padding to the tile);
+ * "MegaMoE 在 MoE 系统谱系中的位置" (section 2.4: per-slot TokenSrcMetadata;
+ * section 2.5: BLOCK_M from the expected tokens per expert; section 2.6:
+ * dropless pool sized T*k + E*(BLOCK_M-1) on one rank; section 2.7: tasks
+ * claimed from an atomic counter, L2 tasks wait for their block's L1 tasks;
+ * section 五: the forward entry points take bf16 or fp8/fp4 tensors).
+ *
+ * Conventions for every entry point:
+ *  - bf16 tensors are passed as `const void*` to 16-byte-aligned, contiguous,
+ *    row-major device memory; fp32 and int32 likewise.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). All GPU work
+ *    is enqueued on it; nothing synchronises the host unless stated.
+ *  - Every function returns a moe_status; no exception crosses the ABI.
+ *  - Device-side failures (a bounded wait that ran out, a routing index out of
+ *    range) are sticky in the workspace and are reported by moe_check().
+ *  - The caller owns all device memory: inputs, weights, outputs and the
+ *    workspace. A plan owns only host state.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct moe_plan* moe_plan_t;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,         /* null pointer, misaligned pointer, T out of range */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2,   /* shape outside the supported set (see moe_plan_create) */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 3, /* bound workspace smaller than moe_plan_workspace_bytes() */
+  MOE_ERR_NO_WORKSPACE = 4,        /* moe_forward before moe_plan_bind_workspace */
+  MOE_ERR_CUDA = 5,                /* a CUDA runtime/driver call failed */
+  MOE_ERR_DEVICE_TIMEOUT = 6,      /* a bounded device-side wait ran out (sticky, via moe_check) */
+  MOE_ERR_DEVICE_BOUNDS = 7,       /* routing metadata held an out-of-range index (sticky) */
+  MOE_ERR_UNSUPPORTED_DEVICE = 8   /* the device is not sm_100 */
+} moe_status;
+
+/* Device views of the routing results inside the bound workspace. Valid after
+ * a moe_forward()/moe_route() on the plan's stream has completed; overwritten
+ * by the next call. Layouts:
+ *   topk_idx      int32 [T, k]   selected experts of token t, ascending expert id
+ *   topk_w        fp32  [T, k]   softmax weights over the k selected logits
+ *   expert_count  int32 [E]      tokens routed to each expert
+ *   expert_offset int32 [E+1]    first slot of each expert; multiples of block_m
+ *   slot_token    int32 [pool]   token of each slot, -1 for padding
+ *   slot_topk     int32 [pool]   top-k position j of each slot, -1 for padding
+ *   num_padded    int32 [1]      slots in use = expert_offset[E]
+ * ("MegaMoE 在 MoE 系统谱系中的位置", section 2.4: the slot record; the rank
+ * field of that record is dropped on one GPU.) */
+typedef struct {
+  int32_t* topk_idx;
+  float* topk_w;
+  int32_t* expert_count;
+  int32_t* expert_offset;
+  int32_t* slot_token;
+  int32_t* slot_topk;
+  int32_t* num_padded;
+  int32_t block_m;
+  int32_t pool_capacity;
+} moe_routing;
+
+/* Static description of a plan. */
+typedef struct {
+  int32_t T_max, H, I, E, k;
+  int32_t block_m;         /* rows per expert block (16, 32, 64 or 128) */
+  int32_t pool_capacity;   /* T_max*k + E*(block_m-1) slots */
+  int32_t num_sms;         /* persistent grid size */
+  size_t workspace_bytes;
+} moe_plan_desc;
+
+/* Create a plan for up to T_max tokens of a layer with hidden size H, expert
+ * intermediate size I, E experts and top-k routing, on CUDA device `device`.
+ * block_m = 0 picks BLOCK_M from n = T_max*k/E: 16 if n <= 16, 32 if n <= 32,
+ * 64 if n <= 64, else 128 (the candidate table of "MegaMoE 在 MoE 系统谱系中
+ * 的位置", section 2.5, cut to the 128-row MMA tile); otherwise it must be one
+ * of 16, 32, 64, 128.
+ * Supported: T_max >= 1; H % 128 == 0; I % 128 == 0; E % 8 == 0, 8 <= E <= 256;
+ * 1 <= k <= min(E, 8). Errors: MOE_ERR_INVALID_ARG (null plan pointer),
+ * MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_UNSUPPORTED_DEVICE, MOE_ERR_CUDA.
+ * Allocates no device memory. */
+int moe_plan_create(moe_plan_t* plan, int T_max, int H, int I, int E, int k, int block_m, int device);
+
+/* Bytes of device workspace the plan needs (routing arrays, scheduler
+ * counters, the bf16 intermediate h [pool, I], the fp32 output accumulator
+ * [T_max, H] and bf16 staging for moe_forward_host). 0 for a null plan. */
+size_t moe_plan_workspace_bytes(moe_plan_t plan);
+
+/* Bind caller-allocated device memory (256-byte aligned, at least
+ * moe_plan_workspace_bytes()) as the plan's workspace. The plan does not take
+ * ownership. Errors: MOE_ERR_INVALID_ARG (null or misaligned),
+ * MOE_ERR_WORKSPACE_TOO_SMALL. Calls sharing one workspace must not overlap in
+ * time on the GPU. */
+int moe_plan_bind_workspace(moe_plan_t plan, void* workspace, size_t bytes);
+
+/* Fill `desc` with the plan's static description. */
+int moe_plan_describe(moe_plan_t plan, moe_plan_desc* desc);
+
+/* Fill `out` with device pointers to the routing results in the workspace. */
+int moe_plan_get_routing(moe_plan_t plan, moe_routing* out);
+
+/* The whole layer forward for T tokens (0 <= T <= T_max):
+ *   x    bf16 [T, H]      device
+ *   Wg   bf16 [H, E]      device
+ *   gate_bias fp32 [E]    device, or NULL for no bias (added to the logits
+ *                         before the top-k and the softmax)
+ *   W1   bf16 [E, H, I]   device (gated branch, SiLU applied)
+ *   W3   bf16 [E, H, I]   device (linear branch)
+ *   W2   bf16 [E, I, H]   device (down projection)
+ *   y    bf16 [T, H]      device, written
+ * Enqueues router, dispatch scan, dispatch scatter, the persistent expert
+ * GEMM and the bf16 cast of the output on `stream`; no host synchronisation
+ * and no host read of routing. T = 0 enqueues nothing. Errors:
+ * MOE_ERR_INVALID_ARG, MOE_ERR_NO_WORKSPACE, MOE_ERR_CUDA (launch failure). */
+int moe_forward(moe_plan_t plan, const void* x, const void* Wg, const float* gate_bias, const void* W1,
+                const void* W3, const void* W2, int T, void* y, void* stream);
+
+/* moe_forward with x and y in HOST memory: copies x [T, H] into the
+ * workspace's staging buffer, runs the layer, copies y [T, H] back, all
+ * enqueued on `stream` (pinned host buffers make the copies asynchronous; the
+ * caller synchronises the stream before reading y). Weights stay on the device. */
+int moe_forward_host(moe_plan_t plan, const void* x_host, const void* Wg, const float* gate_bias, const void* W1,
+                     const void* W3, const void* W2, int T, void* y_host, void* stream);
+
+/* Gate and dispatch only (router, scan, scatter) for T tokens; fills the
+ * routing results exactly as moe_forward does, without the expert FFN. */
+int moe_route(moe_plan_t plan, const void* x, const void* Wg, const float* gate_bias, int T, void* stream);
+
+/* Synchronise `stream`, return the sticky device error of the plan's
+ * workspace (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_BOUNDS) and
+ * clear it; MOE_ERR_CUDA if the stream reports an error. If `detail` is not
+ * NULL it receives the error's detail word (which wait or which block). */
+int moe_check(moe_plan_t plan, void* stream, int32_t* detail);
+
+/* Profiling: when enabled, moe_forward records CUDA events on its stream
+ * around each of its five kernels. moe_plan_profile_read() synchronises on
+ * the last recorded event, writes the summed milliseconds of each kernel
+ * (router, scan, scatter, expert GEMM, finalize) over the forwards recorded
+ * since the previous read into ms[0..4], the number of such forwards into
+ * *count, and resets the sums. At most 256 forwards are kept between reads. */
+int moe_plan_set_profiling(moe_plan_t plan, int enable);
+int moe_plan_profile_read(moe_plan_t plan, float* ms, int* count);
+
+/* Test hooks: the persistent kernel gives up any device-side wait after
+ * timeout_ns nanoseconds (default 2e9) and records MOE_ERR_DEVICE_TIMEOUT;
+ * withhold_block >= 0 makes the kernel never publish the completion of that
+ * L1 block, so the L2 tasks waiting on it time out. -1 restores normal runs. */
+int moe_plan_set_debug(moe_plan_t plan, int withhold_block, uint64_t timeout_ns);
+
+/* Number of kernels one moe_forward launches (for launch accounting). */
+int moe_forward_kernel_count(void);
+
+void moe_plan_destroy(moe_plan_t plan);
+const char* moe_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

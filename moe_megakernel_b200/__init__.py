@@ -1,0 +1,239 @@
+"""Python binding of the single-GPU MoE-layer forward library (libmoe_b200.so).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels. torch supplies device memory (inputs, weights, outputs and the
+workspace) and the stream. If the library has not been built the import of
+the binding fails loudly; there is no other implementation to fall back to.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe_b200.so")
+
+MOE_OK = 0
+STATUS_NAMES = {
+    0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_SHAPE",
+    3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_NO_WORKSPACE", 5: "MOE_ERR_CUDA",
+    6: "MOE_ERR_DEVICE_TIMEOUT", 7: "MOE_ERR_DEVICE_BOUNDS", 8: "MOE_ERR_UNSUPPORTED_DEVICE",
+}
+KERNEL_NAMES = ("router", "dispatch_scan", "dispatch_scatter", "expert_gemm", "finalize")
+
+_c_int, _c_size, _vp = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+
+
+class MoERouting(ctypes.Structure):
+    _fields_ = [("topk_idx", _vp), ("topk_w", _vp), ("expert_count", _vp), ("expert_offset", _vp),
+                ("slot_token", _vp), ("slot_topk", _vp), ("num_padded", _vp),
+                ("block_m", ctypes.c_int32), ("pool_capacity", ctypes.c_int32)]
+
+
+class MoEPlanDesc(ctypes.Structure):
+    _fields_ = [("T_max", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("block_m", ctypes.c_int32),
+                ("pool_capacity", ctypes.c_int32), ("num_sms", ctypes.c_int32),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
+# exported symbol -> (restype, argtypes); the same list as include/moe_b200.h
+SIGNATURES = {
+    "moe_plan_create": (_c_int, [ctypes.POINTER(_vp), _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
+    "moe_plan_workspace_bytes": (_c_size, [_vp]),
+    "moe_plan_bind_workspace": (_c_int, [_vp, _vp, _c_size]),
+    "moe_plan_describe": (_c_int, [_vp, ctypes.POINTER(MoEPlanDesc)]),
+    "moe_plan_get_routing": (_c_int, [_vp, ctypes.POINTER(MoERouting)]),
+    "moe_forward": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
+    "moe_forward_host": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
+    "moe_route": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _vp]),
+    "moe_check": (_c_int, [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]),
+    "moe_plan_set_profiling": (_c_int, [_vp, _c_int]),
+    "moe_plan_profile_read": (_c_int, [_vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_c_int)]),
+    "moe_plan_set_debug": (_c_int, [_vp, _c_int, ctypes.c_uint64]),
+    "moe_forward_kernel_count": (_c_int, []),
+    "moe_plan_destroy": (None, [_vp]),
+    "moe_status_string": (ctypes.c_char_p, [_c_int]),
+}
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libmoe_b200.so and declare every exported entry point."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m moe_megakernel_b200.build` "
+                          "(the CUDA library is the only implementation)")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        name = STATUS_NAMES.get(status, str(status))
+        msg = load_library().moe_status_string(status).decode()
+        super().__init__(f"{what}: {name} ({msg})")
+
+
+def _ok(rc: int, what: str):
+    if rc != MOE_OK:
+        raise MoEError(rc, what)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream, device) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(t: torch.Tensor, name: str, shape, dtype, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: expected {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name}: expected device {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+class MoEPlan:
+    """A plan for one MoE layer shape plus its device workspace.
+
+    ``forward`` runs gate -> dispatch -> expert FFN -> combine for x [T,H]
+    (T <= T_max) and returns y [T,H] bf16. ``routing(T)`` returns views of the
+    routing results of the last call.
+    """
+
+    def __init__(self, T_max: int, H: int, I: int, E: int, k: int, block_m: int = 0, device=None):
+        self.lib = load_library()
+        self.device = torch.device("cuda", torch.cuda.current_device() if device is None
+                                   else torch.device(device).index or 0)
+        self.T_max, self.H, self.I, self.E, self.k = T_max, H, I, E, k
+        self._plan = ctypes.c_void_p()
+        _ok(self.lib.moe_plan_create(ctypes.byref(self._plan), T_max, H, I, E, k, block_m,
+                                     self.device.index), "moe_plan_create")
+        d = MoEPlanDesc()
+        _ok(self.lib.moe_plan_describe(self._plan, ctypes.byref(d)), "moe_plan_describe")
+        self.block_m, self.pool_capacity, self.num_sms = d.block_m, d.pool_capacity, d.num_sms
+        self.workspace_bytes = d.workspace_bytes
+        self.workspace = torch.empty(self.workspace_bytes, dtype=torch.uint8, device=self.device)
+        _ok(self.lib.moe_plan_bind_workspace(self._plan, _ptr(self.workspace), self.workspace_bytes),
+            "moe_plan_bind_workspace")
+
+    # ------------------------------------------------------------------ calls
+    def _check_inputs(self, x, Wg, bias, W=None):
+        T = x.shape[0]
+        _check(x, "x", (T, self.H), torch.bfloat16, self.device)
+        _check(Wg, "Wg", (self.H, self.E), torch.bfloat16, self.device)
+        if bias is not None:
+            _check(bias, "bias", (self.E,), torch.float32, self.device)
+        if W is not None:
+            W1, W3, W2 = W
+            _check(W1, "W1", (self.E, self.H, self.I), torch.bfloat16, self.device)
+            _check(W3, "W3", (self.E, self.H, self.I), torch.bfloat16, self.device)
+            _check(W2, "W2", (self.E, self.I, self.H), torch.bfloat16, self.device)
+        return T
+
+    def forward(self, x, Wg, bias, W1, W3, W2, y=None, stream=None) -> torch.Tensor:
+        T = self._check_inputs(x, Wg, bias, (W1, W3, W2))
+        if y is None:
+            y = torch.empty((T, self.H), dtype=torch.bfloat16, device=self.device)
+        _check(y, "y", (T, self.H), torch.bfloat16, self.device)
+        _ok(self.lib.moe_forward(self._plan, _ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3), _ptr(W2),
+                                 T, _ptr(y), _stream_handle(stream, self.device)), "moe_forward")
+        return y
+
+    def forward_host(self, x_host, Wg, bias, W1, W3, W2, y_host, stream=None):
+        """x_host and y_host are CPU bf16 tensors (pinned for asynchronous copies)."""
+        T = x_host.shape[0]
+        _check(x_host, "x_host", (T, self.H), torch.bfloat16, torch.device("cpu"))
+        _check(y_host, "y_host", (T, self.H), torch.bfloat16, torch.device("cpu"))
+        _check(Wg, "Wg", (self.H, self.E), torch.bfloat16, self.device)
+        _ok(self.lib.moe_forward_host(self._plan, _ptr(x_host), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3),
+                                      _ptr(W2), T, _ptr(y_host), _stream_handle(stream, self.device)),
+            "moe_forward_host")
+        return y_host
+
+    def route(self, x, Wg, bias, stream=None):
+        T = self._check_inputs(x, Wg, bias)
+        _ok(self.lib.moe_route(self._plan, _ptr(x), _ptr(Wg), _ptr(bias), T,
+                               _stream_handle(stream, self.device)), "moe_route")
+
+    def check(self, stream=None) -> int:
+        """Synchronise; raise MoEError on a sticky device error (and clear it)."""
+        detail = ctypes.c_int32(0)
+        rc = self.lib.moe_check(self._plan, _stream_handle(stream, self.device), ctypes.byref(detail))
+        self.last_error_detail = detail.value
+        _ok(rc, "device")
+        return rc
+
+    def routing(self, T: int) -> dict:
+        """Views (into the workspace) of the routing results for the last T-token call."""
+        r = MoERouting()
+        _ok(self.lib.moe_plan_get_routing(self._plan, ctypes.byref(r)), "moe_plan_get_routing")
+        base = self.workspace.data_ptr()
+
+        def view(ptr, n, dtype):
+            off = ptr - base
+            nbytes = n * 4
+            return self.workspace[off:off + nbytes].view(dtype)
+
+        E, k = self.E, self.k
+        return dict(
+            topk_idx=view(r.topk_idx, T * k, torch.int32).view(T, k),
+            topk_w=view(r.topk_w, T * k, torch.float32).view(T, k),
+            expert_count=view(r.expert_count, E, torch.int32),
+            expert_offset=view(r.expert_offset, E + 1, torch.int32),
+            slot_token=view(r.slot_token, r.pool_capacity, torch.int32),
+            slot_topk=view(r.slot_topk, r.pool_capacity, torch.int32),
+            num_padded=view(r.num_padded, 1, torch.int32),
+            block_m=r.block_m,
+        )
+
+    def set_profiling(self, enable: bool):
+        _ok(self.lib.moe_plan_set_profiling(self._plan, 1 if enable else 0), "moe_plan_set_profiling")
+
+    def profile_read(self):
+        """(summed ms per kernel since the last read as a dict, number of forwards)."""
+        ms = (ctypes.c_float * 5)()
+        n = ctypes.c_int(0)
+        _ok(self.lib.moe_plan_profile_read(self._plan, ms, ctypes.byref(n)), "moe_plan_profile_read")
+        return dict(zip(KERNEL_NAMES, list(ms))), n.value
+
+    def set_debug(self, withhold_block: int = -1, timeout_ns: int = 0):
+        _ok(self.lib.moe_plan_set_debug(self._plan, withhold_block, timeout_ns), "moe_plan_set_debug")
+
+    def close(self):
+        if getattr(self, "_plan", None) and self._plan.value:
+            self.lib.moe_plan_destroy(self._plan)
+            self._plan = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def kernels_per_forward() -> int:
+    return load_library().moe_forward_kernel_count()

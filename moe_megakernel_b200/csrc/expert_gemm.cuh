@@ -1,0 +1,512 @@
+// Persistent grouped GEMM over the expert blocks: phase L1 (x W1, x W3 with a
+// fused SwiGLU epilogue, bf16 h out) and phase L2 (h W2 with the combine's
+// gate-weighted scatter-add fused into the epilogue).
+//
+// Prior art this follows, re-done for one B200:
+// * "FlashMoE Kernel", section "架构": one persistent kernel whose blocks run
+//   tile tasks t = (M, *, phi); the two FFN matmuls and the combine's Hadamard
+//   weighting are fused device routines. Here a task is (phase, expert,
+//   m-block, n-tile).
+// * "MegaMoE 在 MoE 系统谱系中的位置", section 2.1: warp roles inside the CTA
+//   (activation TMA, weight TMA, MMA issue, scheduler, epilogue). Here warp 0
+//   is scheduler + TMA producer, warp 1 issues tcgen05 MMAs, warps 2-5 drain
+//   TMEM in the epilogue.
+// * Same page, section 2.7: tasks are claimed from a global atomic counter,
+//   and an L2 task of pool block b waits on an in-kernel counter until the L1
+//   tasks of block b are complete (bounded wait here).
+// * Same page, section 2.4: the slot's (token, top-k) record gives the
+//   combine's write address from the epilogue.
+// * ScatterMoE idea on the same page, section 一: the token gather is fused
+//   into the operand load (TMA gather4 of x rows), no permuted copy of x.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+struct GemmParams {
+  CUtensorMap tm_x;    // x [T, H], box {64, 1}, gather4 rows
+  CUtensorMap tm_w1;   // W1 as [E*H, I], box {64, 64}
+  CUtensorMap tm_w3;   // W3 as [E*H, I], box {64, 64}
+  CUtensorMap tm_w2;   // W2 as [E*I, H], box {64, 64}
+  CUtensorMap tm_h;    // h [pool, I], box {64, BM}
+  const int32_t* slot_token;
+  const int32_t* slot_topk;
+  const float* topk_w;
+  const int32_t* block_start;   // [E+1]
+  int32_t* task_counter;
+  int32_t* l1_done;             // [blocks]
+  int32_t* err;                 // [0] code, [1] detail
+  bf16* h;                      // [pool, I]
+  float* y_acc;                 // [T, H]
+  int T, H, I, E, k, BM, BN2, N1, N2;
+  unsigned long long timeout_ns;
+  int withhold_block;           // test hook: never publish L1 completion of this block (-1: off)
+};
+
+struct Task {
+  int phase;   // 0 = L1, 1 = L2, -1 = no more work
+  int e, b, n;
+};
+
+struct GemmSmem {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t task_full[kTaskRing];
+  uint64_t task_empty[kTaskRing];
+  uint64_t mma_done;
+  Task tasks[kTaskRing];
+  uint32_t tmem_base;
+  int abort;
+  int block_start[257];
+};
+
+constexpr size_t kGemmSmemBytes = 1024 /*alignment slack*/ + (size_t)kStages * kStageBytes + sizeof(GemmSmem);
+
+__device__ __forceinline__ void set_error(const GemmParams& p, GemmSmem& s, int code, int detail) {
+  if (atomicCAS(p.err, 0, code) == 0) p.err[1] = detail;
+  *reinterpret_cast<volatile int*>(&s.abort) = 1;
+}
+
+// Bounded wait of a whole warp on an mbarrier phase. All lanes agree on the result.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const GemmParams& p, GemmSmem& s,
+                                          int where) {
+  bool ok = ptx::mbar_try_wait(bar, parity);
+  if (!ok) {
+    const uint64_t t0 = ptx::globaltimer();
+    while (true) {
+      if (ptx::mbar_try_wait(bar, parity)) {
+        ok = true;
+        break;
+      }
+      if (*reinterpret_cast<volatile int*>(&s.abort)) break;
+      if (ptx::globaltimer() - t0 > p.timeout_ns) {
+        set_error(p, s, kDevTimeout, where);
+        break;
+      }
+    }
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ Task decode_task(int t, const GemmSmem& s, const GemmParams& p) {
+  Task task{-1, 0, 0, 0};
+  const int nb_total = s.block_start[p.E];
+  const int n_l1 = nb_total * p.N1;
+  const int n_l2 = nb_total * p.N2;
+  if (t < 0 || t >= n_l1 + n_l2) return task;
+  int NT, tt;
+  if (t < n_l1) {
+    task.phase = 0;
+    NT = p.N1;
+    tt = t;
+  } else {
+    task.phase = 1;
+    NT = p.N2;
+    tt = t - n_l1;
+  }
+  // expert e owns tasks [block_start[e]*NT, block_start[e+1]*NT); order inside: (n-tile, m-block)
+  const int vb = tt / NT;
+  int lo = 0, hi = p.E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s.block_start[mid] <= vb) lo = mid;
+    else hi = mid - 1;
+  }
+  const int e = lo;
+  const int nb = s.block_start[e + 1] - s.block_start[e];
+  const int local = tt - s.block_start[e] * NT;
+  task.e = e;
+  task.n = local / nb;
+  task.b = s.block_start[e] + (local - task.n * nb);
+  return task;
+}
+
+__device__ __forceinline__ uint8_t* stage_ptr(uint8_t* tiles, int stage) { return tiles + stage * kStageBytes; }
+
+// ---------------------------------------------------------------- producer (warp 0)
+__device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) {
+  const int lane = ptx::lane_id();
+  const uint64_t pol = ptx::policy_evict_normal();
+  int stage = 0;
+  uint32_t phase = 0;
+  int q = 0;
+  uint32_t qphase = 0;
+  uint32_t issued = 0, issued_parity = 0;   // per stage: ever issued, parity of the last issue
+
+  while (true) {
+    int t = 0x7fffffff;
+    if (lane == 0) {
+      const bool stop = *reinterpret_cast<volatile int*>(&s.abort) ||
+                        *reinterpret_cast<volatile int*>(p.err) != 0;
+      if (!stop) t = atomicAdd(p.task_counter, 1);
+    }
+    t = __shfl_sync(0xffffffffu, t, 0);
+    Task task = decode_task(t, s, p);
+
+    if (task.phase == 1) {
+      // the L2 task of block b reads h rows written by all L1 n-tiles of block b
+      bool ok = true;
+      if (lane == 0) {
+        const int* ctr = p.l1_done + task.b;
+        const int need = 4 * p.N1;   // one arrival per epilogue warp per L1 n-tile
+        if (ptx::ld_acquire_gpu(ctr) < need) {
+          const uint64_t t0 = ptx::globaltimer();
+          while (ptx::ld_acquire_gpu(ctr) < need) {
+            if (*reinterpret_cast<volatile int*>(&s.abort) || *reinterpret_cast<volatile int*>(p.err) != 0) {
+              ok = false;
+              break;
+            }
+            if (ptx::globaltimer() - t0 > p.timeout_ns) {
+              set_error(p, s, kDevTimeout, 0x10000 | task.b);
+              ok = false;
+              break;
+            }
+            __nanosleep(256);
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) task.phase = -1;
+      ptx::fence_proxy_async_global();
+    }
+
+    // hand the task to the MMA and epilogue warps
+    if (!warp_wait(&s.task_empty[q], qphase ^ 1, p, s, 1)) break;
+    if (lane == 0) {
+      s.tasks[q] = task;
+      ptx::mbar_arrive(&s.task_full[q]);
+    }
+    __syncwarp();
+    if (++q == kTaskRing) {
+      q = 0;
+      qphase ^= 1;
+    }
+    if (task.phase < 0) break;
+
+    int rows[4] = {0, 0, 0, 0};
+    if (task.phase == 0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = lane * 4 + i;
+        int tok = 0;
+        if (r < p.BM) {
+          tok = p.slot_token[task.b * p.BM + r];
+          if (tok >= p.T) {
+            set_error(p, s, kDevBounds, task.b);
+            tok = 0;
+          }
+          if (tok < 0) tok = 0;   // padding slot: any valid row, the epilogue drops it
+        }
+        rows[i] = tok;
+      }
+    }
+    const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
+    bool ok = true;
+    for (int kb = 0; kb < nk; ++kb) {
+      if (!warp_wait(&s.empty[stage], phase ^ 1, p, s, 2)) {
+        ok = false;
+        break;
+      }
+      uint8_t* sa = stage_ptr(tiles, stage);
+      const uint32_t a_addr = ptx::smem_u32(sa);
+      const uint32_t b_addr = a_addr + kTileABytes;
+      if (task.phase == 0) {
+        if (lane == 0) ptx::mbar_arrive_expect_tx(&s.full[stage], p.BM * 128 + 4 * kBoxBytes);
+        __syncwarp();
+        if (lane * 4 < p.BM)
+          ptx::tma_gather4(a_addr + lane * 512, &p.tm_x, &s.full[stage], kb * kBK, rows[0], rows[1], rows[2],
+                           rows[3], pol);
+        if (lane == 0) {
+          const int wrow = task.e * p.H + kb * kBK;
+          const int n0 = task.n * kL1TileN;
+          ptx::tma_load_2d(b_addr + 0 * kBoxBytes, &p.tm_w1, &s.full[stage], n0, wrow, pol);
+          ptx::tma_load_2d(b_addr + 1 * kBoxBytes, &p.tm_w1, &s.full[stage], n0 + 64, wrow, pol);
+          ptx::tma_load_2d(b_addr + 2 * kBoxBytes, &p.tm_w3, &s.full[stage], n0, wrow, pol);
+          ptx::tma_load_2d(b_addr + 3 * kBoxBytes, &p.tm_w3, &s.full[stage], n0 + 64, wrow, pol);
+        }
+      } else {
+        if (lane == 0) {
+          const int nbox = p.BN2 / 64;
+          ptx::mbar_arrive_expect_tx(&s.full[stage], p.BM * 128 + nbox * kBoxBytes);
+          ptx::tma_load_2d(a_addr, &p.tm_h, &s.full[stage], kb * kBK, task.b * p.BM, pol);
+          const int wrow = task.e * p.I + kb * kBK;
+          for (int j = 0; j < nbox; ++j)
+            ptx::tma_load_2d(b_addr + j * kBoxBytes, &p.tm_w2, &s.full[stage], task.n * p.BN2 + j * 64, wrow,
+                             pol);
+        }
+      }
+      __syncwarp();
+      issued |= 1u << stage;
+      issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+      if (++stage == kStages) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+    if (!ok) break;
+  }
+  // On an early exit, let every issued copy land before the CTA can retire.
+  for (int st = 0; st < kStages; ++st)
+    if (issued & (1u << st)) {
+      const uint32_t par = (issued_parity >> st) & 1u;
+      const uint64_t t0 = ptx::globaltimer();
+      while (!ptx::mbar_try_wait(&s.full[st], par)) {
+        if (ptx::globaltimer() - t0 > p.timeout_ns) break;
+      }
+    }
+}
+
+// ---------------------------------------------------------------- MMA issuer (warp 1)
+__device__ void gemm_mma(const GemmParams& p, GemmSmem& s, uint8_t* tiles, uint32_t tmem_base) {
+  const int lane = ptx::lane_id();
+  const uint32_t idesc_l1 = ptx::idesc_bf16_f32(128, 2 * kL1TileN, false, true);
+  const uint32_t idesc_l2 = ptx::idesc_bf16_f32(128, p.BN2, false, true);
+  int stage = 0;
+  uint32_t phase = 0;
+  int q = 0;
+  uint32_t qphase = 0;
+  int acc = 0;
+  uint32_t acc_phase = 0;
+  bool issued_any = false;
+  while (true) {
+    if (!warp_wait(&s.task_full[q], qphase, p, s, 3)) break;
+    const Task task = s.tasks[q];
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&s.task_empty[q]);
+    if (++q == kTaskRing) {
+      q = 0;
+      qphase ^= 1;
+    }
+    if (task.phase < 0) break;
+    if (!warp_wait(&s.acc_empty[acc], acc_phase ^ 1, p, s, 4)) break;
+    ptx::tc_fence_after();
+    const uint32_t d_tmem = tmem_base + acc * 256;
+    const uint32_t idesc = task.phase == 0 ? idesc_l1 : idesc_l2;
+    const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
+    bool ok = true;
+    for (int kb = 0; kb < nk; ++kb) {
+      if (!warp_wait(&s.full[stage], phase, p, s, 5)) {
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      if (lane == 0) {
+        const uint32_t a_addr = ptx::smem_u32(stage_ptr(tiles, stage));
+        const uint32_t b_addr = a_addr + kTileABytes;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          // A: K-major, 128-byte rows, 8-row groups 1024 B apart; step 16 elements = 32 B along K.
+          const uint64_t ad = ptx::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+          // B: MN-major, 64-column boxes 8 KB apart, 8-row K groups 1024 B apart; step 16 rows = 2 KB.
+          const uint64_t bd = ptx::smem_desc_sw128(b_addr + kk * 2048, kBoxBytes, 1024);
+          ptx::mma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(&s.empty[stage]);
+        issued_any = true;
+      }
+      __syncwarp();
+      if (++stage == kStages) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+    if (!ok) break;
+    if (lane == 0) ptx::mma_commit(&s.acc_full[acc]);
+    __syncwarp();
+    if (++acc == 2) {
+      acc = 0;
+      acc_phase ^= 1;
+    }
+  }
+  // Every MMA must have finished before TMEM is released.
+  issued_any = __any_sync(0xffffffffu, issued_any);
+  if (issued_any) {
+    if (lane == 0) ptx::mma_commit(&s.mma_done);
+    __syncwarp();
+    const uint64_t t0 = ptx::globaltimer();
+    while (!ptx::mbar_try_wait(&s.mma_done, 0)) {
+      if (ptx::globaltimer() - t0 > p.timeout_ns) break;
+    }
+  }
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// ---------------------------------------------------------------- epilogue (warps 2..5)
+__device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_base) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = ptx::lane_id();
+  const int quarter = warp & 3;              // TMEM lanes 32*quarter .. +31
+  const int r = quarter * 32 + lane;         // tile row of this thread
+  int q = 0;
+  uint32_t qphase = 0;
+  int acc = 0;
+  uint32_t acc_phase = 0;
+  while (true) {
+    if (!warp_wait(&s.task_full[q], qphase, p, s, 6)) break;
+    const Task task = s.tasks[q];
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&s.task_empty[q]);
+    if (++q == kTaskRing) {
+      q = 0;
+      qphase ^= 1;
+    }
+    if (task.phase < 0) break;
+    if (!warp_wait(&s.acc_full[acc], acc_phase, p, s, 7)) break;
+    ptx::tc_fence_after();
+    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * 256;
+    const bool valid = r < p.BM;
+    const int slot = task.b * p.BM + r;
+    if (task.phase == 0) {
+      bf16* hrow = p.h + (size_t)slot * p.I + task.n * kL1TileN;
+#pragma unroll 1
+      for (int c = 0; c < kL1TileN / 32; ++c) {
+        uint32_t g[32], u[32];
+        ptx::tmem_ld32(tbase + c * 32, g);
+        ptx::tmem_ld32(tbase + kL1TileN + c * 32, u);
+        ptx::tmem_ld_wait();
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(hrow + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 o;
+            o.x = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 0]), __uint_as_float(u[8 * v + 0])),
+                              silu_mul(__uint_as_float(g[8 * v + 1]), __uint_as_float(u[8 * v + 1])));
+            o.y = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 2]), __uint_as_float(u[8 * v + 2])),
+                              silu_mul(__uint_as_float(g[8 * v + 3]), __uint_as_float(u[8 * v + 3])));
+            o.z = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 4]), __uint_as_float(u[8 * v + 4])),
+                              silu_mul(__uint_as_float(g[8 * v + 5]), __uint_as_float(u[8 * v + 5])));
+            o.w = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 6]), __uint_as_float(u[8 * v + 6])),
+                              silu_mul(__uint_as_float(g[8 * v + 7]), __uint_as_float(u[8 * v + 7])));
+            dst[v] = o;
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&s.acc_empty[acc]);
+      // Publish per warp (no cross-warp barrier): this warp's 32 h rows of the
+      // (block, n-tile) are written. Block b is complete at 4 * N1 arrivals.
+      __threadfence();
+      ptx::fence_proxy_async_global();
+      __syncwarp();
+      if (lane == 0 && task.b != p.withhold_block) ptx::red_release_gpu_add(p.l1_done + task.b, 1);
+    } else {
+      int tok = -1;
+      float w = 0.f;
+      if (valid) {
+        tok = p.slot_token[slot];
+        if (tok >= p.T) {
+          set_error(p, s, kDevBounds, 0x20000 | task.b);
+          tok = -1;
+        }
+        if (tok >= 0) {
+          const int j = p.slot_topk[slot];
+          if (j < 0 || j >= p.k) {
+            set_error(p, s, kDevBounds, 0x30000 | task.b);
+            tok = -1;
+          } else {
+            w = p.topk_w[(size_t)tok * p.k + j];
+          }
+        }
+      }
+      float* yrow = p.y_acc + (size_t)(tok < 0 ? 0 : tok) * p.H + task.n * p.BN2;
+#pragma unroll 1
+      for (int c = 0; c < p.BN2 / 32; ++c) {
+        uint32_t v[32];
+        ptx::tmem_ld32(tbase + c * 32, v);
+        ptx::tmem_ld_wait();
+        if (tok >= 0) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 o = make_float4(w * __uint_as_float(v[4 * i + 0]), w * __uint_as_float(v[4 * i + 1]),
+                                         w * __uint_as_float(v[4 * i + 2]), w * __uint_as_float(v[4 * i + 3]));
+            atomicAdd(reinterpret_cast<float4*>(yrow + c * 32 + 4 * i), o);
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&s.acc_empty[acc]);
+    }
+    if (++acc == 2) {
+      acc = 0;
+      acc_phase ^= 1;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1) moe_expert_gemm_kernel(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  GemmSmem& s = *reinterpret_cast<GemmSmem*>(tiles + (size_t)kStages * kStageBytes);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      ptx::mbar_init(&s.full[i], 1);
+      ptx::mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&s.acc_full[i], 1);
+      ptx::mbar_init(&s.acc_empty[i], 4);
+    }
+    for (int i = 0; i < kTaskRing; ++i) {
+      ptx::mbar_init(&s.task_full[i], 1);
+      ptx::mbar_init(&s.task_empty[i], 5);   // MMA lane 0 + one lane per epilogue warp
+    }
+    ptx::mbar_init(&s.mma_done, 1);
+    s.abort = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&p.tm_x);
+    ptx::prefetch_tmap(&p.tm_w1);
+    ptx::prefetch_tmap(&p.tm_w3);
+    ptx::prefetch_tmap(&p.tm_w2);
+    ptx::prefetch_tmap(&p.tm_h);
+  }
+  for (int e = threadIdx.x; e <= p.E; e += kGemmThreads) s.block_start[e] = p.block_start[e];
+  if (warp == 1) {
+    ptx::tmem_alloc(&s.tmem_base, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  // Rows >= BLOCK_M of the A tiles are never loaded: keep them zero.
+  if (p.BM < kTileM) {
+    const int row_bytes = 128;
+    for (int st = 0; st < kStages; ++st) {
+      uint4* a = reinterpret_cast<uint4*>(stage_ptr(tiles, st) + p.BM * row_bytes);
+      const int n = (kTileM - p.BM) * row_bytes / 16;
+      for (int i = threadIdx.x; i < n; i += kGemmThreads) a[i] = make_uint4(0, 0, 0, 0);
+    }
+    ptx::fence_proxy_async_shared();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = s.tmem_base;
+
+  if (warp == 0) gemm_producer(p, s, tiles);
+  else if (warp == 1) gemm_mma(p, s, tiles, tmem_base);
+  else gemm_epilogue(p, s, tmem_base);
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 1) ptx::tmem_dealloc(tmem_base, kTmemCols);
+}
+
+}  // namespace moe

@@ -1,0 +1,488 @@
+// Host side of the C ABI declared in include/moe_b200.h: plan, workspace
+// layout, TMA descriptors, launch sequence, error and profiling plumbing.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/moe_b200.h"
+#include "common.cuh"
+#include "dispatch.cuh"
+#include "expert_gemm.cuh"
+#include "router.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr int kNumKernels = 5;      // router, scan, scatter, expert GEMM, finalize
+constexpr int kMaxProfiled = 256;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Layout {
+  size_t err, sched, topk_idx, topk_w, rank, chunk_count, expert_count, expert_offset, block_start, num_padded,
+      slot_token, slot_topk, l1_done, h, y_acc, x_stage, y_stage, total;
+};
+
+class DeviceGuard {
+ public:
+  explicit DeviceGuard(int dev) {
+    cudaGetDevice(&prev_);
+    if (prev_ != dev) cudaSetDevice(dev);
+    dev_ = dev;
+  }
+  ~DeviceGuard() {
+    if (prev_ != dev_) cudaSetDevice(prev_);
+  }
+
+ private:
+  int prev_ = 0, dev_ = 0;
+};
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2D bf16 tensor map: `inner` contiguous elements per row, `rows` rows,
+// row pitch `pitch_elems`, box {64, box_rows}, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t pitch_elems,
+              uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {pitch_elems * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int block_m_rule(int T, int k, int E) {
+  // n = T*k/E compared against 16, 32, 64 without rounding
+  const long long tk = (long long)T * k;
+  if (tk <= 16LL * E) return 16;
+  if (tk <= 32LL * E) return 32;
+  if (tk <= 64LL * E) return 64;
+  return 128;
+}
+
+}  // namespace
+
+struct moe_plan {
+  int T_max, H, I, E, k, BM, device, num_sms;
+  int BN2, N1, N2, pool, chunks_max, blocks_max;
+  Layout L;
+  uint8_t* ws = nullptr;
+  size_t ws_bytes = 0;
+  bool profile = false;
+  std::vector<cudaEvent_t> ev;   // kMaxProfiled * (kNumKernels + 1)
+  int ev_used = 0;
+  int withhold = -1;
+  uint64_t timeout_ns = 2000000000ull;
+};
+
+static Layout make_layout(const moe_plan& p) {
+  Layout L{};
+  size_t o = 0;
+  auto take = [&](size_t bytes, size_t align) {
+    o = align_up(o, align);
+    const size_t at = o;
+    o += bytes;
+    return at;
+  };
+  const size_t tk = (size_t)p.T_max * p.k;
+  L.err = take(16 * 4, 256);
+  L.sched = take(16 * 4, 256);
+  L.topk_idx = take(tk * 4, 256);
+  L.topk_w = take(tk * 4, 256);
+  L.rank = take(tk * 4, 256);
+  L.chunk_count = take((size_t)p.chunks_max * p.E * 4, 256);
+  L.expert_count = take((size_t)p.E * 4, 256);
+  L.expert_offset = take((size_t)(p.E + 1) * 4, 256);
+  L.block_start = take((size_t)(p.E + 1) * 4, 256);
+  L.num_padded = L.sched + 2 * 4;
+  L.slot_token = take((size_t)p.pool * 4, 256);
+  L.slot_topk = take((size_t)p.pool * 4, 256);
+  L.l1_done = take((size_t)p.blocks_max * 4, 256);
+  L.h = take((size_t)p.pool * p.I * 2, 1024);
+  L.y_acc = take((size_t)p.T_max * p.H * 4, 1024);
+  L.x_stage = take((size_t)p.T_max * p.H * 2, 1024);
+  L.y_stage = take((size_t)p.T_max * p.H * 2, 1024);
+  L.total = align_up(o, 1024);
+  return L;
+}
+
+template <int EP>
+static cudaError_t launch_router(const RouterParams& rp, int T, cudaStream_t st) {
+  const int grid = (T + kRouterTokens - 1) / kRouterTokens;
+  moe_router_kernel<EP><<<grid, kRouterThreads, RouterSmem<EP>::kBytes, st>>>(rp);
+  return cudaGetLastError();
+}
+
+template <int EP>
+static cudaError_t set_router_smem() {
+  return cudaFuncSetAttribute(moe_router_kernel<EP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              RouterSmem<EP>::kBytes);
+}
+
+static int expert_pad(int E) {
+  int ep = 16;
+  while (ep < E) ep *= 2;
+  return ep;
+}
+
+static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias, const void* W1, const void* W3,
+                   const void* W2, int T, void* y, cudaStream_t st, bool full) {
+  if (p->ws == nullptr) return MOE_ERR_NO_WORKSPACE;
+  if (T < 0 || T > p->T_max) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;   // nothing to do; empty tensors may carry null pointers
+  if (x == nullptr || Wg == nullptr || !aligned16(x) || !aligned16(Wg)) return MOE_ERR_INVALID_ARG;
+  if (bias != nullptr && (reinterpret_cast<uintptr_t>(bias) & 3u)) return MOE_ERR_INVALID_ARG;
+  if (full) {
+    if (W1 == nullptr || W3 == nullptr || W2 == nullptr || y == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(W1) || !aligned16(W3) || !aligned16(W2) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  }
+  DeviceGuard guard(p->device);
+  uint8_t* ws = p->ws;
+  const Layout& L = p->L;
+  const bool prof = p->profile && p->ev_used < kMaxProfiled;
+  cudaEvent_t* ev = prof ? &p->ev[(size_t)p->ev_used * (kNumKernels + 1)] : nullptr;
+  auto mark = [&](int i) {
+    if (prof) cudaEventRecord(ev[i], st);
+  };
+  cudaError_t ce;
+
+  // 1. router (+ per-chunk histogram, + zero the output accumulator)
+  RouterParams rp;
+  rp.x = static_cast<const bf16*>(x);
+  rp.Wg = static_cast<const bf16*>(Wg);
+  rp.bias = bias;
+  rp.topk_idx = reinterpret_cast<int32_t*>(ws + L.topk_idx);
+  rp.topk_w = reinterpret_cast<float*>(ws + L.topk_w);
+  rp.rank = reinterpret_cast<int32_t*>(ws + L.rank);
+  rp.chunk_count = reinterpret_cast<int32_t*>(ws + L.chunk_count);
+  rp.y_acc = reinterpret_cast<float*>(ws + L.y_acc);
+  rp.T = T;
+  rp.H = p->H;
+  rp.E = p->E;
+  rp.k = p->k;
+  mark(0);
+  switch (expert_pad(p->E)) {
+    case 16: ce = launch_router<16>(rp, T, st); break;
+    case 32: ce = launch_router<32>(rp, T, st); break;
+    case 64: ce = launch_router<64>(rp, T, st); break;
+    case 128: ce = launch_router<128>(rp, T, st); break;
+    default: ce = launch_router<256>(rp, T, st); break;
+  }
+  if (ce != cudaSuccess) return MOE_ERR_CUDA;
+
+  // 2. dispatch scan, 3. dispatch scatter
+  DispatchParams dp;
+  dp.topk_idx = rp.topk_idx;
+  dp.rank = rp.rank;
+  dp.chunk_count = rp.chunk_count;
+  dp.expert_count = reinterpret_cast<int32_t*>(ws + L.expert_count);
+  dp.expert_offset = reinterpret_cast<int32_t*>(ws + L.expert_offset);
+  dp.block_start = reinterpret_cast<int32_t*>(ws + L.block_start);
+  dp.slot_token = reinterpret_cast<int32_t*>(ws + L.slot_token);
+  dp.slot_topk = reinterpret_cast<int32_t*>(ws + L.slot_topk);
+  dp.l1_done = reinterpret_cast<int32_t*>(ws + L.l1_done);
+  dp.sched = reinterpret_cast<int32_t*>(ws + L.sched);
+  dp.err = reinterpret_cast<int32_t*>(ws + L.err);
+  dp.T = T;
+  dp.E = p->E;
+  dp.k = p->k;
+  dp.BM = p->BM;
+  dp.num_chunks = (T + kRouterTokens - 1) / kRouterTokens;
+  dp.pool = p->pool;
+  mark(1);
+  moe_dispatch_scan_kernel<<<1, kScanThreads, 0, st>>>(dp);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  mark(2);
+  moe_dispatch_scatter_kernel<<<(T * p->k + 255) / 256, 256, 0, st>>>(dp);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  mark(3);
+  if (!full) {
+    if (prof) {
+      mark(4);
+      mark(5);
+      ++p->ev_used;
+    }
+    return MOE_OK;
+  }
+
+  // 4. persistent expert GEMM (L1 + SwiGLU, L2 + weighted scatter-add)
+  GemmParams gp;
+  std::memset(&gp, 0, sizeof(gp));
+  bf16* h = reinterpret_cast<bf16*>(ws + L.h);
+  const int E = p->E, H = p->H, I = p->I;
+  bool ok = make_map(&gp.tm_x, x, H, T, H, 1) &&
+            make_map(&gp.tm_w1, W1, I, (uint64_t)E * H, I, 64) &&
+            make_map(&gp.tm_w3, W3, I, (uint64_t)E * H, I, 64) &&
+            make_map(&gp.tm_w2, W2, H, (uint64_t)E * I, H, 64) &&
+            make_map(&gp.tm_h, h, I, p->pool, I, p->BM);
+  if (!ok) return MOE_ERR_CUDA;
+  gp.slot_token = dp.slot_token;
+  gp.slot_topk = dp.slot_topk;
+  gp.topk_w = rp.topk_w;
+  gp.block_start = dp.block_start;
+  gp.task_counter = dp.sched;
+  gp.l1_done = dp.l1_done;
+  gp.err = dp.err;
+  gp.h = h;
+  gp.y_acc = rp.y_acc;
+  gp.T = T;
+  gp.H = H;
+  gp.I = I;
+  gp.E = E;
+  gp.k = p->k;
+  gp.BM = p->BM;
+  gp.BN2 = p->BN2;
+  gp.N1 = p->N1;
+  gp.N2 = p->N2;
+  gp.timeout_ns = p->timeout_ns;
+  gp.withhold_block = p->withhold;
+  moe_expert_gemm_kernel<<<p->num_sms, kGemmThreads, kGemmSmemBytes, st>>>(gp);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  mark(4);
+
+  // 5. y = bf16(y_acc)
+  const size_t n4 = (size_t)T * H / 4;
+  const int fgrid = (int)std::min<size_t>((n4 + 255) / 256, (size_t)p->num_sms * 16);
+  moe_finalize_kernel<<<fgrid, 256, 0, st>>>(rp.y_acc, static_cast<bf16*>(y), n4);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  mark(5);
+  if (prof) ++p->ev_used;
+  return MOE_OK;
+}
+
+extern "C" {
+
+int moe_plan_create(moe_plan_t* out, int T_max, int H, int I, int E, int k, int block_m, int device) {
+  if (out == nullptr) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (T_max < 1 || H < 128 || H % 128 || I < 128 || I % 128 || E < 8 || E > 256 || E % 8 || k < 1 || k > 8 ||
+      k > E)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (block_m != 0 && block_m != 16 && block_m != 32 && block_m != 64 && block_m != 128)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  // int32 indexing of slots, h rows and T*k
+  if ((long long)T_max * k + (long long)E * 127 > (1LL << 30)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (device < 0 || device >= ndev) return MOE_ERR_INVALID_ARG;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) return MOE_ERR_CUDA;
+  if (prop.major != 10 || prop.minor != 0) return MOE_ERR_UNSUPPORTED_DEVICE;
+  if (tensor_map_encoder() == nullptr) return MOE_ERR_CUDA;
+
+  moe_plan* p = new (std::nothrow) moe_plan();
+  if (p == nullptr) return MOE_ERR_CUDA;
+  p->T_max = T_max;
+  p->H = H;
+  p->I = I;
+  p->E = E;
+  p->k = k;
+  p->BM = block_m ? block_m : block_m_rule(T_max, k, E);
+  p->device = device;
+  p->num_sms = prop.multiProcessorCount;
+  p->BN2 = (H % 256 == 0) ? 256 : 128;
+  p->N1 = I / kL1TileN;
+  p->N2 = H / p->BN2;
+  p->pool = T_max * k + E * (p->BM - 1);
+  p->pool = (p->pool + p->BM - 1) / p->BM * p->BM;
+  p->chunks_max = (T_max + kRouterTokens - 1) / kRouterTokens;
+  p->blocks_max = p->pool / p->BM;
+  p->L = make_layout(*p);
+
+  DeviceGuard guard(device);
+  cudaError_t ce = cudaFuncSetAttribute(moe_expert_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)kGemmSmemBytes);
+  if (ce == cudaSuccess) ce = set_router_smem<16>();
+  if (ce == cudaSuccess) ce = set_router_smem<32>();
+  if (ce == cudaSuccess) ce = set_router_smem<64>();
+  if (ce == cudaSuccess) ce = set_router_smem<128>();
+  if (ce == cudaSuccess) ce = set_router_smem<256>();
+  if (ce != cudaSuccess) {
+    delete p;
+    return MOE_ERR_CUDA;
+  }
+  *out = p;
+  return MOE_OK;
+}
+
+size_t moe_plan_workspace_bytes(moe_plan_t p) { return p ? p->L.total : 0; }
+
+int moe_plan_bind_workspace(moe_plan_t p, void* ws, size_t bytes) {
+  if (p == nullptr || ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_INVALID_ARG;
+  if (bytes < p->L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  p->ws = static_cast<uint8_t*>(ws);
+  p->ws_bytes = bytes;
+  DeviceGuard guard(p->device);
+  // error word and scheduler counters start at zero
+  if (cudaMemset(p->ws + p->L.err, 0, 16 * 4) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemset(p->ws + p->L.sched, 0, 16 * 4) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+int moe_plan_describe(moe_plan_t p, moe_plan_desc* d) {
+  if (p == nullptr || d == nullptr) return MOE_ERR_INVALID_ARG;
+  d->T_max = p->T_max;
+  d->H = p->H;
+  d->I = p->I;
+  d->E = p->E;
+  d->k = p->k;
+  d->block_m = p->BM;
+  d->pool_capacity = p->pool;
+  d->num_sms = p->num_sms;
+  d->workspace_bytes = p->L.total;
+  return MOE_OK;
+}
+
+int moe_plan_get_routing(moe_plan_t p, moe_routing* r) {
+  if (p == nullptr || r == nullptr) return MOE_ERR_INVALID_ARG;
+  if (p->ws == nullptr) return MOE_ERR_NO_WORKSPACE;
+  r->topk_idx = reinterpret_cast<int32_t*>(p->ws + p->L.topk_idx);
+  r->topk_w = reinterpret_cast<float*>(p->ws + p->L.topk_w);
+  r->expert_count = reinterpret_cast<int32_t*>(p->ws + p->L.expert_count);
+  r->expert_offset = reinterpret_cast<int32_t*>(p->ws + p->L.expert_offset);
+  r->slot_token = reinterpret_cast<int32_t*>(p->ws + p->L.slot_token);
+  r->slot_topk = reinterpret_cast<int32_t*>(p->ws + p->L.slot_topk);
+  r->num_padded = reinterpret_cast<int32_t*>(p->ws + p->L.num_padded);
+  r->block_m = p->BM;
+  r->pool_capacity = p->pool;
+  return MOE_OK;
+}
+
+int moe_forward(moe_plan_t p, const void* x, const void* Wg, const float* bias, const void* W1, const void* W3,
+                const void* W2, int T, void* y, void* stream) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  return enqueue(p, x, Wg, bias, W1, W3, W2, T, y, static_cast<cudaStream_t>(stream), true);
+}
+
+int moe_route(moe_plan_t p, const void* x, const void* Wg, const float* bias, int T, void* stream) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  return enqueue(p, x, Wg, bias, nullptr, nullptr, nullptr, T, nullptr, static_cast<cudaStream_t>(stream), false);
+}
+
+int moe_forward_host(moe_plan_t p, const void* x_host, const void* Wg, const float* bias, const void* W1,
+                     const void* W3, const void* W2, int T, void* y_host, void* stream) {
+  if (p == nullptr || x_host == nullptr || y_host == nullptr) return MOE_ERR_INVALID_ARG;
+  if (p->ws == nullptr) return MOE_ERR_NO_WORKSPACE;
+  if (T < 0 || T > p->T_max) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  DeviceGuard guard(p->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = (size_t)T * p->H * 2;
+  void* xd = p->ws + p->L.x_stage;
+  void* yd = p->ws + p->L.y_stage;
+  if (cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return MOE_ERR_CUDA;
+  const int rc = enqueue(p, xd, Wg, bias, W1, W3, W2, T, yd, st, true);
+  if (rc != MOE_OK) return rc;
+  if (cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+int moe_check(moe_plan_t p, void* stream, int32_t* detail) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  if (p->ws == nullptr) return MOE_ERR_NO_WORKSPACE;
+  DeviceGuard guard(p->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  int32_t e[2] = {0, 0};
+  if (cudaMemcpy(e, p->ws + p->L.err, sizeof(e), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (e[0] != 0 && cudaMemset(p->ws + p->L.err, 0, sizeof(e)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  if (detail) *detail = e[1];
+  switch (e[0]) {
+    case kDevOk: return MOE_OK;
+    case kDevTimeout: return MOE_ERR_DEVICE_TIMEOUT;
+    default: return MOE_ERR_DEVICE_BOUNDS;
+  }
+}
+
+int moe_plan_set_profiling(moe_plan_t p, int enable) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(p->device);
+  if (enable && p->ev.empty()) {
+    p->ev.resize((size_t)kMaxProfiled * (kNumKernels + 1));
+    for (auto& e : p->ev)
+      if (cudaEventCreate(&e) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  p->profile = enable != 0;
+  p->ev_used = 0;
+  return MOE_OK;
+}
+
+int moe_plan_profile_read(moe_plan_t p, float* ms, int* count) {
+  if (p == nullptr || ms == nullptr) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(p->device);
+  for (int i = 0; i < kNumKernels; ++i) ms[i] = 0.f;
+  const int n = p->ev_used;
+  if (n > 0 && cudaEventSynchronize(p->ev[(size_t)(n - 1) * (kNumKernels + 1) + kNumKernels]) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  for (int f = 0; f < n; ++f) {
+    cudaEvent_t* ev = &p->ev[(size_t)f * (kNumKernels + 1)];
+    for (int i = 0; i < kNumKernels; ++i) {
+      float t = 0.f;
+      if (cudaEventElapsedTime(&t, ev[i], ev[i + 1]) != cudaSuccess) return MOE_ERR_CUDA;
+      ms[i] += t;
+    }
+  }
+  if (count) *count = n;
+  p->ev_used = 0;
+  return MOE_OK;
+}
+
+int moe_plan_set_debug(moe_plan_t p, int withhold_block, uint64_t timeout_ns) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  p->withhold = withhold_block;
+  p->timeout_ns = timeout_ns ? timeout_ns : 2000000000ull;
+  return MOE_OK;
+}
+
+int moe_forward_kernel_count(void) { return kNumKernels; }
+
+void moe_plan_destroy(moe_plan_t p) {
+  if (p == nullptr) return;
+  {
+    DeviceGuard guard(p->device);
+    for (auto& e : p->ev) cudaEventDestroy(e);
+  }
+  delete p;
+}
+
+const char* moe_status_string(int s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MOE_ERR_NO_WORKSPACE: return "no workspace bound";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case MOE_ERR_DEVICE_BOUNDS: return "routing index out of range on the device";
+    case MOE_ERR_UNSUPPORTED_DEVICE: return "device is not sm_100";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,251 @@
+// Router: gate GEMM logits = x Wg (+ b), warp-level top-k, softmax over the
+// k selected logits, plus the per-chunk expert histogram and stable in-chunk
+// ranks that the dispatch scan consumes.
+//
+// Gate definition: "FlashMoE Kernel", opening paragraph (gate is the first step
+// of the fused layer); softmax top-k with weights renormalised over the k
+// selected experts. Within a token the k experts are written in ascending
+// expert id; ties in the selection go to the lower id.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace moe {
+
+struct RouterParams {
+  const bf16* x;        // [T, H]
+  const bf16* Wg;       // [H, E]
+  const float* bias;    // [E] or nullptr
+  int32_t* topk_idx;    // [T, k]
+  float* topk_w;        // [T, k]
+  int32_t* rank;        // [T, k]  rank of (t, j) among this chunk's tokens routed to the same expert
+  int32_t* chunk_count; // [num_chunks, E]
+  float* y_acc;         // [T, H] zeroed here, accumulated by the expert GEMM
+  int T, H, E, k;
+};
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  const int n = valid ? 16 : 0;   // zero-fill when out of range
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* p) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(s));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void* p) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(s));
+}
+__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Shared memory of one router CTA, for EP padded experts.
+template <int EP>
+struct RouterSmem {
+  static constexpr int kXStride = kRouterKChunk + 8;  // bf16 per x row (padding: no ldmatrix bank conflicts)
+  static constexpr int kWStride = EP + 8;             // bf16 per Wg row
+  static constexpr int kXBytes = kRouterTokens * kXStride * 2;
+  static constexpr int kWBytes = kRouterKChunk * kWStride * 2;
+  static constexpr int kStageBytes = kXBytes + kWBytes;
+  static constexpr int kLogitStride = EP + 1;         // fp32 per logit row
+  static constexpr int kTileBytes = 2 * kStageBytes;  // double-buffered; logits alias this after the K loop
+  static constexpr int kSelBytes = kRouterTokens * 8 * 4;
+  static constexpr int kBytes = kTileBytes + kSelBytes;
+  static_assert(kRouterTokens * kLogitStride * 4 <= kTileBytes, "logits must fit in the tile buffers");
+};
+
+template <int EP>
+__global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(const RouterParams p) {
+  using S = RouterSmem<EP>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int NT = EP / 8;   // n-tiles of 8 experts
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * kRouterTokens;
+  const int ntok = min(kRouterTokens, p.T - t0);
+
+  float acc[NT][4];
+#pragma unroll
+  for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+
+  auto load_chunk = [&](int stage, int kc) {
+    bf16* xs = reinterpret_cast<bf16*>(smem + stage * S::kStageBytes);
+    bf16* ws = reinterpret_cast<bf16*>(smem + stage * S::kStageBytes + S::kXBytes);
+    const int h0 = kc * kRouterKChunk;
+    // x: 64 rows x 8 chunks of 16 B
+    for (int i = threadIdx.x; i < kRouterTokens * 8; i += kRouterThreads) {
+      const int r = i >> 3, c = i & 7;
+      const bool ok = r < ntok;
+      const bf16* src = p.x + (size_t)(ok ? t0 + r : 0) * p.H + h0 + c * 8;
+      cp_async16(xs + r * S::kXStride + c * 8, src, ok);
+    }
+    // Wg: 64 rows x EP/8 chunks of 16 B (columns >= E zero-filled)
+    constexpr int CPR = EP / 8;
+    for (int i = threadIdx.x; i < kRouterKChunk * CPR; i += kRouterThreads) {
+      const int r = i / CPR, c = i % CPR;
+      const bool ok = c * 8 < p.E;
+      const bf16* src = p.Wg + (size_t)(h0 + r) * p.E + (ok ? c * 8 : 0);
+      cp_async16(ws + r * S::kWStride + c * 8, src, ok);
+    }
+    cp_async_commit();
+  };
+
+  const int nk = p.H / kRouterKChunk;
+  load_chunk(0, 0);
+  for (int kc = 0; kc < nk; ++kc) {
+    const int stage = kc & 1;
+    if (kc + 1 < nk) {
+      load_chunk(stage ^ 1, kc + 1);
+      cp_async_wait_1();
+    } else {
+      cp_async_wait_all();
+    }
+    __syncthreads();
+    const bf16* xs = reinterpret_cast<const bf16*>(smem + stage * S::kStageBytes);
+    const bf16* ws = reinterpret_cast<const bf16*>(smem + stage * S::kStageBytes + S::kXBytes);
+#pragma unroll
+    for (int ks = 0; ks < kRouterKChunk / 16; ++ks) {
+      uint32_t a[4];
+      ldmatrix_x4(a, xs + (warp * 16 + (lane & 15)) * S::kXStride + ks * 16 + (lane >> 4) * 8);
+#pragma unroll
+      for (int np = 0; np < NT / 2; ++np) {
+        uint32_t b[4];
+        const int q = lane >> 3, i = lane & 7;
+        ldmatrix_x4_trans(b, ws + (ks * 16 + (q & 1) * 8 + i) * S::kWStride + np * 16 + (q >> 1) * 8);
+        mma_16816(acc[2 * np], a, b[0], b[1]);
+        mma_16816(acc[2 * np + 1], a, b[2], b[3]);
+      }
+    }
+    __syncthreads();
+  }
+
+  // Logits (+ bias) to shared memory; padded experts get -inf.
+  float* logits = reinterpret_cast<float*>(smem);
+  {
+    const int r0 = warp * 16 + (lane >> 2);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int col = nt * 8 + 2 * (lane & 3) + h;
+        const float b = (col < p.E && p.bias != nullptr) ? p.bias[col] : 0.f;
+        const float v0 = col < p.E ? acc[nt][h] + b : -INFINITY;
+        const float v1 = col < p.E ? acc[nt][2 + h] + b : -INFINITY;
+        logits[r0 * S::kLogitStride + col] = v0;
+        logits[(r0 + 8) * S::kLogitStride + col] = v1;
+      }
+    }
+  }
+  __syncwarp();
+
+  // Warp-level top-k: each warp owns the 16 token rows it computed.
+  int32_t* sel = reinterpret_cast<int32_t*>(smem + S::kTileBytes);   // [64][8] ascending expert ids
+  constexpr int VPL = (EP + 31) / 32;
+  for (int rr = 0; rr < 16; ++rr) {
+    const int row = warp * 16 + rr;
+    if (row >= ntok) break;   // warp-uniform
+    float v[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = lane + 32 * i;
+      v[i] = e < EP ? logits[row * S::kLogitStride + e] : -INFINITY;
+    }
+    int chosen[8];
+    float chosen_l[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      chosen[r] = 0x7fffffff;
+      chosen_l[r] = -INFINITY;
+      if (r < p.k) {
+        float best = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+          const int e = lane + 32 * i;
+          if (e < p.E && (v[i] > best || (v[i] == best && e < bi))) {
+            best = v[i];
+            bi = e;
+          }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+          if (ob > best || (ob == best && oi < bi)) {
+            best = ob;
+            bi = oi;
+          }
+        }
+        chosen[r] = bi;
+        chosen_l[r] = best;
+        if ((bi & 31) == lane) {
+#pragma unroll
+          for (int i = 0; i < VPL; ++i)
+            if (i == (bi >> 5)) v[i] = -INFINITY;
+        }
+      }
+    }
+    // Softmax over the k selected; chosen_l[0] is their maximum.
+    float denom = 0.f;
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      if (r < p.k) denom += expf(chosen_l[r] - chosen_l[0]);
+    int me = 0x7fffffff;
+    float ml = 0.f;
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      if (r == lane) {
+        me = chosen[r];
+        ml = chosen_l[r];
+      }
+    if (lane < p.k) {
+      int pos = 0;   // position in ascending expert order
+#pragma unroll
+      for (int r = 0; r < 8; ++r) pos += (r < p.k && chosen[r] < me) ? 1 : 0;
+      const size_t o = (size_t)(t0 + row) * p.k + pos;
+      p.topk_idx[o] = me;
+      p.topk_w[o] = expf(ml - chosen_l[0]) / denom;
+      sel[row * 8 + pos] = me;
+    }
+  }
+  __syncthreads();
+
+  // Per-chunk histogram and stable ranks (tokens in ascending order).
+  for (int e = threadIdx.x; e < p.E; e += kRouterThreads) {
+    int cnt = 0;
+    for (int t = 0; t < ntok; ++t) {
+      for (int j = 0; j < p.k; ++j) {
+        if (sel[t * 8 + j] == e) {
+          p.rank[(size_t)(t0 + t) * p.k + j] = cnt;
+          ++cnt;
+        }
+      }
+    }
+    p.chunk_count[(size_t)blockIdx.x * p.E + e] = cnt;
+  }
+
+  // Zero this chunk's rows of the fp32 output accumulator.
+  {
+    float4* dst = reinterpret_cast<float4*>(p.y_acc + (size_t)t0 * p.H);
+    const size_t n4 = (size_t)ntok * p.H / 4;
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (size_t i = threadIdx.x; i < n4; i += kRouterThreads) dst[i] = z;
+  }
+}
+
+}  // namespace moe

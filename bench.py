@@ -1,0 +1,338 @@
+"""Benchmark of the single-GPU MoE-layer forward (tokens/s, device-timed).
+
+python bench.py --gpus N --steps K --warmup W [--workload NAME] [--impl reference]
+
+One step = one whole forward of the layer (router, dispatch scan, dispatch
+scatter, persistent expert GEMM, finalize) over one batch of T synthetic
+tokens whose inputs are already resident in HBM. Between timed steps the L2
+cache is flushed by writing a 256 MB buffer (outside the per-step events).
+With N > 1 (torchrun, one process per GPU) every rank runs an independent
+replica on its own T tokens (weak scaling, no collective in the data path);
+the step time is the max over ranks.
+
+The JSON line also carries:
+* roofline: the expert-GEMM kernel's achieved TFLOP/s (6*T*k*H*I algorithmic
+  FLOP per launch / its mean CUDA-event duration on the launching stream)
+  against the measured dense bf16 peak, and the whole layer's fraction of
+  max(FLOP / TC peak, bytes / HBM peak);
+* e2e: the same metric through the host-buffer entry point (x copied in from
+  pinned memory, y copied back, every step);
+* cpu_baseline: the fp64 CPU oracle timed on a bounded sample on rank 0;
+* clocks: SM clock samples and throttle reasons taken during the timed steps.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+BASELINE_METRIC = "MoE-layer fwd tokens/s on 1 B200 (device-timed); % of max(TC, HBM) roofline"
+DEFAULT_WORKLOAD = "mixtral"
+FLUSH_BYTES = 256 << 20
+ORACLE_SAMPLE = {"tiny": 64, "mixtral": 128, "fine_grained_prefill": 24, "decode": 8, "skewed": 512}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def workload_label(s):
+    return f"{s.name}: T={s.T} H={s.H} I={s.I} E={s.E} k={s.k}" + (" zipf-bias" if s.zipf_bias else "")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        rows = []
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) != 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        loaded = [r for r in rows if r[3] >= 50] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[4]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(loaded), "power_w_max": max(r[2] for r in rows)}
+
+
+# ------------------------------------------------------------------ oracle timing
+def time_oracle(inp, n_tokens: int):
+    """The fp64 CPU oracle as it stands, on the first n_tokens tokens (host copies of the inputs)."""
+    import numpy as np
+    import torch
+
+    import oracle.moe_oracle as O
+    x = inp["x"][:n_tokens].double().cpu().numpy()
+    Wg = inp["Wg"].double().cpu().numpy()
+    bias = None if inp["bias"] is None else inp["bias"].double().cpu().numpy()
+    W1c, W3c, W2c = inp["W1"].cpu(), inp["W3"].cpu(), inp["W2"].cpu()
+
+    def load(e):
+        return (W1c[e].double().numpy(), W3c[e].double().numpy(), W2c[e].double().numpy())
+
+    t0 = time.perf_counter()
+    O.moe_forward(x, Wg, bias, load, inp["k"])
+    dt = time.perf_counter() - t0
+    cores = None
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        cores = max([i.get("num_threads", 0) for i in info] + [torch.get_num_threads()])
+    except Exception:
+        cores = torch.get_num_threads()
+    del np
+    return n_tokens / dt, dt, cores
+
+
+# ------------------------------------------------------------------ main GPU arm
+def run_gpu(args, rank, world, local_rank):
+    import torch
+
+    from moe_megakernel_b200 import MoEPlan, kernels_per_forward
+    from synth.moe_inputs import WORKLOADS, make_inputs
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    shape = WORKLOADS[args.workload]
+    inp = make_inputs(shape, device=dev, seed=args.seed)
+    T, H, I, E, k = shape.T, shape.H, shape.I, shape.E, shape.k
+    plan = MoEPlan(T, H, I, E, k, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    args_fwd = (inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"])
+
+    def barrier():
+        if dist is not None:
+            dist.barrier(device_ids=[local_rank])
+
+    for _ in range(args.warmup):
+        plan.forward(*args_fwd, y=y)
+    plan.check()
+
+    # timed device steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    plan.set_profiling(True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        plan.forward(*args_fwd, y=y)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    plan.check()
+    kernel_ms, nprof = plan.profile_read()
+    plan.set_profiling(False)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    mean_ms = sum(step_ms) / len(step_ms)
+    if dist is not None:
+        t = torch.tensor([mean_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        mean_ms = t.item()
+
+    # end to end through the host-buffer entry point
+    x_host = inp["x"].cpu().pin_memory()
+    y_host = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    for _ in range(max(1, args.warmup)):
+        plan.forward_host(x_host, inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], y_host)
+    plan.check()
+    e2e_steps = max(3, args.steps)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        plan.forward_host(x_host, inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], y_host)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    plan.check()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+
+    # routing statistics for the roofline's byte count
+    r = plan.routing(T)
+    counts = r["expert_count"].cpu()
+    active = int((counts > 0).sum())
+    num_padded = int(r["num_padded"].item())
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        n = min(T, ORACLE_SAMPLE.get(args.workload, 64))
+        v, dt, cores = time_oracle(inp, n)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"fp64 oracle (gate, dispatch, expert FFN, combine) on the first {n} of {T} tokens "
+                         f"of the same inputs, {dt:.1f} s wall"}
+
+    if rank == 0:
+        peaks = measured_peaks()
+        flop = 6.0 * T * k * H * I
+        alg_bytes = 2.0 * 3 * H * I * active + 2.0 * H * E + 2.0 * T * H * 2
+        gemm_ms = kernel_ms["expert_gemm"] / max(nprof, 1)
+        achieved_tflops = flop / (gemm_ms * 1e-3) / 1e12
+        # the timed loop runs for seconds under the power cap: sustained peak
+        tc_peak = peaks["bf16_tflops_sustained"]
+        t_tc = flop / (tc_peak * 1e12)
+        t_hbm = alg_bytes / (peaks["hbm_gbs"] * 1e9)
+        bound = "tensor" if t_tc >= t_hbm else "hbm"
+        if bound == "tensor":
+            roof = {"bound": "tensor", "achieved": achieved_tflops, "peak": tc_peak, "unit": "TFLOP/s",
+                    "frac": achieved_tflops / tc_peak}
+        else:
+            gbs = alg_bytes / (gemm_ms * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": gbs / peaks["hbm_gbs"]}
+        roof.update({"kernel": "moe_expert_gemm_kernel", "traffic": None,
+                     "peak_source": f"{peaks['source']} ({'bf16_tflops_sustained' if bound == 'tensor' else 'hbm_gbs'})",
+                     "kernel_ms": gemm_ms,
+                     "layer_t_roof_ms": max(t_tc, t_hbm) * 1e3,
+                     "layer_frac": max(t_tc, t_hbm) * 1e3 / mean_ms,
+                     "kernel_ms_per_step": {kk: v / max(nprof, 1) for kk, v in kernel_ms.items()}})
+        tokens = T * world
+        line = {
+            "metric": BASELINE_METRIC,
+            "value": tokens / (mean_ms * 1e-3),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": mean_ms,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) x, N(0,1/H) Wg/W1/W3, N(0,1/I) W2, bf16; random-init weights)",
+            "config": {"workload": workload_label(shape), "T_per_gpu": T, "H": H, "I": I, "E": E, "k": k,
+                       "block_m": plan.block_m, "active_experts": active, "padded_slots": num_padded,
+                       "l2": "flushed between steps (256 MB write, outside per-step events)",
+                       "parallelism": "replicas" if world > 1 else "single"},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2,
+                    "ms_per_step": e2e_ms, "api": "moe_forward_host (pinned host x and y)"},
+            "gpu_launches": args.steps * kernels_per_forward(),
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier(device_ids=[local_rank])
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ reference arm (the oracle)
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import torch
+
+    from synth.moe_inputs import WORKLOADS, make_inputs
+    shape = WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(shape, device=dev, seed=args.seed)
+    n = min(shape.T, ORACLE_SAMPLE.get(args.workload, 64))
+    for _ in range(args.warmup):
+        time_oracle(inp, max(1, n // 8))
+    times, cores = [], None
+    for _ in range(args.steps):
+        v, dt, cores = time_oracle(inp, n)
+        times.append(dt)
+    value = n * len(times) / sum(times)
+    sample = f"fp64 CPU oracle on the first {n} of {shape.T} tokens per step"
+    print(json.dumps({
+        "impl": "reference", "metric": BASELINE_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sum(times) / len(times) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": workload_label(shape)},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if world != args.gpus:
+        world = max(world, 1)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_gpu(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -31,7 +31,11 @@ constexpr int kBoxBytes = 64 * kBK * 2;            // one 64x64 bf16 box, 8 KB
 constexpr int kTileBBytes = 4 * kBoxBytes;         // 32 KB
 constexpr int kStageBytes = kTileABytes + kTileBBytes;
 constexpr int kTaskRing = 4;
-constexpr int kGemmThreads = 192;                  // producer, MMA, 4 epilogue warps
+#ifndef MOE_GATHER_WARPS
+#define MOE_GATHER_WARPS 4
+#endif
+constexpr int kGatherWarps = MOE_GATHER_WARPS;     // warps that gather routed x rows
+constexpr int kGemmThreads = 192 + 32 * kGatherWarps;   // producer, MMA, 4 epilogue warps, gather warps
 constexpr int kTmemCols = 512;                     // two 256-column fp32 accumulators
 
 }  // namespace moe

@@ -8,16 +8,21 @@
 //   weighting are fused device routines. Here a task is (phase, expert,
 //   m-block, n-tile).
 // * "MegaMoE 在 MoE 系统谱系中的位置", section 2.1: warp roles inside the CTA
-//   (activation TMA, weight TMA, MMA issue, scheduler, epilogue). Here warp 0
-//   is scheduler + TMA producer, warp 1 issues tcgen05 MMAs, warps 2-5 drain
-//   TMEM in the epilogue.
+//   (dispatch/activation loads, weight TMA, MMA issue, scheduler, epilogue).
+//   Here warp 0 is scheduler + TMA producer of the weight tiles (and of the h
+//   tiles in L2), warp 1 issues tcgen05 MMAs, warps 2-5 drain TMEM in the
+//   epilogue, and warps 6.. gather the routed x rows for L1.
 // * Same page, section 2.7: tasks are claimed from a global atomic counter,
 //   and an L2 task of pool block b waits on an in-kernel counter until the L1
 //   tasks of block b are complete (bounded wait here).
 // * Same page, section 2.4: the slot's (token, top-k) record gives the
 //   combine's write address from the epilogue.
 // * ScatterMoE idea on the same page, section 一: the token gather is fused
-//   into the operand load (TMA gather4 of x rows), no permuted copy of x.
+//   into the operand load, no permuted copy of x. The routed x rows are
+//   fetched with 16-byte cp.async by the gather warps straight into the
+//   128-byte-swizzled K-major tile (a 4-row TMA gather costs far more TMA
+//   time than its 512 bytes are worth at this tile shape, and one warp of
+//   cp.async cannot keep up either); the weight tiles use TMA.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -29,7 +34,7 @@
 namespace moe {
 
 struct GemmParams {
-  CUtensorMap tm_x;    // x [T, H], box {64, 1}, gather4 rows
+  const bf16* x;       // [T, H]
   CUtensorMap tm_w1;   // W1 as [E*H, I], box {64, 64}
   CUtensorMap tm_w3;   // W3 as [E*H, I], box {64, 64}
   CUtensorMap tm_w2;   // W2 as [E*I, H], box {64, 64}
@@ -177,7 +182,7 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
       ptx::fence_proxy_async_global();
     }
 
-    // hand the task to the MMA and epilogue warps
+    // hand the task to the MMA, epilogue and gather warps
     if (!warp_wait(&s.task_empty[q], qphase ^ 1, p, s, 1)) break;
     if (lane == 0) {
       s.tasks[q] = task;
@@ -190,23 +195,6 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
     }
     if (task.phase < 0) break;
 
-    int rows[4] = {0, 0, 0, 0};
-    if (task.phase == 0) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = lane * 4 + i;
-        int tok = 0;
-        if (r < p.BM) {
-          tok = p.slot_token[task.b * p.BM + r];
-          if (tok >= p.T) {
-            set_error(p, s, kDevBounds, task.b);
-            tok = 0;
-          }
-          if (tok < 0) tok = 0;   // padding slot: any valid row, the epilogue drops it
-        }
-        rows[i] = tok;
-      }
-    }
     const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
@@ -214,16 +202,12 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
         ok = false;
         break;
       }
-      uint8_t* sa = stage_ptr(tiles, stage);
-      const uint32_t a_addr = ptx::smem_u32(sa);
+      const uint32_t a_addr = ptx::smem_u32(stage_ptr(tiles, stage));
       const uint32_t b_addr = a_addr + kTileABytes;
       if (task.phase == 0) {
-        if (lane == 0) ptx::mbar_arrive_expect_tx(&s.full[stage], p.BM * 128 + 4 * kBoxBytes);
-        __syncwarp();
-        if (lane * 4 < p.BM)
-          ptx::tma_gather4(a_addr + lane * 512, &p.tm_x, &s.full[stage], kb * kBK, rows[0], rows[1], rows[2],
-                           rows[3], pol);
+        // B: 128 columns of W1 next to the same 128 of W3; A comes from the gather warps.
         if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(&s.full[stage], 4 * kBoxBytes);
           const int wrow = task.e * p.H + kb * kBK;
           const int n0 = task.n * kL1TileN;
           ptx::tma_load_2d(b_addr + 0 * kBoxBytes, &p.tm_w1, &s.full[stage], n0, wrow, pol);
@@ -297,6 +281,7 @@ __device__ void gemm_mma(const GemmParams& p, GemmSmem& s, uint8_t* tiles, uint3
         break;
       }
       ptx::tc_fence_after();
+      ptx::fence_proxy_async_shared();   // cp.async-written A rows -> tensor-core reads
       if (lane == 0) {
         const uint32_t a_addr = ptx::smem_u32(stage_ptr(tiles, stage));
         const uint32_t b_addr = a_addr + kTileABytes;
@@ -335,6 +320,81 @@ __device__ void gemm_mma(const GemmParams& p, GemmSmem& s, uint8_t* tiles, uint3
       if (ptx::globaltimer() - t0 > p.timeout_ns) break;
     }
   }
+}
+
+// ---------------------------------------------------------------- gather warps (warps 6 .. 6+G-1)
+// L1 tasks: the A tile is BM routed rows of x, 64 columns per stage. Warp
+// instruction i (4 rows x 128 B, one 16-byte chunk per lane) is issued by
+// gather warp i % G; chunk c of row r lands at chunk c ^ (r % 8) of the
+// row's 128 bytes, the 128-byte swizzle the MMA descriptor expects. Every
+// lane arrives on the stage's full barrier when its own copies have landed.
+// L2 tasks: the producer loads A with TMA; each gather warp arrives for its
+// 32 lanes so that the barrier's arrival count is the same for both phases.
+__device__ void gemm_gather(const GemmParams& p, GemmSmem& s, uint8_t* tiles, int g) {
+  constexpr int kRowsPerLane = (kTileM / 4 + kGatherWarps - 1) / kGatherWarps;   // rows >= BM are skipped
+  const int lane = ptx::lane_id();
+  const int c = lane & 7;
+  int stage = 0;
+  uint32_t phase = 0;
+  int q = 0;
+  uint32_t qphase = 0;
+  while (true) {
+    if (!warp_wait(&s.task_full[q], qphase, p, s, 8)) break;
+    const Task task = s.tasks[q];
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&s.task_empty[q]);
+    if (++q == kTaskRing) {
+      q = 0;
+      qphase ^= 1;
+    }
+    if (task.phase < 0) break;
+    // token row and smem offset of each of this lane's rows
+    int nrows = 0;
+    uint32_t soff[kRowsPerLane];
+    const bf16* src[kRowsPerLane];
+    if (task.phase == 0) {
+#pragma unroll
+      for (int j = 0; j < kRowsPerLane; ++j) {
+        const int r = (j * kGatherWarps + g) * 4 + (lane >> 3);
+        soff[j] = r * 128 + ((c ^ (r & 7)) << 4);
+        src[j] = p.x + c * 8;
+        if (r < p.BM) {
+          int tok = p.slot_token[task.b * p.BM + r];
+          if (tok >= p.T) {
+            set_error(p, s, kDevBounds, task.b);
+            tok = 0;
+          }
+          if (tok < 0) tok = 0;   // padding slot: any valid row, the epilogue drops it
+          src[j] = p.x + (size_t)tok * p.H + c * 8;
+          nrows = j + 1;
+        }
+      }
+    }
+    const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
+    bool ok = true;
+    for (int kb = 0; kb < nk; ++kb) {
+      if (!warp_wait(&s.empty[stage], phase ^ 1, p, s, 9)) {
+        ok = false;
+        break;
+      }
+      if (task.phase == 0) {
+        const uint32_t a_addr = ptx::smem_u32(stage_ptr(tiles, stage));
+#pragma unroll
+        for (int j = 0; j < kRowsPerLane; ++j)
+          if (j < nrows) ptx::cp_async_16(a_addr + soff[j], src[j] + kb * kBK);
+        ptx::cp_async_mbar_arrive_noinc(&s.full[stage]);
+      } else {
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_count(&s.full[stage], 32);
+      }
+      if (++stage == kStages) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+    if (!ok) break;
+  }
+  ptx::cp_async_wait_all();
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
@@ -457,7 +517,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_expert_gemm_kernel(const 
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      ptx::mbar_init(&s.full[i], 1);
+      ptx::mbar_init(&s.full[i], 1 + 32 * kGatherWarps);   // producer + every gather lane
       ptx::mbar_init(&s.empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -466,14 +526,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_expert_gemm_kernel(const 
     }
     for (int i = 0; i < kTaskRing; ++i) {
       ptx::mbar_init(&s.task_full[i], 1);
-      ptx::mbar_init(&s.task_empty[i], 5);   // MMA lane 0 + one lane per epilogue warp
+      ptx::mbar_init(&s.task_empty[i], 5 + kGatherWarps);   // MMA, 4 epilogue warps, gather warps
     }
     ptx::mbar_init(&s.mma_done, 1);
     s.abort = 0;
     ptx::fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    ptx::prefetch_tmap(&p.tm_x);
     ptx::prefetch_tmap(&p.tm_w1);
     ptx::prefetch_tmap(&p.tm_w3);
     ptx::prefetch_tmap(&p.tm_w2);
@@ -501,7 +560,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_expert_gemm_kernel(const 
 
   if (warp == 0) gemm_producer(p, s, tiles);
   else if (warp == 1) gemm_mma(p, s, tiles, tmem_base);
-  else gemm_epilogue(p, s, tmem_base);
+  else if (warp < 6) gemm_epilogue(p, s, tmem_base);
+  else gemm_gather(p, s, tiles, warp - 6);
 
   ptx::tc_fence_before();
   __syncthreads();

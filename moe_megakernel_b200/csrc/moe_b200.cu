@@ -233,12 +233,12 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   std::memset(&gp, 0, sizeof(gp));
   bf16* h = reinterpret_cast<bf16*>(ws + L.h);
   const int E = p->E, H = p->H, I = p->I;
-  bool ok = make_map(&gp.tm_x, x, H, T, H, 1) &&
-            make_map(&gp.tm_w1, W1, I, (uint64_t)E * H, I, 64) &&
+  bool ok = make_map(&gp.tm_w1, W1, I, (uint64_t)E * H, I, 64) &&
             make_map(&gp.tm_w3, W3, I, (uint64_t)E * H, I, 64) &&
             make_map(&gp.tm_w2, W2, H, (uint64_t)E * I, H, 64) &&
             make_map(&gp.tm_h, h, I, p->pool, I, p->BM);
   if (!ok) return MOE_ERR_CUDA;
+  gp.x = static_cast<const bf16*>(x);
   gp.slot_token = dp.slot_token;
   gp.slot_topk = dp.slot_topk;
   gp.topk_w = rp.topk_w;

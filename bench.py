@@ -50,6 +50,28 @@ def measured_peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
+def kernel_source_hash() -> str:
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "moe_megakernel_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str):
+    """ncu DRAM bytes per expert-GEMM launch, if captured on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    cur = kernel_source_hash()
+    for line in open(p):
+        f = line.split()
+        if len(f) >= 3 and not f[0].startswith("#") and f[0] == workload and f[1] == cur:
+            return int(f[2])
+    return None
+
+
 def workload_label(s):
     return f"{s.name}: T={s.T} H={s.H} I={s.I} E={s.E} k={s.k}" + (" zipf-bias" if s.zipf_bias else "")
 
@@ -244,7 +266,8 @@ def run_gpu(args, rank, world, local_rank):
             gbs = alg_bytes / (gemm_ms * 1e-3) / 1e9
             roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": gbs / peaks["hbm_gbs"]}
-        roof.update({"kernel": "moe_expert_gemm_kernel", "traffic": None,
+        roof.update({"kernel": "moe_expert_gemm_kernel", "traffic": measured_traffic(args.workload),
+                     "traffic_unit": "bytes per launch (ncu dram read+write)",
                      "peak_source": f"{peaks['source']} ({'bf16_tflops_sustained' if bound == 'tensor' else 'hbm_gbs'})",
                      "kernel_ms": gemm_ms,
                      "layer_t_roof_ms": max(t_tc, t_hbm) * 1e3,
@@ -314,8 +337,8 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--seed", type=int, default=0)

@@ -55,7 +55,8 @@ typedef enum {
   MOE_ERR_CUDA = 5,                /* a CUDA runtime/driver call failed */
   MOE_ERR_DEVICE_TIMEOUT = 6,      /* a bounded device-side wait ran out (sticky, via moe_check) */
   MOE_ERR_DEVICE_BOUNDS = 7,       /* routing metadata held an out-of-range index (sticky) */
-  MOE_ERR_UNSUPPORTED_DEVICE = 8   /* the device is not sm_100 */
+  MOE_ERR_UNSUPPORTED_DEVICE = 8,  /* the device is not sm_100 */
+  MOE_ERR_STATIC_SCRATCH_LIMIT = 9 /* moe_route_static: sizes exceed its fixed scratch */
 } moe_status;
 
 /* Device views of the routing results inside the bound workspace. Valid after
@@ -168,6 +169,42 @@ int moe_plan_profile_read(moe_plan_t plan, float* ms, int* count);
  * withhold_block >= 0 makes the kernel never publish the completion of that
  * L1 block, so the L2 tasks waiting on it time out. -1 restores normal runs. */
 int moe_plan_set_debug(moe_plan_t plan, int withhold_block, uint64_t timeout_ns);
+
+/* Routing without any device allocation: the gate and the dispatch of
+ * moe_route(), for callers that cannot allocate device memory - for example
+ * code running inside an inference engine's enqueue-style callback where
+ * allocation is not allowed, a process whose device memory is fully
+ * reserved up front by a framework's pool so cudaMalloc would fail, or a
+ * latency-critical loop that cannot afford cudaMalloc's implicit device-wide
+ * synchronisation. It needs no plan and no workspace: its scratch (ranks,
+ * per-chunk counts, counters, error word) lives in a fixed 1 MiB device array
+ * inside this library, which every GPU that loads the library holds until the
+ * process exits. The pages have no counterpart of this entry point.
+ *
+ * Runs on the calling thread's current device; x [T,H] and Wg [H,E] (bf16),
+ * gate_bias [E] (fp32, or NULL) and every output are device pointers on it.
+ * The caller passes the outputs, laid out as in moe_routing:
+ *   topk_idx int32 [T,k], topk_w fp32 [T,k], expert_count int32 [E],
+ *   expert_offset int32 [E+1], slot_token and slot_topk int32 [pool_capacity],
+ *   num_padded int32 [1]; error_word int32 [1] or NULL receives the device
+ *   error code of this call (0 = none, 2 = a routing index out of range).
+ * block_m = 0 applies the same BLOCK_M rule as moe_plan_create. The slots in
+ * use are at most pool = ceil((T*k + E*(BLOCK_M-1)) / BLOCK_M) * BLOCK_M;
+ * pool_capacity must be at least that.
+ * Limit: 128 + T*k + ceil(T/64)*E + (E+1) + pool/BLOCK_M int32 values (each
+ * term rounded up to a multiple of 64) must fit in 262144; larger sizes return
+ * MOE_ERR_STATIC_SCRATCH_LIMIT before anything is enqueued (T = 16384, k = 8,
+ * E = 256 fits). Shape rules as moe_plan_create; T = 0 enqueues nothing.
+ * The first call on each device resolves the array's device address and sets
+ * kernel attributes (host-side set-up, no allocation); make that first call
+ * before any stream capture. Every call shares the one array and clears its
+ * error word itself, so calls whose GPU work overlaps in time (other streams,
+ * other host threads) race on the scratch: serialise them. Allocates nothing
+ * (no cudaMalloc, no cudaFree, no allocating library call). */
+int moe_route_static(const void* x, const void* Wg, const float* gate_bias, int T, int H, int E, int k,
+                     int block_m, int32_t* topk_idx, float* topk_w, int32_t* expert_count, int32_t* expert_offset,
+                     int32_t* slot_token, int32_t* slot_topk, int pool_capacity, int32_t* num_padded,
+                     int32_t* error_word, void* stream);
 
 /* Number of kernels one moe_forward launches (for launch accounting). */
 int moe_forward_kernel_count(void);

@@ -21,6 +21,7 @@ STATUS_NAMES = {
     0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_SHAPE",
     3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_NO_WORKSPACE", 5: "MOE_ERR_CUDA",
     6: "MOE_ERR_DEVICE_TIMEOUT", 7: "MOE_ERR_DEVICE_BOUNDS", 8: "MOE_ERR_UNSUPPORTED_DEVICE",
+    9: "MOE_ERR_STATIC_SCRATCH_LIMIT",
 }
 KERNEL_NAMES = ("router", "dispatch_scan", "dispatch_scatter", "expert_gemm", "finalize")
 
@@ -54,6 +55,8 @@ SIGNATURES = {
     "moe_plan_set_profiling": (_c_int, [_vp, _c_int]),
     "moe_plan_profile_read": (_c_int, [_vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_c_int)]),
     "moe_plan_set_debug": (_c_int, [_vp, _c_int, ctypes.c_uint64]),
+    "moe_route_static": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp,
+                                  _vp, _vp, _c_int, _vp, _vp, _vp]),
     "moe_forward_kernel_count": (_c_int, []),
     "moe_plan_destroy": (None, [_vp]),
     "moe_status_string": (ctypes.c_char_p, [_c_int]),

@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -273,6 +274,145 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   return MOE_OK;
 }
 
+// ---------------------------------------------------------------- routing with no allocation
+// Scratch of moe_route_static(): the error word, the dispatch counters, the
+// in-chunk ranks [T*k], the per-chunk expert counts [ceil(T/64)*E], the block
+// starts [E+1] and the per-block counters the dispatch scan clears. It is a
+// file-scope device array, so every GPU that loads this library holds these
+// 1 MiB until the process exits, and every call on a device uses the same copy.
+namespace {
+constexpr int kStaticScratchInts = 1 << 18;
+constexpr int kStaticMaxDevices = 64;
+std::mutex g_static_mu;
+int32_t* g_static_scratch[kStaticMaxDevices] = {};
+}  // namespace
+
+static __device__ __align__(256) int32_t g_route_scratch[kStaticScratchInts];
+
+// Once per device, with that device current: resolve the array's device
+// address (host code may not use the symbol itself as a pointer) and allow
+// the routing-only router its dynamic shared memory.
+static int static_scratch_for_current_device(int32_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kStaticMaxDevices) return MOE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_scratch[dev] == nullptr) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MOE_ERR_CUDA;
+    if (prop.major != 10 || prop.minor != 0) return MOE_ERR_UNSUPPORTED_DEVICE;
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_route_scratch) != cudaSuccess || ptr == nullptr) return MOE_ERR_CUDA;
+    cudaError_t ce = cudaFuncSetAttribute(moe_router_kernel<16, false>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, RouterSmem<16>::kBytes);
+    if (ce == cudaSuccess)
+      ce = cudaFuncSetAttribute(moe_router_kernel<32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                RouterSmem<32>::kBytes);
+    if (ce == cudaSuccess)
+      ce = cudaFuncSetAttribute(moe_router_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                RouterSmem<64>::kBytes);
+    if (ce == cudaSuccess)
+      ce = cudaFuncSetAttribute(moe_router_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                RouterSmem<128>::kBytes);
+    if (ce == cudaSuccess)
+      ce = cudaFuncSetAttribute(moe_router_kernel<256, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                RouterSmem<256>::kBytes);
+    if (ce != cudaSuccess) return MOE_ERR_CUDA;
+    g_static_scratch[dev] = static_cast<int32_t*>(ptr);
+  }
+  *out = g_static_scratch[dev];
+  return MOE_OK;
+}
+
+extern "C" int moe_route_static(const void* x, const void* Wg, const float* gate_bias, int T, int H, int E, int k,
+                                int block_m, int32_t* topk_idx, float* topk_w, int32_t* expert_count,
+                                int32_t* expert_offset, int32_t* slot_token, int32_t* slot_topk, int pool_capacity,
+                                int32_t* num_padded, int32_t* error_word, void* stream) {
+  if (T < 0 || H < 128 || H % 128 || E < 8 || E > 256 || E % 8 || k < 1 || k > 8 || k > E)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (block_m != 0 && block_m != 16 && block_m != 32 && block_m != 64 && block_m != 128)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  const int BM = block_m ? block_m : block_m_rule(T > 0 ? T : 1, k, E);
+  const long long pool = ((long long)T * k + (long long)E * (BM - 1) + BM - 1) / BM * BM;
+  const long long chunks = (T + kRouterTokens - 1) / kRouterTokens;
+  // scratch regions, each rounded up to 64 ints (256 bytes)
+  auto r64 = [](long long v) { return (v + 63) / 64 * 64; };
+  const long long o_err = 0, o_sched = 64, o_rank = 128;
+  const long long o_chunk = o_rank + r64((long long)T * k);
+  const long long o_bs = o_chunk + r64(chunks * E);
+  const long long o_l1 = o_bs + r64(E + 1);
+  const long long need = o_l1 + r64(pool / BM);
+  if (need > kStaticScratchInts) return MOE_ERR_STATIC_SCRATCH_LIMIT;
+  if (T == 0) return MOE_OK;
+  if (x == nullptr || Wg == nullptr || !aligned16(x) || !aligned16(Wg)) return MOE_ERR_INVALID_ARG;
+  if (gate_bias != nullptr && (reinterpret_cast<uintptr_t>(gate_bias) & 3u)) return MOE_ERR_INVALID_ARG;
+  if (topk_idx == nullptr || topk_w == nullptr || expert_count == nullptr || expert_offset == nullptr ||
+      slot_token == nullptr || slot_topk == nullptr || num_padded == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (pool_capacity < pool) return MOE_ERR_INVALID_ARG;
+  int32_t* scratch = nullptr;
+  int rc = static_scratch_for_current_device(&scratch);
+  if (rc != MOE_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // The error word must start at zero; everything else is fully written below.
+  if (cudaMemsetAsync(scratch + o_err, 0, 2 * sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  RouterParams rp;
+  rp.x = static_cast<const bf16*>(x);
+  rp.Wg = static_cast<const bf16*>(Wg);
+  rp.bias = gate_bias;
+  rp.topk_idx = topk_idx;
+  rp.topk_w = topk_w;
+  rp.rank = scratch + o_rank;
+  rp.chunk_count = scratch + o_chunk;
+  rp.y_acc = nullptr;
+  rp.T = T;
+  rp.H = H;
+  rp.E = E;
+  rp.k = k;
+  const int grid = (int)chunks;
+  switch (expert_pad(E)) {
+    case 16: moe_router_kernel<16, false><<<grid, kRouterThreads, RouterSmem<16>::kBytes, st>>>(rp); break;
+    case 32: moe_router_kernel<32, false><<<grid, kRouterThreads, RouterSmem<32>::kBytes, st>>>(rp); break;
+    case 64: moe_router_kernel<64, false><<<grid, kRouterThreads, RouterSmem<64>::kBytes, st>>>(rp); break;
+    case 128: moe_router_kernel<128, false><<<grid, kRouterThreads, RouterSmem<128>::kBytes, st>>>(rp); break;
+    default: moe_router_kernel<256, false><<<grid, kRouterThreads, RouterSmem<256>::kBytes, st>>>(rp); break;
+  }
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+
+  DispatchParams dp;
+  dp.topk_idx = topk_idx;
+  dp.rank = rp.rank;
+  dp.chunk_count = rp.chunk_count;
+  dp.expert_count = expert_count;
+  dp.expert_offset = expert_offset;
+  dp.block_start = scratch + o_bs;
+  dp.slot_token = slot_token;
+  dp.slot_topk = slot_topk;
+  dp.l1_done = scratch + o_l1;
+  dp.sched = scratch + o_sched;
+  dp.err = scratch + o_err;
+  dp.T = T;
+  dp.E = E;
+  dp.k = k;
+  dp.BM = BM;
+  dp.num_chunks = (int)chunks;
+  dp.pool = (int)pool;
+  moe_dispatch_scan_kernel<<<1, kScanThreads, 0, st>>>(dp);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  moe_dispatch_scatter_kernel<<<(T * k + 255) / 256, 256, 0, st>>>(dp);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  // slots in use (written by the scan) and the device error word, to the caller's buffers
+  if (cudaMemcpyAsync(num_padded, scratch + o_sched + 2, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (error_word != nullptr &&
+      cudaMemcpyAsync(error_word, scratch + o_err, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
 extern "C" {
 
 int moe_plan_create(moe_plan_t* out, int T_max, int H, int I, int E, int k, int block_m, int device) {
@@ -481,6 +621,7 @@ const char* moe_status_string(int s) {
     case MOE_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
     case MOE_ERR_DEVICE_BOUNDS: return "routing index out of range on the device";
     case MOE_ERR_UNSUPPORTED_DEVICE: return "device is not sm_100";
+    case MOE_ERR_STATIC_SCRATCH_LIMIT: return "sizes exceed the fixed scratch of moe_route_static";
     default: return "unknown status";
   }
 }

@@ -70,7 +70,9 @@ struct RouterSmem {
   static_assert(kRouterTokens * kLogitStride * 4 <= kTileBytes, "logits must fit in the tile buffers");
 };
 
-template <int EP>
+// kZeroAcc: also zero this chunk's rows of the fp32 output accumulator (the
+// full forward); routing-only callers without an accumulator pass false.
+template <int EP, bool kZeroAcc = true>
 __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(const RouterParams p) {
   using S = RouterSmem<EP>;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -240,7 +242,7 @@ __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(const Router
   }
 
   // Zero this chunk's rows of the fp32 output accumulator.
-  {
+  if constexpr (kZeroAcc) {
     float4* dst = reinterpret_cast<float4*>(p.y_acc + (size_t)t0 * p.H);
     const size_t n4 = (size_t)ntok * p.H / 4;
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -339,13 +339,23 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    help="named workload, or 'custom' with --shape")
+    ap.add_argument("--shape", default=None,
+                    help="T,H,I,E,k[,zipf] for --workload custom (e.g. a scaled-down case for profiling)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload == "custom":
+        if not args.shape:
+            ap.error("--workload custom needs --shape T,H,I,E,k[,zipf]")
+        from synth.moe_inputs import WORKLOADS, custom_shape
+        f = args.shape.split(",")
+        WORKLOADS["custom"] = custom_shape(*[int(v) for v in f[:5]], zipf=len(f) > 5 and f[5] == "zipf",
+                                           name="custom")
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))

@@ -37,5 +37,6 @@ constexpr int kTaskRing = 4;
 constexpr int kGatherWarps = MOE_GATHER_WARPS;     // warps that gather routed x rows
 constexpr int kGemmThreads = 192 + 32 * kGatherWarps;   // producer, MMA, 4 epilogue warps, gather warps
 constexpr int kTmemCols = 512;                     // two 256-column fp32 accumulators
+constexpr int kMaxGroups = 512;                    // block groups of the expert GEMM's task order
 
 }  // namespace moe

@@ -24,9 +24,13 @@ struct DispatchParams {
   int32_t* slot_token;       // [pool]
   int32_t* slot_topk;        // [pool]
   int32_t* l1_done;          // [pool / BLOCK_M] zeroed here
-  int32_t* sched;            // [0] task counter, [1] blocks, [2] padded slots
+  int32_t* sched;            // [0] task counter, [1] blocks, [2] padded slots, [3] block groups
   int32_t* err;              // sticky device error word
+  // Block groups of the expert GEMM's task order (nullptr: routing only, no groups).
+  int32_t* group_start;      // [max_groups + 1] first block of each group
+  int32_t* l2_done;          // [pool / BLOCK_M] zeroed here
   int T, E, k, BM, num_chunks, pool;
+  int group_min, group_max, max_groups;
 };
 
 constexpr int kScanThreads = 1024;
@@ -70,6 +74,37 @@ __global__ void __launch_bounds__(kScanThreads) moe_dispatch_scan_kernel(const D
     p.sched[0] = 0;
     p.sched[1] = acc;
     p.sched[2] = acc * p.BM;
+    if (p.group_start != nullptr) {
+      // Consecutive blocks form groups of at most group_max blocks; a group is
+      // closed at an expert boundary once it holds group_min blocks, so that
+      // small experts share a group and an expert's blocks rarely straddle two.
+      int ng = 0, cur = 0, start = 0;
+      p.group_start[0] = 0;
+      for (int e = 0; e < p.E; ++e) {
+        int nb = s_nb[e];
+        while (nb > 0) {
+          const int take = min(nb, p.group_max - cur);
+          cur += take;
+          nb -= take;
+          if (cur == p.group_max) {
+            start += cur;
+            cur = 0;
+            if (ng < p.max_groups) p.group_start[++ng] = start;
+          }
+        }
+        if (cur >= p.group_min) {
+          start += cur;
+          cur = 0;
+          if (ng < p.max_groups) p.group_start[++ng] = start;
+        }
+      }
+      if (cur > 0) {
+        start += cur;
+        if (ng < p.max_groups) p.group_start[++ng] = start;
+      }
+      if (start != acc) atomicCAS(p.err, 0, kDevBounds);   // more groups than max_groups
+      p.sched[3] = ng;
+    }
   }
   __syncthreads();
   for (int e = threadIdx.x; e <= p.E; e += kScanThreads) {
@@ -88,6 +123,8 @@ __global__ void __launch_bounds__(kScanThreads) moe_dispatch_scan_kernel(const D
   }
   const int nblocks = s_bs[p.E];
   for (int b = threadIdx.x; b < nblocks; b += kScanThreads) p.l1_done[b] = 0;
+  if (p.l2_done != nullptr)
+    for (int b = threadIdx.x; b < nblocks; b += kScanThreads) p.l2_done[b] = 0;
 }
 
 // One thread per routed pair (t, j): slot = offset[e] + chunk base + in-chunk rank.

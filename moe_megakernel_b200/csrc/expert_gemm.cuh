@@ -26,6 +26,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cstddef>
 #include <cstdint>
 
 #include "common.cuh"
@@ -38,17 +39,22 @@ struct GemmParams {
   CUtensorMap tm_w1;   // W1 as [E*H, I], box {64, 64}
   CUtensorMap tm_w3;   // W3 as [E*H, I], box {64, 64}
   CUtensorMap tm_w2;   // W2 as [E*I, H], box {64, 64}
-  CUtensorMap tm_h;    // h [pool, I], box {64, BM}
+  CUtensorMap tm_h;    // h ring [ring_blocks * BM, I], box {64, BM}
   const int32_t* slot_token;
   const int32_t* slot_topk;
   const float* topk_w;
   const int32_t* block_start;   // [E+1]
+  const int32_t* group_start;   // [groups + 1] first block of each block group
+  const int32_t* num_groups;    // [1]
   int32_t* task_counter;
-  int32_t* l1_done;             // [blocks]
+  int32_t* l1_done;             // [blocks] 4 arrivals per L1 n-tile of the block
+  int32_t* l2_done;             // [blocks] 1 arrival per L2 n-tile of the block
   int32_t* err;                 // [0] code, [1] detail
-  bf16* h;                      // [pool, I]
+  bf16* h;                      // ring of ring_blocks blocks of BM rows x I
   float* y_acc;                 // [T, H]
   int T, H, I, E, k, BM, BN2, N1, N2;
+  int ring_blocks;              // block b uses ring slot b % ring_blocks
+  int max_groups;
   unsigned long long timeout_ns;
   int withhold_block;           // test hook: never publish L1 completion of this block (-1: off)
 };
@@ -59,6 +65,10 @@ struct Task {
 };
 
 struct GemmSmem {
+  // L2 epilogue staging, per epilogue warp: 32 rows x 32 fp32 (rows padded to
+  // 144 B so that the 32 lanes' 16-byte stores hit distinct banks). First
+  // member, so 16-byte aligned as the bulk reduction's source must be.
+  float out_stage[4][32][36];
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t acc_full[2];
@@ -69,8 +79,13 @@ struct GemmSmem {
   Task tasks[kTaskRing];
   uint32_t tmem_base;
   int abort;
+  int num_groups;
   int block_start[257];
+  int group_start[kMaxGroups + 1];
 };
+
+static_assert(offsetof(GemmSmem, out_stage) % 16 == 0, "bulk-reduce source must be 16-byte aligned");
+static_assert((36 * 4) % 16 == 0, "staging rows must stay 16-byte aligned");
 
 constexpr size_t kGemmSmemBytes = 1024 /*alignment slack*/ + (size_t)kStages * kStageBytes + sizeof(GemmSmem);
 
@@ -100,36 +115,79 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xffffffffu, ok);
 }
 
+// Task order. Blocks are cut into groups (expert-aligned where possible) and
+// the phases interleave with a lag of one group:
+//   L1(0), L1(1), L2(0), L1(2), L2(1), ..., L1(G-1), L2(G-2), L2(G-1)
+// so that L2 tasks of a group start once its L1 tasks have had a whole
+// segment to finish, and the h ring only has to hold a few groups. Segment
+// s: s = 0 is L1(0); s = 2g-1 is L1(g) and s = 2g is L2(g-1) for g = 1..G
+// (L1(G) is empty). Inside a segment the order is (expert, n-tile, m-block)
+// so that the m-blocks sharing a weight slice run side by side.
+// Bounded wait (one thread) until *ctr >= need, with acquire semantics.
+__device__ __forceinline__ bool wait_counter(const int* ctr, int need, const GemmParams& p, GemmSmem& s,
+                                             int detail) {
+  if (ptx::ld_acquire_gpu(ctr) >= need) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  while (ptx::ld_acquire_gpu(ctr) < need) {
+    if (*reinterpret_cast<volatile int*>(&s.abort) || *reinterpret_cast<volatile int*>(p.err) != 0) return false;
+    if (ptx::globaltimer() - t0 > p.timeout_ns) {
+      set_error(p, s, kDevTimeout, detail);
+      return false;
+    }
+    __nanosleep(256);
+  }
+  return true;
+}
+
+__device__ __forceinline__ int segment_start(const GemmSmem& s, const GemmParams& p, int seg) {
+  const int G = s.num_groups;
+  if (seg == 0) return 0;
+  const int g = (seg + 1) >> 1;
+  if (seg & 1) return s.group_start[g] * p.N1 + s.group_start[g - 1] * p.N2;           // L1(g)
+  return s.group_start[min(g + 1, G)] * p.N1 + s.group_start[g - 1] * p.N2;            // L2(g-1)
+}
+
 __device__ __forceinline__ Task decode_task(int t, const GemmSmem& s, const GemmParams& p) {
   Task task{-1, 0, 0, 0};
+  const int G = s.num_groups;
   const int nb_total = s.block_start[p.E];
-  const int n_l1 = nb_total * p.N1;
-  const int n_l2 = nb_total * p.N2;
-  if (t < 0 || t >= n_l1 + n_l2) return task;
-  int NT, tt;
-  if (t < n_l1) {
-    task.phase = 0;
-    NT = p.N1;
-    tt = t;
-  } else {
-    task.phase = 1;
-    NT = p.N2;
-    tt = t - n_l1;
-  }
-  // expert e owns tasks [block_start[e]*NT, block_start[e+1]*NT); order inside: (n-tile, m-block)
-  const int vb = tt / NT;
-  int lo = 0, hi = p.E - 1;
+  if (t < 0 || t >= nb_total * (p.N1 + p.N2) || G <= 0) return task;
+  // last segment whose start is <= t (empty segments share the next start)
+  int lo = 0, hi = 2 * G;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (s.block_start[mid] <= vb) lo = mid;
+    if (segment_start(s, p, mid) <= t) lo = mid;
     else hi = mid - 1;
   }
-  const int e = lo;
-  const int nb = s.block_start[e + 1] - s.block_start[e];
-  const int local = tt - s.block_start[e] * NT;
+  const int seg = lo;
+  int g, NT;
+  if (seg == 0 || (seg & 1)) {
+    task.phase = 0;
+    g = (seg + 1) >> 1;
+    NT = p.N1;
+  } else {
+    task.phase = 1;
+    g = (seg >> 1) - 1;
+    NT = p.N2;
+  }
+  const int gb0 = s.group_start[g], gb1 = s.group_start[g + 1];
+  const int tl = t - segment_start(s, p, seg);
+  // expert of the tl-th task: its blocks inside the group occupy consecutive NT-task runs
+  const int vb = gb0 + tl / NT;
+  int elo = 0, ehi = p.E - 1;
+  while (elo < ehi) {
+    const int mid = (elo + ehi + 1) >> 1;
+    if (s.block_start[mid] <= vb) elo = mid;
+    else ehi = mid - 1;
+  }
+  const int e = elo;
+  const int eb0 = max(gb0, s.block_start[e]);
+  const int eb1 = min(gb1, s.block_start[e + 1]);
+  const int nb = eb1 - eb0;
+  const int local = tl - (eb0 - gb0) * NT;
   task.e = e;
   task.n = local / nb;
-  task.b = s.block_start[e] + (local - task.n * nb);
+  task.b = eb0 + (local - task.n * nb);
   return task;
 }
 
@@ -157,26 +215,9 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
 
     if (task.phase == 1) {
       // the L2 task of block b reads h rows written by all L1 n-tiles of block b
+      // (one arrival per epilogue warp per n-tile)
       bool ok = true;
-      if (lane == 0) {
-        const int* ctr = p.l1_done + task.b;
-        const int need = 4 * p.N1;   // one arrival per epilogue warp per L1 n-tile
-        if (ptx::ld_acquire_gpu(ctr) < need) {
-          const uint64_t t0 = ptx::globaltimer();
-          while (ptx::ld_acquire_gpu(ctr) < need) {
-            if (*reinterpret_cast<volatile int*>(&s.abort) || *reinterpret_cast<volatile int*>(p.err) != 0) {
-              ok = false;
-              break;
-            }
-            if (ptx::globaltimer() - t0 > p.timeout_ns) {
-              set_error(p, s, kDevTimeout, 0x10000 | task.b);
-              ok = false;
-              break;
-            }
-            __nanosleep(256);
-          }
-        }
-      }
+      if (lane == 0) ok = wait_counter(p.l1_done + task.b, 4 * p.N1, p, s, 0x10000 | task.b);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) task.phase = -1;
       ptx::fence_proxy_async_global();
@@ -219,7 +260,7 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
         if (lane == 0) {
           const int nbox = p.BN2 / 64;
           ptx::mbar_arrive_expect_tx(&s.full[stage], p.BM * 128 + nbox * kBoxBytes);
-          ptx::tma_load_2d(a_addr, &p.tm_h, &s.full[stage], kb * kBK, task.b * p.BM, pol);
+          ptx::tma_load_2d(a_addr, &p.tm_h, &s.full[stage], kb * kBK, (task.b % p.ring_blocks) * p.BM, pol);
           const int wrow = task.e * p.I + kb * kBK;
           for (int j = 0; j < nbox; ++j)
             ptx::tma_load_2d(b_addr + j * kBoxBytes, &p.tm_w2, &s.full[stage], task.n * p.BN2 + j * 64, wrow,
@@ -430,14 +471,24 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
     const bool valid = r < p.BM;
     const int slot = task.b * p.BM + r;
     if (task.phase == 0) {
-      bf16* hrow = p.h + (size_t)slot * p.I + task.n * kL1TileN;
+      // Ring slot of block b; its previous user, block b - ring_blocks, must
+      // have been read by all of its L2 n-tiles before it is overwritten.
+      bool store = valid;
+      if (task.b >= p.ring_blocks) {
+        bool ok = true;
+        if (lane == 0) ok = wait_counter(p.l2_done + (task.b - p.ring_blocks), p.N2, p, s, 0x40000 | task.b);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        store = store && ok;
+      }
+      const int ring_row = (task.b % p.ring_blocks) * p.BM + r;
+      bf16* hrow = p.h + (size_t)ring_row * p.I + task.n * kL1TileN;
 #pragma unroll 1
       for (int c = 0; c < kL1TileN / 32; ++c) {
         uint32_t g[32], u[32];
         ptx::tmem_ld32(tbase + c * 32, g);
         ptx::tmem_ld32(tbase + kL1TileN + c * 32, u);
         ptx::tmem_ld_wait();
-        if (valid) {
+        if (store) {
           uint4* dst = reinterpret_cast<uint4*>(hrow + c * 32);
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
@@ -464,6 +515,9 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
       __syncwarp();
       if (lane == 0 && task.b != p.withhold_block) ptx::red_release_gpu_add(p.l1_done + task.b, 1);
     } else {
+      // This task's MMAs are complete, so its h tiles have been read: one
+      // arrival on the block's L2 counter frees the ring slot once all N2 land.
+      if (quarter == 0 && lane == 0) ptx::red_release_gpu_add(p.l2_done + task.b, 1);
       int tok = -1;
       float w = 0.f;
       if (valid) {
@@ -482,19 +536,28 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
           }
         }
       }
+      // Combine: stage w * o for this row's 32 columns in shared memory, then
+      // one bulk reduction adds the 128 bytes into y_acc[token] (the L2 does the
+      // fp32 adds). Each lane reuses its own staging row once its previous
+      // reduction has read it.
       float* yrow = p.y_acc + (size_t)(tok < 0 ? 0 : tok) * p.H + task.n * p.BN2;
+      float* srow = &s.out_stage[quarter][lane][0];
+      const uint32_t srow_addr = ptx::smem_u32(srow);
 #pragma unroll 1
       for (int c = 0; c < p.BN2 / 32; ++c) {
         uint32_t v[32];
         ptx::tmem_ld32(tbase + c * 32, v);
         ptx::tmem_ld_wait();
         if (tok >= 0) {
+          ptx::bulk_wait_read_all();
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float4 o = make_float4(w * __uint_as_float(v[4 * i + 0]), w * __uint_as_float(v[4 * i + 1]),
-                                         w * __uint_as_float(v[4 * i + 2]), w * __uint_as_float(v[4 * i + 3]));
-            atomicAdd(reinterpret_cast<float4*>(yrow + c * 32 + 4 * i), o);
-          }
+          for (int i = 0; i < 8; ++i)
+            reinterpret_cast<float4*>(srow)[i] =
+                make_float4(w * __uint_as_float(v[4 * i + 0]), w * __uint_as_float(v[4 * i + 1]),
+                            w * __uint_as_float(v[4 * i + 2]), w * __uint_as_float(v[4 * i + 3]));
+          ptx::fence_proxy_async_shared();
+          ptx::bulk_reduce_add_f32(yrow + c * 32, srow_addr, 128);
+          ptx::bulk_commit();
         }
       }
       ptx::tc_fence_before();
@@ -506,6 +569,7 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
       acc_phase ^= 1;
     }
   }
+  ptx::bulk_wait_all();   // every combine reduction has landed before the CTA retires
 }
 
 __global__ void __launch_bounds__(kGemmThreads, 1) moe_expert_gemm_kernel(const __grid_constant__ GemmParams p) {
@@ -539,6 +603,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_expert_gemm_kernel(const 
     ptx::prefetch_tmap(&p.tm_h);
   }
   for (int e = threadIdx.x; e <= p.E; e += kGemmThreads) s.block_start[e] = p.block_start[e];
+  {
+    const int ng = min(*p.num_groups, min(p.max_groups, kMaxGroups));
+    if (threadIdx.x == 0) s.num_groups = ng;
+    for (int g = threadIdx.x; g <= ng; g += kGemmThreads) s.group_start[g] = p.group_start[g];
+  }
   if (warp == 1) {
     ptx::tmem_alloc(&s.tmem_base, kTmemCols);
     ptx::tmem_relinquish();

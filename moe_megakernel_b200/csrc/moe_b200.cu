@@ -28,7 +28,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Layout {
   size_t err, sched, topk_idx, topk_w, rank, chunk_count, expert_count, expert_offset, block_start, num_padded,
-      slot_token, slot_topk, l1_done, h, y_acc, x_stage, y_stage, total;
+      slot_token, slot_topk, l1_done, l2_done, group_start, h, y_acc, x_stage, y_stage, total;
 };
 
 class DeviceGuard {
@@ -89,6 +89,7 @@ int block_m_rule(int T, int k, int E) {
 struct moe_plan {
   int T_max, H, I, E, k, BM, device, num_sms;
   int BN2, N1, N2, pool, chunks_max, blocks_max;
+  int group_min, group_max, max_groups, ring_blocks;   // expert-GEMM task groups and h ring
   Layout L;
   uint8_t* ws = nullptr;
   size_t ws_bytes = 0;
@@ -122,7 +123,9 @@ static Layout make_layout(const moe_plan& p) {
   L.slot_token = take((size_t)p.pool * 4, 256);
   L.slot_topk = take((size_t)p.pool * 4, 256);
   L.l1_done = take((size_t)p.blocks_max * 4, 256);
-  L.h = take((size_t)p.pool * p.I * 2, 1024);
+  L.l2_done = take((size_t)p.blocks_max * 4, 256);
+  L.group_start = take((size_t)(p.max_groups + 1) * 4, 256);
+  L.h = take((size_t)p.ring_blocks * p.BM * p.I * 2, 1024);
   L.y_acc = take((size_t)p.T_max * p.H * 4, 1024);
   L.x_stage = take((size_t)p.T_max * p.H * 2, 1024);
   L.y_stage = take((size_t)p.T_max * p.H * 2, 1024);
@@ -213,6 +216,11 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   dp.BM = p->BM;
   dp.num_chunks = (T + kRouterTokens - 1) / kRouterTokens;
   dp.pool = p->pool;
+  dp.group_start = reinterpret_cast<int32_t*>(ws + L.group_start);
+  dp.l2_done = reinterpret_cast<int32_t*>(ws + L.l2_done);
+  dp.group_min = p->group_min;
+  dp.group_max = p->group_max;
+  dp.max_groups = p->max_groups;
   mark(1);
   moe_dispatch_scan_kernel<<<1, kScanThreads, 0, st>>>(dp);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
@@ -237,15 +245,20 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   bool ok = make_map(&gp.tm_w1, W1, I, (uint64_t)E * H, I, 64) &&
             make_map(&gp.tm_w3, W3, I, (uint64_t)E * H, I, 64) &&
             make_map(&gp.tm_w2, W2, H, (uint64_t)E * I, H, 64) &&
-            make_map(&gp.tm_h, h, I, p->pool, I, p->BM);
+            make_map(&gp.tm_h, h, I, (uint64_t)p->ring_blocks * p->BM, I, p->BM);
   if (!ok) return MOE_ERR_CUDA;
   gp.x = static_cast<const bf16*>(x);
   gp.slot_token = dp.slot_token;
   gp.slot_topk = dp.slot_topk;
   gp.topk_w = rp.topk_w;
   gp.block_start = dp.block_start;
+  gp.group_start = dp.group_start;
+  gp.num_groups = dp.sched + 3;
   gp.task_counter = dp.sched;
   gp.l1_done = dp.l1_done;
+  gp.l2_done = dp.l2_done;
+  gp.ring_blocks = p->ring_blocks;
+  gp.max_groups = p->max_groups;
   gp.err = dp.err;
   gp.h = h;
   gp.y_acc = rp.y_acc;
@@ -399,6 +412,9 @@ extern "C" int moe_route_static(const void* x, const void* Wg, const float* gate
   dp.BM = BM;
   dp.num_chunks = (int)chunks;
   dp.pool = (int)pool;
+  dp.group_start = nullptr;   // routing only: no expert-GEMM task groups
+  dp.l2_done = nullptr;
+  dp.group_min = dp.group_max = dp.max_groups = 0;
   moe_dispatch_scan_kernel<<<1, kScanThreads, 0, st>>>(dp);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   moe_dispatch_scatter_kernel<<<(T * k + 255) / 256, 256, 0, st>>>(dp);
@@ -450,6 +466,17 @@ int moe_plan_create(moe_plan_t* out, int T_max, int H, int I, int E, int k, int 
   p->pool = (p->pool + p->BM - 1) / p->BM * p->BM;
   p->chunks_max = (T_max + kRouterTokens - 1) / kRouterTokens;
   p->blocks_max = p->pool / p->BM;
+  // Task groups (see the expert GEMM's task order): an L1 segment of at least
+  // two waves of tasks so the one-group lag hides L1 completion; groups up to
+  // an expert's expected block count so weight slices stay shared; at most
+  // kMaxGroups groups. The h ring holds 3 groups: the block that last used a
+  // slot is then two segments back in the task order.
+  p->group_min = (2 * p->num_sms + p->N1 - 1) / p->N1;
+  p->group_min = std::max(p->group_min, (p->blocks_max + kMaxGroups - 3) / (kMaxGroups - 2));
+  const int per_expert = (int)(((long long)T_max * k + (long long)E * p->BM - 1) / ((long long)E * p->BM)) + 1;
+  p->group_max = std::max(2 * p->group_min, per_expert);
+  p->max_groups = p->blocks_max / p->group_min + 2;
+  p->ring_blocks = std::min(3 * p->group_max, p->blocks_max);
   p->L = make_layout(*p);
 
   DeviceGuard guard(device);

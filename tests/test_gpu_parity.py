@@ -175,3 +175,20 @@ def test_profiling_counts_forwards():
         plan.forward(inp["x"], inp["Wg"], None, inp["W1"], inp["W3"], inp["W2"])
     ms, n = plan.profile_read()
     assert n == 3 and all(v >= 0 for v in ms.values()) and ms["expert_gemm"] > 0
+
+
+def test_h_ring_wraps_many_times():
+    """I = 14336 makes the task groups 3-6 blocks, so the h ring is 18 blocks
+    for ~70 expert blocks: every slot is reused several times."""
+    from tests.parity_util import sample_tokens
+    shape = custom_shape(4096, 128, 14336, 32, 2)
+    inp = make_inputs(shape, device=DEV)
+    plan = _plan(shape)
+    _poison(plan)
+    y = plan.forward(inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"])
+    plan.check()
+    rows = sample_tokens(shape.T, 256)
+    ref = oracle_forward(inp, tokens=rows, block_m=plan.block_m)
+    assert_routing_equal(plan.routing(shape.T), ref)
+    assert int(ref["num_padded"]) // plan.block_m > 3 * 18
+    assert_y_close(y[torch.from_numpy(rows).to(y.device)], ref["y"])

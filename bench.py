@@ -72,6 +72,21 @@ def measured_traffic(workload: str):
     return None
 
 
+def reduce_max_over_ranks(value: float, dist, device) -> float:
+    """Max of a per-rank number over all ranks (identity on one process)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's step time."""
+    return tokens_per_rank * world / (max_ms * 1e-3)
+
+
 def workload_label(s):
     return f"{s.name}: T={s.T} H={s.H} I={s.I} E={s.E} k={s.k}" + (" zipf-bias" if s.zipf_bias else "")
 
@@ -206,11 +221,7 @@ def run_gpu(args, rank, world, local_rank):
     kernel_ms, nprof = plan.profile_read()
     plan.set_profiling(False)
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    mean_ms = sum(step_ms) / len(step_ms)
-    if dist is not None:
-        t = torch.tensor([mean_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        mean_ms = t.item()
+    mean_ms = reduce_max_over_ranks(sum(step_ms) / len(step_ms), dist, dev)
 
     # end to end through the host-buffer entry point
     x_host = inp["x"].cpu().pin_memory()
@@ -228,11 +239,7 @@ def run_gpu(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     plan.check()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
+    e2e_ms = reduce_max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dist, dev)
 
     # routing statistics for the roofline's byte count
     r = plan.routing(T)
@@ -273,10 +280,9 @@ def run_gpu(args, rank, world, local_rank):
                      "layer_t_roof_ms": max(t_tc, t_hbm) * 1e3,
                      "layer_frac": max(t_tc, t_hbm) * 1e3 / mean_ms,
                      "kernel_ms_per_step": {kk: v / max(nprof, 1) for kk, v in kernel_ms.items()}})
-        tokens = T * world
         line = {
             "metric": BASELINE_METRIC,
-            "value": tokens / (mean_ms * 1e-3),
+            "value": job_tokens_per_s(T, world, mean_ms),
             "unit": "tokens/s",
             "n_gpus": world,
             "steps": args.steps,
@@ -293,7 +299,7 @@ def run_gpu(args, rank, world, local_rank):
                        "parallelism": "replicas" if world > 1 else "single"},
             "roofline": roof,
             "cpu_baseline": cpu,
-            "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+            "e2e": {"value": job_tokens_per_s(T, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2,
                     "ms_per_step": e2e_ms, "api": "moe_forward_host (pinned host x and y)"},
             "gpu_launches": args.steps * kernels_per_forward(),

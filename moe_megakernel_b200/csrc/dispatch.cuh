@@ -35,53 +35,93 @@ struct DispatchParams {
 
 constexpr int kScanThreads = 1024;
 
-// One CTA. Thread e scans expert e's chunk counts; thread 0 scans the padded
-// block counts over experts (E <= 256 values).
+// One CTA. (1) Expert e's chunk counts are scanned by kScanThreads/E threads,
+// each over a contiguous range of chunks; (2) warp 0 scans the padded block
+// counts over experts with shuffles; (3) thread 0 forms the block groups
+// while the other threads write offsets, padding records and counters.
 __global__ void __launch_bounds__(kScanThreads) moe_dispatch_scan_kernel(const DispatchParams p) {
   __shared__ int32_t s_nb[257];
   __shared__ int32_t s_bs[257];
   __shared__ int32_t s_cnt[256];
-  for (int e = threadIdx.x; e < p.E; e += kScanThreads) {
-    int run = 0;
-    int c = 0;
+  __shared__ int32_t s_part[kScanThreads];
+  const int tid = threadIdx.x;
+  // (1) per-expert scan over chunks: threads per expert tpe (a power of two)
+  int tpe = 1;
+  while (tpe * 2 * p.E <= kScanThreads) tpe *= 2;
+  const int e = tid / tpe, sub = tid % tpe;
+  const int per = (p.num_chunks + tpe - 1) / tpe;
+  const int c0 = min(sub * per, p.num_chunks), c1 = min(c0 + per, p.num_chunks);
+  int local = 0;
+  if (e < p.E)
+    for (int c = c0; c < c1; ++c) local += p.chunk_count[(size_t)c * p.E + e];
+  s_part[tid] = local;
+  __syncthreads();
+  if (e < p.E) {
+    int base = 0;
+    for (int q = 0; q < sub; ++q) base += s_part[e * tpe + q];
+    if (sub == tpe - 1) {
+      const int run = base + local;
+      s_cnt[e] = run;
+      s_nb[e] = (run + p.BM - 1) / p.BM;
+    }
+    // counts -> per-chunk bases, 8 loads in flight before the 8 stores
     constexpr int U = 8;
-    for (; c + U <= p.num_chunks; c += U) {
+    int c = c0;
+    for (; c + U <= c1; c += U) {
       int v[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) v[u] = p.chunk_count[(size_t)(c + u) * p.E + e];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        p.chunk_count[(size_t)(c + u) * p.E + e] = run;
-        run += v[u];
+        p.chunk_count[(size_t)(c + u) * p.E + e] = base;
+        base += v[u];
       }
     }
-    for (; c < p.num_chunks; ++c) {
+    for (; c < c1; ++c) {
       const int v = p.chunk_count[(size_t)c * p.E + e];
-      p.chunk_count[(size_t)c * p.E + e] = run;
-      run += v;
+      p.chunk_count[(size_t)c * p.E + e] = base;
+      base += v;
     }
-    s_cnt[e] = run;
-    s_nb[e] = (run + p.BM - 1) / p.BM;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int e = 0; e < p.E; ++e) {
-      s_bs[e] = acc;
-      acc += s_nb[e];
+  // (2) exclusive scan of the block counts (E <= 256: 8 per lane)
+  if (tid < 32) {
+    int v[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ee = tid * 8 + i;
+      v[i] = ee < p.E ? s_nb[ee] : 0;
+      sum += v[i];
     }
-    s_bs[p.E] = acc;
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (tid >= off) incl += o;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ee = tid * 8 + i;
+      if (ee < p.E) s_bs[ee] = run;
+      run += v[i];
+    }
+    if (tid == 31) s_bs[p.E] = incl;
+  }
+  __syncthreads();
+  const int nblocks = s_bs[p.E];
+  if (tid == 0) {
     p.sched[0] = 0;
-    p.sched[1] = acc;
-    p.sched[2] = acc * p.BM;
+    p.sched[1] = nblocks;
+    p.sched[2] = nblocks * p.BM;
     if (p.group_start != nullptr) {
       // Consecutive blocks form groups of at most group_max blocks; a group is
       // closed at an expert boundary once it holds group_min blocks, so that
       // small experts share a group and an expert's blocks rarely straddle two.
       int ng = 0, cur = 0, start = 0;
       p.group_start[0] = 0;
-      for (int e = 0; e < p.E; ++e) {
-        int nb = s_nb[e];
+      for (int ee = 0; ee < p.E; ++ee) {
+        int nb = s_nb[ee];
         while (nb > 0) {
           const int take = min(nb, p.group_max - cur);
           cur += take;
@@ -102,29 +142,29 @@ __global__ void __launch_bounds__(kScanThreads) moe_dispatch_scan_kernel(const D
         start += cur;
         if (ng < p.max_groups) p.group_start[++ng] = start;
       }
-      if (start != acc) atomicCAS(p.err, 0, kDevBounds);   // more groups than max_groups
+      if (start != nblocks) atomicCAS(p.err, 0, kDevBounds);   // more groups than max_groups
       p.sched[3] = ng;
     }
+    return;
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e <= p.E; e += kScanThreads) {
-    p.block_start[e] = s_bs[e];
-    p.expert_offset[e] = s_bs[e] * p.BM;
-    if (e < p.E) p.expert_count[e] = s_cnt[e];
+  // (3) everything else, on threads 1..
+  for (int ee = tid - 1; ee <= p.E; ee += kScanThreads - 1) {
+    p.block_start[ee] = s_bs[ee];
+    p.expert_offset[ee] = s_bs[ee] * p.BM;
+    if (ee < p.E) p.expert_count[ee] = s_cnt[ee];
   }
   // padding slots of each expert's last block
-  for (int e = threadIdx.x; e < p.E; e += kScanThreads) {
-    const int beg = s_bs[e] * p.BM + s_cnt[e];
-    const int end = (s_bs[e] + s_nb[e]) * p.BM;
-    for (int s = beg; s < end && s < p.pool; ++s) {
-      p.slot_token[s] = -1;
-      p.slot_topk[s] = -1;
+  for (int ee = tid - 1; ee < p.E; ee += kScanThreads - 1) {
+    const int beg = s_bs[ee] * p.BM + s_cnt[ee];
+    const int end = (s_bs[ee] + s_nb[ee]) * p.BM;
+    for (int sl = beg; sl < end && sl < p.pool; ++sl) {
+      p.slot_token[sl] = -1;
+      p.slot_topk[sl] = -1;
     }
   }
-  const int nblocks = s_bs[p.E];
-  for (int b = threadIdx.x; b < nblocks; b += kScanThreads) p.l1_done[b] = 0;
+  for (int b = tid - 1; b < nblocks; b += kScanThreads - 1) p.l1_done[b] = 0;
   if (p.l2_done != nullptr)
-    for (int b = threadIdx.x; b < nblocks; b += kScanThreads) p.l2_done[b] = 0;
+    for (int b = tid - 1; b < nblocks; b += kScanThreads - 1) p.l2_done[b] = 0;
 }
 
 // One thread per routed pair (t, j): slot = offset[e] + chunk base + in-chunk rank.

@@ -80,6 +80,7 @@ struct GemmSmem {
   uint32_t tmem_base;
   int abort;
   int num_groups;
+  int rows[kTaskRing][kTileM];   // token row of each A-tile row, per task-ring slot (L1 tasks)
   int block_start[257];
   int group_start[kMaxGroups + 1];
 };
@@ -194,50 +195,87 @@ __device__ __forceinline__ Task decode_task(int t, const GemmSmem& s, const Gemm
 __device__ __forceinline__ uint8_t* stage_ptr(uint8_t* tiles, int stage) { return tiles + stage * kStageBytes; }
 
 // ---------------------------------------------------------------- producer (warp 0)
+// Scheduler and weight-tile TMA. The next task is claimed as soon as the
+// current one starts, and prepared (decoded; for L1 its routed row indices
+// staged in shared memory; for L2 its dependency counter probed) while the
+// current task's k-loop is being issued, so that task switches cost no
+// global round trip on the critical path.
+__device__ __forceinline__ int claim_task(const GemmParams& p, GemmSmem& s, int lane) {
+  int t = 0x7fffffff;
+  if (lane == 0) {
+    const bool stop =
+        *reinterpret_cast<volatile int*>(&s.abort) || *reinterpret_cast<volatile int*>(p.err) != 0;
+    if (!stop) t = atomicAdd(p.task_counter, 1);
+  }
+  return t;   // valid in lane 0 only
+}
+
+// Decode task t into ring slot q: for L1, stage the token row of every A-tile
+// row in s.rows[q]; for L2, report whether block b's L1 tiles are all done.
+__device__ __forceinline__ Task prepare_task(int t, int q, uint32_t qparity, bool& deps_ready, bool& ok,
+                                             const GemmParams& p, GemmSmem& s, int lane) {
+  Task task = decode_task(t, s, p);
+  deps_ready = true;
+  ok = warp_wait(&s.task_empty[q], qparity, p, s, 1);
+  if (!ok) return task;
+  if (task.phase == 0) {
+    for (int r = lane; r < p.BM; r += 32) {
+      int tok = p.slot_token[task.b * p.BM + r];
+      if (tok >= p.T) {
+        set_error(p, s, kDevBounds, task.b);
+        tok = 0;
+      }
+      s.rows[q][r] = tok < 0 ? 0 : tok;   // padding slot: any valid row, the epilogue drops it
+    }
+  } else if (task.phase == 1) {
+    int ready = 1;
+    if (lane == 0) ready = ptx::ld_acquire_gpu(p.l1_done + task.b) >= 4 * p.N1;
+    deps_ready = __shfl_sync(0xffffffffu, ready, 0) != 0;
+  }
+  __syncwarp();
+  return task;
+}
+
 __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) {
   const int lane = ptx::lane_id();
-  const uint64_t pol = ptx::policy_evict_normal();
+  // Weight tiles are streamed: the few m-blocks sharing a slice read it at
+  // nearly the same time, so mark it first to evict; h keeps the default.
+  const uint64_t pol = ptx::policy_evict_first();
+  const uint64_t polh = ptx::policy_evict_normal();
   int stage = 0;
   uint32_t phase = 0;
   int q = 0;
   uint32_t qphase = 0;
   uint32_t issued = 0, issued_parity = 0;   // per stage: ever issued, parity of the last issue
 
-  while (true) {
-    int t = 0x7fffffff;
-    if (lane == 0) {
-      const bool stop = *reinterpret_cast<volatile int*>(&s.abort) ||
-                        *reinterpret_cast<volatile int*>(p.err) != 0;
-      if (!stop) t = atomicAdd(p.task_counter, 1);
-    }
-    t = __shfl_sync(0xffffffffu, t, 0);
-    Task task = decode_task(t, s, p);
-
-    if (task.phase == 1) {
+  bool deps_ready = true, ok = true;
+  int t = __shfl_sync(0xffffffffu, claim_task(p, s, lane), 0);
+  Task task = prepare_task(t, q, qphase ^ 1, deps_ready, ok, p, s, lane);
+  while (ok) {
+    if (task.phase == 1 && !deps_ready) {
       // the L2 task of block b reads h rows written by all L1 n-tiles of block b
       // (one arrival per epilogue warp per n-tile)
-      bool ok = true;
-      if (lane == 0) ok = wait_counter(p.l1_done + task.b, 4 * p.N1, p, s, 0x10000 | task.b);
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      if (!ok) task.phase = -1;
-      ptx::fence_proxy_async_global();
+      bool fine = true;
+      if (lane == 0) fine = wait_counter(p.l1_done + task.b, 4 * p.N1, p, s, 0x10000 | task.b);
+      if (__shfl_sync(0xffffffffu, fine ? 1 : 0, 0) == 0) task.phase = -1;
     }
+    if (task.phase == 1) ptx::fence_proxy_async_global();   // h written by other CTAs -> TMA reads
 
-    // hand the task to the MMA, epilogue and gather warps
-    if (!warp_wait(&s.task_empty[q], qphase ^ 1, p, s, 1)) break;
+    // hand the task to the MMA, epilogue and gather warps (its slot was freed in prepare_task)
     if (lane == 0) {
       s.tasks[q] = task;
       ptx::mbar_arrive(&s.task_full[q]);
     }
     __syncwarp();
-    if (++q == kTaskRing) {
-      q = 0;
-      qphase ^= 1;
-    }
+    const int qn = (q + 1) % kTaskRing;
+    const uint32_t qphase_n = qn == 0 ? qphase ^ 1 : qphase;
     if (task.phase < 0) break;
 
+    const int t_next_lane0 = claim_task(p, s, lane);   // result consumed after a few stages
+    bool prepared = false;
+    Task next{-1, 0, 0, 0};
     const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
-    bool ok = true;
+    const int prep_at = nk > 2 ? 2 : nk - 1;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait(&s.empty[stage], phase ^ 1, p, s, 2)) {
         ok = false;
@@ -260,7 +298,7 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
         if (lane == 0) {
           const int nbox = p.BN2 / 64;
           ptx::mbar_arrive_expect_tx(&s.full[stage], p.BM * 128 + nbox * kBoxBytes);
-          ptx::tma_load_2d(a_addr, &p.tm_h, &s.full[stage], kb * kBK, (task.b % p.ring_blocks) * p.BM, pol);
+          ptx::tma_load_2d(a_addr, &p.tm_h, &s.full[stage], kb * kBK, (task.b % p.ring_blocks) * p.BM, polh);
           const int wrow = task.e * p.I + kb * kBK;
           for (int j = 0; j < nbox; ++j)
             ptx::tma_load_2d(b_addr + j * kBoxBytes, &p.tm_w2, &s.full[stage], task.n * p.BN2 + j * 64, wrow,
@@ -274,8 +312,21 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
         stage = 0;
         phase ^= 1;
       }
+      if (kb == prep_at) {
+        const int tn = __shfl_sync(0xffffffffu, t_next_lane0, 0);
+        next = prepare_task(tn, qn, qphase_n ^ 1, deps_ready, ok, p, s, lane);
+        prepared = true;
+        if (!ok) break;
+      }
     }
     if (!ok) break;
+    if (!prepared) {
+      const int tn = __shfl_sync(0xffffffffu, t_next_lane0, 0);
+      next = prepare_task(tn, qn, qphase_n ^ 1, deps_ready, ok, p, s, lane);
+    }
+    task = next;
+    q = qn;
+    qphase = qphase_n;
   }
   // On an early exit, let every issued copy land before the CTA can retire.
   for (int st = 0; st < kStages; ++st)
@@ -382,35 +433,31 @@ __device__ void gemm_gather(const GemmParams& p, GemmSmem& s, uint8_t* tiles, in
   while (true) {
     if (!warp_wait(&s.task_full[q], qphase, p, s, 8)) break;
     const Task task = s.tasks[q];
-    __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(&s.task_empty[q]);
+    const int q_task = q;
     if (++q == kTaskRing) {
       q = 0;
       qphase ^= 1;
     }
     if (task.phase < 0) break;
-    // token row and smem offset of each of this lane's rows
+    // smem offset and source row of each of this lane's rows (row indices staged by the producer)
     int nrows = 0;
     uint32_t soff[kRowsPerLane];
     const bf16* src[kRowsPerLane];
     if (task.phase == 0) {
+      const int* rows = s.rows[q_task];
 #pragma unroll
       for (int j = 0; j < kRowsPerLane; ++j) {
         const int r = (j * kGatherWarps + g) * 4 + (lane >> 3);
         soff[j] = r * 128 + ((c ^ (r & 7)) << 4);
         src[j] = p.x + c * 8;
         if (r < p.BM) {
-          int tok = p.slot_token[task.b * p.BM + r];
-          if (tok >= p.T) {
-            set_error(p, s, kDevBounds, task.b);
-            tok = 0;
-          }
-          if (tok < 0) tok = 0;   // padding slot: any valid row, the epilogue drops it
-          src[j] = p.x + (size_t)tok * p.H + c * 8;
+          src[j] = p.x + (size_t)rows[r] * p.H + c * 8;
           nrows = j + 1;
         }
       }
     }
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&s.task_empty[q_task]);   // slot (and its rows) free
     const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {

@@ -28,7 +28,8 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Layout {
   size_t err, sched, topk_idx, topk_w, rank, chunk_count, expert_count, expert_offset, block_start, num_padded,
-      slot_token, slot_topk, l1_done, l2_done, group_start, h, y_acc, x_stage, y_stage, total;
+      slot_token, slot_topk, l1_done, l2_done, group_start, router_partial, router_counter, h, y_acc, x_stage,
+      y_stage, total;
 };
 
 class DeviceGuard {
@@ -125,6 +126,8 @@ static Layout make_layout(const moe_plan& p) {
   L.l1_done = take((size_t)p.blocks_max * 4, 256);
   L.l2_done = take((size_t)p.blocks_max * 4, 256);
   L.group_start = take((size_t)(p.max_groups + 1) * 4, 256);
+  L.router_partial = take((size_t)kRouterSplitTiles * kRouterMaxSplit * kRouterTokens * 256 * 4, 256);
+  L.router_counter = take((size_t)kRouterSplitTiles * 4, 256);
   L.h = take((size_t)p.ring_blocks * p.BM * p.I * 2, 1024);
   L.y_acc = take((size_t)p.T_max * p.H * 4, 1024);
   L.x_stage = take((size_t)p.T_max * p.H * 2, 1024);
@@ -133,9 +136,21 @@ static Layout make_layout(const moe_plan& p) {
   return L;
 }
 
+// Number of H splits for the router: with few token tiles, spread the gate
+// GEMM over more CTAs (the largest divisor of H/64 up to kRouterMaxSplit).
+static int router_splits(int T, int H) {
+  const int tiles = (T + kRouterTokens - 1) / kRouterTokens;
+  if (tiles > kRouterSplitTiles) return 1;
+  const int nk = H / kRouterKChunk;
+  int s = 1;
+  for (int d = 1; d <= kRouterMaxSplit && d <= nk; ++d)
+    if (nk % d == 0) s = d;
+  return s;
+}
+
 template <int EP>
-static cudaError_t launch_router(const RouterParams& rp, int T, cudaStream_t st) {
-  const int grid = (T + kRouterTokens - 1) / kRouterTokens;
+static cudaError_t launch_router(const RouterParams& rp, int T, int splits, cudaStream_t st) {
+  const dim3 grid((T + kRouterTokens - 1) / kRouterTokens, splits);
   moe_router_kernel<EP><<<grid, kRouterThreads, RouterSmem<EP>::kBytes, st>>>(rp);
   return cudaGetLastError();
 }
@@ -183,17 +198,20 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   rp.rank = reinterpret_cast<int32_t*>(ws + L.rank);
   rp.chunk_count = reinterpret_cast<int32_t*>(ws + L.chunk_count);
   rp.y_acc = reinterpret_cast<float*>(ws + L.y_acc);
+  rp.partial = reinterpret_cast<float*>(ws + L.router_partial);
+  rp.tile_counter = reinterpret_cast<int32_t*>(ws + L.router_counter);
   rp.T = T;
   rp.H = p->H;
   rp.E = p->E;
   rp.k = p->k;
+  const int splits = router_splits(T, p->H);
   mark(0);
   switch (expert_pad(p->E)) {
-    case 16: ce = launch_router<16>(rp, T, st); break;
-    case 32: ce = launch_router<32>(rp, T, st); break;
-    case 64: ce = launch_router<64>(rp, T, st); break;
-    case 128: ce = launch_router<128>(rp, T, st); break;
-    default: ce = launch_router<256>(rp, T, st); break;
+    case 16: ce = launch_router<16>(rp, T, splits, st); break;
+    case 32: ce = launch_router<32>(rp, T, splits, st); break;
+    case 64: ce = launch_router<64>(rp, T, splits, st); break;
+    case 128: ce = launch_router<128>(rp, T, splits, st); break;
+    default: ce = launch_router<256>(rp, T, splits, st); break;
   }
   if (ce != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -380,6 +398,8 @@ extern "C" int moe_route_static(const void* x, const void* Wg, const float* gate
   rp.rank = scratch + o_rank;
   rp.chunk_count = scratch + o_chunk;
   rp.y_acc = nullptr;
+  rp.partial = nullptr;   // one CTA per token tile (no H split)
+  rp.tile_counter = nullptr;
   rp.T = T;
   rp.H = H;
   rp.E = E;
@@ -506,6 +526,7 @@ int moe_plan_bind_workspace(moe_plan_t p, void* ws, size_t bytes) {
   // error word and scheduler counters start at zero
   if (cudaMemset(p->ws + p->L.err, 0, 16 * 4) != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaMemset(p->ws + p->L.sched, 0, 16 * 4) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemset(p->ws + p->L.router_counter, 0, kRouterSplitTiles * 4) != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }

@@ -23,6 +23,11 @@ struct RouterParams {
   int32_t* rank;        // [T, k]  rank of (t, j) among this chunk's tokens routed to the same expert
   int32_t* chunk_count; // [num_chunks, E]
   float* y_acc;         // [T, H] zeroed here, accumulated by the expert GEMM
+  // Split of H over gridDim.y CTAs (small T): partial logits of each split,
+  // [tiles][splits][64][EP] fp32, and one arrival counter per token tile (zero
+  // between calls; the last CTA of a tile sums the splits and resets it).
+  float* partial;
+  int32_t* tile_counter;
   int T, H, E, k;
 };
 
@@ -107,12 +112,14 @@ __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(const Router
     cp_async_commit();
   };
 
-  const int nk = p.H / kRouterKChunk;
-  load_chunk(0, 0);
+  // this CTA's share of H: chunks [kc0, kc0 + nk)
+  const int nk = p.H / kRouterKChunk / gridDim.y;
+  const int kc0 = blockIdx.y * nk;
+  load_chunk(0, kc0);
   for (int kc = 0; kc < nk; ++kc) {
     const int stage = kc & 1;
     if (kc + 1 < nk) {
-      load_chunk(stage ^ 1, kc + 1);
+      load_chunk(stage ^ 1, kc0 + kc + 1);
       cp_async_wait_1();
     } else {
       cp_async_wait_all();
@@ -138,7 +145,58 @@ __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(const Router
 
   // Logits (+ bias) to shared memory; padded experts get -inf.
   float* logits = reinterpret_cast<float*>(smem);
-  {
+  if (gridDim.y > 1) {
+    // Split H: publish this split's partial logits; the last CTA of the token
+    // tile to arrive sums all splits in split order (deterministic).
+    __shared__ int s_last;
+    const int tile = blockIdx.x, nsplit = gridDim.y;
+    float* mine = p.partial + ((size_t)tile * nsplit + blockIdx.y) * kRouterTokens * EP;
+    const int r0 = warp * 16 + (lane >> 2);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int col = nt * 8 + 2 * (lane & 3) + h;
+        mine[r0 * EP + col] = acc[nt][h];
+        mine[(r0 + 8) * EP + col] = acc[nt][2 + h];
+      }
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(p.tile_counter + tile, 1) == nsplit - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    // 4 experts per thread and all splits' loads in flight at once; rows past
+    // the last token are not needed.
+    const float4* all = reinterpret_cast<const float4*>(p.partial + (size_t)tile * nsplit * kRouterTokens * EP);
+    const int stride4 = kRouterTokens * EP / 4;
+    for (int i = threadIdx.x; i < ntok * EP / 4; i += kRouterThreads) {
+      float4 part[kRouterMaxSplit];
+#pragma unroll
+      for (int sp = 0; sp < kRouterMaxSplit; ++sp)
+        if (sp < nsplit) part[sp] = __ldcg(all + (size_t)sp * stride4 + i);
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int sp = 0; sp < kRouterMaxSplit; ++sp)
+        if (sp < nsplit) {
+          v.x += part[sp].x;
+          v.y += part[sp].y;
+          v.z += part[sp].z;
+          v.w += part[sp].w;
+        }
+      const int row = (4 * i) / EP, col = (4 * i) % EP;
+      const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int cj = col + j;
+        const float b = (cj < p.E && p.bias != nullptr) ? p.bias[cj] : 0.f;
+        logits[row * S::kLogitStride + cj] = cj < p.E ? vv[j] + b : -INFINITY;
+      }
+    }
+    if (threadIdx.x == 0) p.tile_counter[tile] = 0;   // ready for the next call
+    __syncthreads();
+  } else {
     const int r0 = warp * 16 + (lane >> 2);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {

@@ -50,12 +50,14 @@ def measured_peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
+GEMM_SOURCES = ("common.cuh", "ptx.cuh", "expert_gemm.cuh")   # what the expert-GEMM kernel is built from
+
+
 def kernel_source_hash() -> str:
-    import glob
     import hashlib
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "moe_megakernel_b200", "csrc", "*"))):
-        h.update(open(f, "rb").read())
+    for f in GEMM_SOURCES:
+        h.update(open(os.path.join(ROOT, "moe_megakernel_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 

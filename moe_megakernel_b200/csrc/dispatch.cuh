@@ -116,31 +116,23 @@ __global__ void __launch_bounds__(kScanThreads) moe_dispatch_scan_kernel(const D
     p.sched[2] = nblocks * p.BM;
     if (p.group_start != nullptr) {
       // Consecutive blocks form groups of at most group_max blocks; a group is
-      // closed at an expert boundary once it holds group_min blocks, so that
-      // small experts share a group and an expert's blocks rarely straddle two.
-      int ng = 0, cur = 0, start = 0;
+      // closed at the first expert boundary at least group_min blocks after
+      // its start, so small experts share a group and an expert's blocks
+      // rarely straddle two. One binary search over the expert boundaries per
+      // group (block starts are non-decreasing).
+      int ng = 0, start = 0;
       p.group_start[0] = 0;
-      for (int ee = 0; ee < p.E; ++ee) {
-        int nb = s_nb[ee];
-        while (nb > 0) {
-          const int take = min(nb, p.group_max - cur);
-          cur += take;
-          nb -= take;
-          if (cur == p.group_max) {
-            start += cur;
-            cur = 0;
-            if (ng < p.max_groups) p.group_start[++ng] = start;
-          }
+      while (start < nblocks && ng < p.max_groups) {
+        const int target = start + p.group_min;
+        int lo = 0, hi = p.E;   // first e with block_start[e] >= target (E if none)
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (s_bs[mid] >= target) hi = mid;
+          else lo = mid + 1;
         }
-        if (cur >= p.group_min) {
-          start += cur;
-          cur = 0;
-          if (ng < p.max_groups) p.group_start[++ng] = start;
-        }
-      }
-      if (cur > 0) {
-        start += cur;
-        if (ng < p.max_groups) p.group_start[++ng] = start;
+        const int boundary = s_bs[lo] >= target ? s_bs[lo] : nblocks;
+        start = min(min(boundary, start + p.group_max), nblocks);
+        p.group_start[++ng] = start;
       }
       if (start != nblocks) atomicCAS(p.err, 0, kDevBounds);   // more groups than max_groups
       p.sched[3] = ng;

@@ -16,6 +16,7 @@
 #include "dispatch.cuh"
 #include "expert_gemm.cuh"
 #include "router.cuh"
+#include "router_tc.cuh"
 
 using namespace moe;
 
@@ -206,12 +207,34 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   rp.k = p->k;
   const int splits = router_splits(T, p->H);
   mark(0);
-  switch (expert_pad(p->E)) {
-    case 16: ce = launch_router<16>(rp, T, splits, st); break;
-    case 32: ce = launch_router<32>(rp, T, splits, st); break;
-    case 64: ce = launch_router<64>(rp, T, splits, st); break;
-    case 128: ce = launch_router<128>(rp, T, splits, st); break;
-    default: ce = launch_router<256>(rp, T, splits, st); break;
+  if (p->E % 64 == 0 && splits == 1) {
+    // many tokens, E a multiple of 64: gate GEMM on tcgen05
+    RouterTcParams tp;
+    std::memset(&tp, 0, sizeof(tp));
+    if (!make_map(&tp.tm_x, x, p->H, T, p->H, kRtcTokens) || !make_map(&tp.tm_wg, Wg, p->E, p->H, p->E, 64))
+      return MOE_ERR_CUDA;
+    tp.bias = bias;
+    tp.topk_idx = rp.topk_idx;
+    tp.topk_w = rp.topk_w;
+    tp.rank = rp.rank;
+    tp.chunk_count = rp.chunk_count;
+    tp.y_acc = rp.y_acc;
+    tp.err = reinterpret_cast<int32_t*>(ws + L.err);
+    tp.T = T;
+    tp.H = p->H;
+    tp.E = p->E;
+    tp.k = p->k;
+    tp.timeout_ns = p->timeout_ns;
+    moe_router_tc_kernel<<<(T + kRtcTokens - 1) / kRtcTokens, kRtcThreads, kRtcSmemBytes, st>>>(tp);
+    ce = cudaGetLastError();
+  } else {
+    switch (expert_pad(p->E)) {
+      case 16: ce = launch_router<16>(rp, T, splits, st); break;
+      case 32: ce = launch_router<32>(rp, T, splits, st); break;
+      case 64: ce = launch_router<64>(rp, T, splits, st); break;
+      case 128: ce = launch_router<128>(rp, T, splits, st); break;
+      default: ce = launch_router<256>(rp, T, splits, st); break;
+    }
   }
   if (ce != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -502,6 +525,8 @@ int moe_plan_create(moe_plan_t* out, int T_max, int H, int I, int E, int k, int 
   DeviceGuard guard(device);
   cudaError_t ce = cudaFuncSetAttribute(moe_expert_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)kGemmSmemBytes);
+  if (ce == cudaSuccess)
+    ce = cudaFuncSetAttribute(moe_router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRtcSmemBytes);
   if (ce == cudaSuccess) ce = set_router_smem<16>();
   if (ce == cudaSuccess) ce = set_router_smem<32>();
   if (ce == cudaSuccess) ce = set_router_smem<64>();

@@ -60,6 +60,32 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4],
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Per-chunk histogram and stable ranks for up to `nchunks` chunks of 64
+// tokens whose selected experts are in sel[t * 8 + j] (t local to the CTA):
+// every (t, j) sets bit t%64 of its expert's token mask; the count of an
+// expert is the mask's popcount and the rank of (t, j) the popcount of the
+// mask below bit t, i.e. the number of earlier tokens of the chunk routed to
+// the same expert. `mask` holds nchunks * E 64-bit words of shared memory.
+__device__ __forceinline__ void chunk_histogram(const int32_t* sel, unsigned long long* mask, int ntok,
+                                                int nchunks, int chunk0, int t0, int E, int k, int32_t* rank,
+                                                int32_t* chunk_count, int nthreads) {
+  for (int i = threadIdx.x; i < nchunks * E; i += nthreads) mask[i] = 0ull;
+  __syncthreads();
+  for (int i = threadIdx.x; i < ntok * k; i += nthreads) {
+    const int t = i / k, j = i - t * k;
+    atomicOr(&mask[(t >> 6) * E + sel[t * 8 + j]], 1ull << (t & 63));
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < ntok * k; i += nthreads) {
+    const int t = i / k, j = i - t * k;
+    const unsigned long long m = mask[(t >> 6) * E + sel[t * 8 + j]];
+    rank[(size_t)(t0 + t) * k + j] = __popcll(m & ((1ull << (t & 63)) - 1ull));
+  }
+  const int chunks_used = (ntok + 63) >> 6;
+  for (int i = threadIdx.x; i < chunks_used * E; i += nthreads)
+    chunk_count[(size_t)(chunk0 + i / E) * E + (i % E)] = __popcll(mask[i]);
+}
+
 // Shared memory of one router CTA, for EP padded experts.
 template <int EP>
 struct RouterSmem {
@@ -71,7 +97,8 @@ struct RouterSmem {
   static constexpr int kLogitStride = EP + 1;         // fp32 per logit row
   static constexpr int kTileBytes = 2 * kStageBytes;  // double-buffered; logits alias this after the K loop
   static constexpr int kSelBytes = kRouterTokens * 8 * 4;
-  static constexpr int kBytes = kTileBytes + kSelBytes;
+  static constexpr int kMaskBytes = 256 * 8;           // one 64-token chunk, E <= 256
+  static constexpr int kBytes = kTileBytes + kSelBytes + kMaskBytes;
   static_assert(kRouterTokens * kLogitStride * 4 <= kTileBytes, "logits must fit in the tile buffers");
 };
 
@@ -160,6 +187,14 @@ __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(const Router
         mine[r0 * EP + col] = acc[nt][h];
         mine[(r0 + 8) * EP + col] = acc[nt][2 + h];
       }
+    }
+    if constexpr (kZeroAcc) {
+      // every split zeroes its share of the tile's output-accumulator rows
+      const size_t n4 = (size_t)ntok * p.H / 4;
+      const size_t per = (n4 + nsplit - 1) / nsplit;
+      const size_t b0 = blockIdx.y * per, b1 = min(n4, b0 + per);
+      float4* dst = reinterpret_cast<float4*>(p.y_acc + (size_t)t0 * p.H);
+      for (size_t i = b0 + threadIdx.x; i < b1; i += kRouterThreads) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __threadfence();
     __syncthreads();
@@ -286,21 +321,11 @@ __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(const Router
   __syncthreads();
 
   // Per-chunk histogram and stable ranks (tokens in ascending order).
-  for (int e = threadIdx.x; e < p.E; e += kRouterThreads) {
-    int cnt = 0;
-    for (int t = 0; t < ntok; ++t) {
-      for (int j = 0; j < p.k; ++j) {
-        if (sel[t * 8 + j] == e) {
-          p.rank[(size_t)(t0 + t) * p.k + j] = cnt;
-          ++cnt;
-        }
-      }
-    }
-    p.chunk_count[(size_t)blockIdx.x * p.E + e] = cnt;
-  }
+  chunk_histogram(sel, reinterpret_cast<unsigned long long*>(smem + S::kTileBytes + S::kSelBytes), ntok, 1,
+                  blockIdx.x, t0, p.E, p.k, p.rank, p.chunk_count, kRouterThreads);
 
-  // Zero this chunk's rows of the fp32 output accumulator.
-  if constexpr (kZeroAcc) {
+  // Zero this chunk's rows of the fp32 output accumulator (the splits did it already).
+  if (kZeroAcc && gridDim.y == 1) {
     float4* dst = reinterpret_cast<float4*>(p.y_acc + (size_t)t0 * p.H);
     const size_t n4 = (size_t)ntok * p.H / 4;
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -190,6 +190,8 @@ def run_gpu(args, rank, world, local_rank):
     inp = make_inputs(shape, device=dev, seed=args.seed)
     T, H, I, E, k = shape.T, shape.H, shape.I, shape.E, shape.k
     plan = MoEPlan(T, H, I, E, k, device=dev)
+    if args.cta_pairs is not None:
+        plan.set_cta_pairs(bool(args.cta_pairs))
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
@@ -296,7 +298,7 @@ def run_gpu(args, rank, world, local_rank):
             "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) x, N(0,1/H) Wg/W1/W3, N(0,1/I) W2, bf16; random-init weights)",
             "config": {"workload": workload_label(shape), "T_per_gpu": T, "H": H, "I": I, "E": E, "k": k,
-                       "block_m": plan.block_m, "active_experts": active, "padded_slots": num_padded,
+                       "block_m": plan.block_m, "cta_pairs": bool(args.cta_pairs), "active_experts": active, "padded_slots": num_padded,
                        "l2": "flushed between steps (256 MB write, outside per-step events)",
                        "parallelism": "replicas" if world > 1 else "single"},
             "roofline": roof,
@@ -354,6 +356,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cta-pairs", type=int, default=None, choices=[0, 1],
+                    help="expert GEMM on CTA pairs (1) or one CTA per block (0); default: the plan's")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -89,6 +89,7 @@ typedef struct {
   int32_t block_m;         /* rows per expert block (16, 32, 64 or 128) */
   int32_t pool_capacity;   /* T_max*k + E*(block_m-1) slots */
   int32_t num_sms;         /* persistent grid size */
+  int32_t pair_clusters;   /* co-resident 2-CTA clusters of the CTA-pair expert GEMM */
   size_t workspace_bytes;
 } moe_plan_desc;
 
@@ -205,6 +206,14 @@ int moe_route_static(const void* x, const void* Wg, const float* gate_bias, int 
                      int block_m, int32_t* topk_idx, float* topk_w, int32_t* expert_count, int32_t* expert_offset,
                      int32_t* slot_token, int32_t* slot_topk, int pool_capacity, int32_t* num_padded,
                      int32_t* error_word, void* stream);
+
+/* Expert-GEMM variant: enable != 0 runs the persistent expert GEMM on CTA
+ * pairs (clusters of two CTAs on neighbouring SMs, tcgen05 cta_group::2):
+ * each task covers two consecutive blocks of one expert (256 rows) and each
+ * CTA loads half of the weight tile. enable = 0 runs one CTA per 128-row
+ * block. Results are the same up to fp32 summation order. Takes effect at the
+ * next moe_forward; the workspace size does not depend on it. */
+int moe_plan_set_cta_pairs(moe_plan_t plan, int enable);
 
 /* Number of kernels one moe_forward launches (for launch accounting). */
 int moe_forward_kernel_count(void);

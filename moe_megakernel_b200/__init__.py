@@ -38,7 +38,7 @@ class MoEPlanDesc(ctypes.Structure):
     _fields_ = [("T_max", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
                 ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("block_m", ctypes.c_int32),
                 ("pool_capacity", ctypes.c_int32), ("num_sms", ctypes.c_int32),
-                ("workspace_bytes", ctypes.c_size_t)]
+                ("pair_clusters", ctypes.c_int32), ("workspace_bytes", ctypes.c_size_t)]
 
 
 # exported symbol -> (restype, argtypes); the same list as include/moe_b200.h
@@ -57,6 +57,7 @@ SIGNATURES = {
     "moe_plan_set_debug": (_c_int, [_vp, _c_int, ctypes.c_uint64]),
     "moe_route_static": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp,
                                   _vp, _vp, _c_int, _vp, _vp, _vp]),
+    "moe_plan_set_cta_pairs": (_c_int, [_vp, _c_int]),
     "moe_forward_kernel_count": (_c_int, []),
     "moe_plan_destroy": (None, [_vp]),
     "moe_status_string": (ctypes.c_char_p, [_c_int]),
@@ -138,6 +139,7 @@ class MoEPlan:
         d = MoEPlanDesc()
         _ok(self.lib.moe_plan_describe(self._plan, ctypes.byref(d)), "moe_plan_describe")
         self.block_m, self.pool_capacity, self.num_sms = d.block_m, d.pool_capacity, d.num_sms
+        self.pair_clusters = d.pair_clusters
         self.workspace_bytes = d.workspace_bytes
         self.workspace = torch.empty(self.workspace_bytes, dtype=torch.uint8, device=self.device)
         _ok(self.lib.moe_plan_bind_workspace(self._plan, _ptr(self.workspace), self.workspace_bytes),
@@ -222,6 +224,9 @@ class MoEPlan:
         n = ctypes.c_int(0)
         _ok(self.lib.moe_plan_profile_read(self._plan, ms, ctypes.byref(n)), "moe_plan_profile_read")
         return dict(zip(KERNEL_NAMES, list(ms))), n.value
+
+    def set_cta_pairs(self, enable: bool):
+        _ok(self.lib.moe_plan_set_cta_pairs(self._plan, 1 if enable else 0), "moe_plan_set_cta_pairs")
 
     def set_debug(self, withhold_block: int = -1, timeout_ns: int = 0):
         _ok(self.lib.moe_plan_set_debug(self._plan, withhold_block, timeout_ns), "moe_plan_set_debug")

@@ -27,8 +27,11 @@ struct DispatchParams {
   int32_t* sched;            // [0] task counter, [1] blocks, [2] padded slots, [3] block groups
   int32_t* err;              // sticky device error word
   // Block groups of the expert GEMM's task order (nullptr: routing only, no groups).
-  int32_t* group_start;      // [max_groups + 1] first block of each group
+  int32_t* group_start;      // [max_groups + 1] first block (or pair) of each group
   int32_t* l2_done;          // [pool / BLOCK_M] zeroed here
+  // CTA-pair mode (nullptr: groups over blocks): pairs of consecutive blocks
+  // of one expert, pair_start[e] = first pair of expert e; groups over pairs.
+  int32_t* pair_start;       // [E+1]
   int T, E, k, BM, num_chunks, pool;
   int group_min, group_max, max_groups;
 };
@@ -108,6 +111,30 @@ __global__ void __launch_bounds__(kScanThreads) moe_dispatch_scan_kernel(const D
     }
     if (tid == 31) s_bs[p.E] = incl;
   }
+  __shared__ int32_t s_ps[257];
+  if (p.pair_start != nullptr && tid < 32) {   // exclusive scan of ceil(blocks / 2) per expert
+    int v[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ee = tid * 8 + i;
+      v[i] = ee < p.E ? (s_nb[ee] + 1) / 2 : 0;
+      sum += v[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (tid >= off) incl += o;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ee = tid * 8 + i;
+      if (ee < p.E) s_ps[ee] = run;
+      run += v[i];
+    }
+    if (tid == 31) s_ps[p.E] = incl;
+  }
   __syncthreads();
   const int nblocks = s_bs[p.E];
   if (tid == 0) {
@@ -120,21 +147,23 @@ __global__ void __launch_bounds__(kScanThreads) moe_dispatch_scan_kernel(const D
       // its start, so small experts share a group and an expert's blocks
       // rarely straddle two. One binary search over the expert boundaries per
       // group (block starts are non-decreasing).
+      const int32_t* units = p.pair_start != nullptr ? s_ps : s_bs;   // group over pairs or blocks
+      const int total = units[p.E];
       int ng = 0, start = 0;
       p.group_start[0] = 0;
-      while (start < nblocks && ng < p.max_groups) {
+      while (start < total && ng < p.max_groups) {
         const int target = start + p.group_min;
-        int lo = 0, hi = p.E;   // first e with block_start[e] >= target (E if none)
+        int lo = 0, hi = p.E;   // first e with units[e] >= target (E if none)
         while (lo < hi) {
           const int mid = (lo + hi) >> 1;
-          if (s_bs[mid] >= target) hi = mid;
+          if (units[mid] >= target) hi = mid;
           else lo = mid + 1;
         }
-        const int boundary = s_bs[lo] >= target ? s_bs[lo] : nblocks;
-        start = min(min(boundary, start + p.group_max), nblocks);
+        const int boundary = units[lo] >= target ? units[lo] : total;
+        start = min(min(boundary, start + p.group_max), total);
         p.group_start[++ng] = start;
       }
-      if (start != nblocks) atomicCAS(p.err, 0, kDevBounds);   // more groups than max_groups
+      if (start != total) atomicCAS(p.err, 0, kDevBounds);   // more groups than max_groups
       p.sched[3] = ng;
     }
     return;
@@ -142,6 +171,7 @@ __global__ void __launch_bounds__(kScanThreads) moe_dispatch_scan_kernel(const D
   // (3) everything else, on threads 1..
   for (int ee = tid - 1; ee <= p.E; ee += kScanThreads - 1) {
     p.block_start[ee] = s_bs[ee];
+    if (p.pair_start != nullptr) p.pair_start[ee] = s_ps[ee];
     p.expert_offset[ee] = s_bs[ee] * p.BM;
     if (ee < p.E) p.expert_count[ee] = s_cnt[ee];
   }

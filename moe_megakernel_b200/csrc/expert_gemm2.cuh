@@ -1,0 +1,791 @@
+// Persistent grouped GEMM over the expert blocks on CTA pairs (tcgen05
+// cta_group::2): the same tasks as expert_gemm.cuh (L1 = x W1, x W3 + SwiGLU
+// into the h ring; L2 = h W2 + gate-weighted bulk-reduce combine), but every
+// task covers a PAIR of consecutive blocks of one expert, 256 rows, computed
+// by the two CTAs of a cluster together:
+//
+// * each CTA holds its own block's 128 A rows and HALF of the weight tile
+//   (L1: CTA 0 the 128 W1 columns, CTA 1 the matching 128 W3 columns; L2:
+//   each CTA 128 of the 256 W2 columns), so one weight tile load feeds 256
+//   rows and a stage is 32 KB per CTA instead of 48 KB (6 stages fit);
+// * the leader CTA (rank 0) claims tasks, issues the MMAs for both CTAs and
+//   multicasts its commits to both CTAs' barriers; each CTA's accumulator is
+//   its own 128 rows x 256 columns in its own TMEM;
+// * each CTA's TMA loads and routed-row gathers land on its own stage
+//   barrier; the follower's warp 1 relays the completion of each of its
+//   stages to the leader's barrier with one remote arrival (counting the
+//   follower's bytes on the leader's barrier directly, with the pair form of
+//   the TMA load, measured 2.5x slower here).
+//
+// Prior art: "MegaMoE 在 MoE 系统谱系中的位置", section 2.1 (the MMA warp issues
+// for the leader CTA only; warp roles with their own jobs) and section 2.7
+// (atomic task queue, L2 waits for its L1 tiles). No TMA multicast is used.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "common.cuh"
+#include "expert_gemm.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+constexpr int kStages2 = 6;
+constexpr int kTileB2Bytes = 2 * kBoxBytes;                 // 128 weight columns x 64 rows per CTA
+constexpr int kStage2Bytes = kTileABytes + kTileB2Bytes;    // 32 KB
+
+struct Gemm2Params {
+  const bf16* x;       // [T, H]
+  CUtensorMap tm_w1;   // W1 as [E*H, I], box {64, 64}
+  CUtensorMap tm_w3;   // W3 as [E*H, I], box {64, 64}
+  CUtensorMap tm_w2;   // W2 as [E*I, H], box {64, 64}
+  CUtensorMap tm_h;    // h ring [ring_pairs * 2 * BM, I], box {64, BM}
+  const int32_t* slot_token;
+  const int32_t* slot_topk;
+  const float* topk_w;
+  const int32_t* block_start;   // [E+1]
+  const int32_t* pair_start;    // [E+1] pairs of consecutive blocks per expert
+  const int32_t* group_start;   // [groups + 1] in pairs
+  const int32_t* num_groups;
+  int32_t* task_counter;
+  int32_t* l1_done;             // [pairs] 8 arrivals per L1 n-tile (4 epilogue warps x 2 CTAs)
+  int32_t* l2_done;             // [pairs] 1 arrival per L2 n-tile
+  int32_t* err;
+  bf16* h;
+  float* y_acc;                 // [T, H]
+  int T, H, I, E, k, BM, BN2, N1, N2;
+  int ring_pairs, max_groups;
+  unsigned long long timeout_ns;
+  int withhold_pair;            // test hook: never publish L1 completion of this pair (-1: off)
+};
+
+struct Task2 {
+  int phase;    // 0 = L1, 1 = L2, -1 = no more work
+  int e, p, n;  // expert, pair, n-tile
+  int b0, b1;   // blocks of CTA 0 and CTA 1 (b1 = -1: the expert has an odd block count)
+  int pad0, pad1;
+};
+
+struct Gemm2Smem {
+  float out_stage[4][32][36];   // L2 epilogue staging (see expert_gemm.cuh); first, 16-byte aligned
+  uint64_t full[kStages2];
+  uint64_t empty[kStages2];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t task_full[kTaskRing];
+  uint64_t task_empty[kTaskRing];
+  uint64_t mma_done;
+  Task2 tasks[kTaskRing];
+  uint32_t tmem_base;
+  int abort;
+  int num_groups;
+  int rows[kTaskRing][kTileM];
+  int block_start[257];
+  int pair_start[257];
+  int group_start[kMaxGroups + 1];
+};
+
+static_assert(offsetof(Gemm2Smem, out_stage) % 16 == 0, "bulk-reduce source must be 16-byte aligned");
+static_assert(sizeof(Task2) == 32, "tasks are copied to the peer as 8 words");
+
+constexpr size_t kGemm2SmemBytes = 1024 + (size_t)kStages2 * kStage2Bytes + sizeof(Gemm2Smem);
+
+__device__ __forceinline__ void set_error2(const Gemm2Params& p, Gemm2Smem& s, int code, int detail) {
+  if (atomicCAS(p.err, 0, code) == 0) p.err[1] = detail;
+  *reinterpret_cast<volatile int*>(&s.abort) = 1;
+}
+
+// Bounded wait of a whole warp on a local barrier phase. Arrivals may come
+// from the peer CTA; the per-stage barriers are waited on at CTA scope (the
+// data they guard is TMA- or cp.async-written shared memory read by the
+// tensor core), the task ring of the follower, whose task words and row
+// indices the leader writes through the cluster window, at cluster scope.
+// Gives up on timeout, on this CTA's abort flag, or (checked every few
+// microseconds) on a recorded error.
+template <bool kClusterAcquire = false>
+__device__ __forceinline__ bool warp_wait2(uint64_t* bar, uint32_t parity, const Gemm2Params& p, Gemm2Smem& s,
+                                           int where) {
+  auto poll = [&]() {
+    return kClusterAcquire ? ptx::mbar_try_wait_cluster(bar, parity) : ptx::mbar_try_wait(bar, parity);
+  };
+  bool ok = poll();
+  if (!ok) {
+    const uint64_t t0 = ptx::globaltimer();
+    uint64_t next_check = t0 + 4000;
+    while (true) {
+      if (poll()) {
+        ok = true;
+        break;
+      }
+      if (*reinterpret_cast<volatile int*>(&s.abort)) break;
+      const uint64_t now = ptx::globaltimer();
+      if (now > next_check) {
+        if (*reinterpret_cast<volatile int*>(p.err) != 0) break;
+        next_check = now + 4000;
+      }
+      if (now - t0 > p.timeout_ns) {
+        set_error2(p, s, kDevTimeout, 0x100 | where);
+        break;
+      }
+    }
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ bool wait_counter2(const int* ctr, int need, const Gemm2Params& p, Gemm2Smem& s,
+                                              int detail) {
+  if (ptx::ld_acquire_gpu(ctr) >= need) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  while (ptx::ld_acquire_gpu(ctr) < need) {
+    if (*reinterpret_cast<volatile int*>(&s.abort) || *reinterpret_cast<volatile int*>(p.err) != 0) return false;
+    if (ptx::globaltimer() - t0 > p.timeout_ns) {
+      set_error2(p, s, kDevTimeout, detail);
+      return false;
+    }
+    __nanosleep(256);
+  }
+  return true;
+}
+
+__device__ __forceinline__ int claim_task_any(int32_t* counter, const int32_t* err, const int* abort, int lane) {
+  int t = 0x7fffffff;
+  if (lane == 0) {
+    const bool stop = *reinterpret_cast<const volatile int*>(abort) || *reinterpret_cast<const volatile int*>(err) != 0;
+    if (!stop) t = atomicAdd(counter, 1);
+  }
+  return t;   // valid in lane 0 only
+}
+
+// Task order as in expert_gemm.cuh, in units of block pairs.
+__device__ __forceinline__ int segment_start2(const Gemm2Smem& s, const Gemm2Params& p, int seg) {
+  const int G = s.num_groups;
+  if (seg == 0) return 0;
+  const int g = (seg + 1) >> 1;
+  if (seg & 1) return s.group_start[g] * p.N1 + s.group_start[g - 1] * p.N2;
+  return s.group_start[min(g + 1, G)] * p.N1 + s.group_start[g - 1] * p.N2;
+}
+
+__device__ __forceinline__ Task2 decode_task2(int t, const Gemm2Smem& s, const Gemm2Params& p) {
+  Task2 task{-1, 0, 0, 0, -1, -1, 0, 0};
+  const int G = s.num_groups;
+  const int np_total = s.pair_start[p.E];
+  if (t < 0 || t >= np_total * (p.N1 + p.N2) || G <= 0) return task;
+  int lo = 0, hi = 2 * G;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (segment_start2(s, p, mid) <= t) lo = mid;
+    else hi = mid - 1;
+  }
+  const int seg = lo;
+  int g, NT;
+  if (seg == 0 || (seg & 1)) {
+    task.phase = 0;
+    g = (seg + 1) >> 1;
+    NT = p.N1;
+  } else {
+    task.phase = 1;
+    g = (seg >> 1) - 1;
+    NT = p.N2;
+  }
+  const int gp0 = s.group_start[g], gp1 = s.group_start[g + 1];
+  const int tl = t - segment_start2(s, p, seg);
+  const int vp = gp0 + tl / NT;
+  int elo = 0, ehi = p.E - 1;
+  while (elo < ehi) {
+    const int mid = (elo + ehi + 1) >> 1;
+    if (s.pair_start[mid] <= vp) elo = mid;
+    else ehi = mid - 1;
+  }
+  const int e = elo;
+  const int ep0 = max(gp0, s.pair_start[e]);
+  const int ep1 = min(gp1, s.pair_start[e + 1]);
+  const int np = ep1 - ep0;
+  const int local = tl - (ep0 - gp0) * NT;
+  task.e = e;
+  task.n = local / np;
+  task.p = ep0 + (local - task.n * np);
+  task.b0 = s.block_start[e] + 2 * (task.p - s.pair_start[e]);
+  task.b1 = task.b0 + 1 < s.block_start[e + 1] ? task.b0 + 1 : -1;
+  return task;
+}
+
+__device__ __forceinline__ uint8_t* stage2_ptr(uint8_t* tiles, int stage) { return tiles + stage * kStage2Bytes; }
+
+// ---------------------------------------------------------------- leader warp 0: scheduler + TMA
+__device__ __forceinline__ Task2 prepare_task2(int t, int q, uint32_t qparity, bool& deps_ready, bool& ok,
+                                               const Gemm2Params& p, Gemm2Smem& s, int lane) {
+  Task2 task = decode_task2(t, s, p);
+  deps_ready = true;
+  ok = warp_wait2(&s.task_empty[q], qparity, p, s, 1);
+  if (!ok) return task;
+  if (task.phase == 0) {
+    // token rows of both CTAs' A tiles: CTA 0 locally, CTA 1 through the cluster window
+    const uint32_t peer_rows = ptx::mapa(ptx::smem_u32(&s.rows[q][0]), 1);
+    for (int r = lane; r < p.BM; r += 32) {
+      int tok0 = p.slot_token[task.b0 * p.BM + r];
+      int tok1 = task.b1 >= 0 ? p.slot_token[task.b1 * p.BM + r] : 0;
+      if (tok0 >= p.T || tok1 >= p.T) {
+        set_error2(p, s, kDevBounds, task.p);
+        tok0 = tok0 >= p.T ? 0 : tok0;
+        tok1 = tok1 >= p.T ? 0 : tok1;
+      }
+      s.rows[q][r] = tok0 < 0 ? 0 : tok0;   // padding slot: any valid row, the epilogue drops it
+      ptx::st_cluster_u32(peer_rows + 4 * r, tok1 < 0 ? 0 : tok1);
+    }
+  } else if (task.phase == 1) {
+    int ready = 1;
+    if (lane == 0) ready = ptx::ld_acquire_gpu(p.l1_done + task.p) >= 8 * p.N1;
+    deps_ready = __shfl_sync(0xffffffffu, ready, 0) != 0;
+  }
+  __syncwarp();
+  return task;
+}
+
+__device__ __forceinline__ void push_task2(const Task2& task, int q, Gemm2Smem& s, int lane) {
+  if (lane < 8) {
+    const uint32_t v = reinterpret_cast<const uint32_t*>(&task)[lane];
+    reinterpret_cast<uint32_t*>(&s.tasks[q])[lane] = v;
+    ptx::st_cluster_u32(ptx::mapa(ptx::smem_u32(&s.tasks[q]), 1) + 4 * lane, v);
+  }
+  // every lane's stores into the peer (task words here, row indices in
+  // prepare_task2) are ordered before lane 0's releasing arrive
+  asm volatile("fence.acq_rel.cluster;" ::: "memory");
+  __syncwarp();
+  if (lane == 0) {
+    ptx::mbar_arrive(&s.task_full[q]);
+    ptx::mbar_arrive_remote(ptx::mapa(ptx::smem_u32(&s.task_full[q]), 1));   // releases the stores above
+  }
+  __syncwarp();
+}
+
+__device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles) {
+  const int lane = ptx::lane_id();
+  const uint64_t pol = ptx::policy_evict_first();
+  const uint64_t polh = ptx::policy_evict_normal();
+  int stage = 0;
+  uint32_t phase = 0;
+  int q = 0;
+  uint32_t qphase = 0;
+  uint32_t issued = 0, issued_parity = 0;
+  bool deps_ready = true, ok = true;
+  int t = __shfl_sync(0xffffffffu, claim_task_any(p.task_counter, p.err, &s.abort, lane), 0);
+  Task2 task = prepare_task2(t, q, qphase ^ 1, deps_ready, ok, p, s, lane);
+  while (ok) {
+    if (task.phase == 1 && !deps_ready) {
+      bool fine = true;
+      if (lane == 0) fine = wait_counter2(p.l1_done + task.p, 8 * p.N1, p, s, 0x10000 | task.p);
+      if (__shfl_sync(0xffffffffu, fine ? 1 : 0, 0) == 0) task.phase = -1;
+    }
+    if (task.phase == 1) ptx::fence_proxy_async_global();
+    push_task2(task, q, s, lane);
+    const int qn = (q + 1) % kTaskRing;
+    const uint32_t qphase_n = qn == 0 ? qphase ^ 1 : qphase;
+    if (task.phase < 0) break;
+
+    const int t_next_lane0 = claim_task_any(p.task_counter, p.err, &s.abort, lane);
+    bool prepared = false;
+    Task2 next{-1, 0, 0, 0, -1, -1, 0, 0};
+    const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
+    const int prep_at = nk > 2 ? 2 : nk - 1;
+    for (int kb = 0; kb < nk; ++kb) {
+      if (!warp_wait2(&s.empty[stage], phase ^ 1, p, s, 2)) {
+        ok = false;
+        break;
+      }
+      const uint32_t a_addr = ptx::smem_u32(stage2_ptr(tiles, stage));
+      const uint32_t b_addr = a_addr + kTileABytes;
+      if (lane == 0) {
+        // this CTA's half only; the follower's half lands on the follower's own
+        // barrier and reaches this one through its relay arrival
+        if (task.phase == 0) {
+          ptx::mbar_arrive_expect_tx(&s.full[stage], 2 * kBoxBytes);
+          const int wrow = task.e * p.H + kb * kBK;
+          const int n0 = task.n * kL1TileN;
+          ptx::tma_load_2d(b_addr, &p.tm_w1, &s.full[stage], n0, wrow, pol);
+          ptx::tma_load_2d(b_addr + kBoxBytes, &p.tm_w1, &s.full[stage], n0 + 64, wrow, pol);
+        } else {
+          const int half_boxes = p.BN2 / 128;
+          ptx::mbar_arrive_expect_tx(&s.full[stage], p.BM * 128 + half_boxes * kBoxBytes);
+          ptx::tma_load_2d(a_addr, &p.tm_h, &s.full[stage], kb * kBK, ((task.p % p.ring_pairs) * 2 + 0) * p.BM, polh);
+          const int wrow = task.e * p.I + kb * kBK;
+          for (int j = 0; j < half_boxes; ++j)
+            ptx::tma_load_2d(b_addr + j * kBoxBytes, &p.tm_w2, &s.full[stage], task.n * p.BN2 + j * 64, wrow, pol);
+        }
+      }
+      __syncwarp();
+      issued |= 1u << stage;
+      issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+      if (++stage == kStages2) {
+        stage = 0;
+        phase ^= 1;
+      }
+      if (kb == prep_at) {
+        const int tn = __shfl_sync(0xffffffffu, t_next_lane0, 0);
+        next = prepare_task2(tn, qn, qphase_n ^ 1, deps_ready, ok, p, s, lane);
+        prepared = true;
+        if (!ok) break;
+      }
+    }
+    if (!ok) break;
+    if (!prepared) {
+      const int tn = __shfl_sync(0xffffffffu, t_next_lane0, 0);
+      next = prepare_task2(tn, qn, qphase_n ^ 1, deps_ready, ok, p, s, lane);
+    }
+    task = next;
+    q = qn;
+    qphase = qphase_n;
+  }
+  for (int st = 0; st < kStages2; ++st)
+    if (issued & (1u << st)) {
+      const uint64_t t0 = ptx::globaltimer();
+      while (!ptx::mbar_try_wait(&s.full[st], (issued_parity >> st) & 1u))
+        if (ptx::globaltimer() - t0 > p.timeout_ns) break;
+    }
+}
+
+// Pop the next task from this CTA's ring and release the slot to the leader.
+__device__ __forceinline__ bool pop_task2(Task2& task, int& q, uint32_t& qphase, int* q_popped, bool is_leader,
+                                          const Gemm2Params& p, Gemm2Smem& s, int where, bool release_now) {
+  const int lane = ptx::lane_id();
+  const bool got = is_leader ? warp_wait2(&s.task_full[q], qphase, p, s, where)
+                             : warp_wait2<true>(&s.task_full[q], qphase, p, s, where);
+  if (!got) return false;
+  task = s.tasks[q];
+  if (q_popped) *q_popped = q;
+  if (release_now) {
+    __syncwarp();
+    if (lane == 0) {
+      if (is_leader) ptx::mbar_arrive(&s.task_empty[q]);
+      else ptx::mbar_arrive_remote(ptx::mapa(ptx::smem_u32(&s.task_empty[q]), 0));
+    }
+  }
+  if (++q == kTaskRing) {
+    q = 0;
+    qphase ^= 1;
+  }
+  return true;
+}
+
+__device__ __forceinline__ void release_task_slot2(int q, bool is_leader, Gemm2Smem& s) {
+  __syncwarp();
+  if (ptx::lane_id() == 0) {
+    if (is_leader) ptx::mbar_arrive(&s.task_empty[q]);
+    else ptx::mbar_arrive_remote(ptx::mapa(ptx::smem_u32(&s.task_empty[q]), 0));
+  }
+}
+
+// ---------------------------------------------------------------- follower warp 0: its TMA halves
+__device__ void gemm2_follower_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles) {
+  const int lane = ptx::lane_id();
+  const uint64_t pol = ptx::policy_evict_first();
+  const uint64_t polh = ptx::policy_evict_normal();
+  int stage = 0;
+  uint32_t phase = 0;
+  int q = 0;
+  uint32_t qphase = 0;
+  while (true) {
+    Task2 task;
+    if (!pop_task2(task, q, qphase, nullptr, false, p, s, 3, true)) break;
+    if (task.phase < 0) break;
+    const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
+    bool ok = true;
+    for (int kb = 0; kb < nk; ++kb) {
+      if (!warp_wait2(&s.empty[stage], phase ^ 1, p, s, 4)) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) {
+        const uint32_t a_addr = ptx::smem_u32(stage2_ptr(tiles, stage));
+        const uint32_t b_addr = a_addr + kTileABytes;
+        if (task.phase == 0) {
+          ptx::mbar_arrive_expect_tx(&s.full[stage], 2 * kBoxBytes);
+          const int wrow = task.e * p.H + kb * kBK;
+          const int n0 = task.n * kL1TileN;
+          ptx::tma_load_2d(b_addr, &p.tm_w3, &s.full[stage], n0, wrow, pol);
+          ptx::tma_load_2d(b_addr + kBoxBytes, &p.tm_w3, &s.full[stage], n0 + 64, wrow, pol);
+        } else {
+          const int half_boxes = p.BN2 / 128;
+          ptx::mbar_arrive_expect_tx(&s.full[stage], p.BM * 128 + half_boxes * kBoxBytes);
+          ptx::tma_load_2d(a_addr, &p.tm_h, &s.full[stage], kb * kBK, ((task.p % p.ring_pairs) * 2 + 1) * p.BM, polh);
+          const int wrow = task.e * p.I + kb * kBK;
+          const int n0 = task.n * p.BN2 + p.BN2 / 2;
+          for (int j = 0; j < half_boxes; ++j)
+            ptx::tma_load_2d(b_addr + j * kBoxBytes, &p.tm_w2, &s.full[stage], n0 + j * 64, wrow, pol);
+        }
+      }
+      __syncwarp();
+      if (++stage == kStages2) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+    if (!ok) break;
+  }
+}
+
+// ---------------------------------------------------------------- follower warp 1: stage relay
+// The follower's TMA bytes and gather lanes land on its own stage barrier;
+// once a stage is complete, one arrival on the leader's barrier of that stage.
+__device__ void gemm2_follower_relay(const Gemm2Params& p, Gemm2Smem& s) {
+  const int lane = ptx::lane_id();
+  const uint32_t lead_full0 = ptx::mapa(ptx::smem_u32(&s.full[0]), 0);
+  int stage = 0;
+  uint32_t phase = 0;
+  int q = 0;
+  uint32_t qphase = 0;
+  while (true) {
+    Task2 task;
+    if (!pop_task2(task, q, qphase, nullptr, false, p, s, 5, true)) break;
+    if (task.phase < 0) break;
+    const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
+    bool ok = true;
+    for (int kb = 0; kb < nk; ++kb) {
+      if (!warp_wait2(&s.full[stage], phase, p, s, 6)) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) {
+        ptx::fence_proxy_async_shared();   // cp.async-written rows -> the tensor core's reads
+        ptx::mbar_arrive_peer(lead_full0 + 8 * stage);
+      }
+      __syncwarp();
+      if (++stage == kStages2) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+    if (!ok) break;
+  }
+}
+
+// ---------------------------------------------------------------- leader warp 1: MMA issuer
+__device__ void gemm2_mma(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, uint32_t tmem_base) {
+  const int lane = ptx::lane_id();
+  const uint32_t idesc_l1 = ptx::idesc_bf16_f32(256, 2 * kL1TileN, false, true);
+  const uint32_t idesc_l2 = ptx::idesc_bf16_f32(256, p.BN2, false, true);
+  int stage = 0;
+  uint32_t phase = 0;
+  int q = 0;
+  uint32_t qphase = 0;
+  int acc = 0;
+  uint32_t acc_phase = 0;
+  bool issued_any = false;
+  while (true) {
+    Task2 task;
+    if (!pop_task2(task, q, qphase, nullptr, true, p, s, 7, true)) break;
+    if (task.phase < 0) break;
+    if (!warp_wait2(&s.acc_empty[acc], acc_phase ^ 1, p, s, 8)) break;
+    ptx::tc_fence_after();
+    const uint32_t d_tmem = tmem_base + acc * 256;
+    const uint32_t idesc = task.phase == 0 ? idesc_l1 : idesc_l2;
+    const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
+    bool ok = true;
+    for (int kb = 0; kb < nk; ++kb) {
+      if (!warp_wait2(&s.full[stage], phase, p, s, 9)) {
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      ptx::fence_proxy_async_shared();
+      if (lane == 0) {
+        const uint32_t a_addr = ptx::smem_u32(stage2_ptr(tiles, stage));
+        const uint32_t b_addr = a_addr + kTileABytes;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t ad = ptx::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+          const uint64_t bd = ptx::smem_desc_sw128(b_addr + kk * 2048, kBoxBytes, 1024);
+          ptx::mma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+        ptx::mma_commit_pair_multicast(&s.empty[stage], 0x3);
+        issued_any = true;
+      }
+      __syncwarp();
+      if (++stage == kStages2) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+    if (!ok) break;
+    if (lane == 0) ptx::mma_commit_pair_multicast(&s.acc_full[acc], 0x3);
+    __syncwarp();
+    if (++acc == 2) {
+      acc = 0;
+      acc_phase ^= 1;
+    }
+  }
+  issued_any = __any_sync(0xffffffffu, issued_any);
+  if (issued_any) {
+    if (lane == 0) ptx::mma_commit_pair_multicast(&s.mma_done, 0x1);
+    __syncwarp();
+    const uint64_t t0 = ptx::globaltimer();
+    while (!ptx::mbar_try_wait(&s.mma_done, 0)) {
+      if (ptx::globaltimer() - t0 > p.timeout_ns) break;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- epilogue (warps 2..5 of both CTAs)
+__device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem_base, uint32_t rank) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = ptx::lane_id();
+  const int quarter = warp & 3;
+  const int r = quarter * 32 + lane;
+  const bool is_leader = rank == 0;
+  const uint32_t lead_acc_empty0 = ptx::mapa(ptx::smem_u32(&s.acc_empty[0]), 0);
+  int q = 0;
+  uint32_t qphase = 0;
+  int acc = 0;
+  uint32_t acc_phase = 0;
+  while (true) {
+    Task2 task;
+    if (!pop_task2(task, q, qphase, nullptr, is_leader, p, s, 10, true)) break;
+    if (task.phase < 0) break;
+    if (!warp_wait2(&s.acc_full[acc], acc_phase, p, s, 11)) break;
+    ptx::tc_fence_after();
+    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * 256;
+    const int b_own = rank == 0 ? task.b0 : task.b1;
+    const bool valid = r < p.BM && b_own >= 0;
+    const int slot = (b_own < 0 ? 0 : b_own) * p.BM + r;
+    if (task.phase == 0) {
+      bool store = valid;
+      if (task.p >= p.ring_pairs) {
+        bool ok = true;
+        if (lane == 0) ok = wait_counter2(p.l2_done + (task.p - p.ring_pairs), p.N2, p, s, 0x40000 | task.p);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        store = store && ok;
+      }
+      const int ring_row = ((task.p % p.ring_pairs) * 2 + (int)rank) * p.BM + r;
+      bf16* hrow = p.h + (size_t)ring_row * p.I + task.n * kL1TileN;
+#pragma unroll 1
+      for (int c = 0; c < kL1TileN / 32; ++c) {
+        uint32_t g[32], u[32];
+        ptx::tmem_ld32(tbase + c * 32, g);
+        ptx::tmem_ld32(tbase + kL1TileN + c * 32, u);
+        ptx::tmem_ld_wait();
+        if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(hrow + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 o;
+            o.x = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 0]), __uint_as_float(u[8 * v + 0])),
+                              silu_mul(__uint_as_float(g[8 * v + 1]), __uint_as_float(u[8 * v + 1])));
+            o.y = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 2]), __uint_as_float(u[8 * v + 2])),
+                              silu_mul(__uint_as_float(g[8 * v + 3]), __uint_as_float(u[8 * v + 3])));
+            o.z = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 4]), __uint_as_float(u[8 * v + 4])),
+                              silu_mul(__uint_as_float(g[8 * v + 5]), __uint_as_float(u[8 * v + 5])));
+            o.w = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 6]), __uint_as_float(u[8 * v + 6])),
+                              silu_mul(__uint_as_float(g[8 * v + 7]), __uint_as_float(u[8 * v + 7])));
+            dst[v] = o;
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (is_leader) ptx::mbar_arrive(&s.acc_empty[acc]);
+        else ptx::mbar_arrive_peer(lead_acc_empty0 + 8 * acc);
+      }
+      __threadfence();
+      ptx::fence_proxy_async_global();
+      __syncwarp();
+      if (lane == 0 && task.p != p.withhold_pair) ptx::red_release_gpu_add(p.l1_done + task.p, 1);
+    } else {
+      if (is_leader && quarter == 0 && lane == 0) ptx::red_release_gpu_add(p.l2_done + task.p, 1);
+      int tok = -1;
+      float w = 0.f;
+      if (valid) {
+        tok = p.slot_token[slot];
+        if (tok >= p.T) {
+          set_error2(p, s, kDevBounds, 0x20000 | task.p);
+          tok = -1;
+        }
+        if (tok >= 0) {
+          const int j = p.slot_topk[slot];
+          if (j < 0 || j >= p.k) {
+            set_error2(p, s, kDevBounds, 0x30000 | task.p);
+            tok = -1;
+          } else {
+            w = p.topk_w[(size_t)tok * p.k + j];
+          }
+        }
+      }
+      float* yrow = p.y_acc + (size_t)(tok < 0 ? 0 : tok) * p.H + task.n * p.BN2;
+      float* srow = &s.out_stage[quarter][lane][0];
+      const uint32_t srow_addr = ptx::smem_u32(srow);
+#pragma unroll 1
+      for (int c = 0; c < p.BN2 / 32; ++c) {
+        uint32_t v[32];
+        ptx::tmem_ld32(tbase + c * 32, v);
+        ptx::tmem_ld_wait();
+        if (tok >= 0) {
+          ptx::bulk_wait_read_all();
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            reinterpret_cast<float4*>(srow)[i] =
+                make_float4(w * __uint_as_float(v[4 * i + 0]), w * __uint_as_float(v[4 * i + 1]),
+                            w * __uint_as_float(v[4 * i + 2]), w * __uint_as_float(v[4 * i + 3]));
+          ptx::fence_proxy_async_shared();
+          ptx::bulk_reduce_add_f32(yrow + c * 32, srow_addr, 128);
+          ptx::bulk_commit();
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (is_leader) ptx::mbar_arrive(&s.acc_empty[acc]);
+        else ptx::mbar_arrive_peer(lead_acc_empty0 + 8 * acc);
+      }
+    }
+    if (++acc == 2) {
+      acc = 0;
+      acc_phase ^= 1;
+    }
+  }
+  ptx::bulk_wait_all();
+}
+
+// ---------------------------------------------------------------- gather warps (warps 6.. of both CTAs)
+__device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, int g, uint32_t rank) {
+  constexpr int kRowsPerLane = (kTileM / 4 + kGatherWarps - 1) / kGatherWarps;
+  const int lane = ptx::lane_id();
+  const int c = lane & 7;
+  const bool is_leader = rank == 0;
+  int stage = 0;
+  uint32_t phase = 0;
+  int q = 0;
+  uint32_t qphase = 0;
+  while (true) {
+    Task2 task;
+    int q_task = 0;
+    if (!pop_task2(task, q, qphase, &q_task, is_leader, p, s, 12, false)) break;
+    if (task.phase < 0) break;
+    const int b_own = rank == 0 ? task.b0 : task.b1;
+    int nrows = 0;
+    uint32_t soff[kRowsPerLane];
+    const bf16* src[kRowsPerLane];
+    if (task.phase == 0 && b_own >= 0) {
+      const int* rows = s.rows[q_task];
+#pragma unroll
+      for (int j = 0; j < kRowsPerLane; ++j) {
+        const int rr = (j * kGatherWarps + g) * 4 + (lane >> 3);
+        soff[j] = rr * 128 + ((c ^ (rr & 7)) << 4);
+        src[j] = p.x + c * 8;
+        if (rr < p.BM) {
+          src[j] = p.x + (size_t)rows[rr] * p.H + c * 8;
+          nrows = j + 1;
+        }
+      }
+    }
+    release_task_slot2(q_task, is_leader, s);   // rows read: the slot may be refilled
+    const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
+    bool ok = true;
+    for (int kb = 0; kb < nk; ++kb) {
+      if (!warp_wait2(&s.empty[stage], phase ^ 1, p, s, 13)) {
+        ok = false;
+        break;
+      }
+      if (task.phase == 0) {
+        const uint32_t a_addr = ptx::smem_u32(stage2_ptr(tiles, stage));
+#pragma unroll
+        for (int j = 0; j < kRowsPerLane; ++j)
+          if (j < nrows) ptx::cp_async_16(a_addr + soff[j], src[j] + kb * kBK);
+        ptx::cp_async_mbar_arrive_noinc(&s.full[stage]);
+      } else {
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_count(&s.full[stage], 32);
+      }
+      if (++stage == kStages2) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+    if (!ok) break;
+  }
+  ptx::cp_async_wait_all();
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1) moe_expert_gemm2_kernel(const __grid_constant__ Gemm2Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Gemm2Smem& s = *reinterpret_cast<Gemm2Smem*>(tiles + (size_t)kStages2 * kStage2Bytes);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const bool is_leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages2; ++i) {
+      // leader: its producer, its gather lanes and the follower's relay; follower: its producer
+      // (with its TMA bytes) and its gather lanes
+      ptx::mbar_init(&s.full[i], is_leader ? 1 + 32 * kGatherWarps + 1 : 1 + 32 * kGatherWarps);
+      ptx::mbar_init(&s.empty[i], 1);   // the leader's MMA commit, multicast to both CTAs
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&s.acc_full[i], 1);
+      ptx::mbar_init(&s.acc_empty[i], 8);   // 4 epilogue warps in each CTA (used in the leader)
+    }
+    for (int i = 0; i < kTaskRing; ++i) {
+      ptx::mbar_init(&s.task_full[i], 1);
+      // in the leader: its MMA + 4 epilogue + gather warps, and the follower's producer,
+      // relay, 4 epilogue and gather warps
+      ptx::mbar_init(&s.task_empty[i], (1 + 4 + kGatherWarps) + (2 + 4 + kGatherWarps));
+    }
+    ptx::mbar_init(&s.mma_done, 1);
+    s.abort = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&p.tm_w1);
+    ptx::prefetch_tmap(&p.tm_w3);
+    ptx::prefetch_tmap(&p.tm_w2);
+    ptx::prefetch_tmap(&p.tm_h);
+  }
+  for (int e = threadIdx.x; e <= p.E; e += kGemmThreads) {
+    s.block_start[e] = p.block_start[e];
+    s.pair_start[e] = p.pair_start[e];
+  }
+  {
+    const int ng = min(*p.num_groups, min(p.max_groups, kMaxGroups));
+    if (threadIdx.x == 0) s.num_groups = ng;
+    for (int g = threadIdx.x; g <= ng; g += kGemmThreads) s.group_start[g] = p.group_start[g];
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(&s.tmem_base, kTmemCols);
+    ptx::tmem_relinquish_pair();
+  }
+  if (p.BM < kTileM) {
+    for (int st = 0; st < kStages2; ++st) {
+      uint4* a = reinterpret_cast<uint4*>(stage2_ptr(tiles, st) + p.BM * 128);
+      const int n = (kTileM - p.BM) * 128 / 16;
+      for (int i = threadIdx.x; i < n; i += kGemmThreads) a[i] = make_uint4(0, 0, 0, 0);
+    }
+    ptx::fence_proxy_async_shared();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();   // both CTAs' barriers exist before any remote arrive
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = s.tmem_base;
+
+  if (warp == 0) {
+    if (is_leader) gemm2_leader_producer(p, s, tiles);
+    else gemm2_follower_producer(p, s, tiles);
+  } else if (warp == 1) {
+    if (is_leader) gemm2_mma(p, s, tiles, tmem_base);
+    else gemm2_follower_relay(p, s);
+  } else if (warp < 6) {
+    gemm2_epilogue(p, s, tmem_base, rank);
+  } else {
+    gemm2_gather(p, s, tiles, warp - 6, rank);
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();   // no peer still arrives on or stores into this CTA's shared memory
+  ptx::tc_fence_after();
+  if (warp == 1) ptx::tmem_dealloc_pair(tmem_base, kTmemCols);
+}
+
+}  // namespace moe

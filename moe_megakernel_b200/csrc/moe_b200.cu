@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "dispatch.cuh"
 #include "expert_gemm.cuh"
+#include "expert_gemm2.cuh"
 #include "router.cuh"
 #include "router_tc.cuh"
 
@@ -29,8 +30,8 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Layout {
   size_t err, sched, topk_idx, topk_w, rank, chunk_count, expert_count, expert_offset, block_start, num_padded,
-      slot_token, slot_topk, l1_done, l2_done, group_start, router_partial, router_counter, h, y_acc, x_stage,
-      y_stage, total;
+      slot_token, slot_topk, l1_done, l2_done, group_start, pair_start, router_partial, router_counter, h, y_acc,
+      x_stage, y_stage, total;
 };
 
 class DeviceGuard {
@@ -92,6 +93,10 @@ struct moe_plan {
   int T_max, H, I, E, k, BM, device, num_sms;
   int BN2, N1, N2, pool, chunks_max, blocks_max;
   int group_min, group_max, max_groups, ring_blocks;   // expert-GEMM task groups and h ring
+  bool cta_pairs = false;                              // run the expert GEMM on CTA pairs
+  int pair_clusters = 0;                               // co-resident clusters of the pair kernel
+  int pgroup_min, pgroup_max, pmax_groups, ring_pairs; // the same in units of block pairs
+  int per_expert;                                      // expected blocks per expert + 1
   Layout L;
   uint8_t* ws = nullptr;
   size_t ws_bytes = 0;
@@ -101,6 +106,18 @@ struct moe_plan {
   int withhold = -1;
   uint64_t timeout_ns = 2000000000ull;
 };
+
+// CTA-pair mode: a task is a pair of consecutive blocks run by one cluster of
+// two CTAs, so there are pair_clusters concurrent tasks (groups and ring in pairs).
+static void size_pair_groups(moe_plan* p) {
+  const int pairs_max = p->blocks_max;   // each pair holds at least one block
+  const int clusters = std::max(1, p->pair_clusters > 0 ? p->pair_clusters : p->num_sms / 2);
+  p->pgroup_min = (2 * clusters + p->N1 - 1) / p->N1;
+  p->pgroup_min = std::max(p->pgroup_min, (pairs_max + kMaxGroups - 3) / (kMaxGroups - 2));
+  p->pgroup_max = std::max(2 * p->pgroup_min, (p->per_expert + 1) / 2);
+  p->pmax_groups = pairs_max / p->pgroup_min + 2;
+  p->ring_pairs = std::min(3 * p->pgroup_max, pairs_max);
+}
 
 static Layout make_layout(const moe_plan& p) {
   Layout L{};
@@ -126,10 +143,11 @@ static Layout make_layout(const moe_plan& p) {
   L.slot_topk = take((size_t)p.pool * 4, 256);
   L.l1_done = take((size_t)p.blocks_max * 4, 256);
   L.l2_done = take((size_t)p.blocks_max * 4, 256);
-  L.group_start = take((size_t)(p.max_groups + 1) * 4, 256);
+  L.group_start = take((size_t)(std::max(p.max_groups, p.pmax_groups) + 1) * 4, 256);
+  L.pair_start = take((size_t)(p.E + 1) * 4, 256);
   L.router_partial = take((size_t)kRouterSplitTiles * kRouterMaxSplit * kRouterTokens * 256 * 4, 256);
   L.router_counter = take((size_t)kRouterSplitTiles * 4, 256);
-  L.h = take((size_t)p.ring_blocks * p.BM * p.I * 2, 1024);
+  L.h = take((size_t)std::max(p.ring_blocks, 2 * p.ring_pairs) * p.BM * p.I * 2, 1024);
   L.y_acc = take((size_t)p.T_max * p.H * 4, 1024);
   L.x_stage = take((size_t)p.T_max * p.H * 2, 1024);
   L.y_stage = take((size_t)p.T_max * p.H * 2, 1024);
@@ -259,9 +277,10 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   dp.pool = p->pool;
   dp.group_start = reinterpret_cast<int32_t*>(ws + L.group_start);
   dp.l2_done = reinterpret_cast<int32_t*>(ws + L.l2_done);
-  dp.group_min = p->group_min;
-  dp.group_max = p->group_max;
-  dp.max_groups = p->max_groups;
+  dp.pair_start = p->cta_pairs ? reinterpret_cast<int32_t*>(ws + L.pair_start) : nullptr;
+  dp.group_min = p->cta_pairs ? p->pgroup_min : p->group_min;
+  dp.group_max = p->cta_pairs ? p->pgroup_max : p->group_max;
+  dp.max_groups = p->cta_pairs ? p->pmax_groups : p->max_groups;
   mark(1);
   moe_dispatch_scan_kernel<<<1, kScanThreads, 0, st>>>(dp);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
@@ -279,42 +298,93 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   }
 
   // 4. persistent expert GEMM (L1 + SwiGLU, L2 + weighted scatter-add)
-  GemmParams gp;
-  std::memset(&gp, 0, sizeof(gp));
   bf16* h = reinterpret_cast<bf16*>(ws + L.h);
   const int E = p->E, H = p->H, I = p->I;
-  bool ok = make_map(&gp.tm_w1, W1, I, (uint64_t)E * H, I, 64) &&
-            make_map(&gp.tm_w3, W3, I, (uint64_t)E * H, I, 64) &&
-            make_map(&gp.tm_w2, W2, H, (uint64_t)E * I, H, 64) &&
-            make_map(&gp.tm_h, h, I, (uint64_t)p->ring_blocks * p->BM, I, p->BM);
-  if (!ok) return MOE_ERR_CUDA;
-  gp.x = static_cast<const bf16*>(x);
-  gp.slot_token = dp.slot_token;
-  gp.slot_topk = dp.slot_topk;
-  gp.topk_w = rp.topk_w;
-  gp.block_start = dp.block_start;
-  gp.group_start = dp.group_start;
-  gp.num_groups = dp.sched + 3;
-  gp.task_counter = dp.sched;
-  gp.l1_done = dp.l1_done;
-  gp.l2_done = dp.l2_done;
-  gp.ring_blocks = p->ring_blocks;
-  gp.max_groups = p->max_groups;
-  gp.err = dp.err;
-  gp.h = h;
-  gp.y_acc = rp.y_acc;
-  gp.T = T;
-  gp.H = H;
-  gp.I = I;
-  gp.E = E;
-  gp.k = p->k;
-  gp.BM = p->BM;
-  gp.BN2 = p->BN2;
-  gp.N1 = p->N1;
-  gp.N2 = p->N2;
-  gp.timeout_ns = p->timeout_ns;
-  gp.withhold_block = p->withhold;
-  moe_expert_gemm_kernel<<<p->num_sms, kGemmThreads, kGemmSmemBytes, st>>>(gp);
+  if (p->cta_pairs) {
+    Gemm2Params gp;
+    std::memset(&gp, 0, sizeof(gp));
+    bool ok = make_map(&gp.tm_w1, W1, I, (uint64_t)E * H, I, 64) &&
+              make_map(&gp.tm_w3, W3, I, (uint64_t)E * H, I, 64) &&
+              make_map(&gp.tm_w2, W2, H, (uint64_t)E * I, H, 64) &&
+              make_map(&gp.tm_h, h, I, (uint64_t)p->ring_pairs * 2 * p->BM, I, p->BM);
+    if (!ok) return MOE_ERR_CUDA;
+    gp.x = static_cast<const bf16*>(x);
+    gp.slot_token = dp.slot_token;
+    gp.slot_topk = dp.slot_topk;
+    gp.topk_w = rp.topk_w;
+    gp.block_start = dp.block_start;
+    gp.pair_start = dp.pair_start;
+    gp.group_start = dp.group_start;
+    gp.num_groups = dp.sched + 3;
+    gp.task_counter = dp.sched;
+    gp.l1_done = dp.l1_done;
+    gp.l2_done = dp.l2_done;
+    gp.err = dp.err;
+    gp.h = h;
+    gp.y_acc = rp.y_acc;
+    gp.T = T;
+    gp.H = H;
+    gp.I = I;
+    gp.E = E;
+    gp.k = p->k;
+    gp.BM = p->BM;
+    gp.BN2 = p->BN2;
+    gp.N1 = p->N1;
+    gp.N2 = p->N2;
+    gp.ring_pairs = p->ring_pairs;
+    gp.max_groups = p->pmax_groups;
+    gp.timeout_ns = p->timeout_ns;
+    gp.withhold_pair = p->withhold;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)(2 * p->pair_clusters));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = kGemm2SmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, moe_expert_gemm2_kernel, gp) != cudaSuccess) return MOE_ERR_CUDA;
+  } else {
+    GemmParams gp;
+    std::memset(&gp, 0, sizeof(gp));
+    bool ok = make_map(&gp.tm_w1, W1, I, (uint64_t)E * H, I, 64) &&
+              make_map(&gp.tm_w3, W3, I, (uint64_t)E * H, I, 64) &&
+              make_map(&gp.tm_w2, W2, H, (uint64_t)E * I, H, 64) &&
+              make_map(&gp.tm_h, h, I, (uint64_t)p->ring_blocks * p->BM, I, p->BM);
+    if (!ok) return MOE_ERR_CUDA;
+    gp.x = static_cast<const bf16*>(x);
+    gp.slot_token = dp.slot_token;
+    gp.slot_topk = dp.slot_topk;
+    gp.topk_w = rp.topk_w;
+    gp.block_start = dp.block_start;
+    gp.group_start = dp.group_start;
+    gp.num_groups = dp.sched + 3;
+    gp.task_counter = dp.sched;
+    gp.l1_done = dp.l1_done;
+    gp.l2_done = dp.l2_done;
+    gp.ring_blocks = p->ring_blocks;
+    gp.max_groups = p->max_groups;
+    gp.err = dp.err;
+    gp.h = h;
+    gp.y_acc = rp.y_acc;
+    gp.T = T;
+    gp.H = H;
+    gp.I = I;
+    gp.E = E;
+    gp.k = p->k;
+    gp.BM = p->BM;
+    gp.BN2 = p->BN2;
+    gp.N1 = p->N1;
+    gp.N2 = p->N2;
+    gp.timeout_ns = p->timeout_ns;
+    gp.withhold_block = p->withhold;
+    moe_expert_gemm_kernel<<<p->num_sms, kGemmThreads, kGemmSmemBytes, st>>>(gp);
+  }
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   mark(4);
 
@@ -457,6 +527,7 @@ extern "C" int moe_route_static(const void* x, const void* Wg, const float* gate
   dp.pool = (int)pool;
   dp.group_start = nullptr;   // routing only: no expert-GEMM task groups
   dp.l2_done = nullptr;
+  dp.pair_start = nullptr;
   dp.group_min = dp.group_max = dp.max_groups = 0;
   moe_dispatch_scan_kernel<<<1, kScanThreads, 0, st>>>(dp);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
@@ -520,11 +591,16 @@ int moe_plan_create(moe_plan_t* out, int T_max, int H, int I, int E, int k, int 
   p->group_max = std::max(2 * p->group_min, per_expert);
   p->max_groups = p->blocks_max / p->group_min + 2;
   p->ring_blocks = std::min(3 * p->group_max, p->blocks_max);
+  p->per_expert = per_expert;
+  size_pair_groups(p);
   p->L = make_layout(*p);
 
   DeviceGuard guard(device);
   cudaError_t ce = cudaFuncSetAttribute(moe_expert_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)kGemmSmemBytes);
+  if (ce == cudaSuccess)
+    ce = cudaFuncSetAttribute(moe_expert_gemm2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)kGemm2SmemBytes);
   if (ce == cudaSuccess)
     ce = cudaFuncSetAttribute(moe_router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRtcSmemBytes);
   if (ce == cudaSuccess) ce = set_router_smem<16>();
@@ -535,6 +611,30 @@ int moe_plan_create(moe_plan_t* out, int T_max, int H, int I, int E, int k, int 
   if (ce != cudaSuccess) {
     delete p;
     return MOE_ERR_CUDA;
+  }
+  {
+    // how many 2-CTA clusters of the pair kernel can be resident at once (a
+    // cluster needs two free SMs of one GPC); the pair grid is sized to it
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)(p->num_sms & ~1));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = kGemm2SmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, moe_expert_gemm2_kernel, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      clusters = 0;
+    }
+    p->pair_clusters = clusters;
+    size_pair_groups(p);   // with the real number of concurrent pair tasks
+    p->L = make_layout(*p);
   }
   *out = p;
   return MOE_OK;
@@ -566,6 +666,7 @@ int moe_plan_describe(moe_plan_t p, moe_plan_desc* d) {
   d->block_m = p->BM;
   d->pool_capacity = p->pool;
   d->num_sms = p->num_sms;
+  d->pair_clusters = p->pair_clusters;
   d->workspace_bytes = p->L.total;
   return MOE_OK;
 }
@@ -669,6 +770,13 @@ int moe_plan_set_debug(moe_plan_t p, int withhold_block, uint64_t timeout_ns) {
   if (p == nullptr) return MOE_ERR_INVALID_ARG;
   p->withhold = withhold_block;
   p->timeout_ns = timeout_ns ? timeout_ns : 2000000000ull;
+  return MOE_OK;
+}
+
+int moe_plan_set_cta_pairs(moe_plan_t p, int enable) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  if (enable && p->pair_clusters < 1) return MOE_ERR_UNSUPPORTED_SHAPE;
+  p->cta_pairs = enable != 0;
   return MOE_OK;
 }
 

@@ -1,0 +1,98 @@
+"""Parity of the CTA-pair expert GEMM (tcgen05 cta_group::2) with the oracle.
+
+Same checks as test_gpu_parity / test_gpu_workloads, with the plan switched
+to CTA pairs: two consecutive blocks of an expert per task, each CTA of a
+cluster holding its own block's rows and half of the weight tile. Shapes
+include experts with an odd block count (the second CTA of the last pair has
+no block), BLOCK_M below 128, H % 256 != 0 and a ring that wraps.
+"""
+import numpy as np
+import pytest
+import torch
+
+from synth.moe_inputs import WORKLOADS, custom_shape, make_inputs
+from tests.parity_util import assert_routing_equal, assert_y_close, oracle_forward, sample_tokens
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+PAIR_SHAPES = [
+    # T,   H,   I,   E,  k, block_m, zipf
+    (64, 128, 256, 8, 2, 0, False),
+    (300, 256, 384, 16, 4, 0, False),      # H % 256 != 0 (L2 tile 128 columns)
+    (300, 256, 384, 16, 4, 16, False),
+    (129, 384, 256, 32, 8, 0, True),
+    (1000, 256, 512, 8, 2, 0, False),      # several pairs per expert, odd block counts
+    (500, 512, 256, 128, 8, 0, True),
+    (4096, 128, 14336, 32, 2, 0, False),   # N1 = 112: small groups, the h ring wraps
+]
+
+
+def _plan(shape, block_m=0):
+    from moe_megakernel_b200 import MoEPlan
+    plan = MoEPlan(shape.T, shape.H, shape.I, shape.E, shape.k, block_m=block_m)
+    plan.set_cta_pairs(True)
+    return plan
+
+
+@pytest.mark.parametrize("T,H,I,E,k,bm,zipf", PAIR_SHAPES)
+def test_pairs_forward_matches_oracle(T, H, I, E, k, bm, zipf):
+    shape = custom_shape(T, H, I, E, k, zipf)
+    inp = make_inputs(shape, device=DEV)
+    plan = _plan(shape, bm)
+    plan.workspace.fill_(0xFF)   # poison: unwritten reads show up as NaN
+    plan.lib.moe_plan_bind_workspace(plan._plan, plan.workspace.data_ptr(), plan.workspace_bytes)
+    y = plan.forward(inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"])
+    plan.check()
+    rows = sample_tokens(T, 256)
+    ref = oracle_forward(inp, tokens=rows, block_m=plan.block_m)
+    assert_routing_equal(plan.routing(T), ref)
+    fro, mx = assert_y_close(y[torch.from_numpy(rows).to(y.device)], ref["y"])
+    print(f"pairs T={T} H={H} I={I} E={E} k={k}: rel_fro={fro:.2e} max_abs={mx:.2e}")
+
+
+def test_pairs_and_single_agree_and_repeat():
+    shape = custom_shape(1000, 256, 512, 8, 2)
+    inp = make_inputs(shape, device=DEV)
+    plan = _plan(shape)
+    y_pair = plan.forward(inp["x"], inp["Wg"], None, inp["W1"], inp["W3"], inp["W2"]).float()
+    plan.check()
+    y_pair2 = plan.forward(inp["x"], inp["Wg"], None, inp["W1"], inp["W3"], inp["W2"]).float()
+    plan.check()
+    plan.set_cta_pairs(False)
+    y_single = plan.forward(inp["x"], inp["Wg"], None, inp["W1"], inp["W3"], inp["W2"]).float()
+    plan.check()
+    assert (y_pair - y_single).abs().max().item() <= 1e-2
+    assert (y_pair - y_pair2).abs().max().item() <= 1e-2
+
+
+def test_pairs_bounded_wait_reports_timeout():
+    from moe_megakernel_b200 import MoEError
+    shape = custom_shape(256, 128, 256, 8, 2)
+    inp = make_inputs(shape, device=DEV)
+    plan = _plan(shape)
+    plan.set_debug(withhold_block=0, timeout_ns=20_000_000)   # pair 0's L1 completion never published
+    plan.forward(inp["x"], inp["Wg"], None, inp["W1"], inp["W3"], inp["W2"])
+    with pytest.raises(MoEError) as ei:
+        plan.check()
+    assert ei.value.status == 6
+    plan.set_debug(-1, 0)
+    y = plan.forward(inp["x"], inp["Wg"], None, inp["W1"], inp["W3"], inp["W2"])
+    plan.check()
+    assert_y_close(y, oracle_forward(inp, block_m=plan.block_m)["y"])
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["mixtral", "fine_grained_prefill", "decode", "skewed"])
+def test_pairs_workload_matches_oracle(name):
+    shape = WORKLOADS[name]
+    inp = make_inputs(shape, device=DEV)
+    plan = _plan(shape)
+    y = plan.forward(inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"])
+    plan.check()
+    rows = sample_tokens(shape.T, {"mixtral": 32, "fine_grained_prefill": 12, "decode": 32, "skewed": 96}[name])
+    ref = oracle_forward(inp, tokens=rows, block_m=plan.block_m)
+    assert_routing_equal(plan.routing(shape.T), ref)
+    fro, mx = assert_y_close(y[torch.from_numpy(rows).to(y.device)], ref["y"])
+    print(f"pairs {name}: rel_fro={fro:.2e} max_abs={mx:.2e}")

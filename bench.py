@@ -50,7 +50,7 @@ def measured_peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
-GEMM_SOURCES = ("common.cuh", "ptx.cuh", "expert_gemm.cuh")   # what the expert-GEMM kernel is built from
+GEMM_SOURCES = ("common.cuh", "ptx.cuh", "expert_gemm.cuh", "expert_gemm2.cuh")   # what the expert GEMMs are built from
 
 
 def kernel_source_hash() -> str:
@@ -277,7 +277,8 @@ def run_gpu(args, rank, world, local_rank):
             gbs = alg_bytes / (gemm_ms * 1e-3) / 1e9
             roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": gbs / peaks["hbm_gbs"]}
-        roof.update({"kernel": "moe_expert_gemm_kernel", "traffic": measured_traffic(args.workload),
+        roof.update({"kernel": "moe_expert_gemm2_kernel" if plan.cta_pairs else "moe_expert_gemm_kernel",
+                     "traffic": measured_traffic(args.workload),
                      "traffic_unit": "bytes per launch (ncu dram read+write)",
                      "peak_source": f"{peaks['source']} ({'bf16_tflops_sustained' if bound == 'tensor' else 'hbm_gbs'})",
                      "kernel_ms": gemm_ms,
@@ -298,7 +299,7 @@ def run_gpu(args, rank, world, local_rank):
             "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) x, N(0,1/H) Wg/W1/W3, N(0,1/I) W2, bf16; random-init weights)",
             "config": {"workload": workload_label(shape), "T_per_gpu": T, "H": H, "I": I, "E": E, "k": k,
-                       "block_m": plan.block_m, "cta_pairs": bool(args.cta_pairs), "active_experts": active, "padded_slots": num_padded,
+                       "block_m": plan.block_m, "cta_pairs": plan.cta_pairs, "active_experts": active, "padded_slots": num_padded,
                        "l2": "flushed between steps (256 MB write, outside per-step events)",
                        "parallelism": "replicas" if world > 1 else "single"},
             "roofline": roof,

@@ -90,6 +90,7 @@ typedef struct {
   int32_t pool_capacity;   /* T_max*k + E*(block_m-1) slots */
   int32_t num_sms;         /* persistent grid size */
   int32_t pair_clusters;   /* co-resident 2-CTA clusters of the CTA-pair expert GEMM */
+  int32_t cta_pairs;       /* 1: the expert GEMM runs on CTA pairs (see moe_plan_set_cta_pairs) */
   size_t workspace_bytes;
 } moe_plan_desc;
 
@@ -210,9 +211,12 @@ int moe_route_static(const void* x, const void* Wg, const float* gate_bias, int 
 /* Expert-GEMM variant: enable != 0 runs the persistent expert GEMM on CTA
  * pairs (clusters of two CTAs on neighbouring SMs, tcgen05 cta_group::2):
  * each task covers two consecutive blocks of one expert (256 rows) and each
- * CTA loads half of the weight tile. enable = 0 runs one CTA per 128-row
- * block. Results are the same up to fp32 summation order. Takes effect at the
- * next moe_forward; the workspace size does not depend on it. */
+ * CTA loads half of the weight tile. enable = 0 runs one CTA per block. A new
+ * plan uses pairs when BLOCK_M is 128 and the device can co-schedule 2-CTA
+ * clusters, else one CTA per block. Results are the same up to fp32
+ * summation order. Takes effect at the next moe_forward; the workspace size
+ * does not depend on it. Errors: MOE_ERR_INVALID_ARG (null plan),
+ * MOE_ERR_UNSUPPORTED_SHAPE (pairs requested where no 2-CTA cluster fits). */
 int moe_plan_set_cta_pairs(moe_plan_t plan, int enable);
 
 /* Number of kernels one moe_forward launches (for launch accounting). */

@@ -38,7 +38,8 @@ class MoEPlanDesc(ctypes.Structure):
     _fields_ = [("T_max", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
                 ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("block_m", ctypes.c_int32),
                 ("pool_capacity", ctypes.c_int32), ("num_sms", ctypes.c_int32),
-                ("pair_clusters", ctypes.c_int32), ("workspace_bytes", ctypes.c_size_t)]
+                ("pair_clusters", ctypes.c_int32), ("cta_pairs", ctypes.c_int32),
+                ("workspace_bytes", ctypes.c_size_t)]
 
 
 # exported symbol -> (restype, argtypes); the same list as include/moe_b200.h
@@ -227,6 +228,13 @@ class MoEPlan:
 
     def set_cta_pairs(self, enable: bool):
         _ok(self.lib.moe_plan_set_cta_pairs(self._plan, 1 if enable else 0), "moe_plan_set_cta_pairs")
+
+    @property
+    def cta_pairs(self) -> bool:
+        """Whether the expert GEMM currently runs on CTA pairs."""
+        d = MoEPlanDesc()
+        _ok(self.lib.moe_plan_describe(self._plan, ctypes.byref(d)), "moe_plan_describe")
+        return bool(d.cta_pairs)
 
     def set_debug(self, withhold_block: int = -1, timeout_ns: int = 0):
         _ok(self.lib.moe_plan_set_debug(self._plan, withhold_block, timeout_ns), "moe_plan_set_debug")

@@ -38,6 +38,7 @@ constexpr int kTaskRing = 4;
 #endif
 constexpr int kGatherWarps = MOE_GATHER_WARPS;     // warps that gather routed x rows
 constexpr int kGemmThreads = 192 + 32 * kGatherWarps;   // producer, MMA, 4 epilogue warps, gather warps
+constexpr int kGemm1Threads = kGemmThreads + 32;        // the same plus a scheduler warp (single-CTA kernel)
 constexpr int kTmemCols = 512;                     // two 256-column fp32 accumulators
 constexpr int kMaxGroups = 512;                    // block groups of the expert GEMM's task order
 

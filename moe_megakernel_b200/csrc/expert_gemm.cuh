@@ -9,9 +9,10 @@
 //   m-block, n-tile).
 // * "MegaMoE 在 MoE 系统谱系中的位置", section 2.1: warp roles inside the CTA
 //   (dispatch/activation loads, weight TMA, MMA issue, scheduler, epilogue).
-//   Here warp 0 is scheduler + TMA producer of the weight tiles (and of the h
-//   tiles in L2), warp 1 issues tcgen05 MMAs, warps 2-5 drain TMEM in the
-//   epilogue, and warps 6.. gather the routed x rows for L1.
+//   Here warp 0 is the TMA producer of the weight tiles, warp 1 issues
+//   tcgen05 MMAs, warps 2-5 drain TMEM in the epilogue, warps 6.. load the
+//   A rows (routed x rows in L1, the block's h rows in L2), and the last
+//   warp is the scheduler: it claims, decodes and prepares the next task.
 // * Same page, section 2.7: tasks are claimed from a global atomic counter,
 //   and an L2 task of pool block b waits on an in-kernel counter until the L1
 //   tasks of block b are complete (bounded wait here).
@@ -39,7 +40,6 @@ struct GemmParams {
   CUtensorMap tm_w1;   // W1 as [E*H, I], box {64, 64}
   CUtensorMap tm_w3;   // W3 as [E*H, I], box {64, 64}
   CUtensorMap tm_w2;   // W2 as [E*I, H], box {64, 64}
-  CUtensorMap tm_h;    // h ring [ring_blocks * BM, I], box {64, BM}
   const int32_t* slot_token;
   const int32_t* slot_topk;
   const float* topk_w;
@@ -66,9 +66,10 @@ struct Task {
 
 struct GemmSmem {
   // L2 epilogue staging, per epilogue warp: 32 rows x 32 fp32 (rows padded to
-  // 144 B so that the 32 lanes' 16-byte stores hit distinct banks). First
-  // member, so 16-byte aligned as the bulk reduction's source must be.
+  // 144 B so that row-wise and transposed 16-byte accesses are conflict-free),
+  // and the token of each staged row.
   float out_stage[4][32][36];
+  int out_tok[4][32];
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t acc_full[2];
@@ -79,13 +80,14 @@ struct GemmSmem {
   Task tasks[kTaskRing];
   uint32_t tmem_base;
   int abort;
+  int taken;                     // tasks the producer has taken from the ring
   int num_groups;
   int rows[kTaskRing][kTileM];   // token row of each A-tile row, per task-ring slot (L1 tasks)
   int block_start[257];
   int group_start[kMaxGroups + 1];
 };
 
-static_assert(offsetof(GemmSmem, out_stage) % 16 == 0, "bulk-reduce source must be 16-byte aligned");
+static_assert(offsetof(GemmSmem, out_stage) % 16 == 0, "staging rows are read as float4");
 static_assert((36 * 4) % 16 == 0, "staging rows must stay 16-byte aligned");
 
 constexpr size_t kGemmSmemBytes = 1024 /*alignment slack*/ + (size_t)kStages * kStageBytes + sizeof(GemmSmem);
@@ -194,12 +196,14 @@ __device__ __forceinline__ Task decode_task(int t, const GemmSmem& s, const Gemm
 
 __device__ __forceinline__ uint8_t* stage_ptr(uint8_t* tiles, int stage) { return tiles + stage * kStageBytes; }
 
-// ---------------------------------------------------------------- producer (warp 0)
-// Scheduler and weight-tile TMA. The next task is claimed as soon as the
-// current one starts, and prepared (decoded; for L1 its routed row indices
-// staged in shared memory; for L2 its dependency counter probed) while the
-// current task's k-loop is being issued, so that task switches cost no
-// global round trip on the critical path.
+// ---------------------------------------------------------------- scheduler (last warp)
+// Claims tasks from the global counter, decodes them, stages the routed row
+// indices of L1 tasks in s.rows[q] and waits for the L1 tiles an L2 task
+// reads, then publishes the task in ring slot q. Every global round trip of
+// the task switch happens here, one task ahead of the producer, so the weight
+// stream never pauses for it. It claims the next task only once the producer
+// has taken the last one it published: at most one claimed task waits in the
+// ring, which keeps the end of the kernel balanced across CTAs.
 __device__ __forceinline__ int claim_task(const GemmParams& p, GemmSmem& s, int lane) {
   int t = 0x7fffffff;
   if (lane == 0) {
@@ -207,75 +211,106 @@ __device__ __forceinline__ int claim_task(const GemmParams& p, GemmSmem& s, int 
         *reinterpret_cast<volatile int*>(&s.abort) || *reinterpret_cast<volatile int*>(p.err) != 0;
     if (!stop) t = atomicAdd(p.task_counter, 1);
   }
-  return t;   // valid in lane 0 only
+  return __shfl_sync(0xffffffffu, t, 0);
 }
 
-// Decode task t into ring slot q: for L1, stage the token row of every A-tile
-// row in s.rows[q]; for L2, report whether block b's L1 tiles are all done.
-__device__ __forceinline__ Task prepare_task(int t, int q, uint32_t qparity, bool& deps_ready, bool& ok,
-                                             const GemmParams& p, GemmSmem& s, int lane) {
-  Task task = decode_task(t, s, p);
-  deps_ready = true;
-  ok = warp_wait(&s.task_empty[q], qparity, p, s, 1);
-  if (!ok) return task;
-  if (task.phase == 0) {
-    for (int r = lane; r < p.BM; r += 32) {
-      int tok = p.slot_token[task.b * p.BM + r];
-      if (tok >= p.T) {
-        set_error(p, s, kDevBounds, task.b);
-        tok = 0;
-      }
-      s.rows[q][r] = tok < 0 ? 0 : tok;   // padding slot: any valid row, the epilogue drops it
+// Bounded wait (one thread) until the producer has taken `n` tasks.
+__device__ __forceinline__ bool wait_taken(int n, const GemmParams& p, GemmSmem& s) {
+  if (*reinterpret_cast<volatile int*>(&s.taken) >= n) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  while (*reinterpret_cast<volatile int*>(&s.taken) < n) {
+    if (*reinterpret_cast<volatile int*>(&s.abort)) return false;
+    if (ptx::globaltimer() - t0 > p.timeout_ns) {
+      set_error(p, s, kDevTimeout, 10);
+      return false;
     }
-  } else if (task.phase == 1) {
-    int ready = 1;
-    if (lane == 0) ready = ptx::ld_acquire_gpu(p.l1_done + task.b) >= 4 * p.N1;
-    deps_ready = __shfl_sync(0xffffffffu, ready, 0) != 0;
+    __nanosleep(64);
   }
-  __syncwarp();
-  return task;
+  return true;
 }
 
-__device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) {
+__device__ void gemm_scheduler(const GemmParams& p, GemmSmem& s) {
   const int lane = ptx::lane_id();
-  // Weight tiles are streamed: the few m-blocks sharing a slice read it at
-  // nearly the same time, so mark it first to evict; h keeps the default.
-  const uint64_t pol = ptx::policy_evict_first();
-  const uint64_t polh = ptx::policy_evict_normal();
-  int stage = 0;
-  uint32_t phase = 0;
   int q = 0;
   uint32_t qphase = 0;
-  uint32_t issued = 0, issued_parity = 0;   // per stage: ever issued, parity of the last issue
-
-  bool deps_ready = true, ok = true;
-  int t = __shfl_sync(0xffffffffu, claim_task(p, s, lane), 0);
-  Task task = prepare_task(t, q, qphase ^ 1, deps_ready, ok, p, s, lane);
-  while (ok) {
-    if (task.phase == 1 && !deps_ready) {
+  int pushed = 0;
+  while (true) {
+    bool ok = true;
+    if (lane == 0) ok = wait_taken(pushed, p, s);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    Task task{-1, 0, 0, 0};
+    if (ok) task = decode_task(claim_task(p, s, lane), s, p);
+    if (!warp_wait(&s.task_empty[q], qphase ^ 1, p, s, 1)) break;
+    if (task.phase == 0) {
+      // all loads first (one round trip), then the checks
+      constexpr int kPer = kTileM / 32;
+      int tok[kPer];
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int r = lane + 32 * i;
+        tok[i] = r < p.BM ? p.slot_token[task.b * p.BM + r] : 0;
+      }
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int r = lane + 32 * i;
+        if (r < p.BM) {
+          if (tok[i] >= p.T) {
+            set_error(p, s, kDevBounds, task.b);
+            tok[i] = 0;
+          }
+          s.rows[q][r] = tok[i] < 0 ? 0 : tok[i];   // padding slot: any valid row, the epilogue drops it
+        }
+      }
+    } else if (task.phase == 1) {
       // the L2 task of block b reads h rows written by all L1 n-tiles of block b
       // (one arrival per epilogue warp per n-tile)
       bool fine = true;
       if (lane == 0) fine = wait_counter(p.l1_done + task.b, 4 * p.N1, p, s, 0x10000 | task.b);
       if (__shfl_sync(0xffffffffu, fine ? 1 : 0, 0) == 0) task.phase = -1;
     }
-    if (task.phase == 1) ptx::fence_proxy_async_global();   // h written by other CTAs -> TMA reads
-
-    // hand the task to the MMA, epilogue and gather warps (its slot was freed in prepare_task)
+    __syncwarp();
     if (lane == 0) {
       s.tasks[q] = task;
       ptx::mbar_arrive(&s.task_full[q]);
     }
     __syncwarp();
-    const int qn = (q + 1) % kTaskRing;
-    const uint32_t qphase_n = qn == 0 ? qphase ^ 1 : qphase;
+    ++pushed;
+    if (++q == kTaskRing) {
+      q = 0;
+      qphase ^= 1;
+    }
+    if (task.phase < 0) break;
+  }
+}
+
+// ---------------------------------------------------------------- producer (warp 0)
+// Weight-tile TMA (and the h tiles of L2 tasks) for the tasks the scheduler publishes.
+__device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) {
+  const int lane = ptx::lane_id();
+  // Weight tiles are streamed: the few m-blocks sharing a slice read it at
+  // nearly the same time, so mark it first to evict.
+  const uint64_t pol = ptx::policy_evict_first();
+  int stage = 0;
+  uint32_t phase = 0;
+  int q = 0;
+  uint32_t qphase = 0;
+  uint32_t issued = 0, issued_parity = 0;   // per stage: ever issued, parity of the last issue
+  bool ok = true;
+  while (ok) {
+    if (!warp_wait(&s.task_full[q], qphase, p, s, 11)) break;
+    const Task task = s.tasks[q];
+    __syncwarp();
+    if (lane == 0) {
+      ptx::mbar_arrive(&s.task_empty[q]);
+      *reinterpret_cast<volatile int*>(&s.taken) = *reinterpret_cast<volatile int*>(&s.taken) + 1;
+    }
+    if (++q == kTaskRing) {
+      q = 0;
+      qphase ^= 1;
+    }
     if (task.phase < 0) break;
 
-    const int t_next_lane0 = claim_task(p, s, lane);   // result consumed after a few stages
-    bool prepared = false;
-    Task next{-1, 0, 0, 0};
     const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
-    const int prep_at = nk > 2 ? 2 : nk - 1;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait(&s.empty[stage], phase ^ 1, p, s, 2)) {
         ok = false;
@@ -289,16 +324,16 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
           ptx::mbar_arrive_expect_tx(&s.full[stage], 4 * kBoxBytes);
           const int wrow = task.e * p.H + kb * kBK;
           const int n0 = task.n * kL1TileN;
-          ptx::tma_load_2d(b_addr + 0 * kBoxBytes, &p.tm_w1, &s.full[stage], n0, wrow, pol);
-          ptx::tma_load_2d(b_addr + 1 * kBoxBytes, &p.tm_w1, &s.full[stage], n0 + 64, wrow, pol);
-          ptx::tma_load_2d(b_addr + 2 * kBoxBytes, &p.tm_w3, &s.full[stage], n0, wrow, pol);
-          ptx::tma_load_2d(b_addr + 3 * kBoxBytes, &p.tm_w3, &s.full[stage], n0 + 64, wrow, pol);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            ptx::tma_load_2d(b_addr + j * kBoxBytes, j < 2 ? &p.tm_w1 : &p.tm_w3, &s.full[stage], n0 + (j & 1) * 64,
+                             wrow, pol);
         }
       } else {
+        // B: 256 (or 128) columns of W2; A (the block's h rows) comes from the gather warps.
         if (lane == 0) {
           const int nbox = p.BN2 / 64;
-          ptx::mbar_arrive_expect_tx(&s.full[stage], p.BM * 128 + nbox * kBoxBytes);
-          ptx::tma_load_2d(a_addr, &p.tm_h, &s.full[stage], kb * kBK, (task.b % p.ring_blocks) * p.BM, polh);
+          ptx::mbar_arrive_expect_tx(&s.full[stage], nbox * kBoxBytes);
           const int wrow = task.e * p.I + kb * kBK;
           for (int j = 0; j < nbox; ++j)
             ptx::tma_load_2d(b_addr + j * kBoxBytes, &p.tm_w2, &s.full[stage], task.n * p.BN2 + j * 64, wrow,
@@ -312,21 +347,7 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
         stage = 0;
         phase ^= 1;
       }
-      if (kb == prep_at) {
-        const int tn = __shfl_sync(0xffffffffu, t_next_lane0, 0);
-        next = prepare_task(tn, qn, qphase_n ^ 1, deps_ready, ok, p, s, lane);
-        prepared = true;
-        if (!ok) break;
-      }
     }
-    if (!ok) break;
-    if (!prepared) {
-      const int tn = __shfl_sync(0xffffffffu, t_next_lane0, 0);
-      next = prepare_task(tn, qn, qphase_n ^ 1, deps_ready, ok, p, s, lane);
-    }
-    task = next;
-    q = qn;
-    qphase = qphase_n;
   }
   // On an early exit, let every issued copy land before the CTA can retire.
   for (int st = 0; st < kStages; ++st)
@@ -414,14 +435,14 @@ __device__ void gemm_mma(const GemmParams& p, GemmSmem& s, uint8_t* tiles, uint3
   }
 }
 
-// ---------------------------------------------------------------- gather warps (warps 6 .. 6+G-1)
+// ---------------------------------------------------------------- A-row warps (warps 6 .. 6+G-1)
 // L1 tasks: the A tile is BM routed rows of x, 64 columns per stage. Warp
 // instruction i (4 rows x 128 B, one 16-byte chunk per lane) is issued by
 // gather warp i % G; chunk c of row r lands at chunk c ^ (r % 8) of the
 // row's 128 bytes, the 128-byte swizzle the MMA descriptor expects. Every
 // lane arrives on the stage's full barrier when its own copies have landed.
-// L2 tasks: the producer loads A with TMA; each gather warp arrives for its
-// 32 lanes so that the barrier's arrival count is the same for both phases.
+// L2 tasks: the same for the block's BM rows of h in the ring (a single
+// 128-row TMA box per stage kept the tensor pipe waiting twice as long).
 __device__ void gemm_gather(const GemmParams& p, GemmSmem& s, uint8_t* tiles, int g) {
   constexpr int kRowsPerLane = (kTileM / 4 + kGatherWarps - 1) / kGatherWarps;   // rows >= BM are skipped
   const int lane = ptx::lane_id();
@@ -439,21 +460,21 @@ __device__ void gemm_gather(const GemmParams& p, GemmSmem& s, uint8_t* tiles, in
       qphase ^= 1;
     }
     if (task.phase < 0) break;
-    // smem offset and source row of each of this lane's rows (row indices staged by the producer)
+    // smem offset and source row of each of this lane's rows: L1, the routed x
+    // rows (indices staged by the scheduler); L2, the block's h rows in the ring
     int nrows = 0;
     uint32_t soff[kRowsPerLane];
     const bf16* src[kRowsPerLane];
-    if (task.phase == 0) {
-      const int* rows = s.rows[q_task];
+    const int* rows = s.rows[q_task];
+    const bf16* hblock = p.h + (size_t)(task.b % p.ring_blocks) * p.BM * p.I;
 #pragma unroll
-      for (int j = 0; j < kRowsPerLane; ++j) {
-        const int r = (j * kGatherWarps + g) * 4 + (lane >> 3);
-        soff[j] = r * 128 + ((c ^ (r & 7)) << 4);
-        src[j] = p.x + c * 8;
-        if (r < p.BM) {
-          src[j] = p.x + (size_t)rows[r] * p.H + c * 8;
-          nrows = j + 1;
-        }
+    for (int j = 0; j < kRowsPerLane; ++j) {
+      const int r = (j * kGatherWarps + g) * 4 + (lane >> 3);
+      soff[j] = r * 128 + ((c ^ (r & 7)) << 4);
+      src[j] = p.x + c * 8;
+      if (r < p.BM) {
+        src[j] = task.phase == 0 ? p.x + (size_t)rows[r] * p.H + c * 8 : hblock + (size_t)r * p.I + c * 8;
+        nrows = j + 1;
       }
     }
     __syncwarp();
@@ -465,16 +486,11 @@ __device__ void gemm_gather(const GemmParams& p, GemmSmem& s, uint8_t* tiles, in
         ok = false;
         break;
       }
-      if (task.phase == 0) {
-        const uint32_t a_addr = ptx::smem_u32(stage_ptr(tiles, stage));
+      const uint32_t a_addr = ptx::smem_u32(stage_ptr(tiles, stage));
 #pragma unroll
-        for (int j = 0; j < kRowsPerLane; ++j)
-          if (j < nrows) ptx::cp_async_16(a_addr + soff[j], src[j] + kb * kBK);
-        ptx::cp_async_mbar_arrive_noinc(&s.full[stage]);
-      } else {
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive_count(&s.full[stage], 32);
-      }
+      for (int j = 0; j < kRowsPerLane; ++j)
+        if (j < nrows) ptx::cp_async_16(a_addr + soff[j], src[j] + kb * kBK);
+      ptx::cp_async_mbar_arrive_noinc(&s.full[stage]);
       if (++stage == kStages) {
         stage = 0;
         phase ^= 1;
@@ -490,6 +506,45 @@ __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f +
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Combine of one epilogue warp's 32 accumulator rows (TMEM lanes tbase..+31,
+// columns 0..ncols-1): y_acc[tok_r][c] += w_r * acc[r][c] for every row r with
+// tok_r >= 0. Each lane holds row `lane`; per 32 columns the warp stages w*acc
+// in shared memory (rows padded to 36 floats, conflict-free both ways) and
+// reads it back transposed, so that 8 lanes cover one row's 128 contiguous
+// bytes and every red.v4 instruction adds 4 whole 128-byte row segments.
+__device__ __forceinline__ void combine_rows(uint32_t tbase, int ncols, float w, int tok, float* y_acc, int H,
+                                             int col0, float (*stage)[36], int* stage_tok) {
+  const int lane = ptx::lane_id();
+  stage_tok[lane] = tok;
+  __syncwarp();
+  const int sub = lane >> 3;
+  const int cc = (lane & 7) * 4;
+  float* ybase[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int t = stage_tok[i * 4 + sub];
+    ybase[i] = t >= 0 ? y_acc + (size_t)t * H + col0 + cc : nullptr;
+  }
+  float* srow = stage[lane];
+#pragma unroll 1
+  for (int c = 0; c < ncols / 32; ++c) {
+    uint32_t v[32];
+    ptx::tmem_ld32(tbase + c * 32, v);
+    ptx::tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      reinterpret_cast<float4*>(srow)[i] =
+          make_float4(w * __uint_as_float(v[4 * i + 0]), w * __uint_as_float(v[4 * i + 1]),
+                      w * __uint_as_float(v[4 * i + 2]), w * __uint_as_float(v[4 * i + 3]));
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (ybase[i] != nullptr)
+        ptx::red_add_v4_f32(ybase[i] + c * 32, *reinterpret_cast<const float4*>(&stage[i * 4 + sub][cc]));
+    __syncwarp();
+  }
 }
 
 // ---------------------------------------------------------------- epilogue (warps 2..5)
@@ -558,7 +613,6 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
       // Publish per warp (no cross-warp barrier): this warp's 32 h rows of the
       // (block, n-tile) are written. Block b is complete at 4 * N1 arrivals.
       __threadfence();
-      ptx::fence_proxy_async_global();
       __syncwarp();
       if (lane == 0 && task.b != p.withhold_block) ptx::red_release_gpu_add(p.l1_done + task.b, 1);
     } else {
@@ -583,30 +637,8 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
           }
         }
       }
-      // Combine: stage w * o for this row's 32 columns in shared memory, then
-      // one bulk reduction adds the 128 bytes into y_acc[token] (the L2 does the
-      // fp32 adds). Each lane reuses its own staging row once its previous
-      // reduction has read it.
-      float* yrow = p.y_acc + (size_t)(tok < 0 ? 0 : tok) * p.H + task.n * p.BN2;
-      float* srow = &s.out_stage[quarter][lane][0];
-      const uint32_t srow_addr = ptx::smem_u32(srow);
-#pragma unroll 1
-      for (int c = 0; c < p.BN2 / 32; ++c) {
-        uint32_t v[32];
-        ptx::tmem_ld32(tbase + c * 32, v);
-        ptx::tmem_ld_wait();
-        if (tok >= 0) {
-          ptx::bulk_wait_read_all();
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            reinterpret_cast<float4*>(srow)[i] =
-                make_float4(w * __uint_as_float(v[4 * i + 0]), w * __uint_as_float(v[4 * i + 1]),
-                            w * __uint_as_float(v[4 * i + 2]), w * __uint_as_float(v[4 * i + 3]));
-          ptx::fence_proxy_async_shared();
-          ptx::bulk_reduce_add_f32(yrow + c * 32, srow_addr, 128);
-          ptx::bulk_commit();
-        }
-      }
+      // Combine: y_acc[token] += w * o, 128-byte row segments per red.v4 (the L2 does the fp32 adds).
+      combine_rows(tbase, p.BN2, w, tok, p.y_acc, p.H, task.n * p.BN2, s.out_stage[quarter], s.out_tok[quarter]);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&s.acc_empty[acc]);
@@ -616,10 +648,9 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
       acc_phase ^= 1;
     }
   }
-  ptx::bulk_wait_all();   // every combine reduction has landed before the CTA retires
 }
 
-__global__ void __launch_bounds__(kGemmThreads, 1) moe_expert_gemm_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(kGemm1Threads, 1) moe_expert_gemm_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   GemmSmem& s = *reinterpret_cast<GemmSmem*>(tiles + (size_t)kStages * kStageBytes);
@@ -637,23 +668,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_expert_gemm_kernel(const 
     }
     for (int i = 0; i < kTaskRing; ++i) {
       ptx::mbar_init(&s.task_full[i], 1);
-      ptx::mbar_init(&s.task_empty[i], 5 + kGatherWarps);   // MMA, 4 epilogue warps, gather warps
+      ptx::mbar_init(&s.task_empty[i], 6 + kGatherWarps);   // producer, MMA, 4 epilogue warps, gather warps
     }
     ptx::mbar_init(&s.mma_done, 1);
     s.abort = 0;
+    s.taken = 0;
     ptx::fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     ptx::prefetch_tmap(&p.tm_w1);
     ptx::prefetch_tmap(&p.tm_w3);
     ptx::prefetch_tmap(&p.tm_w2);
-    ptx::prefetch_tmap(&p.tm_h);
   }
-  for (int e = threadIdx.x; e <= p.E; e += kGemmThreads) s.block_start[e] = p.block_start[e];
+  for (int e = threadIdx.x; e <= p.E; e += kGemm1Threads) s.block_start[e] = p.block_start[e];
   {
     const int ng = min(*p.num_groups, min(p.max_groups, kMaxGroups));
     if (threadIdx.x == 0) s.num_groups = ng;
-    for (int g = threadIdx.x; g <= ng; g += kGemmThreads) s.group_start[g] = p.group_start[g];
+    for (int g = threadIdx.x; g <= ng; g += kGemm1Threads) s.group_start[g] = p.group_start[g];
   }
   if (warp == 1) {
     ptx::tmem_alloc(&s.tmem_base, kTmemCols);
@@ -665,7 +696,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_expert_gemm_kernel(const 
     for (int st = 0; st < kStages; ++st) {
       uint4* a = reinterpret_cast<uint4*>(stage_ptr(tiles, st) + p.BM * row_bytes);
       const int n = (kTileM - p.BM) * row_bytes / 16;
-      for (int i = threadIdx.x; i < n; i += kGemmThreads) a[i] = make_uint4(0, 0, 0, 0);
+      for (int i = threadIdx.x; i < n; i += kGemm1Threads) a[i] = make_uint4(0, 0, 0, 0);
     }
     ptx::fence_proxy_async_shared();
   }
@@ -677,7 +708,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_expert_gemm_kernel(const 
   if (warp == 0) gemm_producer(p, s, tiles);
   else if (warp == 1) gemm_mma(p, s, tiles, tmem_base);
   else if (warp < 6) gemm_epilogue(p, s, tmem_base);
-  else gemm_gather(p, s, tiles, warp - 6);
+  else if (warp < 6 + kGatherWarps) gemm_gather(p, s, tiles, warp - 6);
+  else gemm_scheduler(p, s);
 
   ptx::tc_fence_before();
   __syncthreads();

@@ -1,6 +1,6 @@
 // Persistent grouped GEMM over the expert blocks on CTA pairs (tcgen05
 // cta_group::2): the same tasks as expert_gemm.cuh (L1 = x W1, x W3 + SwiGLU
-// into the h ring; L2 = h W2 + gate-weighted bulk-reduce combine), but every
+// into the h ring; L2 = h W2 + gate-weighted scatter-add combine), but every
 // task covers a PAIR of consecutive blocks of one expert, 256 rows, computed
 // by the two CTAs of a cluster together:
 //
@@ -11,8 +11,12 @@
 // * the leader CTA (rank 0) claims tasks, issues the MMAs for both CTAs and
 //   multicasts its commits to both CTAs' barriers; each CTA's accumulator is
 //   its own 128 rows x 256 columns in its own TMEM;
-// * each CTA's TMA loads and routed-row gathers land on its own stage
-//   barrier; the follower's warp 1 relays the completion of each of its
+// * L1 weight halves come by TMA; in L2 the A-row warps load both the h
+//   rows and the CTA's W2 half with cp.async (with a 64x64 TMA box of W2
+//   the L2 tasks ran at about half the tensor-pipe rate, with cp.async at
+//   70-90 %);
+// * each CTA's loads land on its own stage barrier; the follower's warp 1
+//   relays the completion of each of its
 //   stages to the leader's barrier with one remote arrival (counting the
 //   follower's bytes on the leader's barrier directly, with the pair form of
 //   the TMA load, measured 2.5x slower here).
@@ -38,10 +42,9 @@ constexpr int kStage2Bytes = kTileABytes + kTileB2Bytes;    // 32 KB
 
 struct Gemm2Params {
   const bf16* x;       // [T, H]
+  const bf16* w2;      // [E, I, H]
   CUtensorMap tm_w1;   // W1 as [E*H, I], box {64, 64}
   CUtensorMap tm_w3;   // W3 as [E*H, I], box {64, 64}
-  CUtensorMap tm_w2;   // W2 as [E*I, H], box {64, 64}
-  CUtensorMap tm_h;    // h ring [ring_pairs * 2 * BM, I], box {64, BM}
   const int32_t* slot_token;
   const int32_t* slot_topk;
   const float* topk_w;
@@ -69,7 +72,8 @@ struct Task2 {
 };
 
 struct Gemm2Smem {
-  float out_stage[4][32][36];   // L2 epilogue staging (see expert_gemm.cuh); first, 16-byte aligned
+  float out_stage[4][32][36];   // L2 epilogue staging (see combine_rows in expert_gemm.cuh)
+  int out_tok[4][32];
   uint64_t full[kStages2];
   uint64_t empty[kStages2];
   uint64_t acc_full[2];
@@ -87,7 +91,7 @@ struct Gemm2Smem {
   int group_start[kMaxGroups + 1];
 };
 
-static_assert(offsetof(Gemm2Smem, out_stage) % 16 == 0, "bulk-reduce source must be 16-byte aligned");
+static_assert(offsetof(Gemm2Smem, out_stage) % 16 == 0, "staging rows are read as float4");
 static_assert(sizeof(Task2) == 32, "tasks are copied to the peer as 8 words");
 
 constexpr size_t kGemm2SmemBytes = 1024 + (size_t)kStages2 * kStage2Bytes + sizeof(Gemm2Smem);
@@ -263,7 +267,6 @@ __device__ __forceinline__ void push_task2(const Task2& task, int q, Gemm2Smem& 
 __device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles) {
   const int lane = ptx::lane_id();
   const uint64_t pol = ptx::policy_evict_first();
-  const uint64_t polh = ptx::policy_evict_normal();
   int stage = 0;
   uint32_t phase = 0;
   int q = 0;
@@ -278,7 +281,6 @@ __device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_
       if (lane == 0) fine = wait_counter2(p.l1_done + task.p, 8 * p.N1, p, s, 0x10000 | task.p);
       if (__shfl_sync(0xffffffffu, fine ? 1 : 0, 0) == 0) task.phase = -1;
     }
-    if (task.phase == 1) ptx::fence_proxy_async_global();
     push_task2(task, q, s, lane);
     const int qn = (q + 1) % kTaskRing;
     const uint32_t qphase_n = qn == 0 ? qphase ^ 1 : qphase;
@@ -306,12 +308,9 @@ __device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_
           ptx::tma_load_2d(b_addr, &p.tm_w1, &s.full[stage], n0, wrow, pol);
           ptx::tma_load_2d(b_addr + kBoxBytes, &p.tm_w1, &s.full[stage], n0 + 64, wrow, pol);
         } else {
-          const int half_boxes = p.BN2 / 128;
-          ptx::mbar_arrive_expect_tx(&s.full[stage], p.BM * 128 + half_boxes * kBoxBytes);
-          ptx::tma_load_2d(a_addr, &p.tm_h, &s.full[stage], kb * kBK, ((task.p % p.ring_pairs) * 2 + 0) * p.BM, polh);
-          const int wrow = task.e * p.I + kb * kBK;
-          for (int j = 0; j < half_boxes; ++j)
-            ptx::tma_load_2d(b_addr + j * kBoxBytes, &p.tm_w2, &s.full[stage], task.n * p.BN2 + j * 64, wrow, pol);
+          // L2: both operands come from the A-row warps' cp.async (a TMA box of
+          // W2 kept the tensor pipe waiting); only this arrival is the producer's
+          ptx::mbar_arrive(&s.full[stage]);
         }
       }
       __syncwarp();
@@ -380,7 +379,6 @@ __device__ __forceinline__ void release_task_slot2(int q, bool is_leader, Gemm2S
 __device__ void gemm2_follower_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles) {
   const int lane = ptx::lane_id();
   const uint64_t pol = ptx::policy_evict_first();
-  const uint64_t polh = ptx::policy_evict_normal();
   int stage = 0;
   uint32_t phase = 0;
   int q = 0;
@@ -406,13 +404,7 @@ __device__ void gemm2_follower_producer(const Gemm2Params& p, Gemm2Smem& s, uint
           ptx::tma_load_2d(b_addr, &p.tm_w3, &s.full[stage], n0, wrow, pol);
           ptx::tma_load_2d(b_addr + kBoxBytes, &p.tm_w3, &s.full[stage], n0 + 64, wrow, pol);
         } else {
-          const int half_boxes = p.BN2 / 128;
-          ptx::mbar_arrive_expect_tx(&s.full[stage], p.BM * 128 + half_boxes * kBoxBytes);
-          ptx::tma_load_2d(a_addr, &p.tm_h, &s.full[stage], kb * kBK, ((task.p % p.ring_pairs) * 2 + 1) * p.BM, polh);
-          const int wrow = task.e * p.I + kb * kBK;
-          const int n0 = task.n * p.BN2 + p.BN2 / 2;
-          for (int j = 0; j < half_boxes; ++j)
-            ptx::tma_load_2d(b_addr + j * kBoxBytes, &p.tm_w2, &s.full[stage], n0 + j * 64, wrow, pol);
+          ptx::mbar_arrive(&s.full[stage]);   // L2: operands by the A-row warps (see the leader)
         }
       }
       __syncwarp();
@@ -588,7 +580,6 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
         else ptx::mbar_arrive_peer(lead_acc_empty0 + 8 * acc);
       }
       __threadfence();
-      ptx::fence_proxy_async_global();
       __syncwarp();
       if (lane == 0 && task.p != p.withhold_pair) ptx::red_release_gpu_add(p.l1_done + task.p, 1);
     } else {
@@ -611,26 +602,7 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
           }
         }
       }
-      float* yrow = p.y_acc + (size_t)(tok < 0 ? 0 : tok) * p.H + task.n * p.BN2;
-      float* srow = &s.out_stage[quarter][lane][0];
-      const uint32_t srow_addr = ptx::smem_u32(srow);
-#pragma unroll 1
-      for (int c = 0; c < p.BN2 / 32; ++c) {
-        uint32_t v[32];
-        ptx::tmem_ld32(tbase + c * 32, v);
-        ptx::tmem_ld_wait();
-        if (tok >= 0) {
-          ptx::bulk_wait_read_all();
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            reinterpret_cast<float4*>(srow)[i] =
-                make_float4(w * __uint_as_float(v[4 * i + 0]), w * __uint_as_float(v[4 * i + 1]),
-                            w * __uint_as_float(v[4 * i + 2]), w * __uint_as_float(v[4 * i + 3]));
-          ptx::fence_proxy_async_shared();
-          ptx::bulk_reduce_add_f32(yrow + c * 32, srow_addr, 128);
-          ptx::bulk_commit();
-        }
-      }
+      combine_rows(tbase, p.BN2, w, tok, p.y_acc, p.H, task.n * p.BN2, s.out_stage[quarter], s.out_tok[quarter]);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -643,12 +615,12 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
       acc_phase ^= 1;
     }
   }
-  ptx::bulk_wait_all();
 }
 
 // ---------------------------------------------------------------- gather warps (warps 6.. of both CTAs)
 __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, int g, uint32_t rank) {
   constexpr int kRowsPerLane = (kTileM / 4 + kGatherWarps - 1) / kGatherWarps;
+  const uint64_t wpol = ptx::policy_evict_first();
   const int lane = ptx::lane_id();
   const int c = lane & 7;
   const bool is_leader = rank == 0;
@@ -665,20 +637,26 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
     int nrows = 0;
     uint32_t soff[kRowsPerLane];
     const bf16* src[kRowsPerLane];
-    if (task.phase == 0 && b_own >= 0) {
+    if (b_own >= 0) {
+      // L1: the routed x rows of this CTA's block; L2: its h rows in the ring
       const int* rows = s.rows[q_task];
+      const bf16* hblock = p.h + (size_t)((task.p % p.ring_pairs) * 2 + (int)rank) * p.BM * p.I;
 #pragma unroll
       for (int j = 0; j < kRowsPerLane; ++j) {
         const int rr = (j * kGatherWarps + g) * 4 + (lane >> 3);
         soff[j] = rr * 128 + ((c ^ (rr & 7)) << 4);
         src[j] = p.x + c * 8;
         if (rr < p.BM) {
-          src[j] = p.x + (size_t)rows[rr] * p.H + c * 8;
+          src[j] = task.phase == 0 ? p.x + (size_t)rows[rr] * p.H + c * 8 : hblock + (size_t)rr * p.I + c * 8;
           nrows = j + 1;
         }
       }
     }
     release_task_slot2(q_task, is_leader, s);   // rows read: the slot may be refilled
+    // L2: this CTA's half of the W2 tile too (BN2/2 columns: one or two 64x64
+    // boxes, each 64 K-rows of 128 bytes in the same 128-byte swizzle as TMA)
+    const int nhalf = task.phase == 1 ? p.BN2 / 128 : 0;
+    const bf16* w2src = p.w2 + (size_t)task.e * p.I * p.H + task.n * p.BN2 + (int)rank * (p.BN2 / 2) + c * 8;
     const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
@@ -686,16 +664,19 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
         ok = false;
         break;
       }
-      if (task.phase == 0) {
-        const uint32_t a_addr = ptx::smem_u32(stage2_ptr(tiles, stage));
+      const uint32_t a_addr = ptx::smem_u32(stage2_ptr(tiles, stage));
 #pragma unroll
-        for (int j = 0; j < kRowsPerLane; ++j)
-          if (j < nrows) ptx::cp_async_16(a_addr + soff[j], src[j] + kb * kBK);
-        ptx::cp_async_mbar_arrive_noinc(&s.full[stage]);
-      } else {
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive_count(&s.full[stage], 32);
+      for (int j = 0; j < kRowsPerLane; ++j)
+        if (j < nrows) ptx::cp_async_16(a_addr + soff[j], src[j] + kb * kBK);
+      for (int j = 0; j < nhalf; ++j) {
+#pragma unroll
+        for (int i = 0; i < 64 / 4 / kGatherWarps; ++i) {
+          const int kr = (i * kGatherWarps + g) * 4 + (lane >> 3);
+          ptx::cp_async_16_hint(a_addr + kTileABytes + j * kBoxBytes + kr * 128 + ((c ^ (kr & 7)) << 4),
+                                w2src + (size_t)(kb * kBK + kr) * p.H + j * 64, wpol);
+        }
       }
+      ptx::cp_async_mbar_arrive_noinc(&s.full[stage]);
       if (++stage == kStages2) {
         stage = 0;
         phase ^= 1;
@@ -739,8 +720,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_expert_gemm2_kernel(const
   if (warp == 0 && lane == 0) {
     ptx::prefetch_tmap(&p.tm_w1);
     ptx::prefetch_tmap(&p.tm_w3);
-    ptx::prefetch_tmap(&p.tm_w2);
-    ptx::prefetch_tmap(&p.tm_h);
   }
   for (int e = threadIdx.x; e <= p.E; e += kGemmThreads) {
     s.block_start[e] = p.block_start[e];

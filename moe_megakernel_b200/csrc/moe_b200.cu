@@ -304,11 +304,10 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     Gemm2Params gp;
     std::memset(&gp, 0, sizeof(gp));
     bool ok = make_map(&gp.tm_w1, W1, I, (uint64_t)E * H, I, 64) &&
-              make_map(&gp.tm_w3, W3, I, (uint64_t)E * H, I, 64) &&
-              make_map(&gp.tm_w2, W2, H, (uint64_t)E * I, H, 64) &&
-              make_map(&gp.tm_h, h, I, (uint64_t)p->ring_pairs * 2 * p->BM, I, p->BM);
+              make_map(&gp.tm_w3, W3, I, (uint64_t)E * H, I, 64);
     if (!ok) return MOE_ERR_CUDA;
     gp.x = static_cast<const bf16*>(x);
+    gp.w2 = static_cast<const bf16*>(W2);
     gp.slot_token = dp.slot_token;
     gp.slot_topk = dp.slot_topk;
     gp.topk_w = rp.topk_w;
@@ -354,8 +353,7 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     std::memset(&gp, 0, sizeof(gp));
     bool ok = make_map(&gp.tm_w1, W1, I, (uint64_t)E * H, I, 64) &&
               make_map(&gp.tm_w3, W3, I, (uint64_t)E * H, I, 64) &&
-              make_map(&gp.tm_w2, W2, H, (uint64_t)E * I, H, 64) &&
-              make_map(&gp.tm_h, h, I, (uint64_t)p->ring_blocks * p->BM, I, p->BM);
+              make_map(&gp.tm_w2, W2, H, (uint64_t)E * I, H, 64);
     if (!ok) return MOE_ERR_CUDA;
     gp.x = static_cast<const bf16*>(x);
     gp.slot_token = dp.slot_token;
@@ -383,7 +381,7 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     gp.N2 = p->N2;
     gp.timeout_ns = p->timeout_ns;
     gp.withhold_block = p->withhold;
-    moe_expert_gemm_kernel<<<p->num_sms, kGemmThreads, kGemmSmemBytes, st>>>(gp);
+    moe_expert_gemm_kernel<<<p->num_sms, kGemm1Threads, kGemmSmemBytes, st>>>(gp);
   }
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   mark(4);
@@ -635,6 +633,9 @@ int moe_plan_create(moe_plan_t* out, int T_max, int H, int I, int E, int k, int 
     p->pair_clusters = clusters;
     size_pair_groups(p);   // with the real number of concurrent pair tasks
     p->L = make_layout(*p);
+    // Full 128-row blocks run on CTA pairs (half the weight-tile traffic per
+    // SM); smaller blocks keep the single-CTA kernel.
+    p->cta_pairs = p->BM == 128 && clusters > 0;
   }
   *out = p;
   return MOE_OK;
@@ -667,6 +668,7 @@ int moe_plan_describe(moe_plan_t p, moe_plan_desc* d) {
   d->pool_capacity = p->pool;
   d->num_sms = p->num_sms;
   d->pair_clusters = p->pair_clusters;
+  d->cta_pairs = p->cta_pairs ? 1 : 0;
   d->workspace_bytes = p->L.total;
   return MOE_OK;
 }

@@ -92,6 +92,11 @@ __device__ __forceinline__ uint64_t policy_evict_normal() {
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
+// The same with an L2 eviction-priority hint.
+__device__ __forceinline__ void cp_async_16_hint(uint32_t dst, const void* src, uint64_t policy) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "l"(policy)
+               : "memory");
+}
 // Arrive on `bar` once this thread's cp.async copies have landed, counted
 // against the barrier's expected arrivals (no pending-count increment).
 __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
@@ -183,6 +188,12 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
 }
 __device__ __forceinline__ void red_release_gpu_add(int* p, int v) {
   asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Fire-and-forget fp32 vector reduction: p[0..3] += v (16-byte aligned).
+__device__ __forceinline__ void red_add_v4_f32(float* p, float4 v) {
+  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05

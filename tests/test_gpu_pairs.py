@@ -1,10 +1,12 @@
-"""Parity of the CTA-pair expert GEMM (tcgen05 cta_group::2) with the oracle.
+"""Parity of both expert-GEMM kernels with the oracle, each forced on.
 
-Same checks as test_gpu_parity / test_gpu_workloads, with the plan switched
-to CTA pairs: two consecutive blocks of an expert per task, each CTA of a
-cluster holding its own block's rows and half of the weight tile. Shapes
-include experts with an odd block count (the second CTA of the last pair has
-no block), BLOCK_M below 128, H % 256 != 0 and a ring that wraps.
+The plan runs 128-row blocks on CTA pairs (tcgen05 cta_group::2: two
+consecutive blocks of an expert per task, each CTA of a cluster holding its
+own block's rows and half of the weight tile) and smaller blocks on the
+single-CTA kernel. Here every shape runs on both, and the full workloads on
+the kernel the plan would not pick. Shapes include experts with an odd block
+count (the second CTA of the last pair has no block), BLOCK_M below 128,
+H % 256 != 0 and a ring that wraps.
 """
 import numpy as np
 import pytest
@@ -29,18 +31,20 @@ PAIR_SHAPES = [
 ]
 
 
-def _plan(shape, block_m=0):
+def _plan(shape, block_m=0, pairs=True):
     from moe_megakernel_b200 import MoEPlan
     plan = MoEPlan(shape.T, shape.H, shape.I, shape.E, shape.k, block_m=block_m)
-    plan.set_cta_pairs(True)
+    plan.set_cta_pairs(pairs)
     return plan
 
 
+@pytest.mark.parametrize("pairs", [True, False], ids=["pairs", "single"])
 @pytest.mark.parametrize("T,H,I,E,k,bm,zipf", PAIR_SHAPES)
-def test_pairs_forward_matches_oracle(T, H, I, E, k, bm, zipf):
+def test_pairs_forward_matches_oracle(T, H, I, E, k, bm, zipf, pairs):
+    """Both expert-GEMM kernels on every shape, whichever the plan would pick."""
     shape = custom_shape(T, H, I, E, k, zipf)
     inp = make_inputs(shape, device=DEV)
-    plan = _plan(shape, bm)
+    plan = _plan(shape, bm, pairs)
     plan.workspace.fill_(0xFF)   # poison: unwritten reads show up as NaN
     plan.lib.moe_plan_bind_workspace(plan._plan, plan.workspace.data_ptr(), plan.workspace_bytes)
     y = plan.forward(inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"])
@@ -49,7 +53,7 @@ def test_pairs_forward_matches_oracle(T, H, I, E, k, bm, zipf):
     ref = oracle_forward(inp, tokens=rows, block_m=plan.block_m)
     assert_routing_equal(plan.routing(T), ref)
     fro, mx = assert_y_close(y[torch.from_numpy(rows).to(y.device)], ref["y"])
-    print(f"pairs T={T} H={H} I={I} E={E} k={k}: rel_fro={fro:.2e} max_abs={mx:.2e}")
+    print(f"{'pairs' if pairs else 'single'} T={T} H={H} I={I} E={E} k={k}: rel_fro={fro:.2e} max_abs={mx:.2e}")
 
 
 def test_pairs_and_single_agree_and_repeat():
@@ -86,13 +90,15 @@ def test_pairs_bounded_wait_reports_timeout():
 @pytest.mark.slow
 @pytest.mark.parametrize("name", ["mixtral", "fine_grained_prefill", "decode", "skewed"])
 def test_pairs_workload_matches_oracle(name):
+    """The full workloads on the kernel the plan does NOT pick by default."""
     shape = WORKLOADS[name]
     inp = make_inputs(shape, device=DEV)
     plan = _plan(shape)
+    plan.set_cta_pairs(plan.block_m != 128)
     y = plan.forward(inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"])
     plan.check()
     rows = sample_tokens(shape.T, {"mixtral": 32, "fine_grained_prefill": 12, "decode": 32, "skewed": 96}[name])
     ref = oracle_forward(inp, tokens=rows, block_m=plan.block_m)
     assert_routing_equal(plan.routing(shape.T), ref)
     fro, mx = assert_y_close(y[torch.from_numpy(rows).to(y.device)], ref["y"])
-    print(f"pairs {name}: rel_fro={fro:.2e} max_abs={mx:.2e}")
+    print(f"{'pairs' if plan.block_m != 128 else 'single'} {name}: rel_fro={fro:.2e} max_abs={mx:.2e}")

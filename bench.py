@@ -95,51 +95,76 @@ def workload_label(s):
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    """SM clock, power and throttle reasons polled through NVML every 2 ms in a
+    thread (read-only queries); stats cover the samples taken between
+    begin() and end(), i.e. during the timed steps. Falls back to one
+    nvidia-smi query per sample if NVML cannot be loaded."""
+
+    REASON_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+                   "sw_power_cap": 0x4}
 
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
-        self.proc = None
-        self.lines = []
+        self.samples = []          # (t, sm_mhz, power_w, reasons_mask)
+        self.t0 = self.t1 = None
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._nvml = None
+
+    def _poll_nvml(self, nv, h):
+        while not self._stop.is_set():
+            try:
+                self.samples.append((time.perf_counter(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                     nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+            except Exception:
+                return
+            time.sleep(0.002)
+
+    def _poll_smi(self):
+        q = "clocks.sm,power.draw,clocks_event_reasons.active"
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={q}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip().split(",")
+                self.samples.append((time.perf_counter(), float(out[0]), float(out[1]), int(out[2].strip(), 16)))
+            except Exception:
+                return
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            threading.Thread(target=self._read, daemon=True).start()
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByIndex(self.idx)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self._nvml = nv
+            self._thread = threading.Thread(target=self._poll_nvml, args=(nv, h), daemon=True)
+        except Exception:
+            self._thread = threading.Thread(target=self._poll_smi, daemon=True)
+        self._thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def begin(self):
+        self.t0 = time.perf_counter()
+
+    def end(self):
+        self.t1 = time.perf_counter()
 
     def stop(self):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-        rows = []
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) != 8:
-                continue
-            try:
-                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
-            except ValueError:
-                continue
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=10)
+        rows = [r for r in self.samples if self.t0 is not None and self.t1 is not None and self.t0 <= r[0] <= self.t1]
+        if not rows and self.samples and self.t1 is not None:
+            rows = [min(self.samples, key=lambda r: abs(r[0] - self.t1))]
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        loaded = [r for r in rows if r[3] >= 50] or rows
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[4]) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(loaded), "power_w_max": max(r[2] for r in rows)}
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"], "samples": 0}
+        reasons = sorted({n for r in rows for n, b in self.REASON_BITS.items() if r[3] & b})
+        return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_min_mhz": min(r[1] for r in rows),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(r[2] for r in rows),
+                "source": "nvml" if self._nvml is not None else "nvidia-smi"}
 
 
 # ------------------------------------------------------------------ oracle timing
@@ -212,13 +237,14 @@ def run_gpu(args, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize(dev)
     clocks.start()
-    time.sleep(0.3)
+    clocks.begin()
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record(stream)
         plan.forward(*args_fwd, y=y)
         ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
+    clocks.end()
     barrier()
     clk = clocks.stop()
     plan.check()

@@ -37,8 +37,8 @@ constexpr int kTaskRing = 4;
 #define MOE_GATHER_WARPS 4
 #endif
 constexpr int kGatherWarps = MOE_GATHER_WARPS;     // warps that gather routed x rows
-constexpr int kGemmThreads = 192 + 32 * kGatherWarps;   // producer, MMA, 4 epilogue warps, gather warps
-constexpr int kGemm1Threads = kGemmThreads + 32;        // the same plus a scheduler warp (single-CTA kernel)
+// expert-GEMM CTA: producer, MMA (or relay), 4 epilogue warps, A-row warps, scheduler
+constexpr int kGemm1Threads = 224 + 32 * kGatherWarps;
 constexpr int kTmemCols = 512;                     // two 256-column fp32 accumulators
 constexpr int kMaxGroups = 512;                    // block groups of the expert GEMM's task order
 

@@ -509,13 +509,34 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 }
 
 // Combine of one epilogue warp's 32 accumulator rows (TMEM lanes tbase..+31,
-// columns 0..ncols-1): y_acc[tok_r][c] += w_r * acc[r][c] for every row r with
-// tok_r >= 0. Each lane holds row `lane`; per 32 columns the warp stages w*acc
-// in shared memory (rows padded to 36 floats, conflict-free both ways) and
-// reads it back transposed, so that 8 lanes cover one row's 128 contiguous
-// bytes and every red.v4 instruction adds 4 whole 128-byte row segments.
+// columns 0..ncols-1, ncols a multiple of 64): y_acc[tok_r][c] += w_r *
+// acc[r][c] for every row r with tok_r >= 0. Each lane holds row `lane`; per
+// 32 columns the warp stages w*acc in shared memory (rows padded to 36 floats,
+// conflict-free both ways) and reads it back transposed, so that 8 lanes
+// cover one row's 128 contiguous bytes and every red.v4 instruction adds 4
+// whole 128-byte row segments. The TMEM load of the next 32 columns is in
+// flight while the current ones are staged and reduced, and `release()` runs
+// as soon as the last TMEM load has landed, so the MMA warp can reuse the
+// accumulator while the last reductions are still being issued.
+__device__ __forceinline__ void combine_stage_and_reduce(const uint32_t (&v)[32], int c, float w, float* srow,
+                                                         float (*stage)[36], float* const (&ybase)[8], int sub,
+                                                         int cc) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    reinterpret_cast<float4*>(srow)[i] =
+        make_float4(w * __uint_as_float(v[4 * i + 0]), w * __uint_as_float(v[4 * i + 1]),
+                    w * __uint_as_float(v[4 * i + 2]), w * __uint_as_float(v[4 * i + 3]));
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (ybase[i] != nullptr)
+      ptx::red_add_v4_f32(ybase[i] + c * 32, *reinterpret_cast<const float4*>(&stage[i * 4 + sub][cc]));
+  __syncwarp();
+}
+
+template <typename Release>
 __device__ __forceinline__ void combine_rows(uint32_t tbase, int ncols, float w, int tok, float* y_acc, int H,
-                                             int col0, float (*stage)[36], int* stage_tok) {
+                                             int col0, float (*stage)[36], int* stage_tok, Release release) {
   const int lane = ptx::lane_id();
   stage_tok[lane] = tok;
   __syncwarp();
@@ -528,22 +549,17 @@ __device__ __forceinline__ void combine_rows(uint32_t tbase, int ncols, float w,
     ybase[i] = t >= 0 ? y_acc + (size_t)t * H + col0 + cc : nullptr;
   }
   float* srow = stage[lane];
+  uint32_t va[32], vb[32];
+  ptx::tmem_ld32(tbase, va);
 #pragma unroll 1
-  for (int c = 0; c < ncols / 32; ++c) {
-    uint32_t v[32];
-    ptx::tmem_ld32(tbase + c * 32, v);
-    ptx::tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      reinterpret_cast<float4*>(srow)[i] =
-          make_float4(w * __uint_as_float(v[4 * i + 0]), w * __uint_as_float(v[4 * i + 1]),
-                      w * __uint_as_float(v[4 * i + 2]), w * __uint_as_float(v[4 * i + 3]));
-    __syncwarp();
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (ybase[i] != nullptr)
-        ptx::red_add_v4_f32(ybase[i] + c * 32, *reinterpret_cast<const float4*>(&stage[i * 4 + sub][cc]));
-    __syncwarp();
+  for (int c = 0; c < ncols / 32; c += 2) {
+    ptx::tmem_ld_wait();                                         // va holds columns 32c ..
+    ptx::tmem_ld32(tbase + (c + 1) * 32, vb);
+    combine_stage_and_reduce(va, c, w, srow, stage, ybase, sub, cc);
+    ptx::tmem_ld_wait();                                         // vb holds columns 32(c+1) ..
+    if (c + 2 < ncols / 32) ptx::tmem_ld32(tbase + (c + 2) * 32, va);
+    else release();                                              // no TMEM reads left
+    combine_stage_and_reduce(vb, c + 1, w, srow, stage, ybase, sub, cc);
   }
 }
 
@@ -638,10 +654,12 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
         }
       }
       // Combine: y_acc[token] += w * o, 128-byte row segments per red.v4 (the L2 does the fp32 adds).
-      combine_rows(tbase, p.BN2, w, tok, p.y_acc, p.H, task.n * p.BN2, s.out_stage[quarter], s.out_tok[quarter]);
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&s.acc_empty[acc]);
+      combine_rows(tbase, p.BN2, w, tok, p.y_acc, p.H, task.n * p.BN2, s.out_stage[quarter], s.out_tok[quarter],
+                   [&]() {
+                     ptx::tc_fence_before();
+                     __syncwarp();
+                     if (lane == 0) ptx::mbar_arrive(&s.acc_empty[acc]);
+                   });
     }
     if (++acc == 2) {
       acc = 0;

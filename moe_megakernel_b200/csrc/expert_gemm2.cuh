@@ -8,9 +8,10 @@
 //   (L1: CTA 0 the 128 W1 columns, CTA 1 the matching 128 W3 columns; L2:
 //   each CTA 128 of the 256 W2 columns), so one weight tile load feeds 256
 //   rows and a stage is 32 KB per CTA instead of 48 KB (6 stages fit);
-// * the leader CTA (rank 0) claims tasks, issues the MMAs for both CTAs and
-//   multicasts its commits to both CTAs' barriers; each CTA's accumulator is
-//   its own 128 rows x 256 columns in its own TMEM;
+// * the leader CTA (rank 0) claims and prepares tasks in its scheduler warp,
+//   publishes them in both CTAs' task rings, issues the MMAs for both CTAs
+//   and multicasts its commits to both CTAs' barriers; each CTA's
+//   accumulator is its own 128 rows x 256 columns in its own TMEM;
 // * L1 weight halves come by TMA; in L2 the A-row warps load both the h
 //   rows and the CTA's W2 half with cp.async (with a 64x64 TMA box of W2
 //   the L2 tasks ran at about half the tensor-pipe rate, with cp.async at
@@ -84,6 +85,7 @@ struct Gemm2Smem {
   Task2 tasks[kTaskRing];
   uint32_t tmem_base;
   int abort;
+  int taken;   // tasks the leader's producer has taken from the ring
   int num_groups;
   int rows[kTaskRing][kTileM];
   int block_start[257];
@@ -217,34 +219,48 @@ __device__ __forceinline__ Task2 decode_task2(int t, const Gemm2Smem& s, const G
 
 __device__ __forceinline__ uint8_t* stage2_ptr(uint8_t* tiles, int stage) { return tiles + stage * kStage2Bytes; }
 
-// ---------------------------------------------------------------- leader warp 0: scheduler + TMA
-__device__ __forceinline__ Task2 prepare_task2(int t, int q, uint32_t qparity, bool& deps_ready, bool& ok,
-                                               const Gemm2Params& p, Gemm2Smem& s, int lane) {
-  Task2 task = decode_task2(t, s, p);
-  deps_ready = true;
-  ok = warp_wait2(&s.task_empty[q], qparity, p, s, 1);
-  if (!ok) return task;
+// ---------------------------------------------------------------- leader scheduler (last warp)
+// Claims tasks, decodes them, stages the token rows of both CTAs' A tiles
+// (L1) or waits for the L1 tiles of the pair (L2), and publishes each task in
+// both CTAs' rings; as in expert_gemm.cuh it runs one task ahead of the
+// leader's producer and never further.
+__device__ __forceinline__ bool prepare_task2(Task2& task, int q, uint32_t qparity, const Gemm2Params& p,
+                                              Gemm2Smem& s, int lane) {
+  if (!warp_wait2(&s.task_empty[q], qparity, p, s, 1)) return false;
   if (task.phase == 0) {
     // token rows of both CTAs' A tiles: CTA 0 locally, CTA 1 through the cluster window
+    // (all loads first, one round trip)
+    constexpr int kPer = kTileM / 32;
+    int tok0[kPer], tok1[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int r = lane + 32 * i;
+      tok0[i] = r < p.BM ? p.slot_token[task.b0 * p.BM + r] : 0;
+      tok1[i] = r < p.BM && task.b1 >= 0 ? p.slot_token[task.b1 * p.BM + r] : 0;
+    }
     const uint32_t peer_rows = ptx::mapa(ptx::smem_u32(&s.rows[q][0]), 1);
-    for (int r = lane; r < p.BM; r += 32) {
-      int tok0 = p.slot_token[task.b0 * p.BM + r];
-      int tok1 = task.b1 >= 0 ? p.slot_token[task.b1 * p.BM + r] : 0;
-      if (tok0 >= p.T || tok1 >= p.T) {
-        set_error2(p, s, kDevBounds, task.p);
-        tok0 = tok0 >= p.T ? 0 : tok0;
-        tok1 = tok1 >= p.T ? 0 : tok1;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int r = lane + 32 * i;
+      if (r < p.BM) {
+        if (tok0[i] >= p.T || tok1[i] >= p.T) {
+          set_error2(p, s, kDevBounds, task.p);
+          tok0[i] = tok0[i] >= p.T ? 0 : tok0[i];
+          tok1[i] = tok1[i] >= p.T ? 0 : tok1[i];
+        }
+        s.rows[q][r] = tok0[i] < 0 ? 0 : tok0[i];   // padding slot: any valid row, the epilogue drops it
+        ptx::st_cluster_u32(peer_rows + 4 * r, tok1[i] < 0 ? 0 : tok1[i]);
       }
-      s.rows[q][r] = tok0 < 0 ? 0 : tok0;   // padding slot: any valid row, the epilogue drops it
-      ptx::st_cluster_u32(peer_rows + 4 * r, tok1 < 0 ? 0 : tok1);
     }
   } else if (task.phase == 1) {
-    int ready = 1;
-    if (lane == 0) ready = ptx::ld_acquire_gpu(p.l1_done + task.p) >= 8 * p.N1;
-    deps_ready = __shfl_sync(0xffffffffu, ready, 0) != 0;
+    // the L2 task of pair p reads h rows written by all L1 n-tiles of the pair
+    // (one arrival per epilogue warp of both CTAs per n-tile)
+    bool fine = true;
+    if (lane == 0) fine = wait_counter2(p.l1_done + task.p, 8 * p.N1, p, s, 0x10000 | task.p);
+    if (__shfl_sync(0xffffffffu, fine ? 1 : 0, 0) == 0) task.phase = -1;
   }
   __syncwarp();
-  return task;
+  return true;
 }
 
 __device__ __forceinline__ void push_task2(const Task2& task, int q, Gemm2Smem& s, int lane) {
@@ -264,6 +280,47 @@ __device__ __forceinline__ void push_task2(const Task2& task, int q, Gemm2Smem& 
   __syncwarp();
 }
 
+// Bounded wait (one thread) until the leader's producer has taken `n` tasks.
+__device__ __forceinline__ bool wait_taken2(int n, const Gemm2Params& p, Gemm2Smem& s) {
+  if (*reinterpret_cast<volatile int*>(&s.taken) >= n) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  while (*reinterpret_cast<volatile int*>(&s.taken) < n) {
+    if (*reinterpret_cast<volatile int*>(&s.abort)) return false;
+    if (ptx::globaltimer() - t0 > p.timeout_ns) {
+      set_error2(p, s, kDevTimeout, 0x10a);
+      return false;
+    }
+    __nanosleep(64);
+  }
+  return true;
+}
+
+__device__ void gemm2_scheduler(const Gemm2Params& p, Gemm2Smem& s) {
+  const int lane = ptx::lane_id();
+  int q = 0;
+  uint32_t qphase = 0;
+  int pushed = 0;
+  while (true) {
+    bool ok = true;
+    if (lane == 0) ok = wait_taken2(pushed, p, s);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    Task2 task{-1, 0, 0, 0, -1, -1, 0, 0};
+    if (ok) {
+      const int t = __shfl_sync(0xffffffffu, claim_task_any(p.task_counter, p.err, &s.abort, lane), 0);
+      task = decode_task2(t, s, p);
+    }
+    if (!prepare_task2(task, q, qphase ^ 1, p, s, lane)) break;
+    push_task2(task, q, s, lane);
+    ++pushed;
+    if (++q == kTaskRing) {
+      q = 0;
+      qphase ^= 1;
+    }
+    if (task.phase < 0) break;
+  }
+}
+
+// ---------------------------------------------------------------- leader warp 0: TMA
 __device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles) {
   const int lane = ptx::lane_id();
   const uint64_t pol = ptx::policy_evict_first();
@@ -272,25 +329,21 @@ __device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_
   int q = 0;
   uint32_t qphase = 0;
   uint32_t issued = 0, issued_parity = 0;
-  bool deps_ready = true, ok = true;
-  int t = __shfl_sync(0xffffffffu, claim_task_any(p.task_counter, p.err, &s.abort, lane), 0);
-  Task2 task = prepare_task2(t, q, qphase ^ 1, deps_ready, ok, p, s, lane);
+  bool ok = true;
   while (ok) {
-    if (task.phase == 1 && !deps_ready) {
-      bool fine = true;
-      if (lane == 0) fine = wait_counter2(p.l1_done + task.p, 8 * p.N1, p, s, 0x10000 | task.p);
-      if (__shfl_sync(0xffffffffu, fine ? 1 : 0, 0) == 0) task.phase = -1;
+    if (!warp_wait2(&s.task_full[q], qphase, p, s, 14)) break;
+    const Task2 task = s.tasks[q];
+    __syncwarp();
+    if (lane == 0) {
+      ptx::mbar_arrive(&s.task_empty[q]);
+      *reinterpret_cast<volatile int*>(&s.taken) = *reinterpret_cast<volatile int*>(&s.taken) + 1;
     }
-    push_task2(task, q, s, lane);
-    const int qn = (q + 1) % kTaskRing;
-    const uint32_t qphase_n = qn == 0 ? qphase ^ 1 : qphase;
+    if (++q == kTaskRing) {
+      q = 0;
+      qphase ^= 1;
+    }
     if (task.phase < 0) break;
-
-    const int t_next_lane0 = claim_task_any(p.task_counter, p.err, &s.abort, lane);
-    bool prepared = false;
-    Task2 next{-1, 0, 0, 0, -1, -1, 0, 0};
     const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
-    const int prep_at = nk > 2 ? 2 : nk - 1;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait2(&s.empty[stage], phase ^ 1, p, s, 2)) {
         ok = false;
@@ -320,21 +373,7 @@ __device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_
         stage = 0;
         phase ^= 1;
       }
-      if (kb == prep_at) {
-        const int tn = __shfl_sync(0xffffffffu, t_next_lane0, 0);
-        next = prepare_task2(tn, qn, qphase_n ^ 1, deps_ready, ok, p, s, lane);
-        prepared = true;
-        if (!ok) break;
-      }
     }
-    if (!ok) break;
-    if (!prepared) {
-      const int tn = __shfl_sync(0xffffffffu, t_next_lane0, 0);
-      next = prepare_task2(tn, qn, qphase_n ^ 1, deps_ready, ok, p, s, lane);
-    }
-    task = next;
-    q = qn;
-    qphase = qphase_n;
   }
   for (int st = 0; st < kStages2; ++st)
     if (issued & (1u << st)) {
@@ -602,13 +641,15 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
           }
         }
       }
-      combine_rows(tbase, p.BN2, w, tok, p.y_acc, p.H, task.n * p.BN2, s.out_stage[quarter], s.out_tok[quarter]);
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (is_leader) ptx::mbar_arrive(&s.acc_empty[acc]);
-        else ptx::mbar_arrive_peer(lead_acc_empty0 + 8 * acc);
-      }
+      combine_rows(tbase, p.BN2, w, tok, p.y_acc, p.H, task.n * p.BN2, s.out_stage[quarter], s.out_tok[quarter],
+                   [&]() {
+                     ptx::tc_fence_before();
+                     __syncwarp();
+                     if (lane == 0) {
+                       if (is_leader) ptx::mbar_arrive(&s.acc_empty[acc]);
+                       else ptx::mbar_arrive_peer(lead_acc_empty0 + 8 * acc);
+                     }
+                   });
     }
     if (++acc == 2) {
       acc = 0;
@@ -687,7 +728,7 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
   ptx::cp_async_wait_all();
 }
 
-__global__ void __launch_bounds__(kGemmThreads, 1) moe_expert_gemm2_kernel(const __grid_constant__ Gemm2Params p) {
+__global__ void __launch_bounds__(kGemm1Threads, 1) moe_expert_gemm2_kernel(const __grid_constant__ Gemm2Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Gemm2Smem& s = *reinterpret_cast<Gemm2Smem*>(tiles + (size_t)kStages2 * kStage2Bytes);
@@ -709,26 +750,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_expert_gemm2_kernel(const
     }
     for (int i = 0; i < kTaskRing; ++i) {
       ptx::mbar_init(&s.task_full[i], 1);
-      // in the leader: its MMA + 4 epilogue + gather warps, and the follower's producer,
-      // relay, 4 epilogue and gather warps
-      ptx::mbar_init(&s.task_empty[i], (1 + 4 + kGatherWarps) + (2 + 4 + kGatherWarps));
+      // in the leader: its producer, MMA, 4 epilogue and gather warps, and the
+      // follower's producer, relay, 4 epilogue and gather warps
+      ptx::mbar_init(&s.task_empty[i], (2 + 4 + kGatherWarps) + (2 + 4 + kGatherWarps));
     }
     ptx::mbar_init(&s.mma_done, 1);
     s.abort = 0;
+    s.taken = 0;
     ptx::fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     ptx::prefetch_tmap(&p.tm_w1);
     ptx::prefetch_tmap(&p.tm_w3);
   }
-  for (int e = threadIdx.x; e <= p.E; e += kGemmThreads) {
+  for (int e = threadIdx.x; e <= p.E; e += kGemm1Threads) {
     s.block_start[e] = p.block_start[e];
     s.pair_start[e] = p.pair_start[e];
   }
   {
     const int ng = min(*p.num_groups, min(p.max_groups, kMaxGroups));
     if (threadIdx.x == 0) s.num_groups = ng;
-    for (int g = threadIdx.x; g <= ng; g += kGemmThreads) s.group_start[g] = p.group_start[g];
+    for (int g = threadIdx.x; g <= ng; g += kGemm1Threads) s.group_start[g] = p.group_start[g];
   }
   if (warp == 1) {
     ptx::tmem_alloc_pair(&s.tmem_base, kTmemCols);
@@ -738,7 +780,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_expert_gemm2_kernel(const
     for (int st = 0; st < kStages2; ++st) {
       uint4* a = reinterpret_cast<uint4*>(stage2_ptr(tiles, st) + p.BM * 128);
       const int n = (kTileM - p.BM) * 128 / 16;
-      for (int i = threadIdx.x; i < n; i += kGemmThreads) a[i] = make_uint4(0, 0, 0, 0);
+      for (int i = threadIdx.x; i < n; i += kGemm1Threads) a[i] = make_uint4(0, 0, 0, 0);
     }
     ptx::fence_proxy_async_shared();
   }
@@ -756,8 +798,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) moe_expert_gemm2_kernel(const
     else gemm2_follower_relay(p, s);
   } else if (warp < 6) {
     gemm2_epilogue(p, s, tmem_base, rank);
-  } else {
+  } else if (warp < 6 + kGatherWarps) {
     gemm2_gather(p, s, tiles, warp - 6, rank);
+  } else if (is_leader) {
+    gemm2_scheduler(p, s);
   }
 
   ptx::tc_fence_before();

@@ -337,7 +337,7 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3((unsigned)(2 * p->pair_clusters));
-    cfg.blockDim = dim3(kGemmThreads);
+    cfg.blockDim = dim3(kGemm1Threads);
     cfg.dynamicSmemBytes = kGemm2SmemBytes;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -616,7 +616,7 @@ int moe_plan_create(moe_plan_t* out, int T_max, int H, int I, int E, int k, int 
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3((unsigned)(p->num_sms & ~1));
-    cfg.blockDim = dim3(kGemmThreads);
+    cfg.blockDim = dim3(kGemm1Threads);
     cfg.dynamicSmemBytes = kGemm2SmemBytes;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;

@@ -36,6 +36,12 @@ Readings where the pages are silent (each is also listed in the design notes):
 * BLOCK_M rule for one GPU: with n = T*k/E expected tokens per expert,
   BLOCK_M = 16 if n <= 16, 32 if n <= 32, 64 if n <= 64, else 128.
 * Padding slots of the per-expert blocks hold the record (-1, -1).
+* Shared experts ("MegaMoE 在 MoE 系统谱系中的位置", section 2.7: the shared
+  experts' two GEMM phases run in the same task queue as the routed ones):
+  each of the S shared experts is the same SwiGLU FFN (same H and I, same
+  bf16 rounding of the activation) applied to every token with weight 1 and
+  added to the routed combine: y[t] += sum_s FFN_shared_s(x[t]). Routing and
+  dispatch do not see them.
 
 Everything is fp64 on inputs given as fp64 arrays holding bf16 values.
 """
@@ -200,13 +206,16 @@ def stacked_expert_weights(W1, W3, W2) -> Callable[[int], tuple]:
 
 
 def moe_forward(x, Wg, bias, expert_weights: Callable[[int], tuple], k: int,
-                block_m: Optional[int] = None, tokens: Optional[Sequence[int]] = None) -> dict:
+                block_m: Optional[int] = None, tokens: Optional[Sequence[int]] = None,
+                shared_weights: Optional[Callable[[int], tuple]] = None, n_shared: int = 0) -> dict:
     """The whole layer: gate, dispatch, expert FFN, gate-weighted combine.
 
     x [T,H] fp64; Wg [H,E] fp64; bias [E] or None; ``expert_weights(e)``
     returns (W1[e], W3[e], W2[e]) as fp64. If ``tokens`` is given, y is
     computed only for those token rows (routing and dispatch always cover all
-    T tokens). y[t] = sum_j w[t,j] * FFN_{idx[t,j]}(x[t]).
+    T tokens). y[t] = sum_j w[t,j] * FFN_{idx[t,j]}(x[t])
+                      + sum_{s < n_shared} FFN_shared_s(x[t]),
+    with ``shared_weights(s)`` returning the shared expert's (W1, W3, W2).
     """
     x = np.asarray(x, np.float64)
     T, H = x.shape
@@ -225,4 +234,15 @@ def moe_forward(x, Wg, bias, expert_weights: Callable[[int], tuple], k: int,
         o = expert_ffn(x[rows[hit[0]]], W1e, W3e, W2e)
         wt = w[rows[hit[0]], hit[1]]
         np.add.at(y, hit[0], wt[:, None] * o)
+    if n_shared:
+        y += shared_ffn_sum(x[rows], shared_weights, n_shared)
     return dict(topk_idx=idx, topk_w=w, logits=logits, y=y, tokens=rows, **disp)
+
+
+def shared_ffn_sum(xr: np.ndarray, shared_weights: Callable[[int], tuple], n_shared: int) -> np.ndarray:
+    """sum over the n_shared shared experts of FFN_shared_s(xr), each with weight 1."""
+    out = np.zeros((xr.shape[0], xr.shape[1]), dtype=np.float64)
+    for sh in range(n_shared):
+        W1s, W3s, W2s = shared_weights(sh)
+        out += expert_ffn(xr, W1s, W3s, W2s)
+    return out

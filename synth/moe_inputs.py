@@ -39,6 +39,7 @@ GAP_MIN = 1e-2          # minimum gap between the k-th and (k+1)-th gate logit
 MAX_REDRAWS = 64        # redraw rounds before giving up
 
 _STREAM_X, _STREAM_WG, _STREAM_W1, _STREAM_W3, _STREAM_W2 = 1, 2, 3, 4, 5
+_STREAM_WS1, _STREAM_WS3, _STREAM_WS2 = 6, 7, 8   # shared experts
 _STREAM_REDRAW = 100    # + attempt number
 
 
@@ -147,14 +148,37 @@ def make_expert_weights(shape: MoEShape, device="cpu", seed: int = 0):
     return W1, W3, W2
 
 
-def make_inputs(shape, device="cpu", seed: int = 0, T: Optional[int] = None):
-    """All inputs of one workload as a dict of tensors on ``device``."""
+def make_shared_weights(shape: MoEShape, n_shared: int, device="cpu", seed: int = 0):
+    """Shared experts Ws1, Ws3 [S,H,I] and Ws2 [S,I,H], bf16, same init as the routed experts
+    (their own generator streams)."""
+    device = torch.device(device)
+    H, I = shape.H, shape.I
+    Ws1 = torch.empty((n_shared, H, I), dtype=torch.bfloat16, device=device)
+    Ws3 = torch.empty((n_shared, H, I), dtype=torch.bfloat16, device=device)
+    Ws2 = torch.empty((n_shared, I, H), dtype=torch.bfloat16, device=device)
+    g1 = _gen(device, seed, _STREAM_WS1)
+    g3 = _gen(device, seed, _STREAM_WS3)
+    g2 = _gen(device, seed, _STREAM_WS2)
+    s_h, s_i = 1.0 / math.sqrt(H), 1.0 / math.sqrt(I)
+    for e in range(n_shared):
+        Ws1[e] = _normal_bf16((H, I), s_h, g1, device)
+        Ws3[e] = _normal_bf16((H, I), s_h, g3, device)
+        Ws2[e] = _normal_bf16((I, H), s_i, g2, device)
+    return Ws1, Ws3, Ws2
+
+
+def make_inputs(shape, device="cpu", seed: int = 0, T: Optional[int] = None, n_shared: int = 0):
+    """All inputs of one workload as a dict of tensors on ``device`` (plus
+    ``n_shared`` shared experts Ws1/Ws3/Ws2 when asked for)."""
     if isinstance(shape, str):
         shape = WORKLOADS[shape]
     x, Wg, bias, redrawn = make_router_inputs(shape, device, seed, T)
     W1, W3, W2 = make_expert_weights(shape, device, seed)
-    return dict(shape=shape, x=x, Wg=Wg, bias=bias, W1=W1, W3=W3, W2=W2,
-                k=shape.k, redrawn=redrawn)
+    out = dict(shape=shape, x=x, Wg=Wg, bias=bias, W1=W1, W3=W3, W2=W2,
+               k=shape.k, redrawn=redrawn, n_shared=n_shared)
+    if n_shared:
+        out["Ws1"], out["Ws3"], out["Ws2"] = make_shared_weights(shape, n_shared, device, seed)
+    return out
 
 
 def custom_shape(T, H, I, E, k, zipf=False, name="custom") -> MoEShape:

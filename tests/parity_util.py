@@ -39,8 +39,10 @@ def oracle_forward(inp: dict, tokens=None, block_m=None):
     x = to_f64(inp["x"])
     Wg = to_f64(inp["Wg"])
     bias = None if inp["bias"] is None else to_f64(inp["bias"])
+    S = inp.get("n_shared", 0)
+    shared = expert_loader(inp["Ws1"], inp["Ws3"], inp["Ws2"]) if S else None
     return O.moe_forward(x, Wg, bias, expert_loader(inp["W1"], inp["W3"], inp["W2"]), inp["k"],
-                         block_m=block_m, tokens=tokens)
+                         block_m=block_m, tokens=tokens, shared_weights=shared, n_shared=S)
 
 
 def oracle_route(inp: dict, block_m: int):

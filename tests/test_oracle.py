@@ -258,6 +258,55 @@ def test_token_subset_matches_full():
     np.testing.assert_allclose(sub["y"], full["y"][[3, 17, 29, 0]], rtol=1e-14, atol=1e-16)
 
 
+# ----------------------------------------------------------------- shared experts
+
+def test_shared_experts_add_dense_ffns():
+    """With the routed experts' W2 = 0 the routed combine is exactly 0, so y is
+    the sum of the shared experts' textbook dense FFNs (weight 1 each)."""
+    rng = _rng(11)
+    x, Wg, W1, W3, W2 = _tiny_layer(rng)
+    S = 2
+    Ws1 = _bf16_vals(rng, (S, x.shape[1], W1.shape[2]), 0.25)
+    Ws3 = _bf16_vals(rng, (S, x.shape[1], W1.shape[2]), 0.25)
+    Ws2 = _bf16_vals(rng, (S, W1.shape[2], x.shape[1]), 0.2)
+    r = O.moe_forward(x, Wg, None, O.stacked_expert_weights(W1, W3, 0 * W2), 2,
+                      shared_weights=O.stacked_expert_weights(Ws1, Ws3, Ws2), n_shared=S)
+    ref = sum(_torch_ffn(x, Ws1[s], Ws3[s], Ws2[s]) for s in range(S))
+    np.testing.assert_allclose(r["y"], ref, rtol=1e-12, atol=1e-14)
+    # routing and dispatch do not see the shared experts
+    r0 = O.moe_forward(x, Wg, None, O.stacked_expert_weights(W1, W3, W2), 2)
+    for key in ("topk_idx", "offset", "slot_token", "slot_topk"):
+        np.testing.assert_array_equal(r[key], r0[key])
+
+
+def test_shared_expert_equal_to_routed_doubles_y():
+    """Every token routed to expert 0 with weight 1 (bias +100, k = 1) and one
+    shared expert with expert 0's weights: y = 2 * FFN_0(x)."""
+    rng = _rng(12)
+    x, Wg, W1, W3, W2 = _tiny_layer(rng)
+    b = np.zeros(Wg.shape[1])
+    b[0] = 100.0
+    r = O.moe_forward(x, Wg, b, O.stacked_expert_weights(W1, W3, W2), 1,
+                      shared_weights=O.stacked_expert_weights(W1[:1], W3[:1], W2[:1]), n_shared=1)
+    np.testing.assert_allclose(r["y"], 2 * _torch_ffn(x, W1[0], W3[0], W2[0]), rtol=1e-12, atol=1e-14)
+
+
+def test_two_shared_experts_equal_one_of_double_width():
+    """Shared experts add up: S experts of width I equal one of width S*I
+    (W1/W3 concatenated along I, W2 along I), since the activation is rounded
+    element by element."""
+    rng = _rng(13)
+    x, Wg, W1, W3, W2 = _tiny_layer(rng)
+    H, I = x.shape[1], W1.shape[2]
+    Ws1 = _bf16_vals(rng, (2, H, I), 0.25)
+    Ws3 = _bf16_vals(rng, (2, H, I), 0.25)
+    Ws2 = _bf16_vals(rng, (2, I, H), 0.2)
+    two = O.shared_ffn_sum(x, O.stacked_expert_weights(Ws1, Ws3, Ws2), 2)
+    wide = O.expert_ffn(x, np.concatenate([Ws1[0], Ws1[1]], 1), np.concatenate([Ws3[0], Ws3[1]], 1),
+                        np.concatenate([Ws2[0], Ws2[1]], 0))
+    np.testing.assert_allclose(two, wide, rtol=1e-12, atol=1e-14)
+
+
 # ----------------------------------------------------------------- planted mistakes
 
 _MUTANTS = {
@@ -271,6 +320,8 @@ _MUTANTS = {
     "descending_order": ("top_k_select", lambda l, k: np.argsort(-l, axis=1, kind="stable")[:, :k]),
     "round_half_away": ("bf16_round", lambda a: np.ldexp(np.floor(np.ldexp(np.frexp(np.asarray(a, float))[0], 8) + 0.5),
                                                           np.frexp(np.asarray(a, float))[1] - 8)),
+    "shared_averaged": ("shared_ffn_sum", lambda xr, sw, S: sum(O.expert_ffn(xr, *sw(s)) for s in range(S)) / S),
+    "shared_first_only": ("shared_ffn_sum", lambda xr, sw, S: O.expert_ffn(xr, *sw(0))),
 }
 
 
@@ -279,7 +330,8 @@ def _pins_pass():
              test_routing_golden, test_weights_are_full_softmax_renormalised, test_brute_force_dense_masked,
              test_k_equals_E_uniform_weights_is_mean_of_experts,
              lambda: test_top_k_matches_torch_topk(8, 2),
-             lambda: test_single_expert_is_dense_ffn("bias")]
+             lambda: test_single_expert_is_dense_ffn("bias"),
+             test_shared_experts_add_dense_ffns, test_shared_expert_equal_to_routed_doubles_y]
     for t in tests:
         try:
             t()

@@ -89,8 +89,9 @@ def job_tokens_per_s(tokens_per_rank: int, world: int, max_ms: float) -> float:
     return tokens_per_rank * world / (max_ms * 1e-3)
 
 
-def workload_label(s):
-    return f"{s.name}: T={s.T} H={s.H} I={s.I} E={s.E} k={s.k}" + (" zipf-bias" if s.zipf_bias else "")
+def workload_label(s, n_shared=0):
+    return (f"{s.name}: T={s.T} H={s.H} I={s.I} E={s.E} k={s.k}" + (" zipf-bias" if s.zipf_bias else "")
+            + (f" +{n_shared} shared" if n_shared else ""))
 
 
 # ------------------------------------------------------------------ clocks
@@ -178,12 +179,17 @@ def time_oracle(inp, n_tokens: int):
     Wg = inp["Wg"].double().cpu().numpy()
     bias = None if inp["bias"] is None else inp["bias"].double().cpu().numpy()
     W1c, W3c, W2c = inp["W1"].cpu(), inp["W3"].cpu(), inp["W2"].cpu()
+    S = inp.get("n_shared", 0)
+    Wsc = [inp[n].cpu() for n in ("Ws1", "Ws3", "Ws2")] if S else None
 
     def load(e):
         return (W1c[e].double().numpy(), W3c[e].double().numpy(), W2c[e].double().numpy())
 
+    def load_shared(s):
+        return tuple(w[s].double().numpy() for w in Wsc)
+
     t0 = time.perf_counter()
-    O.moe_forward(x, Wg, bias, load, inp["k"])
+    O.moe_forward(x, Wg, bias, load, inp["k"], shared_weights=load_shared if S else None, n_shared=S)
     dt = time.perf_counter() - t0
     cores = None
     try:
@@ -212,9 +218,11 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     shape = WORKLOADS[args.workload]
-    inp = make_inputs(shape, device=dev, seed=args.seed)
+    S = args.shared
+    inp = make_inputs(shape, device=dev, seed=args.seed, n_shared=S)
     T, H, I, E, k = shape.T, shape.H, shape.I, shape.E, shape.k
-    plan = MoEPlan(T, H, I, E, k, device=dev)
+    plan = MoEPlan(T, H, I, E, k, device=dev, n_shared=S)
+    shared_kw = dict(Ws1=inp["Ws1"], Ws3=inp["Ws3"], Ws2=inp["Ws2"]) if S else {}
     if args.cta_pairs is not None:
         plan.set_cta_pairs(bool(args.cta_pairs))
     stream = torch.cuda.current_stream(dev)
@@ -227,7 +235,7 @@ def run_gpu(args, rank, world, local_rank):
             dist.barrier(device_ids=[local_rank])
 
     for _ in range(args.warmup):
-        plan.forward(*args_fwd, y=y)
+        plan.forward(*args_fwd, y=y, **shared_kw)
     plan.check()
 
     # timed device steps
@@ -241,7 +249,7 @@ def run_gpu(args, rank, world, local_rank):
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record(stream)
-        plan.forward(*args_fwd, y=y)
+        plan.forward(*args_fwd, y=y, **shared_kw)
         ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     clocks.end()
@@ -257,7 +265,7 @@ def run_gpu(args, rank, world, local_rank):
     x_host = inp["x"].cpu().pin_memory()
     y_host = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
     for _ in range(max(1, args.warmup)):
-        plan.forward_host(x_host, inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], y_host)
+        plan.forward_host(x_host, inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], y_host, **shared_kw)
     plan.check()
     e2e_steps = max(3, args.steps)
     barrier()
@@ -265,7 +273,7 @@ def run_gpu(args, rank, world, local_rank):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        plan.forward_host(x_host, inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], y_host)
+        plan.forward_host(x_host, inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], y_host, **shared_kw)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     plan.check()
@@ -287,8 +295,8 @@ def run_gpu(args, rank, world, local_rank):
 
     if rank == 0:
         peaks = measured_peaks()
-        flop = 6.0 * T * k * H * I
-        alg_bytes = 2.0 * 3 * H * I * active + 2.0 * H * E + 2.0 * T * H * 2
+        flop = 6.0 * T * (k + S) * H * I                     # routed pairs and shared-expert rows
+        alg_bytes = 2.0 * 3 * H * I * (active + S) + 2.0 * H * E + 2.0 * T * H * 2
         gemm_ms = kernel_ms["expert_gemm"] / max(nprof, 1)
         achieved_tflops = flop / (gemm_ms * 1e-3) / 1e12
         # the timed loop runs for seconds under the power cap: sustained peak
@@ -324,7 +332,7 @@ def run_gpu(args, rank, world, local_rank):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) x, N(0,1/H) Wg/W1/W3, N(0,1/I) W2, bf16; random-init weights)",
-            "config": {"workload": workload_label(shape), "T_per_gpu": T, "H": H, "I": I, "E": E, "k": k,
+            "config": {"workload": workload_label(shape, S), "T_per_gpu": T, "H": H, "I": I, "E": E, "k": k,
                        "block_m": plan.block_m, "cta_pairs": plan.cta_pairs, "active_experts": active, "padded_slots": num_padded,
                        "l2": "flushed between steps (256 MB write, outside per-step events)",
                        "parallelism": "replicas" if world > 1 else "single"},
@@ -351,7 +359,7 @@ def run_reference(args, rank, world):
     from synth.moe_inputs import WORKLOADS, make_inputs
     shape = WORKLOADS[args.workload]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    inp = make_inputs(shape, device=dev, seed=args.seed)
+    inp = make_inputs(shape, device=dev, seed=args.seed, n_shared=args.shared)
     n = min(shape.T, ORACLE_SAMPLE.get(args.workload, 64))
     for _ in range(args.warmup):
         time_oracle(inp, max(1, n // 8))
@@ -365,7 +373,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": BASELINE_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sum(times) / len(times) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": workload_label(shape)},
+        "data": "synthetic", "config": {"workload": workload_label(shape, args.shared)},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
@@ -382,6 +390,8 @@ def main():
                     help="T,H,I,E,k[,zipf] for --workload custom (e.g. a scaled-down case for profiling)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--shared", type=int, default=0,
+                    help="shared experts (weight 1, every token) on top of the workload's routed experts")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cta-pairs", type=int, default=None, choices=[0, 1],
                     help="expert GEMM on CTA pairs (1) or one CTA per block (0); default: the plan's")

@@ -68,7 +68,10 @@ typedef enum {
  *   expert_offset int32 [E+1]    first slot of each expert; multiples of block_m
  *   slot_token    int32 [pool]   token of each slot, -1 for padding
  *   slot_topk     int32 [pool]   top-k position j of each slot, -1 for padding
- *   num_padded    int32 [1]      slots in use = expert_offset[E]
+ *   num_padded    int32 [1]      slots in use by routed experts = expert_offset[E]
+ * With shared experts (moe_plan_create_shared) the slots after the routed
+ * ones hold every token once per shared expert, in token order, with
+ * slot_topk = -2 (combine weight 1), padded to block_m with (-1, -1).
  * ("MegaMoE 在 MoE 系统谱系中的位置", section 2.4: the slot record; the rank
  * field of that record is dropped on one GPU.) */
 typedef struct {
@@ -87,10 +90,12 @@ typedef struct {
 typedef struct {
   int32_t T_max, H, I, E, k;
   int32_t block_m;         /* rows per expert block (16, 32, 64 or 128) */
-  int32_t pool_capacity;   /* T_max*k + E*(block_m-1) slots */
+  int32_t pool_capacity;   /* T_max*k + E*(block_m-1) slots rounded up to block_m, plus
+                              n_shared * ceil(T_max/block_m) * block_m */
   int32_t num_sms;         /* persistent grid size */
   int32_t pair_clusters;   /* co-resident 2-CTA clusters of the CTA-pair expert GEMM */
   int32_t cta_pairs;       /* 1: the expert GEMM runs on CTA pairs (see moe_plan_set_cta_pairs) */
+  int32_t n_shared;        /* shared experts (moe_plan_create_shared) */
   size_t workspace_bytes;
 } moe_plan_desc;
 
@@ -105,6 +110,18 @@ typedef struct {
  * MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_UNSUPPORTED_DEVICE, MOE_ERR_CUDA.
  * Allocates no device memory. */
 int moe_plan_create(moe_plan_t* plan, int T_max, int H, int I, int E, int k, int block_m, int device);
+
+/* The same with n_shared (0 .. 8) shared experts ("MegaMoE 在 MoE 系统谱系中
+ * 的位置", section 2.7: the shared experts' two GEMM phases are scheduled in
+ * the routed experts' task queue). A shared expert is a SwiGLU FFN of the
+ * same H and I applied to every token with weight 1; its output is added to
+ * the routed combine: y[t] = sum_j w[t,j] FFN_{e_j}(x[t]) + sum_s FFNs_s(x[t]).
+ * Routing and BLOCK_M do not depend on it. Such a plan runs with
+ * moe_forward_shared / moe_forward_host_shared (moe_forward and
+ * moe_forward_host return MOE_ERR_INVALID_ARG for it). Errors as for
+ * moe_plan_create; n_shared outside 0..8 is MOE_ERR_UNSUPPORTED_SHAPE. */
+int moe_plan_create_shared(moe_plan_t* plan, int T_max, int H, int I, int E, int k, int n_shared, int block_m,
+                           int device);
 
 /* Bytes of device workspace the plan needs (routing arrays, scheduler
  * counters, the bf16 intermediate h [pool, I], the fp32 output accumulator
@@ -140,12 +157,29 @@ int moe_plan_get_routing(moe_plan_t plan, moe_routing* out);
 int moe_forward(moe_plan_t plan, const void* x, const void* Wg, const float* gate_bias, const void* W1,
                 const void* W3, const void* W2, int T, void* y, void* stream);
 
+/* moe_forward for a plan with shared experts (moe_plan_create_shared), which
+ * run as more blocks of the same persistent expert GEMM:
+ *   Ws1  bf16 [S, H, I]   device (shared experts' gated branch)
+ *   Ws3  bf16 [S, H, I]   device (linear branch)
+ *   Ws2  bf16 [S, I, H]   device (down projection)
+ * With S = 0 the shared pointers are ignored and may be NULL. Errors as for
+ * moe_forward; a NULL or misaligned shared pointer with S > 0 is
+ * MOE_ERR_INVALID_ARG. */
+int moe_forward_shared(moe_plan_t plan, const void* x, const void* Wg, const float* gate_bias, const void* W1,
+                       const void* W3, const void* W2, const void* Ws1, const void* Ws3, const void* Ws2, int T,
+                       void* y, void* stream);
+
 /* moe_forward with x and y in HOST memory: copies x [T, H] into the
  * workspace's staging buffer, runs the layer, copies y [T, H] back, all
  * enqueued on `stream` (pinned host buffers make the copies asynchronous; the
  * caller synchronises the stream before reading y). Weights stay on the device. */
 int moe_forward_host(moe_plan_t plan, const void* x_host, const void* Wg, const float* gate_bias, const void* W1,
                      const void* W3, const void* W2, int T, void* y_host, void* stream);
+
+/* moe_forward_host for a plan with shared experts (see moe_forward_shared). */
+int moe_forward_host_shared(moe_plan_t plan, const void* x_host, const void* Wg, const float* gate_bias,
+                            const void* W1, const void* W3, const void* W2, const void* Ws1, const void* Ws3,
+                            const void* Ws2, int T, void* y_host, void* stream);
 
 /* Gate and dispatch only (router, scan, scatter) for T tokens; fills the
  * routing results exactly as moe_forward does, without the expert FFN. */

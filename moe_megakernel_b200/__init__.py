@@ -39,18 +39,22 @@ class MoEPlanDesc(ctypes.Structure):
                 ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("block_m", ctypes.c_int32),
                 ("pool_capacity", ctypes.c_int32), ("num_sms", ctypes.c_int32),
                 ("pair_clusters", ctypes.c_int32), ("cta_pairs", ctypes.c_int32),
-                ("workspace_bytes", ctypes.c_size_t)]
+                ("n_shared", ctypes.c_int32), ("workspace_bytes", ctypes.c_size_t)]
 
 
 # exported symbol -> (restype, argtypes); the same list as include/moe_b200.h
 SIGNATURES = {
     "moe_plan_create": (_c_int, [ctypes.POINTER(_vp), _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
+    "moe_plan_create_shared": (_c_int, [ctypes.POINTER(_vp), _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                        _c_int]),
     "moe_plan_workspace_bytes": (_c_size, [_vp]),
     "moe_plan_bind_workspace": (_c_int, [_vp, _vp, _c_size]),
     "moe_plan_describe": (_c_int, [_vp, ctypes.POINTER(MoEPlanDesc)]),
     "moe_plan_get_routing": (_c_int, [_vp, ctypes.POINTER(MoERouting)]),
     "moe_forward": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
     "moe_forward_host": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
+    "moe_forward_shared": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
+    "moe_forward_host_shared": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
     "moe_route": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _vp]),
     "moe_check": (_c_int, [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]),
     "moe_plan_set_profiling": (_c_int, [_vp, _c_int]),
@@ -129,14 +133,15 @@ class MoEPlan:
     routing results of the last call.
     """
 
-    def __init__(self, T_max: int, H: int, I: int, E: int, k: int, block_m: int = 0, device=None):
+    def __init__(self, T_max: int, H: int, I: int, E: int, k: int, block_m: int = 0, device=None,
+                 n_shared: int = 0):
         self.lib = load_library()
         self.device = torch.device("cuda", torch.cuda.current_device() if device is None
                                    else torch.device(device).index or 0)
-        self.T_max, self.H, self.I, self.E, self.k = T_max, H, I, E, k
+        self.T_max, self.H, self.I, self.E, self.k, self.n_shared = T_max, H, I, E, k, n_shared
         self._plan = ctypes.c_void_p()
-        _ok(self.lib.moe_plan_create(ctypes.byref(self._plan), T_max, H, I, E, k, block_m,
-                                     self.device.index), "moe_plan_create")
+        _ok(self.lib.moe_plan_create_shared(ctypes.byref(self._plan), T_max, H, I, E, k, n_shared, block_m,
+                                            self.device.index), "moe_plan_create_shared")
         d = MoEPlanDesc()
         _ok(self.lib.moe_plan_describe(self._plan, ctypes.byref(d)), "moe_plan_describe")
         self.block_m, self.pool_capacity, self.num_sms = d.block_m, d.pool_capacity, d.num_sms
@@ -147,7 +152,7 @@ class MoEPlan:
             "moe_plan_bind_workspace")
 
     # ------------------------------------------------------------------ calls
-    def _check_inputs(self, x, Wg, bias, W=None):
+    def _check_inputs(self, x, Wg, bias, W=None, Ws=None):
         T = x.shape[0]
         _check(x, "x", (T, self.H), torch.bfloat16, self.device)
         _check(Wg, "Wg", (self.H, self.E), torch.bfloat16, self.device)
@@ -158,26 +163,35 @@ class MoEPlan:
             _check(W1, "W1", (self.E, self.H, self.I), torch.bfloat16, self.device)
             _check(W3, "W3", (self.E, self.H, self.I), torch.bfloat16, self.device)
             _check(W2, "W2", (self.E, self.I, self.H), torch.bfloat16, self.device)
+        if self.n_shared and Ws is not None:
+            Ws1, Ws3, Ws2 = Ws
+            S = self.n_shared
+            _check(Ws1, "Ws1", (S, self.H, self.I), torch.bfloat16, self.device)
+            _check(Ws3, "Ws3", (S, self.H, self.I), torch.bfloat16, self.device)
+            _check(Ws2, "Ws2", (S, self.I, self.H), torch.bfloat16, self.device)
         return T
 
-    def forward(self, x, Wg, bias, W1, W3, W2, y=None, stream=None) -> torch.Tensor:
-        T = self._check_inputs(x, Wg, bias, (W1, W3, W2))
+    def forward(self, x, Wg, bias, W1, W3, W2, y=None, stream=None, Ws1=None, Ws3=None, Ws2=None) -> torch.Tensor:
+        """Ws1/Ws3/Ws2: the shared experts' weights, required when the plan has n_shared > 0."""
+        T = self._check_inputs(x, Wg, bias, (W1, W3, W2), (Ws1, Ws3, Ws2))
         if y is None:
             y = torch.empty((T, self.H), dtype=torch.bfloat16, device=self.device)
         _check(y, "y", (T, self.H), torch.bfloat16, self.device)
-        _ok(self.lib.moe_forward(self._plan, _ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3), _ptr(W2),
-                                 T, _ptr(y), _stream_handle(stream, self.device)), "moe_forward")
+        _ok(self.lib.moe_forward_shared(self._plan, _ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3), _ptr(W2),
+                                        _ptr(Ws1), _ptr(Ws3), _ptr(Ws2), T, _ptr(y),
+                                        _stream_handle(stream, self.device)), "moe_forward_shared")
         return y
 
-    def forward_host(self, x_host, Wg, bias, W1, W3, W2, y_host, stream=None):
+    def forward_host(self, x_host, Wg, bias, W1, W3, W2, y_host, stream=None, Ws1=None, Ws3=None, Ws2=None):
         """x_host and y_host are CPU bf16 tensors (pinned for asynchronous copies)."""
         T = x_host.shape[0]
         _check(x_host, "x_host", (T, self.H), torch.bfloat16, torch.device("cpu"))
         _check(y_host, "y_host", (T, self.H), torch.bfloat16, torch.device("cpu"))
         _check(Wg, "Wg", (self.H, self.E), torch.bfloat16, self.device)
-        _ok(self.lib.moe_forward_host(self._plan, _ptr(x_host), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3),
-                                      _ptr(W2), T, _ptr(y_host), _stream_handle(stream, self.device)),
-            "moe_forward_host")
+        _ok(self.lib.moe_forward_host_shared(self._plan, _ptr(x_host), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3),
+                                             _ptr(W2), _ptr(Ws1), _ptr(Ws3), _ptr(Ws2), T, _ptr(y_host),
+                                             _stream_handle(stream, self.device)),
+            "moe_forward_host_shared")
         return y_host
 
     def route(self, x, Wg, bias, stream=None):

@@ -41,5 +41,8 @@ constexpr int kGatherWarps = MOE_GATHER_WARPS;     // warps that gather routed x
 constexpr int kGemm1Threads = 224 + 32 * kGatherWarps;
 constexpr int kTmemCols = 512;                     // two 256-column fp32 accumulators
 constexpr int kMaxGroups = 512;                    // block groups of the expert GEMM's task order
+constexpr int kMaxExperts = 256;                   // routed experts per plan
+constexpr int kMaxShared = 8;                      // shared experts per plan
+constexpr int kMaxExpertsAll = kMaxExperts + kMaxShared;
 
 }  // namespace moe

@@ -1,6 +1,9 @@
 // Dispatch: exclusive scans of the router's per-chunk histograms, padding of
 // every expert to a multiple of BLOCK_M, and the stable token -> slot
-// permutation with its (token, top-k position) record per slot.
+// permutation with its (token, top-k position) record per slot. Shared
+// experts (same page, section 2.7: their two GEMM phases share the routed
+// experts' task queue) follow the routed pool as experts E .. E+S-1 whose
+// blocks hold every token once, in order, with the record (t, kSharedTopk).
 //
 // "MegaMoE 在 MoE 系统谱系中的位置", section 2.4 (TokenSrcMetadata: each pool
 // slot records where its token came from, and the combine writes through that
@@ -19,8 +22,8 @@ struct DispatchParams {
   const int32_t* rank;       // [T, k]
   int32_t* chunk_count;      // [num_chunks, E]: counts in, per-chunk bases out
   int32_t* expert_count;     // [E]
-  int32_t* expert_offset;    // [E+1] slot offsets (multiples of BLOCK_M)
-  int32_t* block_start;      // [E+1] the same in blocks
+  int32_t* expert_offset;    // [E+1] slot offsets of the routed experts (multiples of BLOCK_M)
+  int32_t* block_start;      // [E+S+1] first block of every expert, shared ones last
   int32_t* slot_token;       // [pool]
   int32_t* slot_topk;        // [pool]
   int32_t* l1_done;          // [pool / BLOCK_M] zeroed here
@@ -31,21 +34,26 @@ struct DispatchParams {
   int32_t* l2_done;          // [pool / BLOCK_M] zeroed here
   // CTA-pair mode (nullptr: groups over blocks): pairs of consecutive blocks
   // of one expert, pair_start[e] = first pair of expert e; groups over pairs.
-  int32_t* pair_start;       // [E+1]
-  int T, E, k, BM, num_chunks, pool;
+  int32_t* pair_start;       // [E+S+1]
+  int T, E, S, k, BM, num_chunks, pool;
   int group_min, group_max, max_groups;
 };
 
 constexpr int kScanThreads = 1024;
 
+// slot_topk of a shared expert's slot: combine weight 1, no top-k position.
+constexpr int kSharedTopk = -2;
+
 // One CTA. (1) Expert e's chunk counts are scanned by kScanThreads/E threads,
 // each over a contiguous range of chunks; (2) warp 0 scans the padded block
-// counts over experts with shuffles; (3) thread 0 forms the block groups
-// while the other threads write offsets, padding records and counters.
+// counts over the routed and shared experts with shuffles; (3) thread 0 forms
+// the block groups while the other threads write offsets, padding and
+// shared-expert records and counters.
 __global__ void __launch_bounds__(kScanThreads) moe_dispatch_scan_kernel(const DispatchParams p) {
-  __shared__ int32_t s_nb[257];
-  __shared__ int32_t s_bs[257];
-  __shared__ int32_t s_cnt[256];
+  constexpr int kPerLane = (kMaxExpertsAll + 31) / 32;
+  __shared__ int32_t s_nb[kMaxExpertsAll + 1];
+  __shared__ int32_t s_bs[kMaxExpertsAll + 1];
+  __shared__ int32_t s_cnt[kMaxExperts];
   __shared__ int32_t s_part[kScanThreads];
   const int tid = threadIdx.x;
   // (1) per-expert scan over chunks: threads per expert tpe (a power of two)
@@ -86,14 +94,16 @@ __global__ void __launch_bounds__(kScanThreads) moe_dispatch_scan_kernel(const D
       base += v;
     }
   }
+  const int EA = p.E + p.S;   // routed + shared experts
+  if (tid < p.S) s_nb[p.E + tid] = (p.T + p.BM - 1) / p.BM;   // a shared expert sees every token
   __syncthreads();
-  // (2) exclusive scan of the block counts (E <= 256: 8 per lane)
+  // (2) exclusive scan of the block counts (E + S <= kMaxExpertsAll)
   if (tid < 32) {
-    int v[8], sum = 0;
+    int v[kPerLane], sum = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int ee = tid * 8 + i;
-      v[i] = ee < p.E ? s_nb[ee] : 0;
+    for (int i = 0; i < kPerLane; ++i) {
+      const int ee = tid * kPerLane + i;
+      v[i] = ee < EA ? s_nb[ee] : 0;
       sum += v[i];
     }
     int incl = sum;
@@ -104,20 +114,20 @@ __global__ void __launch_bounds__(kScanThreads) moe_dispatch_scan_kernel(const D
     }
     int run = incl - sum;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int ee = tid * 8 + i;
-      if (ee < p.E) s_bs[ee] = run;
+    for (int i = 0; i < kPerLane; ++i) {
+      const int ee = tid * kPerLane + i;
+      if (ee < EA) s_bs[ee] = run;
       run += v[i];
     }
-    if (tid == 31) s_bs[p.E] = incl;
+    if (tid == 31) s_bs[EA] = incl;
   }
-  __shared__ int32_t s_ps[257];
+  __shared__ int32_t s_ps[kMaxExpertsAll + 1];
   if (p.pair_start != nullptr && tid < 32) {   // exclusive scan of ceil(blocks / 2) per expert
-    int v[8], sum = 0;
+    int v[kPerLane], sum = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int ee = tid * 8 + i;
-      v[i] = ee < p.E ? (s_nb[ee] + 1) / 2 : 0;
+    for (int i = 0; i < kPerLane; ++i) {
+      const int ee = tid * kPerLane + i;
+      v[i] = ee < EA ? (s_nb[ee] + 1) / 2 : 0;
       sum += v[i];
     }
     int incl = sum;
@@ -128,19 +138,19 @@ __global__ void __launch_bounds__(kScanThreads) moe_dispatch_scan_kernel(const D
     }
     int run = incl - sum;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int ee = tid * 8 + i;
-      if (ee < p.E) s_ps[ee] = run;
+    for (int i = 0; i < kPerLane; ++i) {
+      const int ee = tid * kPerLane + i;
+      if (ee < EA) s_ps[ee] = run;
       run += v[i];
     }
-    if (tid == 31) s_ps[p.E] = incl;
+    if (tid == 31) s_ps[EA] = incl;
   }
   __syncthreads();
-  const int nblocks = s_bs[p.E];
+  const int nblocks = s_bs[EA];
   if (tid == 0) {
     p.sched[0] = 0;
     p.sched[1] = nblocks;
-    p.sched[2] = nblocks * p.BM;
+    p.sched[2] = s_bs[p.E] * p.BM;   // routed slots (the routing result)
     if (p.group_start != nullptr) {
       // Consecutive blocks form groups of at most group_max blocks; a group is
       // closed at the first expert boundary at least group_min blocks after
@@ -148,12 +158,12 @@ __global__ void __launch_bounds__(kScanThreads) moe_dispatch_scan_kernel(const D
       // rarely straddle two. One binary search over the expert boundaries per
       // group (block starts are non-decreasing).
       const int32_t* units = p.pair_start != nullptr ? s_ps : s_bs;   // group over pairs or blocks
-      const int total = units[p.E];
+      const int total = units[EA];
       int ng = 0, start = 0;
       p.group_start[0] = 0;
       while (start < total && ng < p.max_groups) {
         const int target = start + p.group_min;
-        int lo = 0, hi = p.E;   // first e with units[e] >= target (E if none)
+        int lo = 0, hi = EA;   // first e with units[e] >= target (EA if none)
         while (lo < hi) {
           const int mid = (lo + hi) >> 1;
           if (units[mid] >= target) hi = mid;
@@ -169,11 +179,21 @@ __global__ void __launch_bounds__(kScanThreads) moe_dispatch_scan_kernel(const D
     return;
   }
   // (3) everything else, on threads 1..
-  for (int ee = tid - 1; ee <= p.E; ee += kScanThreads - 1) {
+  for (int ee = tid - 1; ee <= EA; ee += kScanThreads - 1) {
     p.block_start[ee] = s_bs[ee];
     if (p.pair_start != nullptr) p.pair_start[ee] = s_ps[ee];
-    p.expert_offset[ee] = s_bs[ee] * p.BM;
+    if (ee <= p.E) p.expert_offset[ee] = s_bs[ee] * p.BM;
     if (ee < p.E) p.expert_count[ee] = s_cnt[ee];
+  }
+  // shared experts: slot (first slot of expert E+s) + t holds token t
+  for (int i = tid - 1; i < p.S * s_nb[p.E] * p.BM; i += kScanThreads - 1) {
+    const int per = s_nb[p.E] * p.BM;
+    const int t = i % per;
+    const int sl = s_bs[p.E] * p.BM + i;
+    if (sl < p.pool) {
+      p.slot_token[sl] = t < p.T ? t : -1;
+      p.slot_topk[sl] = t < p.T ? kSharedTopk : -1;
+    }
   }
   // padding slots of each expert's last block
   for (int ee = tid - 1; ee < p.E; ee += kScanThreads - 1) {

@@ -40,10 +40,13 @@ struct GemmParams {
   CUtensorMap tm_w1;   // W1 as [E*H, I], box {64, 64}
   CUtensorMap tm_w3;   // W3 as [E*H, I], box {64, 64}
   CUtensorMap tm_w2;   // W2 as [E*I, H], box {64, 64}
+  CUtensorMap tm_ws1;  // shared experts' W1 as [S*H, I] (experts E .. E+S-1; unused when S = 0)
+  CUtensorMap tm_ws3;  // shared experts' W3 as [S*H, I]
+  CUtensorMap tm_ws2;  // shared experts' W2 as [S*I, H]
   const int32_t* slot_token;
   const int32_t* slot_topk;
   const float* topk_w;
-  const int32_t* block_start;   // [E+1]
+  const int32_t* block_start;   // [E+S+1]
   const int32_t* group_start;   // [groups + 1] first block of each block group
   const int32_t* num_groups;    // [1]
   int32_t* task_counter;
@@ -53,6 +56,7 @@ struct GemmParams {
   bf16* h;                      // ring of ring_blocks blocks of BM rows x I
   float* y_acc;                 // [T, H]
   int T, H, I, E, k, BM, BN2, N1, N2;
+  int S;                        // shared experts (0 .. kMaxShared)
   int ring_blocks;              // block b uses ring slot b % ring_blocks
   int max_groups;
   unsigned long long timeout_ns;
@@ -83,7 +87,7 @@ struct GemmSmem {
   int taken;                     // tasks the producer has taken from the ring
   int num_groups;
   int rows[kTaskRing][kTileM];   // token row of each A-tile row, per task-ring slot (L1 tasks)
-  int block_start[257];
+  int block_start[kMaxExpertsAll + 1];
   int group_start[kMaxGroups + 1];
 };
 
@@ -153,7 +157,7 @@ __device__ __forceinline__ int segment_start(const GemmSmem& s, const GemmParams
 __device__ __forceinline__ Task decode_task(int t, const GemmSmem& s, const GemmParams& p) {
   Task task{-1, 0, 0, 0};
   const int G = s.num_groups;
-  const int nb_total = s.block_start[p.E];
+  const int nb_total = s.block_start[p.E + p.S];
   if (t < 0 || t >= nb_total * (p.N1 + p.N2) || G <= 0) return task;
   // last segment whose start is <= t (empty segments share the next start)
   int lo = 0, hi = 2 * G;
@@ -177,7 +181,7 @@ __device__ __forceinline__ Task decode_task(int t, const GemmSmem& s, const Gemm
   const int tl = t - segment_start(s, p, seg);
   // expert of the tl-th task: its blocks inside the group occupy consecutive NT-task runs
   const int vb = gb0 + tl / NT;
-  int elo = 0, ehi = p.E - 1;
+  int elo = 0, ehi = p.E + p.S - 1;
   while (elo < ehi) {
     const int mid = (elo + ehi + 1) >> 1;
     if (s.block_start[mid] <= vb) elo = mid;
@@ -322,22 +326,25 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
         // B: 128 columns of W1 next to the same 128 of W3; A comes from the gather warps.
         if (lane == 0) {
           ptx::mbar_arrive_expect_tx(&s.full[stage], 4 * kBoxBytes);
-          const int wrow = task.e * p.H + kb * kBK;
+          const bool sh = task.e >= p.E;   // shared expert: its own weight tensors
+          const int wrow = (sh ? task.e - p.E : task.e) * p.H + kb * kBK;
           const int n0 = task.n * kL1TileN;
+          const CUtensorMap* m1 = sh ? &p.tm_ws1 : &p.tm_w1;
+          const CUtensorMap* m3 = sh ? &p.tm_ws3 : &p.tm_w3;
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            ptx::tma_load_2d(b_addr + j * kBoxBytes, j < 2 ? &p.tm_w1 : &p.tm_w3, &s.full[stage], n0 + (j & 1) * 64,
-                             wrow, pol);
+            ptx::tma_load_2d(b_addr + j * kBoxBytes, j < 2 ? m1 : m3, &s.full[stage], n0 + (j & 1) * 64, wrow, pol);
         }
       } else {
         // B: 256 (or 128) columns of W2; A (the block's h rows) comes from the gather warps.
         if (lane == 0) {
           const int nbox = p.BN2 / 64;
           ptx::mbar_arrive_expect_tx(&s.full[stage], nbox * kBoxBytes);
-          const int wrow = task.e * p.I + kb * kBK;
+          const bool sh = task.e >= p.E;
+          const int wrow = (sh ? task.e - p.E : task.e) * p.I + kb * kBK;
           for (int j = 0; j < nbox; ++j)
-            ptx::tma_load_2d(b_addr + j * kBoxBytes, &p.tm_w2, &s.full[stage], task.n * p.BN2 + j * 64, wrow,
-                             pol);
+            ptx::tma_load_2d(b_addr + j * kBoxBytes, sh ? &p.tm_ws2 : &p.tm_w2, &s.full[stage], task.n * p.BN2 + j * 64,
+                             wrow, pol);
         }
       }
       __syncwarp();
@@ -645,7 +652,9 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
         }
         if (tok >= 0) {
           const int j = p.slot_topk[slot];
-          if (j < 0 || j >= p.k) {
+          if (task.e >= p.E) {
+            w = 1.f;   // shared expert: every token, weight 1
+          } else if (j < 0 || j >= p.k) {
             set_error(p, s, kDevBounds, 0x30000 | task.b);
             tok = -1;
           } else {
@@ -697,8 +706,13 @@ __global__ void __launch_bounds__(kGemm1Threads, 1) moe_expert_gemm_kernel(const
     ptx::prefetch_tmap(&p.tm_w1);
     ptx::prefetch_tmap(&p.tm_w3);
     ptx::prefetch_tmap(&p.tm_w2);
+    if (p.S > 0) {
+      ptx::prefetch_tmap(&p.tm_ws1);
+      ptx::prefetch_tmap(&p.tm_ws3);
+      ptx::prefetch_tmap(&p.tm_ws2);
+    }
   }
-  for (int e = threadIdx.x; e <= p.E; e += kGemm1Threads) s.block_start[e] = p.block_start[e];
+  for (int e = threadIdx.x; e <= p.E + p.S; e += kGemm1Threads) s.block_start[e] = p.block_start[e];
   {
     const int ng = min(*p.num_groups, min(p.max_groups, kMaxGroups));
     if (threadIdx.x == 0) s.num_groups = ng;

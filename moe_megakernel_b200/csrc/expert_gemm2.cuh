@@ -44,8 +44,11 @@ constexpr int kStage2Bytes = kTileABytes + kTileB2Bytes;    // 32 KB
 struct Gemm2Params {
   const bf16* x;       // [T, H]
   const bf16* w2;      // [E, I, H]
+  const bf16* ws2;     // [S, I, H] shared experts (experts E .. E+S-1), or null when S = 0
   CUtensorMap tm_w1;   // W1 as [E*H, I], box {64, 64}
   CUtensorMap tm_w3;   // W3 as [E*H, I], box {64, 64}
+  CUtensorMap tm_ws1;  // shared experts' W1 as [S*H, I] (unused when S = 0)
+  CUtensorMap tm_ws3;  // shared experts' W3 as [S*H, I]
   const int32_t* slot_token;
   const int32_t* slot_topk;
   const float* topk_w;
@@ -60,6 +63,7 @@ struct Gemm2Params {
   bf16* h;
   float* y_acc;                 // [T, H]
   int T, H, I, E, k, BM, BN2, N1, N2;
+  int S;                        // shared experts (0 .. kMaxShared)
   int ring_pairs, max_groups;
   unsigned long long timeout_ns;
   int withhold_pair;            // test hook: never publish L1 completion of this pair (-1: off)
@@ -88,8 +92,8 @@ struct Gemm2Smem {
   int taken;   // tasks the leader's producer has taken from the ring
   int num_groups;
   int rows[kTaskRing][kTileM];
-  int block_start[257];
-  int pair_start[257];
+  int block_start[kMaxExpertsAll + 1];
+  int pair_start[kMaxExpertsAll + 1];
   int group_start[kMaxGroups + 1];
 };
 
@@ -176,7 +180,7 @@ __device__ __forceinline__ int segment_start2(const Gemm2Smem& s, const Gemm2Par
 __device__ __forceinline__ Task2 decode_task2(int t, const Gemm2Smem& s, const Gemm2Params& p) {
   Task2 task{-1, 0, 0, 0, -1, -1, 0, 0};
   const int G = s.num_groups;
-  const int np_total = s.pair_start[p.E];
+  const int np_total = s.pair_start[p.E + p.S];
   if (t < 0 || t >= np_total * (p.N1 + p.N2) || G <= 0) return task;
   int lo = 0, hi = 2 * G;
   while (lo < hi) {
@@ -198,7 +202,7 @@ __device__ __forceinline__ Task2 decode_task2(int t, const Gemm2Smem& s, const G
   const int gp0 = s.group_start[g], gp1 = s.group_start[g + 1];
   const int tl = t - segment_start2(s, p, seg);
   const int vp = gp0 + tl / NT;
-  int elo = 0, ehi = p.E - 1;
+  int elo = 0, ehi = p.E + p.S - 1;
   while (elo < ehi) {
     const int mid = (elo + ehi + 1) >> 1;
     if (s.pair_start[mid] <= vp) elo = mid;
@@ -356,10 +360,12 @@ __device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_
         // barrier and reaches this one through its relay arrival
         if (task.phase == 0) {
           ptx::mbar_arrive_expect_tx(&s.full[stage], 2 * kBoxBytes);
-          const int wrow = task.e * p.H + kb * kBK;
+          const bool sh = task.e >= p.E;   // shared expert: its own weight tensors
+          const int wrow = (sh ? task.e - p.E : task.e) * p.H + kb * kBK;
           const int n0 = task.n * kL1TileN;
-          ptx::tma_load_2d(b_addr, &p.tm_w1, &s.full[stage], n0, wrow, pol);
-          ptx::tma_load_2d(b_addr + kBoxBytes, &p.tm_w1, &s.full[stage], n0 + 64, wrow, pol);
+          const CUtensorMap* m1 = sh ? &p.tm_ws1 : &p.tm_w1;
+          ptx::tma_load_2d(b_addr, m1, &s.full[stage], n0, wrow, pol);
+          ptx::tma_load_2d(b_addr + kBoxBytes, m1, &s.full[stage], n0 + 64, wrow, pol);
         } else {
           // L2: both operands come from the A-row warps' cp.async (a TMA box of
           // W2 kept the tensor pipe waiting); only this arrival is the producer's
@@ -438,10 +444,12 @@ __device__ void gemm2_follower_producer(const Gemm2Params& p, Gemm2Smem& s, uint
         const uint32_t b_addr = a_addr + kTileABytes;
         if (task.phase == 0) {
           ptx::mbar_arrive_expect_tx(&s.full[stage], 2 * kBoxBytes);
-          const int wrow = task.e * p.H + kb * kBK;
+          const bool sh = task.e >= p.E;
+          const int wrow = (sh ? task.e - p.E : task.e) * p.H + kb * kBK;
           const int n0 = task.n * kL1TileN;
-          ptx::tma_load_2d(b_addr, &p.tm_w3, &s.full[stage], n0, wrow, pol);
-          ptx::tma_load_2d(b_addr + kBoxBytes, &p.tm_w3, &s.full[stage], n0 + 64, wrow, pol);
+          const CUtensorMap* m3 = sh ? &p.tm_ws3 : &p.tm_w3;
+          ptx::tma_load_2d(b_addr, m3, &s.full[stage], n0, wrow, pol);
+          ptx::tma_load_2d(b_addr + kBoxBytes, m3, &s.full[stage], n0 + 64, wrow, pol);
         } else {
           ptx::mbar_arrive(&s.full[stage]);   // L2: operands by the A-row warps (see the leader)
         }
@@ -633,7 +641,9 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
         }
         if (tok >= 0) {
           const int j = p.slot_topk[slot];
-          if (j < 0 || j >= p.k) {
+          if (task.e >= p.E) {
+            w = 1.f;   // shared expert: every token, weight 1
+          } else if (j < 0 || j >= p.k) {
             set_error2(p, s, kDevBounds, 0x30000 | task.p);
             tok = -1;
           } else {
@@ -697,7 +707,8 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
     // L2: this CTA's half of the W2 tile too (BN2/2 columns: one or two 64x64
     // boxes, each 64 K-rows of 128 bytes in the same 128-byte swizzle as TMA)
     const int nhalf = task.phase == 1 ? p.BN2 / 128 : 0;
-    const bf16* w2src = p.w2 + (size_t)task.e * p.I * p.H + task.n * p.BN2 + (int)rank * (p.BN2 / 2) + c * 8;
+    const bf16* w2src = (task.e >= p.E ? p.ws2 + (size_t)(task.e - p.E) * p.I * p.H : p.w2 + (size_t)task.e * p.I * p.H) +
+                        task.n * p.BN2 + (int)rank * (p.BN2 / 2) + c * 8;
     const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
@@ -762,8 +773,12 @@ __global__ void __launch_bounds__(kGemm1Threads, 1) moe_expert_gemm2_kernel(cons
   if (warp == 0 && lane == 0) {
     ptx::prefetch_tmap(&p.tm_w1);
     ptx::prefetch_tmap(&p.tm_w3);
+    if (p.S > 0) {
+      ptx::prefetch_tmap(&p.tm_ws1);
+      ptx::prefetch_tmap(&p.tm_ws3);
+    }
   }
-  for (int e = threadIdx.x; e <= p.E; e += kGemm1Threads) {
+  for (int e = threadIdx.x; e <= p.E + p.S; e += kGemm1Threads) {
     s.block_start[e] = p.block_start[e];
     s.pair_start[e] = p.pair_start[e];
   }

@@ -91,6 +91,7 @@ int block_m_rule(int T, int k, int E) {
 
 struct moe_plan {
   int T_max, H, I, E, k, BM, device, num_sms;
+  int S = 0;                                           // shared experts
   int BN2, N1, N2, pool, chunks_max, blocks_max;
   int group_min, group_max, max_groups, ring_blocks;   // expert-GEMM task groups and h ring
   bool cta_pairs = false;                              // run the expert GEMM on CTA pairs
@@ -137,14 +138,14 @@ static Layout make_layout(const moe_plan& p) {
   L.chunk_count = take((size_t)p.chunks_max * p.E * 4, 256);
   L.expert_count = take((size_t)p.E * 4, 256);
   L.expert_offset = take((size_t)(p.E + 1) * 4, 256);
-  L.block_start = take((size_t)(p.E + 1) * 4, 256);
+  L.block_start = take((size_t)(p.E + p.S + 1) * 4, 256);
   L.num_padded = L.sched + 2 * 4;
   L.slot_token = take((size_t)p.pool * 4, 256);
   L.slot_topk = take((size_t)p.pool * 4, 256);
   L.l1_done = take((size_t)p.blocks_max * 4, 256);
   L.l2_done = take((size_t)p.blocks_max * 4, 256);
   L.group_start = take((size_t)(std::max(p.max_groups, p.pmax_groups) + 1) * 4, 256);
-  L.pair_start = take((size_t)(p.E + 1) * 4, 256);
+  L.pair_start = take((size_t)(p.E + p.S + 1) * 4, 256);
   L.router_partial = take((size_t)kRouterSplitTiles * kRouterMaxSplit * kRouterTokens * 256 * 4, 256);
   L.router_counter = take((size_t)kRouterSplitTiles * 4, 256);
   L.h = take((size_t)std::max(p.ring_blocks, 2 * p.ring_pairs) * p.BM * p.I * 2, 1024);
@@ -186,8 +187,14 @@ static int expert_pad(int E) {
   return ep;
 }
 
+struct SharedWeights {
+  const void* Ws1;   // [S, H, I]
+  const void* Ws3;   // [S, H, I]
+  const void* Ws2;   // [S, I, H]
+};
+
 static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias, const void* W1, const void* W3,
-                   const void* W2, int T, void* y, cudaStream_t st, bool full) {
+                   const void* W2, const SharedWeights& sw, int T, void* y, cudaStream_t st, bool full) {
   if (p->ws == nullptr) return MOE_ERR_NO_WORKSPACE;
   if (T < 0 || T > p->T_max) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;   // nothing to do; empty tensors may carry null pointers
@@ -196,6 +203,10 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   if (full) {
     if (W1 == nullptr || W3 == nullptr || W2 == nullptr || y == nullptr) return MOE_ERR_INVALID_ARG;
     if (!aligned16(W1) || !aligned16(W3) || !aligned16(W2) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+    if (p->S > 0) {
+      if (sw.Ws1 == nullptr || sw.Ws3 == nullptr || sw.Ws2 == nullptr) return MOE_ERR_INVALID_ARG;
+      if (!aligned16(sw.Ws1) || !aligned16(sw.Ws3) || !aligned16(sw.Ws2)) return MOE_ERR_INVALID_ARG;
+    }
   }
   DeviceGuard guard(p->device);
   uint8_t* ws = p->ws;
@@ -271,6 +282,7 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   dp.err = reinterpret_cast<int32_t*>(ws + L.err);
   dp.T = T;
   dp.E = p->E;
+  dp.S = p->S;
   dp.k = p->k;
   dp.BM = p->BM;
   dp.num_chunks = (T + kRouterTokens - 1) / kRouterTokens;
@@ -305,9 +317,14 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     std::memset(&gp, 0, sizeof(gp));
     bool ok = make_map(&gp.tm_w1, W1, I, (uint64_t)E * H, I, 64) &&
               make_map(&gp.tm_w3, W3, I, (uint64_t)E * H, I, 64);
+    if (ok && p->S > 0)
+      ok = make_map(&gp.tm_ws1, sw.Ws1, I, (uint64_t)p->S * H, I, 64) &&
+           make_map(&gp.tm_ws3, sw.Ws3, I, (uint64_t)p->S * H, I, 64);
     if (!ok) return MOE_ERR_CUDA;
     gp.x = static_cast<const bf16*>(x);
     gp.w2 = static_cast<const bf16*>(W2);
+    gp.ws2 = static_cast<const bf16*>(sw.Ws2);
+    gp.S = p->S;
     gp.slot_token = dp.slot_token;
     gp.slot_topk = dp.slot_topk;
     gp.topk_w = rp.topk_w;
@@ -354,7 +371,12 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     bool ok = make_map(&gp.tm_w1, W1, I, (uint64_t)E * H, I, 64) &&
               make_map(&gp.tm_w3, W3, I, (uint64_t)E * H, I, 64) &&
               make_map(&gp.tm_w2, W2, H, (uint64_t)E * I, H, 64);
+    if (ok && p->S > 0)
+      ok = make_map(&gp.tm_ws1, sw.Ws1, I, (uint64_t)p->S * H, I, 64) &&
+           make_map(&gp.tm_ws3, sw.Ws3, I, (uint64_t)p->S * H, I, 64) &&
+           make_map(&gp.tm_ws2, sw.Ws2, H, (uint64_t)p->S * I, H, 64);
     if (!ok) return MOE_ERR_CUDA;
+    gp.S = p->S;
     gp.x = static_cast<const bf16*>(x);
     gp.slot_token = dp.slot_token;
     gp.slot_topk = dp.slot_topk;
@@ -544,15 +566,21 @@ extern "C" int moe_route_static(const void* x, const void* Wg, const float* gate
 extern "C" {
 
 int moe_plan_create(moe_plan_t* out, int T_max, int H, int I, int E, int k, int block_m, int device) {
+  return moe_plan_create_shared(out, T_max, H, I, E, k, 0, block_m, device);
+}
+
+int moe_plan_create_shared(moe_plan_t* out, int T_max, int H, int I, int E, int k, int n_shared, int block_m,
+                           int device) {
   if (out == nullptr) return MOE_ERR_INVALID_ARG;
   *out = nullptr;
-  if (T_max < 1 || H < 128 || H % 128 || I < 128 || I % 128 || E < 8 || E > 256 || E % 8 || k < 1 || k > 8 ||
-      k > E)
+  if (T_max < 1 || H < 128 || H % 128 || I < 128 || I % 128 || E < 8 || E > kMaxExperts || E % 8 || k < 1 ||
+      k > 8 || k > E || n_shared < 0 || n_shared > kMaxShared)
     return MOE_ERR_UNSUPPORTED_SHAPE;
   if (block_m != 0 && block_m != 16 && block_m != 32 && block_m != 64 && block_m != 128)
     return MOE_ERR_UNSUPPORTED_SHAPE;
   // int32 indexing of slots, h rows and T*k
-  if ((long long)T_max * k + (long long)E * 127 > (1LL << 30)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)T_max * (k + n_shared) + (long long)(E + n_shared) * 127 > (1LL << 30))
+    return MOE_ERR_UNSUPPORTED_SHAPE;
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess) return MOE_ERR_CUDA;
   if (device < 0 || device >= ndev) return MOE_ERR_INVALID_ARG;
@@ -574,8 +602,10 @@ int moe_plan_create(moe_plan_t* out, int T_max, int H, int I, int E, int k, int 
   p->BN2 = (H % 256 == 0) ? 256 : 128;
   p->N1 = I / kL1TileN;
   p->N2 = H / p->BN2;
+  p->S = n_shared;
   p->pool = T_max * k + E * (p->BM - 1);
   p->pool = (p->pool + p->BM - 1) / p->BM * p->BM;
+  p->pool += n_shared * ((T_max + p->BM - 1) / p->BM) * p->BM;   // shared experts: every token once each
   p->chunks_max = (T_max + kRouterTokens - 1) / kRouterTokens;
   p->blocks_max = p->pool / p->BM;
   // Task groups (see the expert GEMM's task order): an L1 segment of at least
@@ -668,6 +698,7 @@ int moe_plan_describe(moe_plan_t p, moe_plan_desc* d) {
   d->pool_capacity = p->pool;
   d->num_sms = p->num_sms;
   d->pair_clusters = p->pair_clusters;
+  d->n_shared = p->S;
   d->cta_pairs = p->cta_pairs ? 1 : 0;
   d->workspace_bytes = p->L.total;
   return MOE_OK;
@@ -690,17 +721,26 @@ int moe_plan_get_routing(moe_plan_t p, moe_routing* r) {
 
 int moe_forward(moe_plan_t p, const void* x, const void* Wg, const float* bias, const void* W1, const void* W3,
                 const void* W2, int T, void* y, void* stream) {
+  if (p == nullptr || p->S > 0) return MOE_ERR_INVALID_ARG;
+  return enqueue(p, x, Wg, bias, W1, W3, W2, SharedWeights{}, T, y, static_cast<cudaStream_t>(stream), true);
+}
+
+int moe_forward_shared(moe_plan_t p, const void* x, const void* Wg, const float* bias, const void* W1,
+                       const void* W3, const void* W2, const void* Ws1, const void* Ws3, const void* Ws2, int T,
+                       void* y, void* stream) {
   if (p == nullptr) return MOE_ERR_INVALID_ARG;
-  return enqueue(p, x, Wg, bias, W1, W3, W2, T, y, static_cast<cudaStream_t>(stream), true);
+  return enqueue(p, x, Wg, bias, W1, W3, W2, SharedWeights{Ws1, Ws3, Ws2}, T, y, static_cast<cudaStream_t>(stream),
+                 true);
 }
 
 int moe_route(moe_plan_t p, const void* x, const void* Wg, const float* bias, int T, void* stream) {
   if (p == nullptr) return MOE_ERR_INVALID_ARG;
-  return enqueue(p, x, Wg, bias, nullptr, nullptr, nullptr, T, nullptr, static_cast<cudaStream_t>(stream), false);
+  return enqueue(p, x, Wg, bias, nullptr, nullptr, nullptr, SharedWeights{}, T, nullptr,
+                 static_cast<cudaStream_t>(stream), false);
 }
 
-int moe_forward_host(moe_plan_t p, const void* x_host, const void* Wg, const float* bias, const void* W1,
-                     const void* W3, const void* W2, int T, void* y_host, void* stream) {
+static int forward_host(moe_plan_t p, const void* x_host, const void* Wg, const float* bias, const void* W1,
+                        const void* W3, const void* W2, const SharedWeights& sw, int T, void* y_host, void* stream) {
   if (p == nullptr || x_host == nullptr || y_host == nullptr) return MOE_ERR_INVALID_ARG;
   if (p->ws == nullptr) return MOE_ERR_NO_WORKSPACE;
   if (T < 0 || T > p->T_max) return MOE_ERR_INVALID_ARG;
@@ -711,10 +751,22 @@ int moe_forward_host(moe_plan_t p, const void* x_host, const void* Wg, const flo
   void* xd = p->ws + p->L.x_stage;
   void* yd = p->ws + p->L.y_stage;
   if (cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return MOE_ERR_CUDA;
-  const int rc = enqueue(p, xd, Wg, bias, W1, W3, W2, T, yd, st, true);
+  const int rc = enqueue(p, xd, Wg, bias, W1, W3, W2, sw, T, yd, st, true);
   if (rc != MOE_OK) return rc;
   if (cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
+}
+
+int moe_forward_host(moe_plan_t p, const void* x_host, const void* Wg, const float* bias, const void* W1,
+                     const void* W3, const void* W2, int T, void* y_host, void* stream) {
+  if (p != nullptr && p->S > 0) return MOE_ERR_INVALID_ARG;
+  return forward_host(p, x_host, Wg, bias, W1, W3, W2, SharedWeights{}, T, y_host, stream);
+}
+
+int moe_forward_host_shared(moe_plan_t p, const void* x_host, const void* Wg, const float* bias, const void* W1,
+                            const void* W3, const void* W2, const void* Ws1, const void* Ws3, const void* Ws2, int T,
+                            void* y_host, void* stream) {
+  return forward_host(p, x_host, Wg, bias, W1, W3, W2, SharedWeights{Ws1, Ws3, Ws2}, T, y_host, stream);
 }
 
 int moe_check(moe_plan_t p, void* stream, int32_t* detail) {

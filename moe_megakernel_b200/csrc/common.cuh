@@ -18,8 +18,7 @@ enum DeviceError : int {
 constexpr int kRouterTokens = 64;
 constexpr int kRouterThreads = 128;
 constexpr int kRouterKChunk = 64;
-constexpr int kRouterSplitTiles = 8;    // token tiles up to which H is split across CTAs
-constexpr int kRouterMaxSplit = 16;     // at most this many H splits
+constexpr int kRouterMaxSplit = 64;     // at most this many H splits (only while tiles < SMs)
 
 // Expert GEMM tile: M = 128 rows (one tcgen05 MMA), K block = 64 bf16 = one
 // 128-byte swizzle row, N = 256 (L1: 128 columns of W1 next to the same 128 of

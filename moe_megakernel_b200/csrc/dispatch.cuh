@@ -51,6 +51,10 @@ constexpr int kSharedTopk = -2;
 // shared-expert records and counters.
 __global__ void __launch_bounds__(kScanThreads) moe_dispatch_scan_kernel(const DispatchParams p) {
   constexpr int kPerLane = (kMaxExpertsAll + 31) / 32;
+  if (p.E < 1 || p.E > kMaxExperts || p.S < 0 || p.S > kMaxShared) {   // the host validates; never trust it blindly
+    if (threadIdx.x == 0) atomicCAS(p.err, 0, kDevBounds);
+    return;
+  }
   __shared__ int32_t s_nb[kMaxExpertsAll + 1];
   __shared__ int32_t s_bs[kMaxExpertsAll + 1];
   __shared__ int32_t s_cnt[kMaxExperts];

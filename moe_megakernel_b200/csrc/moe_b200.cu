@@ -146,8 +146,9 @@ static Layout make_layout(const moe_plan& p) {
   L.l2_done = take((size_t)p.blocks_max * 4, 256);
   L.group_start = take((size_t)(std::max(p.max_groups, p.pmax_groups) + 1) * 4, 256);
   L.pair_start = take((size_t)(p.E + p.S + 1) * 4, 256);
-  L.router_partial = take((size_t)kRouterSplitTiles * kRouterMaxSplit * kRouterTokens * 256 * 4, 256);
-  L.router_counter = take((size_t)kRouterSplitTiles * 4, 256);
+  // split-H router: per token tile (fewer tiles than SMs) a logits accumulator and an arrival counter
+  L.router_partial = take((size_t)p.num_sms * kRouterTokens * 256 * 4, 256);
+  L.router_counter = take((size_t)p.num_sms * 4, 256);
   L.h = take((size_t)std::max(p.ring_blocks, 2 * p.ring_pairs) * p.BM * p.I * 2, 1024);
   L.y_acc = take((size_t)p.T_max * p.H * 4, 1024);
   L.x_stage = take((size_t)p.T_max * p.H * 2, 1024);
@@ -156,14 +157,16 @@ static Layout make_layout(const moe_plan& p) {
   return L;
 }
 
-// Number of H splits for the router: with few token tiles, spread the gate
-// GEMM over more CTAs (the largest divisor of H/64 up to kRouterMaxSplit).
-static int router_splits(int T, int H) {
+// Number of H splits for the router: with fewer 64-token tiles than SMs,
+// spread the gate GEMM over about two CTAs per SM (the largest divisor of
+// H/64 up to kRouterMaxSplit and that target).
+static int router_splits(int T, int H, int num_sms) {
   const int tiles = (T + kRouterTokens - 1) / kRouterTokens;
-  if (tiles > kRouterSplitTiles) return 1;
+  if (tiles >= num_sms) return 1;
+  const int want = (2 * num_sms + tiles - 1) / tiles;
   const int nk = H / kRouterKChunk;
   int s = 1;
-  for (int d = 1; d <= kRouterMaxSplit && d <= nk; ++d)
+  for (int d = 1; d <= kRouterMaxSplit && d <= nk && d <= want; ++d)
     if (nk % d == 0) s = d;
   return s;
 }
@@ -219,7 +222,7 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   cudaError_t ce;
 
   // 1. router (+ per-chunk histogram, + zero the output accumulator)
-  RouterParams rp;
+  RouterParams rp{};
   rp.x = static_cast<const bf16*>(x);
   rp.Wg = static_cast<const bf16*>(Wg);
   rp.bias = bias;
@@ -234,7 +237,7 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   rp.H = p->H;
   rp.E = p->E;
   rp.k = p->k;
-  const int splits = router_splits(T, p->H);
+  const int splits = router_splits(T, p->H, p->num_sms);
   mark(0);
   if (p->E % 64 == 0 && splits == 1) {
     // many tokens, E a multiple of 64: gate GEMM on tcgen05
@@ -268,7 +271,7 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   if (ce != cudaSuccess) return MOE_ERR_CUDA;
 
   // 2. dispatch scan, 3. dispatch scatter
-  DispatchParams dp;
+  DispatchParams dp{};
   dp.topk_idx = rp.topk_idx;
   dp.rank = rp.rank;
   dp.chunk_count = rp.chunk_count;
@@ -502,7 +505,7 @@ extern "C" int moe_route_static(const void* x, const void* Wg, const float* gate
   // The error word must start at zero; everything else is fully written below.
   if (cudaMemsetAsync(scratch + o_err, 0, 2 * sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
 
-  RouterParams rp;
+  RouterParams rp{};
   rp.x = static_cast<const bf16*>(x);
   rp.Wg = static_cast<const bf16*>(Wg);
   rp.bias = gate_bias;
@@ -527,7 +530,7 @@ extern "C" int moe_route_static(const void* x, const void* Wg, const float* gate
   }
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
 
-  DispatchParams dp;
+  DispatchParams dp{};
   dp.topk_idx = topk_idx;
   dp.rank = rp.rank;
   dp.chunk_count = rp.chunk_count;
@@ -682,7 +685,10 @@ int moe_plan_bind_workspace(moe_plan_t p, void* ws, size_t bytes) {
   // error word and scheduler counters start at zero
   if (cudaMemset(p->ws + p->L.err, 0, 16 * 4) != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaMemset(p->ws + p->L.sched, 0, 16 * 4) != cudaSuccess) return MOE_ERR_CUDA;
-  if (cudaMemset(p->ws + p->L.router_counter, 0, kRouterSplitTiles * 4) != cudaSuccess) return MOE_ERR_CUDA;
+  // split-H router state: accumulators and counters are zero between calls
+  if (cudaMemset(p->ws + p->L.router_counter, 0, (size_t)p->num_sms * 4) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemset(p->ws + p->L.router_partial, 0, (size_t)p->num_sms * kRouterTokens * 256 * 4) != cudaSuccess)
+    return MOE_ERR_CUDA;
   if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }

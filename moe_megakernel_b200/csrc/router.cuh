@@ -11,6 +11,7 @@
 #include <cstdint>
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace moe {
 
@@ -23,9 +24,10 @@ struct RouterParams {
   int32_t* rank;        // [T, k]  rank of (t, j) among this chunk's tokens routed to the same expert
   int32_t* chunk_count; // [num_chunks, E]
   float* y_acc;         // [T, H] zeroed here, accumulated by the expert GEMM
-  // Split of H over gridDim.y CTAs (small T): partial logits of each split,
-  // [tiles][splits][64][EP] fp32, and one arrival counter per token tile (zero
-  // between calls; the last CTA of a tile sums the splits and resets it).
+  // Split of H over gridDim.y CTAs (fewer token tiles than SMs): every split
+  // adds its partial logits into the tile's accumulator [tiles][64][EP] fp32
+  // and arrives on the tile's counter; the last CTA to arrive reads the sums,
+  // and leaves accumulator and counter at zero for the next call.
   float* partial;
   int32_t* tile_counter;
   int T, H, E, k;
@@ -173,20 +175,19 @@ __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(const Router
   // Logits (+ bias) to shared memory; padded experts get -inf.
   float* logits = reinterpret_cast<float*>(smem);
   if (gridDim.y > 1) {
-    // Split H: publish this split's partial logits; the last CTA of the token
-    // tile to arrive sums all splits in split order (deterministic).
+    // Split H: add this split's partial logits into the tile's accumulator
+    // (fp32 vector reductions at L2; the summation order over splits varies
+    // run to run, at fp32 rounding level); the last CTA of the tile to arrive
+    // takes the sums.
     __shared__ int s_last;
     const int tile = blockIdx.x, nsplit = gridDim.y;
-    float* mine = p.partial + ((size_t)tile * nsplit + blockIdx.y) * kRouterTokens * EP;
+    float* tacc = p.partial + (size_t)tile * kRouterTokens * EP;
     const int r0 = warp * 16 + (lane >> 2);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int col = nt * 8 + 2 * (lane & 3) + h;
-        mine[r0 * EP + col] = acc[nt][h];
-        mine[(r0 + 8) * EP + col] = acc[nt][2 + h];
-      }
+      const int col = nt * 8 + 2 * (lane & 3);
+      if (r0 < ntok) ptx::red_add_v2_f32(tacc + r0 * EP + col, acc[nt][0], acc[nt][1]);
+      if (r0 + 8 < ntok) ptx::red_add_v2_f32(tacc + (r0 + 8) * EP + col, acc[nt][2], acc[nt][3]);
     }
     if constexpr (kZeroAcc) {
       // every split zeroes its share of the tile's output-accumulator rows
@@ -202,24 +203,12 @@ __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(const Router
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    // 4 experts per thread and all splits' loads in flight at once; rows past
-    // the last token are not needed.
-    const float4* all = reinterpret_cast<const float4*>(p.partial + (size_t)tile * nsplit * kRouterTokens * EP);
-    const int stride4 = kRouterTokens * EP / 4;
+    // read the sums (L2) and leave the accumulator at zero for the next call
+    float4* all = reinterpret_cast<float4*>(tacc);
+#pragma unroll 4
     for (int i = threadIdx.x; i < ntok * EP / 4; i += kRouterThreads) {
-      float4 part[kRouterMaxSplit];
-#pragma unroll
-      for (int sp = 0; sp < kRouterMaxSplit; ++sp)
-        if (sp < nsplit) part[sp] = __ldcg(all + (size_t)sp * stride4 + i);
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int sp = 0; sp < kRouterMaxSplit; ++sp)
-        if (sp < nsplit) {
-          v.x += part[sp].x;
-          v.y += part[sp].y;
-          v.z += part[sp].z;
-          v.w += part[sp].w;
-        }
+      const float4 v = __ldcg(all + i);
+      __stcg(all + i, make_float4(0.f, 0.f, 0.f, 0.f));
       const int row = (4 * i) / EP, col = (4 * i) % EP;
       const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -248,11 +237,13 @@ __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(const Router
   }
   __syncwarp();
 
-  // Warp-level top-k: each warp owns the 16 token rows it computed.
+  // Warp-level top-k over the logits in shared memory; rows are dealt to the
+  // 4 warps round-robin so that a partly filled tile still uses all of them.
+  __syncthreads();
   int32_t* sel = reinterpret_cast<int32_t*>(smem + S::kTileBytes);   // [64][8] ascending expert ids
   constexpr int VPL = (EP + 31) / 32;
   for (int rr = 0; rr < 16; ++rr) {
-    const int row = warp * 16 + rr;
+    const int row = rr * 4 + warp;
     if (row >= ntok) break;   // warp-uniform
     float v[VPL];
 #pragma unroll

@@ -73,14 +73,18 @@ __device__ __forceinline__ void chunk_histogram(const int32_t* sel, unsigned lon
                                                 int32_t* chunk_count, int nthreads) {
   for (int i = threadIdx.x; i < nchunks * E; i += nthreads) mask[i] = 0ull;
   __syncthreads();
+  // (an expert id outside [0, E) -- only possible after an aborted top-k --
+  // is left out here; the dispatch scatter reports it as a bounds error)
   for (int i = threadIdx.x; i < ntok * k; i += nthreads) {
     const int t = i / k, j = i - t * k;
-    atomicOr(&mask[(t >> 6) * E + sel[t * 8 + j]], 1ull << (t & 63));
+    const int e = sel[t * 8 + j];
+    if (e >= 0 && e < E) atomicOr(&mask[(t >> 6) * E + e], 1ull << (t & 63));
   }
   __syncthreads();
   for (int i = threadIdx.x; i < ntok * k; i += nthreads) {
     const int t = i / k, j = i - t * k;
-    const unsigned long long m = mask[(t >> 6) * E + sel[t * 8 + j]];
+    const int e = sel[t * 8 + j];
+    const unsigned long long m = (e >= 0 && e < E) ? mask[(t >> 6) * E + e] : 0ull;
     rank[(size_t)(t0 + t) * k + j] = __popcll(m & ((1ull << (t & 63)) - 1ull));
   }
   const int chunks_used = (ntok + 63) >> 6;

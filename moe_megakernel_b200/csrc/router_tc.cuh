@@ -212,6 +212,12 @@ __global__ void __launch_bounds__(kRtcThreads, 1) moe_router_tc_kernel(const __g
         }
       }
     }
+    if (!ok && r < ntok) {
+      // aborted (bounded wait ran out): no selection; mark the rows invalid
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s.sel[r][j] = -1;
+      if (r == 0) atomicCAS(p.err, 0, kDevTimeout);
+    }
     if (ok && r < ntok) {
       // softmax over the k kept logits (best[0] is their maximum)
       float denom = 0.f;

@@ -134,6 +134,20 @@ def test_route_only_matches_oracle():
     assert_routing_equal(plan.routing(700), oracle_route(inp, plan.block_m))
 
 
+def test_route_only_tcgen05_router_back_to_back():
+    """Routing-only calls on the tcgen05 router (at least one 64-token tile per
+    SM, E a multiple of 64), three in a row without a host sync, then the
+    result against the oracle."""
+    shape = custom_shape(10000, 256, 128, 64, 4)
+    plan = _plan(shape)
+    inp = make_inputs(shape, device=DEV)
+    for _ in range(3):
+        plan.route(inp["x"], inp["Wg"], inp["bias"])
+    plan.check()
+    from tests.parity_util import oracle_route
+    assert_routing_equal(plan.routing(shape.T), oracle_route(inp, plan.block_m))
+
+
 def test_host_io_entry_matches_device_entry():
     shape = custom_shape(128, 256, 256, 8, 2)
     plan = _plan(shape)

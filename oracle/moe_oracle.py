@@ -43,6 +43,17 @@ Readings where the pages are silent (each is also listed in the design notes):
   added to the routed combine: y[t] += sum_s FFN_shared_s(x[t]). Routing and
   dispatch do not see them.
 
+* FP8 first GEMM (optional; "MegaMoE 在 MoE 系统谱系中的位置", section 一: the
+  Mega MoE kernel runs its GEMMs on 8-bit operands with scale factors loaded
+  beside them, and section 2.1: its epilogue quantizes with an amax). Reading
+  taken here: x and W1/W3 as OCP FP8 E4M3 (1 sign, 4 exponent bits with bias
+  7, 3 mantissa bits, largest finite 448, round to nearest even, saturating),
+  with power-of-two scales: one per token over H for x, one per (expert,
+  column i) over H for W1 and W3; the scale is the smallest power of two p
+  with amax / p <= 448 (1 for an all-zero row). g = sx[t] * s1[e,i] *
+  sum_h xq[t,h] W1q[e,h,i], the same for u; the activation and the second
+  GEMM are as in the bf16 layer.
+
 Everything is fp64 on inputs given as fp64 arrays holding bf16 values.
 """
 from __future__ import annotations
@@ -78,6 +89,39 @@ def bf16_round(a) -> np.ndarray:
     out[finite] = r
     out[~finite] = a[~finite]
     return out
+
+
+E4M3_MAX = 448.0
+
+
+def e4m3_round(a) -> np.ndarray:
+    """Round fp64 values to the nearest FP8 E4M3 value (ties to even), as fp64,
+    saturating at +-448.
+
+    Written from the format: normal values (1 + m/8) * 2**e for e in -6..8, so
+    for |a| in [2**e, 2**(e+1)) the grid step is 2**(e-3); below 2**-6 the
+    subnormal step is 2**-9.
+    """
+    a = np.asarray(a, dtype=np.float64)
+    m, e = np.frexp(a)                      # a = m * 2**e, |m| in [0.5, 1)
+    step_exp = np.maximum(e - 1, -6) - 3    # exponent of the grid step
+    r = np.ldexp(np.rint(np.ldexp(a, -step_exp)), step_exp)
+    return np.clip(r, -E4M3_MAX, E4M3_MAX)
+
+
+def pow2_scale(amax) -> np.ndarray:
+    """Smallest power of two p with amax / p <= 448 (1 where amax == 0)."""
+    amax = np.asarray(amax, dtype=np.float64)
+    q = amax / E4M3_MAX
+    m, e = np.frexp(q)                      # q = m * 2**e, m in [0.5, 1)
+    k = np.where(m == 0.5, e - 1, e)        # 2**k >= q, and 2**(k-1) < q
+    return np.where(amax > 0, np.ldexp(1.0, k), 1.0)
+
+
+def quantize_fp8(a: np.ndarray, axis: int):
+    """(codes, scales): scales = pow2_scale(max |a| along `axis`), codes = e4m3_round(a / scales)."""
+    sc = pow2_scale(np.max(np.abs(a), axis=axis, keepdims=True))
+    return e4m3_round(a / sc), sc
 
 
 # --------------------------------------------------------------------------
@@ -197,6 +241,16 @@ def expert_ffn(xr: np.ndarray, W1e: np.ndarray, W3e: np.ndarray, W2e: np.ndarray
     return a @ W2e
 
 
+def expert_ffn_fp8(xq: np.ndarray, sx: np.ndarray, W1q: np.ndarray, s1: np.ndarray, W3q: np.ndarray,
+                   s3: np.ndarray, W2e: np.ndarray) -> np.ndarray:
+    """The expert FFN with an FP8 first GEMM: xq [n,H] codes with scales sx [n,1];
+    W1q, W3q [H,I] codes with column scales s1, s3 [1,I]; W2e [I,H] as in the bf16 layer."""
+    g = (xq @ W1q) * sx * s1
+    u = (xq @ W3q) * sx * s3
+    a = bf16_round(silu(g) * u)
+    return a @ W2e
+
+
 def stacked_expert_weights(W1, W3, W2) -> Callable[[int], tuple]:
     """Expert loader over stacked arrays W1,W3 [E,H,I], W2 [E,I,H] (any float dtype)."""
     def load(e):
@@ -207,7 +261,8 @@ def stacked_expert_weights(W1, W3, W2) -> Callable[[int], tuple]:
 
 def moe_forward(x, Wg, bias, expert_weights: Callable[[int], tuple], k: int,
                 block_m: Optional[int] = None, tokens: Optional[Sequence[int]] = None,
-                shared_weights: Optional[Callable[[int], tuple]] = None, n_shared: int = 0) -> dict:
+                shared_weights: Optional[Callable[[int], tuple]] = None, n_shared: int = 0,
+                fp8: bool = False) -> dict:
     """The whole layer: gate, dispatch, expert FFN, gate-weighted combine.
 
     x [T,H] fp64; Wg [H,E] fp64; bias [E] or None; ``expert_weights(e)``
@@ -216,6 +271,8 @@ def moe_forward(x, Wg, bias, expert_weights: Callable[[int], tuple], k: int,
     T tokens). y[t] = sum_j w[t,j] * FFN_{idx[t,j]}(x[t])
                       + sum_{s < n_shared} FFN_shared_s(x[t]),
     with ``shared_weights(s)`` returning the shared expert's (W1, W3, W2).
+    fp8=True runs the first GEMM on FP8 E4M3 operands (see the module notes):
+    x is quantized per token, W1/W3 per (expert, column); no shared experts.
     """
     x = np.asarray(x, np.float64)
     T, H = x.shape
@@ -225,13 +282,22 @@ def moe_forward(x, Wg, bias, expert_weights: Callable[[int], tuple], k: int,
     disp = dispatch(idx, E, bm)
     rows = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
     y = np.zeros((len(rows), H), dtype=np.float64)
+    if fp8:
+        if n_shared:
+            raise ValueError("the FP8 first GEMM is defined without shared experts")
+        xq, sx = quantize_fp8(x, axis=1)
     for e in range(E):
         # (row position in `rows`, top-k position) of every selected pair routed to e
         hit = np.nonzero(idx[rows] == e)
         if hit[0].size == 0:
             continue
         W1e, W3e, W2e = expert_weights(e)
-        o = expert_ffn(x[rows[hit[0]]], W1e, W3e, W2e)
+        if fp8:
+            W1q, s1 = quantize_fp8(W1e, axis=0)
+            W3q, s3 = quantize_fp8(W3e, axis=0)
+            o = expert_ffn_fp8(xq[rows[hit[0]]], sx[rows[hit[0]]], W1q, s1, W3q, s3, W2e)
+        else:
+            o = expert_ffn(x[rows[hit[0]]], W1e, W3e, W2e)
         wt = w[rows[hit[0]], hit[1]]
         np.add.at(y, hit[0], wt[:, None] * o)
     if n_shared:

@@ -307,6 +307,62 @@ def test_two_shared_experts_equal_one_of_double_width():
     np.testing.assert_allclose(two, wide, rtol=1e-12, atol=1e-14)
 
 
+# ----------------------------------------------------------------- FP8 first GEMM
+
+def test_e4m3_round_golden_and_matches_torch():
+    """E4M3 rounding: hand-derived values (ties to even on the 1/8 mantissa
+    grid, the 2**-9 subnormal grid, saturation at 448) and torch's float8
+    conversion on 20000 random in-range values."""
+    golden = {1.0: 1.0, 1.0625: 1.0, 1.1875: 1.25, 3.5: 3.5, 2.0 ** -9: 2.0 ** -9,
+              1.5 * 2.0 ** -9: 2.0 ** -8, 2.0 ** -10: 0.0, 447.0: 448.0, 460.0: 448.0, -0.3: -0.3125}
+    for v, want in golden.items():
+        assert O.e4m3_round(v) == want, (v, O.e4m3_round(v), want)
+    rng = _rng(21)
+    v = np.clip(rng.standard_normal(20000) * np.exp(rng.uniform(-12, 6, 20000)), -448, 448)
+    t = torch.from_numpy(v).to(torch.float32)
+    np.testing.assert_array_equal(O.e4m3_round(t.double().numpy()), t.to(torch.float8_e4m3fn).double().numpy())
+
+
+def test_pow2_scale_is_the_smallest_power_of_two():
+    rng = _rng(22)
+    amax = np.concatenate([np.exp(rng.uniform(-20, 20, 5000)), [448.0, 896.0, 224.0, 1.0]])
+    p = O.pow2_scale(amax)
+    k = np.log2(p)
+    assert np.all(k == np.round(k))                       # powers of two
+    assert np.all(amax / p <= 448.0) and np.all(amax / (p / 2) > 448.0)
+    assert O.pow2_scale(0.0) == 1.0 and O.pow2_scale(448.0) == 1.0 and O.pow2_scale(449.0) == 2.0
+
+
+def test_fp8_forward_matches_textbook_dequantized_ffn():
+    """fp8=True equals the bf16 layer's combine with x, W1, W3 replaced by their
+    dequantized FP8 values (quantized here with torch's float8 cast and scales
+    from torch log2/ceil)."""
+    rng = _rng(23)
+    x, Wg, W1, W3, W2 = _tiny_layer(rng, T=20, H=32, I=48, E=4)
+    k = 2
+
+    def tq(a, dim):
+        amax = torch.from_numpy(np.abs(a)).amax(dim=dim, keepdim=True)
+        sc = torch.where(amax > 0, torch.exp2(torch.ceil(torch.log2(amax / 448.0))), torch.ones_like(amax))
+        q = (torch.from_numpy(a) / sc).to(torch.float32).to(torch.float8_e4m3fn).double()
+        return (q * sc).numpy()
+
+    xd = tq(x, 1)
+    W1d = np.stack([tq(W1[e], 0) for e in range(W1.shape[0])])
+    W3d = np.stack([tq(W3[e], 0) for e in range(W3.shape[0])])
+    r = O.moe_forward(x, Wg, None, O.stacked_expert_weights(W1, W3, W2), k, fp8=True)
+    idx, w = r["topk_idx"], r["topk_w"]
+    y = np.zeros_like(x)
+    for t in range(x.shape[0]):
+        for j in range(k):
+            e = idx[t, j]
+            y[t] += w[t, j] * _torch_ffn(xd[t:t + 1], W1d[e], W3d[e], W2[e])[0]
+    np.testing.assert_allclose(r["y"], y, rtol=1e-12, atol=1e-14)
+    # and it stays near the bf16 layer (FP8 has 3 mantissa bits)
+    b = O.moe_forward(x, Wg, None, O.stacked_expert_weights(W1, W3, W2), k)
+    assert np.linalg.norm(r["y"] - b["y"]) / np.linalg.norm(b["y"]) < 0.1
+
+
 # ----------------------------------------------------------------- planted mistakes
 
 _MUTANTS = {
@@ -322,6 +378,13 @@ _MUTANTS = {
                                                           np.frexp(np.asarray(a, float))[1] - 8)),
     "shared_averaged": ("shared_ffn_sum", lambda xr, sw, S: sum(O.expert_ffn(xr, *sw(s)) for s in range(S)) / S),
     "shared_first_only": ("shared_ffn_sum", lambda xr, sw, S: O.expert_ffn(xr, *sw(0))),
+    "e4m3_truncation": ("e4m3_round", lambda a: np.clip(np.ldexp(np.trunc(np.ldexp(np.asarray(a, float),
+                        -(np.maximum(np.frexp(np.asarray(a, float))[1] - 1, -6) - 3))),
+                        np.maximum(np.frexp(np.asarray(a, float))[1] - 1, -6) - 3), -448, 448)),
+    "fp8_scale_dropped": ("expert_ffn_fp8", lambda xq, sx, W1q, s1, W3q, s3, W2e:
+                          O.bf16_round(O.silu((xq @ W1q) * s1) * ((xq @ W3q) * s3)) @ W2e),
+    "pow2_scale_floor": ("pow2_scale", lambda amax: np.where(np.asarray(amax) > 0, np.ldexp(1.0, np.frexp(
+                         np.asarray(amax, float) / 448.0)[1] - 1), 1.0)),
 }
 
 
@@ -331,7 +394,9 @@ def _pins_pass():
              test_k_equals_E_uniform_weights_is_mean_of_experts,
              lambda: test_top_k_matches_torch_topk(8, 2),
              lambda: test_single_expert_is_dense_ffn("bias"),
-             test_shared_experts_add_dense_ffns, test_shared_expert_equal_to_routed_doubles_y]
+             test_shared_experts_add_dense_ffns, test_shared_expert_equal_to_routed_doubles_y,
+             test_e4m3_round_golden_and_matches_torch, test_pow2_scale_is_the_smallest_power_of_two,
+             test_fp8_forward_matches_textbook_dequantized_ffn]
     for t in tests:
         try:
             t()

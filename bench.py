@@ -89,9 +89,9 @@ def job_tokens_per_s(tokens_per_rank: int, world: int, max_ms: float) -> float:
     return tokens_per_rank * world / (max_ms * 1e-3)
 
 
-def workload_label(s, n_shared=0):
+def workload_label(s, n_shared=0, fp8=False):
     return (f"{s.name}: T={s.T} H={s.H} I={s.I} E={s.E} k={s.k}" + (" zipf-bias" if s.zipf_bias else "")
-            + (f" +{n_shared} shared" if n_shared else ""))
+            + (f" +{n_shared} shared" if n_shared else "") + (" fp8-e4m3 first GEMM" if fp8 else ""))
 
 
 # ------------------------------------------------------------------ clocks
@@ -169,7 +169,7 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ oracle timing
-def time_oracle(inp, n_tokens: int):
+def time_oracle(inp, n_tokens: int, fp8: bool = False):
     """The fp64 CPU oracle as it stands, on the first n_tokens tokens (host copies of the inputs)."""
     import numpy as np
     import torch
@@ -189,7 +189,7 @@ def time_oracle(inp, n_tokens: int):
         return tuple(w[s].double().numpy() for w in Wsc)
 
     t0 = time.perf_counter()
-    O.moe_forward(x, Wg, bias, load, inp["k"], shared_weights=load_shared if S else None, n_shared=S)
+    O.moe_forward(x, Wg, bias, load, inp["k"], shared_weights=load_shared if S else None, n_shared=S, fp8=fp8)
     dt = time.perf_counter() - t0
     cores = None
     try:
@@ -206,7 +206,7 @@ def time_oracle(inp, n_tokens: int):
 def run_gpu(args, rank, world, local_rank):
     import torch
 
-    from moe_megakernel_b200 import MoEPlan, kernels_per_forward
+    from moe_megakernel_b200 import MoEPlan, kernels_per_forward, quantize_weights_fp8
     from synth.moe_inputs import WORKLOADS, make_inputs
 
     dist = None
@@ -229,13 +229,30 @@ def run_gpu(args, rank, world, local_rank):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     args_fwd = (inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"])
+    if args.fp8:
+        # weights are quantized once, like loading a checkpoint (outside every timed region)
+        W1q, s1 = quantize_weights_fp8(inp["W1"])
+        W3q, s3 = quantize_weights_fp8(inp["W3"])
+        fp8_w = (W1q, s1, W3q, s3, inp["W2"])
+
+    def fwd():
+        if args.fp8:
+            plan.forward_fp8(inp["x"], inp["Wg"], inp["bias"], *fp8_w, y=y)
+        else:
+            plan.forward(*args_fwd, y=y, **shared_kw)
+
+    def fwd_host(x_host, y_host):
+        if args.fp8:
+            plan.forward_host_fp8(x_host, inp["Wg"], inp["bias"], *fp8_w, y_host)
+        else:
+            plan.forward_host(x_host, inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], y_host, **shared_kw)
 
     def barrier():
         if dist is not None:
             dist.barrier(device_ids=[local_rank])
 
     for _ in range(args.warmup):
-        plan.forward(*args_fwd, y=y, **shared_kw)
+        fwd()
     plan.check()
 
     # timed device steps
@@ -249,7 +266,7 @@ def run_gpu(args, rank, world, local_rank):
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record(stream)
-        plan.forward(*args_fwd, y=y, **shared_kw)
+        fwd()
         ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     clocks.end()
@@ -265,7 +282,7 @@ def run_gpu(args, rank, world, local_rank):
     x_host = inp["x"].cpu().pin_memory()
     y_host = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
     for _ in range(max(1, args.warmup)):
-        plan.forward_host(x_host, inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], y_host, **shared_kw)
+        fwd_host(x_host, y_host)
     plan.check()
     e2e_steps = max(3, args.steps)
     barrier()
@@ -273,7 +290,7 @@ def run_gpu(args, rank, world, local_rank):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        plan.forward_host(x_host, inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], y_host, **shared_kw)
+        fwd_host(x_host, y_host)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     plan.check()
@@ -288,19 +305,25 @@ def run_gpu(args, rank, world, local_rank):
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
         n = min(T, ORACLE_SAMPLE.get(args.workload, 64))
-        v, dt, cores = time_oracle(inp, n)
+        v, dt, cores = time_oracle(inp, n, fp8=args.fp8)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"fp64 oracle (gate, dispatch, expert FFN, combine) on the first {n} of {T} tokens "
-                         f"of the same inputs, {dt:.1f} s wall"}
+               "sample": f"fp64 oracle (gate, dispatch, expert FFN, combine{', FP8 first GEMM' if args.fp8 else ''}) "
+                         f"on the first {n} of {T} tokens of the same inputs, {dt:.1f} s wall"}
 
     if rank == 0:
         peaks = measured_peaks()
         flop = 6.0 * T * (k + S) * H * I                     # routed pairs and shared-expert rows
         alg_bytes = 2.0 * 3 * H * I * (active + S) + 2.0 * H * E + 2.0 * T * H * 2
+        if args.fp8:   # W1/W3 as 1-byte codes plus fp32 column scales
+            alg_bytes += (-2.0 * H * I + 8.0 * I) * active
         gemm_ms = kernel_ms["expert_gemm"] / max(nprof, 1)
         achieved_tflops = flop / (gemm_ms * 1e-3) / 1e12
         # the timed loop runs for seconds under the power cap: sustained peak
         tc_peak = peaks["bf16_tflops_sustained"]
+        if args.fp8:
+            # 4/6 of the FLOPs (x.W1, x.W3) at the FP8 rate, taken as 2x the measured bf16 rate
+            # (nominal dense 4.5 vs 2.25 PFLOP/s), 2/6 (h.W2) at the bf16 rate: 6 / (4/2 + 2) = 1.5x
+            tc_peak = 1.5 * tc_peak
         t_tc = flop / (tc_peak * 1e12)
         t_hbm = alg_bytes / (peaks["hbm_gbs"] * 1e9)
         bound = "tensor" if t_tc >= t_hbm else "hbm"
@@ -312,9 +335,11 @@ def run_gpu(args, rank, world, local_rank):
             roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": gbs / peaks["hbm_gbs"]}
         roof.update({"kernel": "moe_expert_gemm2_kernel" if plan.cta_pairs else "moe_expert_gemm_kernel",
-                     "traffic": measured_traffic(args.workload),
+                     "traffic": measured_traffic(args.workload + ("+fp8" if args.fp8 else "")),
                      "traffic_unit": "bytes per launch (ncu dram read+write)",
-                     "peak_source": f"{peaks['source']} ({'bf16_tflops_sustained' if bound == 'tensor' else 'hbm_gbs'})",
+                     "peak_source": f"{peaks['source']} ({'bf16_tflops_sustained' if bound == 'tensor' else 'hbm_gbs'})"
+                                    + (" x 1.5: FP8 first GEMM at 2x the bf16 rate" if args.fp8 and bound == "tensor"
+                                       else ""),
                      "kernel_ms": gemm_ms,
                      "layer_t_roof_ms": max(t_tc, t_hbm) * 1e3,
                      "layer_frac": max(t_tc, t_hbm) * 1e3 / mean_ms,
@@ -330,9 +355,9 @@ def run_gpu(args, rank, world, local_rank):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "bf16",
+            "dtype": "e4m3 x.W1/x.W3 + bf16" if args.fp8 else "bf16",
             "data": "synthetic (seeded N(0,1) x, N(0,1/H) Wg/W1/W3, N(0,1/I) W2, bf16; random-init weights)",
-            "config": {"workload": workload_label(shape, S), "T_per_gpu": T, "H": H, "I": I, "E": E, "k": k,
+            "config": {"workload": workload_label(shape, S, args.fp8), "T_per_gpu": T, "H": H, "I": I, "E": E, "k": k,
                        "block_m": plan.block_m, "cta_pairs": plan.cta_pairs, "active_experts": active, "padded_slots": num_padded,
                        "l2": "flushed between steps (256 MB write, outside per-step events)",
                        "parallelism": "replicas" if world > 1 else "single"},
@@ -340,8 +365,9 @@ def run_gpu(args, rank, world, local_rank):
             "cpu_baseline": cpu,
             "e2e": {"value": job_tokens_per_s(T, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2,
-                    "ms_per_step": e2e_ms, "api": "moe_forward_host (pinned host x and y)"},
-            "gpu_launches": args.steps * kernels_per_forward(),
+                    "ms_per_step": e2e_ms,
+                    "api": f"moe_forward_host{'_fp8' if args.fp8 else ''} (pinned host x and y)"},
+            "gpu_launches": args.steps * (kernels_per_forward() + (1 if args.fp8 else 0)),
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
@@ -362,10 +388,10 @@ def run_reference(args, rank, world):
     inp = make_inputs(shape, device=dev, seed=args.seed, n_shared=args.shared)
     n = min(shape.T, ORACLE_SAMPLE.get(args.workload, 64))
     for _ in range(args.warmup):
-        time_oracle(inp, max(1, n // 8))
+        time_oracle(inp, max(1, n // 8), fp8=args.fp8)
     times, cores = [], None
     for _ in range(args.steps):
-        v, dt, cores = time_oracle(inp, n)
+        v, dt, cores = time_oracle(inp, n, fp8=args.fp8)
         times.append(dt)
     value = n * len(times) / sum(times)
     sample = f"fp64 CPU oracle on the first {n} of {shape.T} tokens per step"
@@ -373,7 +399,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": BASELINE_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sum(times) / len(times) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": workload_label(shape, args.shared)},
+        "data": "synthetic", "config": {"workload": workload_label(shape, args.shared, args.fp8)},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
@@ -392,12 +418,16 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--shared", type=int, default=0,
                     help="shared experts (weight 1, every token) on top of the workload's routed experts")
+    ap.add_argument("--fp8", action="store_true",
+                    help="FP8 E4M3 first GEMM (x.W1, x.W3) with power-of-two per-token / per-column scales")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cta-pairs", type=int, default=None, choices=[0, 1],
                     help="expert GEMM on CTA pairs (1) or one CTA per block (0); default: the plan's")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.fp8 and args.shared:
+        ap.error("--fp8 runs without shared experts")
     if args.workload == "custom":
         if not args.shape:
             ap.error("--workload custom needs --shape T,H,I,E,k[,zipf]")

@@ -55,6 +55,10 @@ SIGNATURES = {
     "moe_forward_host": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
     "moe_forward_shared": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
     "moe_forward_host_shared": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
+    "moe_forward_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
+    "moe_forward_host_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
+    "moe_quantize_weights_fp8": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp]),
+    "moe_quantize_x_fp8": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _vp]),
     "moe_route": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _vp]),
     "moe_check": (_c_int, [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]),
     "moe_plan_set_profiling": (_c_int, [_vp, _c_int]),
@@ -194,6 +198,38 @@ class MoEPlan:
             "moe_forward_host_shared")
         return y_host
 
+    def _check_fp8(self, W1q, s1, W3q, s3, W2):
+        E, H, I = self.E, self.H, self.I
+        _check(W1q, "W1q", (E, I, H), torch.uint8, self.device)
+        _check(W3q, "W3q", (E, I, H), torch.uint8, self.device)
+        _check(s1, "s1", (E, I), torch.float32, self.device)
+        _check(s3, "s3", (E, I), torch.float32, self.device)
+        _check(W2, "W2", (E, I, H), torch.bfloat16, self.device)
+
+    def forward_fp8(self, x, Wg, bias, W1q, s1, W3q, s3, W2, y=None, stream=None) -> torch.Tensor:
+        """Forward with the FP8 E4M3 first GEMM; W1q/s1 and W3q/s3 from quantize_weights_fp8."""
+        T = self._check_inputs(x, Wg, bias)
+        self._check_fp8(W1q, s1, W3q, s3, W2)
+        if y is None:
+            y = torch.empty((T, self.H), dtype=torch.bfloat16, device=self.device)
+        _check(y, "y", (T, self.H), torch.bfloat16, self.device)
+        _ok(self.lib.moe_forward_fp8(self._plan, _ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1q), _ptr(s1), _ptr(W3q),
+                                     _ptr(s3), _ptr(W2), T, _ptr(y), _stream_handle(stream, self.device)),
+            "moe_forward_fp8")
+        return y
+
+    def forward_host_fp8(self, x_host, Wg, bias, W1q, s1, W3q, s3, W2, y_host, stream=None):
+        """forward_fp8 with x_host / y_host CPU bf16 tensors (pinned for asynchronous copies)."""
+        T = x_host.shape[0]
+        _check(x_host, "x_host", (T, self.H), torch.bfloat16, torch.device("cpu"))
+        _check(y_host, "y_host", (T, self.H), torch.bfloat16, torch.device("cpu"))
+        _check(Wg, "Wg", (self.H, self.E), torch.bfloat16, self.device)
+        self._check_fp8(W1q, s1, W3q, s3, W2)
+        _ok(self.lib.moe_forward_host_fp8(self._plan, _ptr(x_host), _ptr(Wg), _ptr(bias), _ptr(W1q), _ptr(s1),
+                                          _ptr(W3q), _ptr(s3), _ptr(W2), T, _ptr(y_host),
+                                          _stream_handle(stream, self.device)), "moe_forward_host_fp8")
+        return y_host
+
     def route(self, x, Wg, bias, stream=None):
         T = self._check_inputs(x, Wg, bias)
         _ok(self.lib.moe_route(self._plan, _ptr(x), _ptr(Wg), _ptr(bias), T,
@@ -263,6 +299,32 @@ class MoEPlan:
             self.close()
         except Exception:
             pass
+
+
+def quantize_weights_fp8(W: torch.Tensor, stream=None):
+    """W bf16 [E, H, I] (W1 or W3) -> (K-major E4M3 codes u8 [E, I, H], column scales fp32 [E, I])."""
+    if not isinstance(W, torch.Tensor) or W.dim() != 3:
+        raise TypeError("W must be a 3-D torch.Tensor [E, H, I]")
+    E, H, I = W.shape
+    _check(W, "W", (E, H, I), torch.bfloat16, None)
+    Wq = torch.empty((E, I, H), dtype=torch.uint8, device=W.device)
+    sc = torch.empty((E, I), dtype=torch.float32, device=W.device)
+    _ok(load_library().moe_quantize_weights_fp8(_ptr(W), _ptr(Wq), _ptr(sc), E, H, I,
+                                                _stream_handle(stream, W.device)), "moe_quantize_weights_fp8")
+    return Wq, sc
+
+
+def quantize_x_fp8(x: torch.Tensor, stream=None):
+    """x bf16 [T, H] -> (E4M3 codes u8 [T, H], per-token scales fp32 [T]), as the FP8 forward forms them."""
+    if not isinstance(x, torch.Tensor) or x.dim() != 2:
+        raise TypeError("x must be a 2-D torch.Tensor [T, H]")
+    T, H = x.shape
+    _check(x, "x", (T, H), torch.bfloat16, None)
+    xq = torch.empty((T, H), dtype=torch.uint8, device=x.device)
+    sx = torch.empty((T,), dtype=torch.float32, device=x.device)
+    _ok(load_library().moe_quantize_x_fp8(_ptr(x), _ptr(xq), _ptr(sx), T, H, _stream_handle(stream, x.device)),
+        "moe_quantize_x_fp8")
+    return xq, sx
 
 
 def kernels_per_forward() -> int:

@@ -37,8 +37,8 @@ namespace moe {
 
 struct GemmParams {
   const bf16* x;       // [T, H]
-  CUtensorMap tm_w1;   // W1 as [E*H, I], box {64, 64}
-  CUtensorMap tm_w3;   // W3 as [E*H, I], box {64, 64}
+  CUtensorMap tm_w1;   // W1 as [E*H, I], box {64, 64}; FP8 first GEMM: W1q as [E*I, H] bytes, box {128, 64}
+  CUtensorMap tm_w3;   // W3 likewise
   CUtensorMap tm_w2;   // W2 as [E*I, H], box {64, 64}
   CUtensorMap tm_ws1;  // shared experts' W1 as [S*H, I] (experts E .. E+S-1; unused when S = 0)
   CUtensorMap tm_ws3;  // shared experts' W3 as [S*H, I]
@@ -57,6 +57,13 @@ struct GemmParams {
   float* y_acc;                 // [T, H]
   int T, H, I, E, k, BM, BN2, N1, N2;
   int S;                        // shared experts (0 .. kMaxShared)
+  // FP8 E4M3 first GEMM (fp8 != 0): x codes [T, H] with per-token scales,
+  // W1/W3 codes K-major [E, I, H] (tensor maps above) with column scales [E, I]
+  int fp8;
+  const uint8_t* xq;
+  const float* sx;
+  const float* s1;
+  const float* s3;
   int ring_blocks;              // block b uses ring slot b % ring_blocks
   int max_groups;
   unsigned long long timeout_ns;
@@ -200,6 +207,9 @@ __device__ __forceinline__ Task decode_task(int t, const GemmSmem& s, const Gemm
 
 __device__ __forceinline__ uint8_t* stage_ptr(uint8_t* tiles, int stage) { return tiles + stage * kStageBytes; }
 
+// K blocks of an L1 task: 64 bf16 or 128 FP8 elements, one 128-byte swizzle row either way.
+__device__ __forceinline__ int l1_ksteps(const GemmParams& p) { return p.fp8 ? p.H / 128 : p.H / kBK; }
+
 // ---------------------------------------------------------------- scheduler (last warp)
 // Claims tasks from the global counter, decodes them, stages the routed row
 // indices of L1 tasks in s.rows[q] and waits for the L1 tiles an L2 task
@@ -314,7 +324,7 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
     }
     if (task.phase < 0) break;
 
-    const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
+    const int nk = task.phase == 0 ? l1_ksteps(p) : p.I / kBK;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait(&s.empty[stage], phase ^ 1, p, s, 2)) {
         ok = false;
@@ -326,14 +336,23 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
         // B: 128 columns of W1 next to the same 128 of W3; A comes from the gather warps.
         if (lane == 0) {
           ptx::mbar_arrive_expect_tx(&s.full[stage], 4 * kBoxBytes);
-          const bool sh = task.e >= p.E;   // shared expert: its own weight tensors
-          const int wrow = (sh ? task.e - p.E : task.e) * p.H + kb * kBK;
           const int n0 = task.n * kL1TileN;
-          const CUtensorMap* m1 = sh ? &p.tm_ws1 : &p.tm_w1;
-          const CUtensorMap* m3 = sh ? &p.tm_ws3 : &p.tm_w3;
+          if (p.fp8) {
+            // K-major FP8 codes: 64 rows (columns of I) x 128 bytes (K) per box
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            ptx::tma_load_2d(b_addr + j * kBoxBytes, j < 2 ? m1 : m3, &s.full[stage], n0 + (j & 1) * 64, wrow, pol);
+            for (int j = 0; j < 4; ++j)
+              ptx::tma_load_2d(b_addr + j * kBoxBytes, j < 2 ? &p.tm_w1 : &p.tm_w3, &s.full[stage], kb * 128,
+                               task.e * p.I + n0 + (j & 1) * 64, pol);
+          } else {
+            const bool sh = task.e >= p.E;   // shared expert: its own weight tensors
+            const int wrow = (sh ? task.e - p.E : task.e) * p.H + kb * kBK;
+            const CUtensorMap* m1 = sh ? &p.tm_ws1 : &p.tm_w1;
+            const CUtensorMap* m3 = sh ? &p.tm_ws3 : &p.tm_w3;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              ptx::tma_load_2d(b_addr + j * kBoxBytes, j < 2 ? m1 : m3, &s.full[stage], n0 + (j & 1) * 64, wrow,
+                               pol);
+          }
         }
       } else {
         // B: 256 (or 128) columns of W2; A (the block's h rows) comes from the gather warps.
@@ -370,7 +389,9 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
 // ---------------------------------------------------------------- MMA issuer (warp 1)
 __device__ void gemm_mma(const GemmParams& p, GemmSmem& s, uint8_t* tiles, uint32_t tmem_base) {
   const int lane = ptx::lane_id();
-  const uint32_t idesc_l1 = ptx::idesc_bf16_f32(128, 2 * kL1TileN, false, true);
+  const uint32_t idesc_l1 =
+      p.fp8 ? ptx::idesc_e4m3_f32(128, 2 * kL1TileN) : ptx::idesc_bf16_f32(128, 2 * kL1TileN, false, true);
+  const bool f8 = p.fp8 != 0;
   const uint32_t idesc_l2 = ptx::idesc_bf16_f32(128, p.BN2, false, true);
   int stage = 0;
   uint32_t phase = 0;
@@ -393,7 +414,7 @@ __device__ void gemm_mma(const GemmParams& p, GemmSmem& s, uint8_t* tiles, uint3
     ptx::tc_fence_after();
     const uint32_t d_tmem = tmem_base + acc * 256;
     const uint32_t idesc = task.phase == 0 ? idesc_l1 : idesc_l2;
-    const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
+    const int nk = task.phase == 0 ? l1_ksteps(p) : p.I / kBK;
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait(&s.full[stage], phase, p, s, 5)) {
@@ -406,12 +427,19 @@ __device__ void gemm_mma(const GemmParams& p, GemmSmem& s, uint8_t* tiles, uint3
         const uint32_t a_addr = ptx::smem_u32(stage_ptr(tiles, stage));
         const uint32_t b_addr = a_addr + kTileABytes;
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-          // A: K-major, 128-byte rows, 8-row groups 1024 B apart; step 16 elements = 32 B along K.
+        for (int kk = 0; kk < 4; ++kk) {
+          // A: K-major, 128-byte rows, 8-row groups 1024 B apart; step 32 B along K
+          // (16 bf16 or 32 FP8 elements per MMA).
           const uint64_t ad = ptx::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
-          // B: MN-major, 64-column boxes 8 KB apart, 8-row K groups 1024 B apart; step 16 rows = 2 KB.
-          const uint64_t bd = ptx::smem_desc_sw128(b_addr + kk * 2048, kBoxBytes, 1024);
-          ptx::mma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          if (f8 && task.phase == 0) {
+            // B: K-major FP8 codes, 256 rows of 128 bytes
+            const uint64_t bd = ptx::smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+            ptx::mma_f8(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          } else {
+            // B: MN-major, 64-column boxes 8 KB apart, 8-row K groups 1024 B apart; step 16 rows = 2 KB.
+            const uint64_t bd = ptx::smem_desc_sw128(b_addr + kk * 2048, kBoxBytes, 1024);
+            ptx::mma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
         }
         ptx::mma_commit(&s.empty[stage]);
         issued_any = true;
@@ -469,24 +497,27 @@ __device__ void gemm_gather(const GemmParams& p, GemmSmem& s, uint8_t* tiles, in
     if (task.phase < 0) break;
     // smem offset and source row of each of this lane's rows: L1, the routed x
     // rows (indices staged by the scheduler); L2, the block's h rows in the ring
+    // (byte addresses: a stage takes the next 128 bytes of every row, 64 bf16 or 128 FP8 codes)
     int nrows = 0;
     uint32_t soff[kRowsPerLane];
-    const bf16* src[kRowsPerLane];
+    const uint8_t* src[kRowsPerLane];
     const int* rows = s.rows[q_task];
-    const bf16* hblock = p.h + (size_t)(task.b % p.ring_blocks) * p.BM * p.I;
+    const uint8_t* hblock = reinterpret_cast<const uint8_t*>(p.h + (size_t)(task.b % p.ring_blocks) * p.BM * p.I);
+    const uint8_t* xrows = p.fp8 ? p.xq : reinterpret_cast<const uint8_t*>(p.x);
+    const size_t xpitch = p.fp8 ? (size_t)p.H : (size_t)p.H * 2;
 #pragma unroll
     for (int j = 0; j < kRowsPerLane; ++j) {
       const int r = (j * kGatherWarps + g) * 4 + (lane >> 3);
       soff[j] = r * 128 + ((c ^ (r & 7)) << 4);
-      src[j] = p.x + c * 8;
+      src[j] = xrows + c * 16;
       if (r < p.BM) {
-        src[j] = task.phase == 0 ? p.x + (size_t)rows[r] * p.H + c * 8 : hblock + (size_t)r * p.I + c * 8;
+        src[j] = task.phase == 0 ? xrows + (size_t)rows[r] * xpitch + c * 16 : hblock + (size_t)r * p.I * 2 + c * 16;
         nrows = j + 1;
       }
     }
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive(&s.task_empty[q_task]);   // slot (and its rows) free
-    const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
+    const int nk = task.phase == 0 ? l1_ksteps(p) : p.I / kBK;
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait(&s.empty[stage], phase ^ 1, p, s, 9)) {
@@ -496,7 +527,7 @@ __device__ void gemm_gather(const GemmParams& p, GemmSmem& s, uint8_t* tiles, in
       const uint32_t a_addr = ptx::smem_u32(stage_ptr(tiles, stage));
 #pragma unroll
       for (int j = 0; j < kRowsPerLane; ++j)
-        if (j < nrows) ptx::cp_async_16(a_addr + soff[j], src[j] + kb * kBK);
+        if (j < nrows) ptx::cp_async_16(a_addr + soff[j], src[j] + (size_t)kb * 128);
       ptx::cp_async_mbar_arrive_noinc(&s.full[stage]);
       if (++stage == kStages) {
         stage = 0;
@@ -509,6 +540,24 @@ __device__ void gemm_gather(const GemmParams& p, GemmSmem& s, uint8_t* tiles, in
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+// FP8 first GEMM: g[i] *= sx * s1[col0 + i], u[i] *= sx * s3[col0 + i] for 32 columns
+// (the column scales are the same for every lane: broadcast loads).
+__device__ __forceinline__ void fp8_scale_columns(uint32_t (&g)[32], uint32_t (&u)[32], float tscale,
+                                                  const float* s1, const float* s3, size_t col0) {
+  const float4* a = reinterpret_cast<const float4*>(s1 + col0);
+  const float4* b = reinterpret_cast<const float4*>(s3 + col0);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 sa = __ldg(a + q), sb = __ldg(b + q);
+    const float fa[4] = {sa.x, sa.y, sa.z, sa.w}, fb[4] = {sb.x, sb.y, sb.z, sb.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      g[4 * q + i] = __float_as_uint(__uint_as_float(g[4 * q + i]) * (tscale * fa[i]));
+      u[4 * q + i] = __float_as_uint(__uint_as_float(u[4 * q + i]) * (tscale * fb[i]));
+    }
+  }
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
@@ -607,12 +656,18 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
       }
       const int ring_row = (task.b % p.ring_blocks) * p.BM + r;
       bf16* hrow = p.h + (size_t)ring_row * p.I + task.n * kL1TileN;
+      float tscale = 1.f;   // FP8 first GEMM: the token's scale (padding rows: any)
+      if (p.fp8 && valid) {
+        const int tok = p.slot_token[slot];
+        tscale = (tok >= 0 && tok < p.T) ? p.sx[tok] : 0.f;
+      }
 #pragma unroll 1
       for (int c = 0; c < kL1TileN / 32; ++c) {
         uint32_t g[32], u[32];
         ptx::tmem_ld32(tbase + c * 32, g);
         ptx::tmem_ld32(tbase + kL1TileN + c * 32, u);
         ptx::tmem_ld_wait();
+        if (p.fp8) fp8_scale_columns(g, u, tscale, p.s1, p.s3, (size_t)task.e * p.I + task.n * kL1TileN + c * 32);
         if (store) {
           uint4* dst = reinterpret_cast<uint4*>(hrow + c * 32);
 #pragma unroll

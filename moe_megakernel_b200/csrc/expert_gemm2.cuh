@@ -64,6 +64,13 @@ struct Gemm2Params {
   float* y_acc;                 // [T, H]
   int T, H, I, E, k, BM, BN2, N1, N2;
   int S;                        // shared experts (0 .. kMaxShared)
+  // FP8 E4M3 first GEMM (see GemmParams): x codes, token scales, K-major W1/W3
+  // codes in tm_w1 / tm_w3 (box {128, 64}), column scales
+  int fp8;
+  const uint8_t* xq;
+  const float* sx;
+  const float* s1;
+  const float* s3;
   int ring_pairs, max_groups;
   unsigned long long timeout_ns;
   int withhold_pair;            // test hook: never publish L1 completion of this pair (-1: off)
@@ -223,6 +230,9 @@ __device__ __forceinline__ Task2 decode_task2(int t, const Gemm2Smem& s, const G
 
 __device__ __forceinline__ uint8_t* stage2_ptr(uint8_t* tiles, int stage) { return tiles + stage * kStage2Bytes; }
 
+// K blocks of an L1 task: 64 bf16 or 128 FP8 elements (one 128-byte swizzle row).
+__device__ __forceinline__ int l1_ksteps2(const Gemm2Params& p) { return p.fp8 ? p.H / 128 : p.H / kBK; }
+
 // ---------------------------------------------------------------- leader scheduler (last warp)
 // Claims tasks, decodes them, stages the token rows of both CTAs' A tiles
 // (L1) or waits for the L1 tiles of the pair (L2), and publishes each task in
@@ -347,7 +357,7 @@ __device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_
       qphase ^= 1;
     }
     if (task.phase < 0) break;
-    const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
+    const int nk = task.phase == 0 ? l1_ksteps2(p) : p.I / kBK;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait2(&s.empty[stage], phase ^ 1, p, s, 2)) {
         ok = false;
@@ -360,12 +370,17 @@ __device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_
         // barrier and reaches this one through its relay arrival
         if (task.phase == 0) {
           ptx::mbar_arrive_expect_tx(&s.full[stage], 2 * kBoxBytes);
-          const bool sh = task.e >= p.E;   // shared expert: its own weight tensors
-          const int wrow = (sh ? task.e - p.E : task.e) * p.H + kb * kBK;
           const int n0 = task.n * kL1TileN;
-          const CUtensorMap* m1 = sh ? &p.tm_ws1 : &p.tm_w1;
-          ptx::tma_load_2d(b_addr, m1, &s.full[stage], n0, wrow, pol);
-          ptx::tma_load_2d(b_addr + kBoxBytes, m1, &s.full[stage], n0 + 64, wrow, pol);
+          if (p.fp8) {   // K-major FP8 codes: 64 rows (columns of I) x 128 bytes per box
+            ptx::tma_load_2d(b_addr, &p.tm_w1, &s.full[stage], kb * 128, task.e * p.I + n0, pol);
+            ptx::tma_load_2d(b_addr + kBoxBytes, &p.tm_w1, &s.full[stage], kb * 128, task.e * p.I + n0 + 64, pol);
+          } else {
+            const bool sh = task.e >= p.E;   // shared expert: its own weight tensors
+            const int wrow = (sh ? task.e - p.E : task.e) * p.H + kb * kBK;
+            const CUtensorMap* m1 = sh ? &p.tm_ws1 : &p.tm_w1;
+            ptx::tma_load_2d(b_addr, m1, &s.full[stage], n0, wrow, pol);
+            ptx::tma_load_2d(b_addr + kBoxBytes, m1, &s.full[stage], n0 + 64, wrow, pol);
+          }
         } else {
           // L2: both operands come from the A-row warps' cp.async (a TMA box of
           // W2 kept the tensor pipe waiting); only this arrival is the producer's
@@ -432,7 +447,7 @@ __device__ void gemm2_follower_producer(const Gemm2Params& p, Gemm2Smem& s, uint
     Task2 task;
     if (!pop_task2(task, q, qphase, nullptr, false, p, s, 3, true)) break;
     if (task.phase < 0) break;
-    const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
+    const int nk = task.phase == 0 ? l1_ksteps2(p) : p.I / kBK;
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait2(&s.empty[stage], phase ^ 1, p, s, 4)) {
@@ -444,12 +459,17 @@ __device__ void gemm2_follower_producer(const Gemm2Params& p, Gemm2Smem& s, uint
         const uint32_t b_addr = a_addr + kTileABytes;
         if (task.phase == 0) {
           ptx::mbar_arrive_expect_tx(&s.full[stage], 2 * kBoxBytes);
-          const bool sh = task.e >= p.E;
-          const int wrow = (sh ? task.e - p.E : task.e) * p.H + kb * kBK;
           const int n0 = task.n * kL1TileN;
-          const CUtensorMap* m3 = sh ? &p.tm_ws3 : &p.tm_w3;
-          ptx::tma_load_2d(b_addr, m3, &s.full[stage], n0, wrow, pol);
-          ptx::tma_load_2d(b_addr + kBoxBytes, m3, &s.full[stage], n0 + 64, wrow, pol);
+          if (p.fp8) {
+            ptx::tma_load_2d(b_addr, &p.tm_w3, &s.full[stage], kb * 128, task.e * p.I + n0, pol);
+            ptx::tma_load_2d(b_addr + kBoxBytes, &p.tm_w3, &s.full[stage], kb * 128, task.e * p.I + n0 + 64, pol);
+          } else {
+            const bool sh = task.e >= p.E;
+            const int wrow = (sh ? task.e - p.E : task.e) * p.H + kb * kBK;
+            const CUtensorMap* m3 = sh ? &p.tm_ws3 : &p.tm_w3;
+            ptx::tma_load_2d(b_addr, m3, &s.full[stage], n0, wrow, pol);
+            ptx::tma_load_2d(b_addr + kBoxBytes, m3, &s.full[stage], n0 + 64, wrow, pol);
+          }
         } else {
           ptx::mbar_arrive(&s.full[stage]);   // L2: operands by the A-row warps (see the leader)
         }
@@ -478,7 +498,7 @@ __device__ void gemm2_follower_relay(const Gemm2Params& p, Gemm2Smem& s) {
     Task2 task;
     if (!pop_task2(task, q, qphase, nullptr, false, p, s, 5, true)) break;
     if (task.phase < 0) break;
-    const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
+    const int nk = task.phase == 0 ? l1_ksteps2(p) : p.I / kBK;
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait2(&s.full[stage], phase, p, s, 6)) {
@@ -502,7 +522,9 @@ __device__ void gemm2_follower_relay(const Gemm2Params& p, Gemm2Smem& s) {
 // ---------------------------------------------------------------- leader warp 1: MMA issuer
 __device__ void gemm2_mma(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, uint32_t tmem_base) {
   const int lane = ptx::lane_id();
-  const uint32_t idesc_l1 = ptx::idesc_bf16_f32(256, 2 * kL1TileN, false, true);
+  const uint32_t idesc_l1 =
+      p.fp8 ? ptx::idesc_e4m3_f32(256, 2 * kL1TileN) : ptx::idesc_bf16_f32(256, 2 * kL1TileN, false, true);
+  const bool f8 = p.fp8 != 0;
   const uint32_t idesc_l2 = ptx::idesc_bf16_f32(256, p.BN2, false, true);
   int stage = 0;
   uint32_t phase = 0;
@@ -519,7 +541,7 @@ __device__ void gemm2_mma(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, ui
     ptx::tc_fence_after();
     const uint32_t d_tmem = tmem_base + acc * 256;
     const uint32_t idesc = task.phase == 0 ? idesc_l1 : idesc_l2;
-    const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
+    const int nk = task.phase == 0 ? l1_ksteps2(p) : p.I / kBK;
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait2(&s.full[stage], phase, p, s, 9)) {
@@ -532,10 +554,16 @@ __device__ void gemm2_mma(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, ui
         const uint32_t a_addr = ptx::smem_u32(stage2_ptr(tiles, stage));
         const uint32_t b_addr = a_addr + kTileABytes;
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
+        for (int kk = 0; kk < 4; ++kk) {
           const uint64_t ad = ptx::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
-          const uint64_t bd = ptx::smem_desc_sw128(b_addr + kk * 2048, kBoxBytes, 1024);
-          ptx::mma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          if (f8 && task.phase == 0) {
+            // B half: K-major FP8 codes, 128 rows of 128 bytes in each CTA
+            const uint64_t bd = ptx::smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+            ptx::mma_f8_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          } else {
+            const uint64_t bd = ptx::smem_desc_sw128(b_addr + kk * 2048, kBoxBytes, 1024);
+            ptx::mma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
         }
         ptx::mma_commit_pair_multicast(&s.empty[stage], 0x3);
         issued_any = true;
@@ -597,12 +625,18 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
       }
       const int ring_row = ((task.p % p.ring_pairs) * 2 + (int)rank) * p.BM + r;
       bf16* hrow = p.h + (size_t)ring_row * p.I + task.n * kL1TileN;
+      float tscale = 1.f;   // FP8 first GEMM: the token's scale (padding rows: any)
+      if (p.fp8 && valid) {
+        const int tok = p.slot_token[slot];
+        tscale = (tok >= 0 && tok < p.T) ? p.sx[tok] : 0.f;
+      }
 #pragma unroll 1
       for (int c = 0; c < kL1TileN / 32; ++c) {
         uint32_t g[32], u[32];
         ptx::tmem_ld32(tbase + c * 32, g);
         ptx::tmem_ld32(tbase + kL1TileN + c * 32, u);
         ptx::tmem_ld_wait();
+        if (p.fp8) fp8_scale_columns(g, u, tscale, p.s1, p.s3, (size_t)task.e * p.I + task.n * kL1TileN + c * 32);
         if (store) {
           uint4* dst = reinterpret_cast<uint4*>(hrow + c * 32);
 #pragma unroll
@@ -687,18 +721,22 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
     const int b_own = rank == 0 ? task.b0 : task.b1;
     int nrows = 0;
     uint32_t soff[kRowsPerLane];
-    const bf16* src[kRowsPerLane];
+    const uint8_t* src[kRowsPerLane];   // byte addresses; a stage takes the next 128 bytes of a row
     if (b_own >= 0) {
-      // L1: the routed x rows of this CTA's block; L2: its h rows in the ring
+      // L1: the routed x rows (bf16, or FP8 codes) of this CTA's block; L2: its h rows in the ring
       const int* rows = s.rows[q_task];
-      const bf16* hblock = p.h + (size_t)((task.p % p.ring_pairs) * 2 + (int)rank) * p.BM * p.I;
+      const uint8_t* hblock =
+          reinterpret_cast<const uint8_t*>(p.h + (size_t)((task.p % p.ring_pairs) * 2 + (int)rank) * p.BM * p.I);
+      const uint8_t* xrows = p.fp8 ? p.xq : reinterpret_cast<const uint8_t*>(p.x);
+      const size_t xpitch = p.fp8 ? (size_t)p.H : (size_t)p.H * 2;
 #pragma unroll
       for (int j = 0; j < kRowsPerLane; ++j) {
         const int rr = (j * kGatherWarps + g) * 4 + (lane >> 3);
         soff[j] = rr * 128 + ((c ^ (rr & 7)) << 4);
-        src[j] = p.x + c * 8;
+        src[j] = xrows + c * 16;
         if (rr < p.BM) {
-          src[j] = task.phase == 0 ? p.x + (size_t)rows[rr] * p.H + c * 8 : hblock + (size_t)rr * p.I + c * 8;
+          src[j] = task.phase == 0 ? xrows + (size_t)rows[rr] * xpitch + c * 16
+                                   : hblock + (size_t)rr * p.I * 2 + c * 16;
           nrows = j + 1;
         }
       }
@@ -709,7 +747,7 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
     const int nhalf = task.phase == 1 ? p.BN2 / 128 : 0;
     const bf16* w2src = (task.e >= p.E ? p.ws2 + (size_t)(task.e - p.E) * p.I * p.H : p.w2 + (size_t)task.e * p.I * p.H) +
                         task.n * p.BN2 + (int)rank * (p.BN2 / 2) + c * 8;
-    const int nk = task.phase == 0 ? p.H / kBK : p.I / kBK;
+    const int nk = task.phase == 0 ? l1_ksteps2(p) : p.I / kBK;
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait2(&s.empty[stage], phase ^ 1, p, s, 13)) {
@@ -719,7 +757,7 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
       const uint32_t a_addr = ptx::smem_u32(stage2_ptr(tiles, stage));
 #pragma unroll
       for (int j = 0; j < kRowsPerLane; ++j)
-        if (j < nrows) ptx::cp_async_16(a_addr + soff[j], src[j] + kb * kBK);
+        if (j < nrows) ptx::cp_async_16(a_addr + soff[j], src[j] + (size_t)kb * 128);
       for (int j = 0; j < nhalf; ++j) {
 #pragma unroll
         for (int i = 0; i < 64 / 4 / kGatherWarps; ++i) {

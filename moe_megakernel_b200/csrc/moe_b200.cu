@@ -16,6 +16,7 @@
 #include "dispatch.cuh"
 #include "expert_gemm.cuh"
 #include "expert_gemm2.cuh"
+#include "quant.cuh"
 #include "router.cuh"
 #include "router_tc.cuh"
 
@@ -31,7 +32,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 struct Layout {
   size_t err, sched, topk_idx, topk_w, rank, chunk_count, expert_count, expert_offset, block_start, num_padded,
       slot_token, slot_topk, l1_done, l2_done, group_start, pair_start, router_partial, router_counter, h, y_acc,
-      x_stage, y_stage, total;
+      x_stage, y_stage, x_q, s_x, total;
 };
 
 class DeviceGuard {
@@ -72,6 +73,20 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2D FP8 (byte) tensor map of K-major codes: `inner` bytes per row, `rows`
+// rows, box {128, 64} (one 128-byte swizzle row per box row), 128-byte swizzle.
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {128, 64};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -153,6 +168,8 @@ static Layout make_layout(const moe_plan& p) {
   L.y_acc = take((size_t)p.T_max * p.H * 4, 1024);
   L.x_stage = take((size_t)p.T_max * p.H * 2, 1024);
   L.y_stage = take((size_t)p.T_max * p.H * 2, 1024);
+  L.x_q = take((size_t)p.T_max * p.H, 1024);   // FP8 first GEMM: x codes and token scales
+  L.s_x = take((size_t)p.T_max * 4, 256);
   L.total = align_up(o, 1024);
   return L;
 }
@@ -196,13 +213,28 @@ struct SharedWeights {
   const void* Ws2;   // [S, I, H]
 };
 
+// FP8 E4M3 first GEMM: K-major codes of W1 / W3 [E, I, H] and their column scales [E, I].
+struct Fp8First {
+  const void* W1q;
+  const float* s1;
+  const void* W3q;
+  const float* s3;
+};
+
 static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias, const void* W1, const void* W3,
-                   const void* W2, const SharedWeights& sw, int T, void* y, cudaStream_t st, bool full) {
+                   const void* W2, const SharedWeights& sw, int T, void* y, cudaStream_t st, bool full,
+                   const Fp8First* f8 = nullptr) {
   if (p->ws == nullptr) return MOE_ERR_NO_WORKSPACE;
   if (T < 0 || T > p->T_max) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;   // nothing to do; empty tensors may carry null pointers
   if (x == nullptr || Wg == nullptr || !aligned16(x) || !aligned16(Wg)) return MOE_ERR_INVALID_ARG;
   if (bias != nullptr && (reinterpret_cast<uintptr_t>(bias) & 3u)) return MOE_ERR_INVALID_ARG;
+  if (f8 != nullptr) {   // the FP8 operands stand in for W1 / W3
+    if (p->S > 0 || f8->s1 == nullptr || f8->s3 == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(f8->s1) || !aligned16(f8->s3)) return MOE_ERR_INVALID_ARG;
+    W1 = f8->W1q;
+    W3 = f8->W3q;
+  }
   if (full) {
     if (W1 == nullptr || W3 == nullptr || W2 == nullptr || y == nullptr) return MOE_ERR_INVALID_ARG;
     if (!aligned16(W1) || !aligned16(W3) || !aligned16(W2) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
@@ -239,6 +271,11 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   rp.k = p->k;
   const int splits = router_splits(T, p->H, p->num_sms);
   mark(0);
+  if (f8 != nullptr) {   // x codes and token scales for the FP8 first GEMM
+    moe_quantize_x_kernel<<<(T + 7) / 8, 256, 0, st>>>(static_cast<const bf16*>(x), ws + L.x_q,
+                                                       reinterpret_cast<float*>(ws + L.s_x), T, p->H);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  }
   if (p->E % 64 == 0 && splits == 1) {
     // many tokens, E a multiple of 64: gate GEMM on tcgen05
     RouterTcParams tp;
@@ -318,13 +355,21 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   if (p->cta_pairs) {
     Gemm2Params gp;
     std::memset(&gp, 0, sizeof(gp));
-    bool ok = make_map(&gp.tm_w1, W1, I, (uint64_t)E * H, I, 64) &&
-              make_map(&gp.tm_w3, W3, I, (uint64_t)E * H, I, 64);
+    bool ok = f8 != nullptr ? make_map_u8(&gp.tm_w1, W1, H, (uint64_t)E * I) && make_map_u8(&gp.tm_w3, W3, H, (uint64_t)E * I)
+                            : make_map(&gp.tm_w1, W1, I, (uint64_t)E * H, I, 64) &&
+                                  make_map(&gp.tm_w3, W3, I, (uint64_t)E * H, I, 64);
     if (ok && p->S > 0)
       ok = make_map(&gp.tm_ws1, sw.Ws1, I, (uint64_t)p->S * H, I, 64) &&
            make_map(&gp.tm_ws3, sw.Ws3, I, (uint64_t)p->S * H, I, 64);
     if (!ok) return MOE_ERR_CUDA;
     gp.x = static_cast<const bf16*>(x);
+    if (f8 != nullptr) {
+      gp.fp8 = 1;
+      gp.xq = ws + L.x_q;
+      gp.sx = reinterpret_cast<const float*>(ws + L.s_x);
+      gp.s1 = f8->s1;
+      gp.s3 = f8->s3;
+    }
     gp.w2 = static_cast<const bf16*>(W2);
     gp.ws2 = static_cast<const bf16*>(sw.Ws2);
     gp.S = p->S;
@@ -371,8 +416,10 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   } else {
     GemmParams gp;
     std::memset(&gp, 0, sizeof(gp));
-    bool ok = make_map(&gp.tm_w1, W1, I, (uint64_t)E * H, I, 64) &&
-              make_map(&gp.tm_w3, W3, I, (uint64_t)E * H, I, 64) &&
+    bool ok = (f8 != nullptr ? make_map_u8(&gp.tm_w1, W1, H, (uint64_t)E * I) &&
+                                   make_map_u8(&gp.tm_w3, W3, H, (uint64_t)E * I)
+                             : make_map(&gp.tm_w1, W1, I, (uint64_t)E * H, I, 64) &&
+                                   make_map(&gp.tm_w3, W3, I, (uint64_t)E * H, I, 64)) &&
               make_map(&gp.tm_w2, W2, H, (uint64_t)E * I, H, 64);
     if (ok && p->S > 0)
       ok = make_map(&gp.tm_ws1, sw.Ws1, I, (uint64_t)p->S * H, I, 64) &&
@@ -381,6 +428,13 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     if (!ok) return MOE_ERR_CUDA;
     gp.S = p->S;
     gp.x = static_cast<const bf16*>(x);
+    if (f8 != nullptr) {
+      gp.fp8 = 1;
+      gp.xq = ws + L.x_q;
+      gp.sx = reinterpret_cast<const float*>(ws + L.s_x);
+      gp.s1 = f8->s1;
+      gp.s3 = f8->s3;
+    }
     gp.slot_token = dp.slot_token;
     gp.slot_topk = dp.slot_topk;
     gp.topk_w = rp.topk_w;
@@ -746,7 +800,8 @@ int moe_route(moe_plan_t p, const void* x, const void* Wg, const float* bias, in
 }
 
 static int forward_host(moe_plan_t p, const void* x_host, const void* Wg, const float* bias, const void* W1,
-                        const void* W3, const void* W2, const SharedWeights& sw, int T, void* y_host, void* stream) {
+                        const void* W3, const void* W2, const SharedWeights& sw, int T, void* y_host, void* stream,
+                        const Fp8First* f8 = nullptr) {
   if (p == nullptr || x_host == nullptr || y_host == nullptr) return MOE_ERR_INVALID_ARG;
   if (p->ws == nullptr) return MOE_ERR_NO_WORKSPACE;
   if (T < 0 || T > p->T_max) return MOE_ERR_INVALID_ARG;
@@ -757,7 +812,7 @@ static int forward_host(moe_plan_t p, const void* x_host, const void* Wg, const 
   void* xd = p->ws + p->L.x_stage;
   void* yd = p->ws + p->L.y_stage;
   if (cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return MOE_ERR_CUDA;
-  const int rc = enqueue(p, xd, Wg, bias, W1, W3, W2, sw, T, yd, st, true);
+  const int rc = enqueue(p, xd, Wg, bias, W1, W3, W2, sw, T, yd, st, true, f8);
   if (rc != MOE_OK) return rc;
   if (cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
@@ -773,6 +828,47 @@ int moe_forward_host_shared(moe_plan_t p, const void* x_host, const void* Wg, co
                             const void* W3, const void* W2, const void* Ws1, const void* Ws3, const void* Ws2, int T,
                             void* y_host, void* stream) {
   return forward_host(p, x_host, Wg, bias, W1, W3, W2, SharedWeights{Ws1, Ws3, Ws2}, T, y_host, stream);
+}
+
+int moe_forward_fp8(moe_plan_t p, const void* x, const void* Wg, const float* bias, const void* W1q, const float* s1,
+                    const void* W3q, const float* s3, const void* W2, int T, void* y, void* stream) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  const Fp8First f8{W1q, s1, W3q, s3};
+  return enqueue(p, x, Wg, bias, nullptr, nullptr, W2, SharedWeights{}, T, y, static_cast<cudaStream_t>(stream), true,
+                 &f8);
+}
+
+int moe_forward_host_fp8(moe_plan_t p, const void* x_host, const void* Wg, const float* bias, const void* W1q,
+                         const float* s1, const void* W3q, const float* s3, const void* W2, int T, void* y_host,
+                         void* stream) {
+  const Fp8First f8{W1q, s1, W3q, s3};
+  return forward_host(p, x_host, Wg, bias, nullptr, nullptr, W2, SharedWeights{}, T, y_host, stream, &f8);
+}
+
+int moe_quantize_x_fp8(const void* x, void* xq, float* sx, int T, int H, void* stream) {
+  if (T < 0 || H < 8 || H % 8) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (x == nullptr || xq == nullptr || sx == nullptr || !aligned16(x) || (reinterpret_cast<uintptr_t>(xq) & 7u) ||
+      (reinterpret_cast<uintptr_t>(sx) & 3u))
+    return MOE_ERR_INVALID_ARG;
+  moe_quantize_x_kernel<<<(T + 7) / 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const bf16*>(x), static_cast<uint8_t*>(xq), sx, T, H);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_quantize_weights_fp8(const void* W, void* Wq, float* scale, int E, int H, int I, void* stream) {
+  if (E < 1 || H < 64 || H % 64 || I < 64 || I % 64) return MOE_ERR_INVALID_ARG;
+  if (W == nullptr || Wq == nullptr || scale == nullptr || !aligned16(Wq) || (reinterpret_cast<uintptr_t>(W) & 1u) ||
+      (reinterpret_cast<uintptr_t>(scale) & 3u))
+    return MOE_ERR_INVALID_ARG;
+  if (E > 65535 || (long long)E * H * I > (1LL << 40)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  moe_weight_scales_kernel<<<dim3((unsigned)(I / 32), (unsigned)E), 256, 0, st>>>(static_cast<const bf16*>(W), scale,
+                                                                                 H, I);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  moe_weight_quant_kernel<<<dim3((unsigned)(I / 64), (unsigned)(H / 64), (unsigned)E), 256, 0, st>>>(
+      static_cast<const bf16*>(W), scale, static_cast<uint8_t*>(Wq), H, I);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int moe_check(moe_plan_t p, void* stream, int32_t* detail) {

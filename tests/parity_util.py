@@ -35,14 +35,14 @@ def expert_loader(W1: torch.Tensor, W3: torch.Tensor, W2: torch.Tensor):
     return load
 
 
-def oracle_forward(inp: dict, tokens=None, block_m=None):
+def oracle_forward(inp: dict, tokens=None, block_m=None, fp8: bool = False):
     x = to_f64(inp["x"])
     Wg = to_f64(inp["Wg"])
     bias = None if inp["bias"] is None else to_f64(inp["bias"])
     S = inp.get("n_shared", 0)
     shared = expert_loader(inp["Ws1"], inp["Ws3"], inp["Ws2"]) if S else None
     return O.moe_forward(x, Wg, bias, expert_loader(inp["W1"], inp["W3"], inp["W2"]), inp["k"],
-                         block_m=block_m, tokens=tokens, shared_weights=shared, n_shared=S)
+                         block_m=block_m, tokens=tokens, shared_weights=shared, n_shared=S, fp8=fp8)
 
 
 def oracle_route(inp: dict, block_m: int):

@@ -1,0 +1,176 @@
+"""FP8 E4M3 first GEMM on the GPU against the oracle.
+
+"MegaMoE 在 MoE 系统谱系中的位置", section 一 (the expert GEMMs take 8-bit
+operands with scale factors beside them) and section 2.1 (activation amax and
+quantization): x is quantized per token, W1 / W3 per (expert, column), with
+power-of-two scales, and x.W1, x.W3 run on tcgen05 kind::f8f6f4; h and W2
+stay bf16. Codes and scales are compared bit-exactly with the oracle's
+(both sides convert the same fp32 / fp64-exact quotient with round to nearest
+even), y with the layer tolerances on the oracle's FP8 layer.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.moe_oracle as O
+from synth.moe_inputs import WORKLOADS, custom_shape, make_inputs
+from tests.parity_util import assert_routing_equal, assert_y_close, oracle_forward, sample_tokens, to_f64
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """Value of each E4M3 byte: sign, 4 exponent bits (bias 7), 3 mantissa bits;
+    exponent 0 is subnormal (m/8 * 2**-6); 0x7f / 0xff are NaN."""
+    b = codes.astype(np.int64)
+    s = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 15
+    m = b & 7
+    v = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1 + m / 8.0) * np.ldexp(1.0, e - 7))
+    v = np.where((b & 0x7F) == 0x7F, np.nan, v)
+    return s * v
+
+
+def _x_cases(T=261, H=512, seed=3):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn((T, H), generator=g)
+    x *= torch.exp2(torch.randint(-24, 24, (T, 1), generator=g).float())   # scales across 48 binades
+    x[0] = 0.0                          # amax 0: scale 1, codes 0
+    x[1, :] = 0.001
+    x[1, 7] = 448.0 * 8                 # amax exactly 448 * 2**3: scale 8, code 448
+    x[2, :] = 1.0 + 1.0 / 16           # halfway between E4M3 1.0 and 1.125 after scaling by 1
+    x[2, 0] = 300.0
+    x[3, :] = -2.0 ** -10               # E4M3 subnormal range after scaling
+    x[3, 1] = 1.0
+    return x.to(torch.bfloat16)
+
+
+def test_quantize_x_codes_and_scales_match_oracle():
+    from moe_megakernel_b200 import quantize_x_fp8
+    x = _x_cases()
+    xq, sx = quantize_x_fp8(x.to(DEV))
+    torch.cuda.synchronize()
+    codes_ref, sc_ref = O.quantize_fp8(to_f64(x), axis=1)
+    np.testing.assert_array_equal(sx.cpu().numpy().astype(np.float64), sc_ref[:, 0])
+    np.testing.assert_array_equal(e4m3_decode(xq.cpu().numpy()), codes_ref)
+    assert sx[0].item() == 1.0 and sx[1].item() == 8.0
+    assert (xq[0] == 0).all()
+
+
+def test_quantize_weights_codes_and_scales_match_oracle():
+    from moe_megakernel_b200 import quantize_weights_fp8
+    E, H, I = 3, 320, 192
+    g = torch.Generator().manual_seed(5)
+    W = torch.randn((E, H, I), generator=g) * 0.02
+    W *= torch.exp2(torch.randint(-6, 6, (E, 1, I), generator=g).float())   # per-column magnitudes
+    W[1, :, 5] = 0.0                                                        # an all-zero column
+    W = W.to(torch.bfloat16)
+    Wq, sc = quantize_weights_fp8(W.to(DEV))
+    torch.cuda.synchronize()
+    assert Wq.shape == (E, I, H) and sc.shape == (E, I)
+    Wq, sc = Wq.cpu().numpy(), sc.cpu().numpy().astype(np.float64)
+    for e in range(E):
+        codes_ref, s_ref = O.quantize_fp8(to_f64(W[e]), axis=0)   # [H, I], [1, I]
+        np.testing.assert_array_equal(sc[e], s_ref[0])
+        np.testing.assert_array_equal(e4m3_decode(Wq[e]).T, codes_ref)
+    assert sc[1, 5] == 1.0
+
+
+SHAPES = [
+    # T,   H,   I,   E,  k, block_m, zipf
+    (64, 128, 256, 8, 2, 0, False),
+    (300, 256, 384, 16, 4, 0, False),    # H % 256 != 0
+    (129, 384, 256, 32, 8, 0, True),     # ragged T, bias
+    (1000, 256, 512, 8, 2, 0, False),    # several full blocks per expert
+    (40, 256, 256, 64, 8, 0, False),     # BLOCK_M 16 (decode-like)
+    (500, 512, 256, 16, 2, 32, False),   # forced BLOCK_M 32
+    (500, 512, 256, 16, 2, 64, False),   # forced BLOCK_M 64
+]
+
+
+def _fp8_weights(inp):
+    from moe_megakernel_b200 import quantize_weights_fp8
+    W1q, s1 = quantize_weights_fp8(inp["W1"])
+    W3q, s3 = quantize_weights_fp8(inp["W3"])
+    return W1q, s1, W3q, s3
+
+
+@pytest.mark.parametrize("pairs", [True, False], ids=["pairs", "single"])
+@pytest.mark.parametrize("T,H,I,E,k,bm,zipf", SHAPES)
+def test_fp8_forward_matches_oracle(T, H, I, E, k, bm, zipf, pairs):
+    from moe_megakernel_b200 import MoEPlan
+    shape = custom_shape(T, H, I, E, k, zipf)
+    inp = make_inputs(shape, device=DEV)
+    plan = MoEPlan(T, H, I, E, k, block_m=bm)
+    plan.set_cta_pairs(pairs)
+    plan.workspace.fill_(0xFF)   # poison: unwritten reads show up as NaN
+    plan.lib.moe_plan_bind_workspace(plan._plan, plan.workspace.data_ptr(), plan.workspace_bytes)
+    W1q, s1, W3q, s3 = _fp8_weights(inp)
+    y = plan.forward_fp8(inp["x"], inp["Wg"], inp["bias"], W1q, s1, W3q, s3, inp["W2"])
+    plan.check()
+    ref = oracle_forward(inp, block_m=plan.block_m, fp8=True)
+    assert_routing_equal(plan.routing(T), ref)
+    fro, mx = assert_y_close(y, ref["y"], "y (fp8)")
+    # the FP8 layer differs from the bf16 one by the quantization, well above the kernel's own error
+    ref16 = oracle_forward(inp, block_m=plan.block_m)
+    q_err = np.linalg.norm(ref["y"] - ref16["y"]) / np.linalg.norm(ref16["y"])
+    print(f"fp8 {'pairs' if pairs else 'single'} T={T} H={H} I={I} E={E} k={k} BM={plan.block_m}: "
+          f"rel_fro={fro:.2e} max_abs={mx:.2e} (fp8 vs bf16 layer {q_err:.2e})")
+
+
+def test_fp8_forward_rejects_shared_plan_and_bad_pointers():
+    from moe_megakernel_b200 import MoEPlan
+    shape = custom_shape(64, 128, 256, 8, 2)
+    inp = make_inputs(shape, device=DEV)
+    W1q, s1, W3q, s3 = _fp8_weights(inp)
+    y = torch.empty_like(inp["x"])
+    shared = MoEPlan(64, 128, 256, 8, 2, n_shared=1)
+    rc = shared.lib.moe_forward_fp8(shared._plan, inp["x"].data_ptr(), inp["Wg"].data_ptr(), None,
+                                    W1q.data_ptr(), s1.data_ptr(), W3q.data_ptr(), s3.data_ptr(),
+                                    inp["W2"].data_ptr(), 64, y.data_ptr(), None)
+    assert rc == 1   # MOE_ERR_INVALID_ARG: FP8 first GEMM without shared experts
+    plan = MoEPlan(64, 128, 256, 8, 2)
+    rc = plan.lib.moe_forward_fp8(plan._plan, inp["x"].data_ptr(), inp["Wg"].data_ptr(), None,
+                                  W1q.data_ptr(), None, W3q.data_ptr(), s3.data_ptr(),
+                                  inp["W2"].data_ptr(), 64, y.data_ptr(), None)
+    assert rc == 1   # missing column scales
+    with pytest.raises(ValueError):
+        plan.forward_fp8(inp["x"], inp["Wg"], None, inp["W1"], s1, W3q, s3, inp["W2"])   # bf16 W1: wrong layout
+    shared.check()
+    plan.check()
+
+
+def test_fp8_host_entry_matches_device_entry():
+    from moe_megakernel_b200 import MoEPlan
+    shape = custom_shape(300, 256, 384, 16, 4)
+    inp = make_inputs(shape, device=DEV)
+    W1q, s1, W3q, s3 = _fp8_weights(inp)
+    plan = MoEPlan(shape.T, shape.H, shape.I, shape.E, shape.k)
+    y = plan.forward_fp8(inp["x"], inp["Wg"], None, W1q, s1, W3q, s3, inp["W2"]).float()
+    plan.check()
+    x_host = inp["x"].cpu().pin_memory()
+    y_host = torch.empty((shape.T, shape.H), dtype=torch.bfloat16).pin_memory()
+    plan.forward_host_fp8(x_host, inp["Wg"], None, W1q, s1, W3q, s3, inp["W2"], y_host)
+    plan.check()
+    assert (y_host.float() - y.cpu()).abs().max().item() <= 1e-2
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["mixtral", "fine_grained_prefill", "decode"])
+def test_fp8_workload_matches_oracle(name):
+    """Full-size layers with the FP8 first GEMM, y on sampled tokens."""
+    from moe_megakernel_b200 import MoEPlan
+    shape = WORKLOADS[name]
+    inp = make_inputs(shape, device=DEV)
+    W1q, s1, W3q, s3 = _fp8_weights(inp)
+    plan = MoEPlan(shape.T, shape.H, shape.I, shape.E, shape.k)
+    y = plan.forward_fp8(inp["x"], inp["Wg"], inp["bias"], W1q, s1, W3q, s3, inp["W2"])
+    plan.check()
+    rows = sample_tokens(shape.T, {"mixtral": 8, "fine_grained_prefill": 4, "decode": 4}[name])
+    # (few tokens: the oracle quantizes every expert a sampled token reaches, in fp64)
+    ref = oracle_forward(inp, tokens=rows, block_m=plan.block_m, fp8=True)
+    assert_routing_equal(plan.routing(shape.T), ref)
+    fro, mx = assert_y_close(y[torch.from_numpy(rows).to(y.device)], ref["y"], "y (fp8)")
+    print(f"fp8 {name}: rel_fro={fro:.2e} max_abs={mx:.2e}")

@@ -43,16 +43,19 @@ Readings where the pages are silent (each is also listed in the design notes):
   added to the routed combine: y[t] += sum_s FFN_shared_s(x[t]). Routing and
   dispatch do not see them.
 
-* FP8 first GEMM (optional; "MegaMoE 在 MoE 系统谱系中的位置", section 一: the
-  Mega MoE kernel runs its GEMMs on 8-bit operands with scale factors loaded
-  beside them, and section 2.1: its epilogue quantizes with an amax). Reading
-  taken here: x and W1/W3 as OCP FP8 E4M3 (1 sign, 4 exponent bits with bias
-  7, 3 mantissa bits, largest finite 448, round to nearest even, saturating),
-  with power-of-two scales: one per token over H for x, one per (expert,
-  column i) over H for W1 and W3; the scale is the smallest power of two p
-  with amax / p <= 448 (1 for an all-zero row). g = sx[t] * s1[e,i] *
-  sum_h xq[t,h] W1q[e,h,i], the same for u; the activation and the second
-  GEMM are as in the bf16 layer.
+* FP8 expert GEMMs (optional; "MegaMoE 在 MoE 系统谱系中的位置", section 一:
+  the Mega MoE kernel runs its GEMMs on 8-bit operands with scale factors
+  loaded beside them, and section 2.1: the activation is quantized from its
+  amax between the two GEMMs). Reading taken here: every operand of both
+  expert GEMMs as OCP FP8 E4M3 (1 sign, 4 exponent bits with bias 7, 3
+  mantissa bits, largest finite 448, round to nearest even, saturating), with
+  power-of-two scales, the smallest power of two p with amax / p <= 448 (1
+  for an all-zero row or column): one per token over H for x; one per
+  (expert, column i) over H for W1 and W3; one per token over I for the
+  activation a = bf16(silu(g) * u) (rounded to bf16 first, as in the bf16
+  layer); one per (expert, output column) over I for W2.
+  g = sx[t] * s1[e,i] * sum_h xq[t,h] W1q[e,h,i], the same for u;
+  o[t,c] = sa[t] * s2[e,c] * sum_i aq[t,i] W2q[e,i,c].
 
 Everything is fp64 on inputs given as fp64 arrays holding bf16 values.
 """
@@ -242,13 +245,15 @@ def expert_ffn(xr: np.ndarray, W1e: np.ndarray, W3e: np.ndarray, W2e: np.ndarray
 
 
 def expert_ffn_fp8(xq: np.ndarray, sx: np.ndarray, W1q: np.ndarray, s1: np.ndarray, W3q: np.ndarray,
-                   s3: np.ndarray, W2e: np.ndarray) -> np.ndarray:
-    """The expert FFN with an FP8 first GEMM: xq [n,H] codes with scales sx [n,1];
-    W1q, W3q [H,I] codes with column scales s1, s3 [1,I]; W2e [I,H] as in the bf16 layer."""
+                   s3: np.ndarray, W2q: np.ndarray, s2: np.ndarray) -> np.ndarray:
+    """The expert FFN on FP8 operands: xq [n,H] codes with scales sx [n,1];
+    W1q, W3q [H,I] codes with column scales s1, s3 [1,I]; W2q [I,H] codes with
+    column scales s2 [1,H]. The bf16-rounded activation is quantized per row."""
     g = (xq @ W1q) * sx * s1
     u = (xq @ W3q) * sx * s3
     a = bf16_round(silu(g) * u)
-    return a @ W2e
+    aq, sa = quantize_fp8(a, axis=1)
+    return (aq @ W2q) * sa * s2
 
 
 def stacked_expert_weights(W1, W3, W2) -> Callable[[int], tuple]:
@@ -271,8 +276,8 @@ def moe_forward(x, Wg, bias, expert_weights: Callable[[int], tuple], k: int,
     T tokens). y[t] = sum_j w[t,j] * FFN_{idx[t,j]}(x[t])
                       + sum_{s < n_shared} FFN_shared_s(x[t]),
     with ``shared_weights(s)`` returning the shared expert's (W1, W3, W2).
-    fp8=True runs the first GEMM on FP8 E4M3 operands (see the module notes):
-    x is quantized per token, W1/W3 per (expert, column); no shared experts.
+    fp8=True runs both expert GEMMs on FP8 E4M3 operands (see the module notes):
+    x and the activation per token, W1/W3/W2 per (expert, column); no shared experts.
     """
     x = np.asarray(x, np.float64)
     T, H = x.shape
@@ -284,7 +289,7 @@ def moe_forward(x, Wg, bias, expert_weights: Callable[[int], tuple], k: int,
     y = np.zeros((len(rows), H), dtype=np.float64)
     if fp8:
         if n_shared:
-            raise ValueError("the FP8 first GEMM is defined without shared experts")
+            raise ValueError("the FP8 layer is defined without shared experts")
         xq, sx = quantize_fp8(x, axis=1)
     for e in range(E):
         # (row position in `rows`, top-k position) of every selected pair routed to e
@@ -295,7 +300,8 @@ def moe_forward(x, Wg, bias, expert_weights: Callable[[int], tuple], k: int,
         if fp8:
             W1q, s1 = quantize_fp8(W1e, axis=0)
             W3q, s3 = quantize_fp8(W3e, axis=0)
-            o = expert_ffn_fp8(xq[rows[hit[0]]], sx[rows[hit[0]]], W1q, s1, W3q, s3, W2e)
+            W2q, s2 = quantize_fp8(W2e, axis=0)
+            o = expert_ffn_fp8(xq[rows[hit[0]]], sx[rows[hit[0]]], W1q, s1, W3q, s3, W2q, s2)
         else:
             o = expert_ffn(x[rows[hit[0]]], W1e, W3e, W2e)
         wt = w[rows[hit[0]], hit[1]]

@@ -307,7 +307,7 @@ def test_two_shared_experts_equal_one_of_double_width():
     np.testing.assert_allclose(two, wide, rtol=1e-12, atol=1e-14)
 
 
-# ----------------------------------------------------------------- FP8 first GEMM
+# ----------------------------------------------------------------- FP8 expert GEMMs
 
 def test_e4m3_round_golden_and_matches_torch():
     """E4M3 rounding: hand-derived values (ties to even on the 1/8 mantissa
@@ -334,9 +334,10 @@ def test_pow2_scale_is_the_smallest_power_of_two():
 
 
 def test_fp8_forward_matches_textbook_dequantized_ffn():
-    """fp8=True equals the bf16 layer's combine with x, W1, W3 replaced by their
-    dequantized FP8 values (quantized here with torch's float8 cast and scales
-    from torch log2/ceil)."""
+    """fp8=True equals the bf16 layer's combine with x, W1, W3, W2 and the
+    bf16 activation replaced by their dequantized FP8 values (quantized here
+    with torch's float8 cast and scales from torch log2/ceil; x and the
+    activation per row, the weights per column)."""
     rng = _rng(23)
     x, Wg, W1, W3, W2 = _tiny_layer(rng, T=20, H=32, I=48, E=4)
     k = 2
@@ -350,13 +351,17 @@ def test_fp8_forward_matches_textbook_dequantized_ffn():
     xd = tq(x, 1)
     W1d = np.stack([tq(W1[e], 0) for e in range(W1.shape[0])])
     W3d = np.stack([tq(W3[e], 0) for e in range(W3.shape[0])])
+    W2d = np.stack([tq(W2[e], 0) for e in range(W2.shape[0])])
     r = O.moe_forward(x, Wg, None, O.stacked_expert_weights(W1, W3, W2), k, fp8=True)
     idx, w = r["topk_idx"], r["topk_w"]
     y = np.zeros_like(x)
     for t in range(x.shape[0]):
         for j in range(k):
             e = idx[t, j]
-            y[t] += w[t, j] * _torch_ffn(xd[t:t + 1], W1d[e], W3d[e], W2[e])[0]
+            xt = torch.from_numpy(xd[t:t + 1])
+            g, u = xt @ torch.from_numpy(W1d[e]), xt @ torch.from_numpy(W3d[e])
+            a = (torch.nn.functional.silu(g) * u).to(torch.bfloat16).double().numpy()
+            y[t] += w[t, j] * (torch.from_numpy(tq(a, 1)) @ torch.from_numpy(W2d[e])).numpy()[0]
     np.testing.assert_allclose(r["y"], y, rtol=1e-12, atol=1e-14)
     # and it stays near the bf16 layer (FP8 has 3 mantissa bits)
     b = O.moe_forward(x, Wg, None, O.stacked_expert_weights(W1, W3, W2), k)
@@ -381,8 +386,14 @@ _MUTANTS = {
     "e4m3_truncation": ("e4m3_round", lambda a: np.clip(np.ldexp(np.trunc(np.ldexp(np.asarray(a, float),
                         -(np.maximum(np.frexp(np.asarray(a, float))[1] - 1, -6) - 3))),
                         np.maximum(np.frexp(np.asarray(a, float))[1] - 1, -6) - 3), -448, 448)),
-    "fp8_scale_dropped": ("expert_ffn_fp8", lambda xq, sx, W1q, s1, W3q, s3, W2e:
-                          O.bf16_round(O.silu((xq @ W1q) * s1) * ((xq @ W3q) * s3)) @ W2e),
+    "fp8_scale_dropped": ("expert_ffn_fp8", lambda xq, sx, W1q, s1, W3q, s3, W2q, s2:
+                          (O.quantize_fp8(O.bf16_round(O.silu((xq @ W1q) * s1) * ((xq @ W3q) * s3)), 1)[0] @ W2q)
+                          * O.quantize_fp8(O.bf16_round(O.silu((xq @ W1q) * s1) * ((xq @ W3q) * s3)), 1)[1] * s2),
+    "fp8_activation_not_quantized": ("expert_ffn_fp8", lambda xq, sx, W1q, s1, W3q, s3, W2q, s2:
+                                     (O.bf16_round(O.silu((xq @ W1q) * sx * s1) * ((xq @ W3q) * sx * s3)) @ W2q) * s2),
+    "fp8_second_scale_dropped": ("expert_ffn_fp8", lambda xq, sx, W1q, s1, W3q, s3, W2q, s2:
+                                 (O.quantize_fp8(O.bf16_round(O.silu((xq @ W1q) * sx * s1) * ((xq @ W3q) * sx * s3)),
+                                                 1)[0] @ W2q) * s2),
     "pow2_scale_floor": ("pow2_scale", lambda amax: np.where(np.asarray(amax) > 0, np.ldexp(1.0, np.frexp(
                          np.asarray(amax, float) / 448.0)[1] - 1), 1.0)),
 }

@@ -51,12 +51,9 @@ Readings where the pages are silent (each is also listed in the design notes):
   mantissa bits, largest finite 448, round to nearest even, saturating), with
   power-of-two scales, the smallest power of two p with amax / p <= 448 (1
   for an all-zero row or column): one per token over H for x; one per
-  (expert, column i) over H for W1 and W3; one per (expert, output column)
-  over I for W2; and for the activation a = bf16(silu(g) * u) (rounded to
-  bf16 first, as in the bf16 layer) one per 128-column tile of a token's row,
-  the granularity of the epilogue that produces it, re-expressed at the
-  token's scale over I (the largest tile scale) for the second GEMM (see
-  quantize_activation_fp8).
+  (expert, column i) over H for W1 and W3; one per token over I for the
+  activation a = bf16(silu(g) * u) (rounded to bf16 first, as in the bf16
+  layer); one per (expert, output column) over I for W2.
   g = sx[t] * s1[e,i] * sum_h xq[t,h] W1q[e,h,i], the same for u;
   o[t,c] = sa[t] * s2[e,c] * sum_i aq[t,i] W2q[e,i,c].
 
@@ -128,28 +125,6 @@ def quantize_fp8(a: np.ndarray, axis: int):
     """(codes, scales): scales = pow2_scale(max |a| along `axis`), codes = e4m3_round(a / scales)."""
     sc = pow2_scale(np.max(np.abs(a), axis=axis, keepdims=True))
     return e4m3_round(a / sc), sc
-
-
-ACT_TILE = 128   # columns of the activation quantized together in the first GEMM's epilogue
-
-
-def quantize_activation_fp8(a: np.ndarray):
-    """Codes and row scales of the activation a [n, I] (I a multiple of ACT_TILE).
-
-    Each ACT_TILE-column tile of a row is quantized with its own scale s_t =
-    pow2_scale(tile amax) (what an epilogue that holds one tile can do); the
-    codes are then re-expressed at the row's scale S = max_t s_t (=
-    pow2_scale(row amax)), e4m3_round(codes * s_t / S), so that one scale per
-    row serves the second GEMM. s_t / S is a power of two <= 1: the second
-    rounding changes a code only where the result falls below the normal
-    E4M3 range.
-    """
-    n, I = a.shape
-    at = a.reshape(n, I // ACT_TILE, ACT_TILE)
-    st = pow2_scale(np.max(np.abs(at), axis=2, keepdims=True))     # [n, tiles, 1]
-    c1 = e4m3_round(at / st)
-    S = np.max(st, axis=1, keepdims=True)                            # [n, 1, 1]
-    return e4m3_round(c1 * (st / S)).reshape(n, I), S.reshape(n, 1)
 
 
 # --------------------------------------------------------------------------
@@ -277,7 +252,7 @@ def expert_ffn_fp8(xq: np.ndarray, sx: np.ndarray, W1q: np.ndarray, s1: np.ndarr
     g = (xq @ W1q) * sx * s1
     u = (xq @ W3q) * sx * s3
     a = bf16_round(silu(g) * u)
-    aq, sa = quantize_activation_fp8(a)
+    aq, sa = quantize_fp8(a, axis=1)
     return (aq @ W2q) * sa * s2
 
 

@@ -333,46 +333,13 @@ def test_pow2_scale_is_the_smallest_power_of_two():
     assert O.pow2_scale(0.0) == 1.0 and O.pow2_scale(448.0) == 1.0 and O.pow2_scale(449.0) == 2.0
 
 
-def test_activation_quantization_two_level():
-    """Tile-then-row quantization of the activation: with one tile per row it is
-    plain per-row quantization; its scale is pow2_scale of the row amax; for
-    normal-range results the codes equal direct per-row quantization (scaling
-    by a power of two commutes with the rounding). A hand case pins the
-    second rounding."""
-    rng = _rng(24)
-    a = rng.standard_normal((6, 128)) * np.exp(rng.uniform(-3, 3, (6, 1)))
-    q1, s1 = O.quantize_activation_fp8(a)
-    qd, sd = O.quantize_fp8(a, axis=1)
-    np.testing.assert_array_equal(q1, qd)
-    np.testing.assert_array_equal(s1, sd)
-    b = rng.standard_normal((5, 512))
-    b[:, 256:384] *= 0.1                       # a tile with a 16x smaller scale
-    q, S = O.quantize_activation_fp8(b)
-    qd, Sd = O.quantize_fp8(b, axis=1)
-    np.testing.assert_array_equal(S, Sd)
-    normal = np.abs(qd) >= 2.0 ** -6
-    np.testing.assert_array_equal(q[normal], qd[normal])
-    # hand case: row amax 448 (S = 1), a second tile with amax 0.875 (s_t = 2**-9):
-    # 0.8125 -> code 416 at s_t, back at S exactly 0.8125; v = 1.0625 * 2**-10 -> v / s_t =
-    # 0.53125 = 1.0625 * 2**-1, a tie on the 1/8 mantissa grid -> 0.5 (even), then 0.5 * 2**-9
-    # is a tie on the 2**-9 subnormal grid -> 0 (even). Direct rounding at S gives 2**-9.
-    h = np.zeros((1, 256))
-    h[0, 0] = 448.0
-    h[0, 128], h[0, 129], h[0, 130] = 0.875, 0.8125, 1.0625 * 2.0 ** -10
-    q, S = O.quantize_activation_fp8(h)
-    assert S[0, 0] == 1.0
-    assert q[0, 0] == 448.0 and q[0, 128] == 0.875 and q[0, 129] == 0.8125 and q[0, 130] == 0.0
-    assert O.quantize_fp8(h, axis=1)[0][0, 130] == 2.0 ** -9
-
-
 def test_fp8_forward_matches_textbook_dequantized_ffn():
     """fp8=True equals the bf16 layer's combine with x, W1, W3, W2 and the
     bf16 activation replaced by their dequantized FP8 values (quantized here
-    with torch's float8 cast and scales from torch log2/ceil; x per row, the
-    weights per column, the activation per 128-column tile and then at the
-    row's scale)."""
+    with torch's float8 cast and scales from torch log2/ceil; x and the
+    activation per row, the weights per column)."""
     rng = _rng(23)
-    x, Wg, W1, W3, W2 = _tiny_layer(rng, T=20, H=32, I=256, E=4)
+    x, Wg, W1, W3, W2 = _tiny_layer(rng, T=20, H=32, I=48, E=4)
     k = 2
 
     def tq(a, dim):
@@ -380,13 +347,6 @@ def test_fp8_forward_matches_textbook_dequantized_ffn():
         sc = torch.where(amax > 0, torch.exp2(torch.ceil(torch.log2(amax / 448.0))), torch.ones_like(amax))
         q = (torch.from_numpy(a) / sc).to(torch.float32).to(torch.float8_e4m3fn).double()
         return (q * sc).numpy()
-
-    def tq_act(a):   # per 128-column tile, then the tile codes at the row scale, dequantized
-        tiles = [tq(a[:, i:i + 128], 1) for i in range(0, a.shape[1], 128)]
-        amax = torch.from_numpy(np.abs(a)).amax(dim=1, keepdim=True)
-        S = torch.where(amax > 0, torch.exp2(torch.ceil(torch.log2(amax / 448.0))), torch.ones_like(amax))
-        t = torch.from_numpy(np.concatenate(tiles, axis=1))
-        return ((t / S).to(torch.float32).to(torch.float8_e4m3fn).double() * S).numpy()
 
     xd = tq(x, 1)
     W1d = np.stack([tq(W1[e], 0) for e in range(W1.shape[0])])
@@ -401,7 +361,7 @@ def test_fp8_forward_matches_textbook_dequantized_ffn():
             xt = torch.from_numpy(xd[t:t + 1])
             g, u = xt @ torch.from_numpy(W1d[e]), xt @ torch.from_numpy(W3d[e])
             a = (torch.nn.functional.silu(g) * u).to(torch.bfloat16).double().numpy()
-            y[t] += w[t, j] * (torch.from_numpy(tq_act(a)) @ torch.from_numpy(W2d[e])).numpy()[0]
+            y[t] += w[t, j] * (torch.from_numpy(tq(a, 1)) @ torch.from_numpy(W2d[e])).numpy()[0]
     np.testing.assert_allclose(r["y"], y, rtol=1e-12, atol=1e-14)
     # and it stays near the bf16 layer (FP8 has 3 mantissa bits)
     b = O.moe_forward(x, Wg, None, O.stacked_expert_weights(W1, W3, W2), k)
@@ -429,12 +389,6 @@ _MUTANTS = {
     "fp8_scale_dropped": ("expert_ffn_fp8", lambda xq, sx, W1q, s1, W3q, s3, W2q, s2:
                           (O.quantize_fp8(O.bf16_round(O.silu((xq @ W1q) * s1) * ((xq @ W3q) * s3)), 1)[0] @ W2q)
                           * O.quantize_fp8(O.bf16_round(O.silu((xq @ W1q) * s1) * ((xq @ W3q) * s3)), 1)[1] * s2),
-    "activation_row_scale_only": ("quantize_activation_fp8", lambda a: O.quantize_fp8(a, axis=1)),
-    "activation_tile_codes_kept": ("quantize_activation_fp8", lambda a: (
-        (O.e4m3_round(a.reshape(a.shape[0], -1, 128) / O.pow2_scale(np.abs(a.reshape(a.shape[0], -1, 128)).max(
-            2, keepdims=True))) * O.pow2_scale(np.abs(a.reshape(a.shape[0], -1, 128)).max(2, keepdims=True))
-         / O.pow2_scale(np.abs(a).max(1, keepdims=True))[:, :, None]).reshape(a.shape),
-        O.pow2_scale(np.abs(a).max(1, keepdims=True)))),
     "fp8_activation_not_quantized": ("expert_ffn_fp8", lambda xq, sx, W1q, s1, W3q, s3, W2q, s2:
                                      (O.bf16_round(O.silu((xq @ W1q) * sx * s1) * ((xq @ W3q) * sx * s3)) @ W2q) * s2),
     "fp8_second_scale_dropped": ("expert_ffn_fp8", lambda xq, sx, W1q, s1, W3q, s3, W2q, s2:
@@ -453,7 +407,7 @@ def _pins_pass():
              lambda: test_single_expert_is_dense_ffn("bias"),
              test_shared_experts_add_dense_ffns, test_shared_expert_equal_to_routed_doubles_y,
              test_e4m3_round_golden_and_matches_torch, test_pow2_scale_is_the_smallest_power_of_two,
-             test_fp8_forward_matches_textbook_dequantized_ffn, test_activation_quantization_two_level]
+             test_fp8_forward_matches_textbook_dequantized_ffn]
     for t in tests:
         try:
             t()

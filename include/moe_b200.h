@@ -181,23 +181,27 @@ int moe_forward_host_shared(moe_plan_t plan, const void* x_host, const void* Wg,
                             const void* W1, const void* W3, const void* W2, const void* Ws1, const void* Ws3,
                             const void* Ws2, int T, void* y_host, void* stream);
 
-/* ---- FP8 E4M3 first GEMM ("MegaMoE 在 MoE 系统谱系中的位置", section 一: the
- * expert GEMMs take 8-bit operands whose scale factors are loaded beside
- * them; section 2.1: amax and quantization of activations). Scales are powers
- * of two: for a row (or column) with largest magnitude amax the scale is the
- * smallest 2**k with amax / 2**k <= 448 (1 when amax == 0), so dividing by it
- * is exact; a code is the E4M3 value nearest to value / scale (ties to even,
- * saturating at +-448). Only x.W1 and x.W3 run on FP8 (tcgen05 kind::f8f6f4,
- * fp32 accumulation; the product is multiplied by the token scale and the
- * column scale before SwiGLU); h and W2 stay bf16. */
+/* ---- FP8 E4M3 expert GEMMs ("MegaMoE 在 MoE 系统谱系中的位置", section 一:
+ * the expert GEMMs take 8-bit operands whose scale factors are loaded beside
+ * them; section 2.1: the activation is quantized from its amax between the
+ * two GEMMs). Scales are powers of two: for a row (or column) with largest
+ * magnitude amax the scale is the smallest 2**k with amax / 2**k <= 448 (1
+ * when amax == 0), so dividing by it is exact; a code is the E4M3 value
+ * nearest to value / scale (ties to even, saturating at +-448). Both GEMMs
+ * run on tcgen05 kind::f8f6f4 with fp32 accumulation: x per token, W1 / W3 /
+ * W2 per (expert, output column), and the activation h = bf16(silu(g) * u)
+ * per token over I (its amax is gathered by the first GEMM's epilogues, and
+ * each row is quantized once before the second GEMM). Accumulators are
+ * multiplied by the row and column scales in the epilogues. */
 
 /* Codes and scales of a weight tensor, done once per set of weights:
- *   W     bf16 [E, H, I]  device (W1 or W3 as moe_forward takes them)
- *   Wq    u8   [E, I, H]  device, written: K-major E4M3 codes, 16-byte aligned
- *   scale fp32 [E, I]     device, written: per (expert, column) scale over H
- * H % 64 == 0 and I % 64 == 0. Enqueued on `stream`. Errors:
- * MOE_ERR_INVALID_ARG (null, misaligned or bad sizes), MOE_ERR_UNSUPPORTED_SHAPE,
- * MOE_ERR_CUDA. */
+ *   W     bf16 [E, K, N]  device (W1 or W3: K = H, N = I; W2: K = I, N = H,
+ *                         as moe_forward takes them)
+ *   Wq    u8   [E, N, K]  device, written: K-major E4M3 codes, 16-byte aligned
+ *   scale fp32 [E, N]     device, written: per (expert, column) scale over K
+ * K % 64 == 0 and N % 64 == 0 (the arguments H and I are K and N). Enqueued
+ * on `stream`. Errors: MOE_ERR_INVALID_ARG (null, misaligned or bad sizes),
+ * MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_CUDA. */
 int moe_quantize_weights_fp8(const void* W, void* Wq, float* scale, int E, int H, int I, void* stream);
 
 /* Codes and scales of activations, as moe_forward_fp8 forms them inside its
@@ -207,18 +211,30 @@ int moe_quantize_weights_fp8(const void* W, void* Wq, float* scale, int E, int H
  * H % 8 == 0. Errors: MOE_ERR_INVALID_ARG, MOE_ERR_CUDA. */
 int moe_quantize_x_fp8(const void* x, void* xq, float* sx, int T, int H, void* stream);
 
-/* moe_forward with the FP8 first GEMM. W1q / W3q and s1 / s3 come from
- * moe_quantize_weights_fp8 (u8 [E, I, H], fp32 [E, I]; 16-byte aligned); W2
- * stays bf16 [E, I, H]. x is quantized per token on the device at the start of
- * each call (into the workspace). Plans with shared experts are rejected
- * (MOE_ERR_INVALID_ARG). Other errors as for moe_forward. */
+/* Give the plan the workspace regions of the FP8 forward (enable = 1) or
+ * drop them (0): the activation of all blocks at once (bf16 and E4M3 codes)
+ * and its per-row amax and scale, so moe_plan_workspace_bytes grows. Unbinds
+ * the workspace: call moe_plan_bind_workspace again afterwards. Plans with
+ * shared experts: MOE_ERR_UNSUPPORTED_SHAPE. */
+int moe_plan_set_fp8(moe_plan_t plan, int enable);
+
+/* moe_forward with FP8 expert GEMMs (the plan needs moe_plan_set_fp8(plan, 1)). W1q / W3q, s1 / s3 (u8 [E, I, H], fp32
+ * [E, I]) and W2q / s2 (u8 [E, H, I], fp32 [E, H]) come from
+ * moe_quantize_weights_fp8; all 16-byte aligned. x is quantized per token on
+ * the device at the start of each call (into the workspace); the gate and
+ * routing are the bf16 layer's. The expert GEMM runs as two launches: the
+ * first GEMM with the bf16 activation and its row amax, then (after the
+ * activation rows are quantized once each) the second GEMM. A plan without
+ * FP8 regions or with shared experts: MOE_ERR_INVALID_ARG. Other errors as
+ * for moe_forward. */
 int moe_forward_fp8(moe_plan_t plan, const void* x, const void* Wg, const float* gate_bias, const void* W1q,
-                    const float* s1, const void* W3q, const float* s3, const void* W2, int T, void* y, void* stream);
+                    const float* s1, const void* W3q, const float* s3, const void* W2q, const float* s2, int T,
+                    void* y, void* stream);
 
 /* moe_forward_fp8 with x and y in HOST memory (see moe_forward_host). */
 int moe_forward_host_fp8(moe_plan_t plan, const void* x_host, const void* Wg, const float* gate_bias,
-                         const void* W1q, const float* s1, const void* W3q, const float* s3, const void* W2, int T,
-                         void* y_host, void* stream);
+                         const void* W1q, const float* s1, const void* W3q, const float* s3, const void* W2q,
+                         const float* s2, int T, void* y_host, void* stream);
 
 /* Gate and dispatch only (router, scan, scatter) for T tokens; fills the
  * routing results exactly as moe_forward does, without the expert FFN. */

@@ -55,8 +55,8 @@ SIGNATURES = {
     "moe_forward_host": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
     "moe_forward_shared": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
     "moe_forward_host_shared": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
-    "moe_forward_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
-    "moe_forward_host_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
+    "moe_forward_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
+    "moe_forward_host_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
     "moe_quantize_weights_fp8": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp]),
     "moe_quantize_x_fp8": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _vp]),
     "moe_route": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _vp]),
@@ -67,6 +67,7 @@ SIGNATURES = {
     "moe_route_static": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp,
                                   _vp, _vp, _c_int, _vp, _vp, _vp]),
     "moe_plan_set_cta_pairs": (_c_int, [_vp, _c_int]),
+    "moe_plan_set_fp8": (_c_int, [_vp, _c_int]),
     "moe_forward_kernel_count": (_c_int, []),
     "moe_plan_destroy": (None, [_vp]),
     "moe_status_string": (ctypes.c_char_p, [_c_int]),
@@ -138,7 +139,7 @@ class MoEPlan:
     """
 
     def __init__(self, T_max: int, H: int, I: int, E: int, k: int, block_m: int = 0, device=None,
-                 n_shared: int = 0):
+                 n_shared: int = 0, fp8: bool = False):
         self.lib = load_library()
         self.device = torch.device("cuda", torch.cuda.current_device() if device is None
                                    else torch.device(device).index or 0)
@@ -146,6 +147,9 @@ class MoEPlan:
         self._plan = ctypes.c_void_p()
         _ok(self.lib.moe_plan_create_shared(ctypes.byref(self._plan), T_max, H, I, E, k, n_shared, block_m,
                                             self.device.index), "moe_plan_create_shared")
+        self.fp8 = bool(fp8)
+        if fp8:   # workspace regions of forward_fp8
+            _ok(self.lib.moe_plan_set_fp8(self._plan, 1), "moe_plan_set_fp8")
         d = MoEPlanDesc()
         _ok(self.lib.moe_plan_describe(self._plan, ctypes.byref(d)), "moe_plan_describe")
         self.block_m, self.pool_capacity, self.num_sms = d.block_m, d.pool_capacity, d.num_sms
@@ -198,35 +202,36 @@ class MoEPlan:
             "moe_forward_host_shared")
         return y_host
 
-    def _check_fp8(self, W1q, s1, W3q, s3, W2):
+    def _check_fp8(self, W1q, s1, W3q, s3, W2q, s2):
         E, H, I = self.E, self.H, self.I
         _check(W1q, "W1q", (E, I, H), torch.uint8, self.device)
         _check(W3q, "W3q", (E, I, H), torch.uint8, self.device)
+        _check(W2q, "W2q", (E, H, I), torch.uint8, self.device)
         _check(s1, "s1", (E, I), torch.float32, self.device)
         _check(s3, "s3", (E, I), torch.float32, self.device)
-        _check(W2, "W2", (E, I, H), torch.bfloat16, self.device)
+        _check(s2, "s2", (E, H), torch.float32, self.device)
 
-    def forward_fp8(self, x, Wg, bias, W1q, s1, W3q, s3, W2, y=None, stream=None) -> torch.Tensor:
-        """Forward with the FP8 E4M3 first GEMM; W1q/s1 and W3q/s3 from quantize_weights_fp8."""
+    def forward_fp8(self, x, Wg, bias, W1q, s1, W3q, s3, W2q, s2, y=None, stream=None) -> torch.Tensor:
+        """Forward with FP8 E4M3 expert GEMMs; (W1q, s1), (W3q, s3), (W2q, s2) from quantize_weights_fp8."""
         T = self._check_inputs(x, Wg, bias)
-        self._check_fp8(W1q, s1, W3q, s3, W2)
+        self._check_fp8(W1q, s1, W3q, s3, W2q, s2)
         if y is None:
             y = torch.empty((T, self.H), dtype=torch.bfloat16, device=self.device)
         _check(y, "y", (T, self.H), torch.bfloat16, self.device)
         _ok(self.lib.moe_forward_fp8(self._plan, _ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1q), _ptr(s1), _ptr(W3q),
-                                     _ptr(s3), _ptr(W2), T, _ptr(y), _stream_handle(stream, self.device)),
+                                     _ptr(s3), _ptr(W2q), _ptr(s2), T, _ptr(y), _stream_handle(stream, self.device)),
             "moe_forward_fp8")
         return y
 
-    def forward_host_fp8(self, x_host, Wg, bias, W1q, s1, W3q, s3, W2, y_host, stream=None):
+    def forward_host_fp8(self, x_host, Wg, bias, W1q, s1, W3q, s3, W2q, s2, y_host, stream=None):
         """forward_fp8 with x_host / y_host CPU bf16 tensors (pinned for asynchronous copies)."""
         T = x_host.shape[0]
         _check(x_host, "x_host", (T, self.H), torch.bfloat16, torch.device("cpu"))
         _check(y_host, "y_host", (T, self.H), torch.bfloat16, torch.device("cpu"))
         _check(Wg, "Wg", (self.H, self.E), torch.bfloat16, self.device)
-        self._check_fp8(W1q, s1, W3q, s3, W2)
+        self._check_fp8(W1q, s1, W3q, s3, W2q, s2)
         _ok(self.lib.moe_forward_host_fp8(self._plan, _ptr(x_host), _ptr(Wg), _ptr(bias), _ptr(W1q), _ptr(s1),
-                                          _ptr(W3q), _ptr(s3), _ptr(W2), T, _ptr(y_host),
+                                          _ptr(W3q), _ptr(s3), _ptr(W2q), _ptr(s2), T, _ptr(y_host),
                                           _stream_handle(stream, self.device)), "moe_forward_host_fp8")
         return y_host
 
@@ -302,9 +307,10 @@ class MoEPlan:
 
 
 def quantize_weights_fp8(W: torch.Tensor, stream=None):
-    """W bf16 [E, H, I] (W1 or W3) -> (K-major E4M3 codes u8 [E, I, H], column scales fp32 [E, I])."""
+    """W bf16 [E, K, N] (W1 / W3: K = H, N = I; W2: K = I, N = H) ->
+    (K-major E4M3 codes u8 [E, N, K], per-column scales over K fp32 [E, N])."""
     if not isinstance(W, torch.Tensor) or W.dim() != 3:
-        raise TypeError("W must be a 3-D torch.Tensor [E, H, I]")
+        raise TypeError("W must be a 3-D torch.Tensor [E, K, N]")
     E, H, I = W.shape
     _check(W, "W", (E, H, I), torch.bfloat16, None)
     Wq = torch.empty((E, I, H), dtype=torch.uint8, device=W.device)

@@ -32,14 +32,15 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace moe {
 
 struct GemmParams {
   const bf16* x;       // [T, H]
-  CUtensorMap tm_w1;   // W1 as [E*H, I], box {64, 64}; FP8 first GEMM: W1q as [E*I, H] bytes, box {128, 64}
+  CUtensorMap tm_w1;   // W1 as [E*H, I], box {64, 64}; FP8: W1q as [E*I, H] bytes, box {128, 64}
   CUtensorMap tm_w3;   // W3 likewise
-  CUtensorMap tm_w2;   // W2 as [E*I, H], box {64, 64}
+  CUtensorMap tm_w2;   // W2 as [E*I, H], box {64, 64}; FP8: W2q as [E*H, I] bytes, box {128, 64}
   CUtensorMap tm_ws1;  // shared experts' W1 as [S*H, I] (experts E .. E+S-1; unused when S = 0)
   CUtensorMap tm_ws3;  // shared experts' W3 as [S*H, I]
   CUtensorMap tm_ws2;  // shared experts' W2 as [S*I, H]
@@ -57,13 +58,23 @@ struct GemmParams {
   float* y_acc;                 // [T, H]
   int T, H, I, E, k, BM, BN2, N1, N2;
   int S;                        // shared experts (0 .. kMaxShared)
-  // FP8 E4M3 first GEMM (fp8 != 0): x codes [T, H] with per-token scales,
-  // W1/W3 codes K-major [E, I, H] (tensor maps above) with column scales [E, I]
+  // FP8 E4M3 expert GEMMs (fp8 != 0): x codes [T, H] with per-token scales,
+  // W1/W3 codes K-major [E, I, H] with column scales [E, I], W2 codes K-major
+  // [E, H, I] with column scales [E, H] (tensor maps above). The two GEMMs run
+  // as two launches (phase_only 0, then 1) around the activation quantizer:
+  // the first stores the bf16 activation in h and raises act_amax of its row
+  // (zero before the launch) to the row's largest |h|; the quantizer writes
+  // the row's codes to h8 and its scale to act_scale; the second reads them.
   int fp8;
   const uint8_t* xq;
   const float* sx;
   const float* s1;
   const float* s3;
+  const float* s2;
+  float* act_amax;           // [h rows]
+  const float* act_scale;    // [h rows]
+  const uint8_t* h8;         // [h rows, I]
+  int phase_only;            // -1: both phases in one launch; 0: first GEMM only; 1: second GEMM only
   int ring_blocks;              // block b uses ring slot b % ring_blocks
   int max_groups;
   unsigned long long timeout_ns;
@@ -165,6 +176,9 @@ __device__ __forceinline__ Task decode_task(int t, const GemmSmem& s, const Gemm
   Task task{-1, 0, 0, 0};
   const int G = s.num_groups;
   const int nb_total = s.block_start[p.E + p.S];
+  // one-phase launches (a single block group): the second GEMM's tasks follow the first's
+  if (p.phase_only == 1) t += nb_total * p.N1;
+  else if (p.phase_only == 0 && t >= nb_total * p.N1) return task;
   if (t < 0 || t >= nb_total * (p.N1 + p.N2) || G <= 0) return task;
   // last segment whose start is <= t (empty segments share the next start)
   int lo = 0, hi = 2 * G;
@@ -209,6 +223,7 @@ __device__ __forceinline__ uint8_t* stage_ptr(uint8_t* tiles, int stage) { retur
 
 // K blocks of an L1 task: 64 bf16 or 128 FP8 elements, one 128-byte swizzle row either way.
 __device__ __forceinline__ int l1_ksteps(const GemmParams& p) { return p.fp8 ? p.H / 128 : p.H / kBK; }
+__device__ __forceinline__ int l2_ksteps(const GemmParams& p) { return p.fp8 ? p.I / 128 : p.I / kBK; }
 
 // ---------------------------------------------------------------- scheduler (last warp)
 // Claims tasks from the global counter, decodes them, stages the routed row
@@ -324,7 +339,7 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
     }
     if (task.phase < 0) break;
 
-    const int nk = task.phase == 0 ? l1_ksteps(p) : p.I / kBK;
+    const int nk = task.phase == 0 ? l1_ksteps(p) : l2_ksteps(p);
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait(&s.empty[stage], phase ^ 1, p, s, 2)) {
         ok = false;
@@ -356,7 +371,13 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
         }
       } else {
         // B: 256 (or 128) columns of W2; A (the block's h rows) comes from the gather warps.
-        if (lane == 0) {
+        if (lane == 0 && p.fp8) {   // K-major E4M3 codes: BN2 rows of 128 bytes, 64 per box
+          const int nbox = p.BN2 / 64;
+          ptx::mbar_arrive_expect_tx(&s.full[stage], nbox * kBoxBytes);
+          for (int j = 0; j < nbox; ++j)
+            ptx::tma_load_2d(b_addr + j * kBoxBytes, &p.tm_w2, &s.full[stage], kb * 128,
+                             task.e * p.H + task.n * p.BN2 + j * 64, pol);
+        } else if (lane == 0) {
           const int nbox = p.BN2 / 64;
           ptx::mbar_arrive_expect_tx(&s.full[stage], nbox * kBoxBytes);
           const bool sh = task.e >= p.E;
@@ -392,7 +413,7 @@ __device__ void gemm_mma(const GemmParams& p, GemmSmem& s, uint8_t* tiles, uint3
   const uint32_t idesc_l1 =
       p.fp8 ? ptx::idesc_e4m3_f32(128, 2 * kL1TileN) : ptx::idesc_bf16_f32(128, 2 * kL1TileN, false, true);
   const bool f8 = p.fp8 != 0;
-  const uint32_t idesc_l2 = ptx::idesc_bf16_f32(128, p.BN2, false, true);
+  const uint32_t idesc_l2 = p.fp8 ? ptx::idesc_e4m3_f32(128, p.BN2) : ptx::idesc_bf16_f32(128, p.BN2, false, true);
   int stage = 0;
   uint32_t phase = 0;
   int q = 0;
@@ -414,7 +435,7 @@ __device__ void gemm_mma(const GemmParams& p, GemmSmem& s, uint8_t* tiles, uint3
     ptx::tc_fence_after();
     const uint32_t d_tmem = tmem_base + acc * 256;
     const uint32_t idesc = task.phase == 0 ? idesc_l1 : idesc_l2;
-    const int nk = task.phase == 0 ? l1_ksteps(p) : p.I / kBK;
+    const int nk = task.phase == 0 ? l1_ksteps(p) : l2_ksteps(p);
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait(&s.full[stage], phase, p, s, 5)) {
@@ -431,8 +452,8 @@ __device__ void gemm_mma(const GemmParams& p, GemmSmem& s, uint8_t* tiles, uint3
           // A: K-major, 128-byte rows, 8-row groups 1024 B apart; step 32 B along K
           // (16 bf16 or 32 FP8 elements per MMA).
           const uint64_t ad = ptx::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
-          if (f8 && task.phase == 0) {
-            // B: K-major FP8 codes, 256 rows of 128 bytes
+          if (f8) {
+            // B: K-major FP8 codes (W1 | W3, or W2), rows of 128 bytes
             const uint64_t bd = ptx::smem_desc_sw128(b_addr + kk * 32, 16, 1024);
             ptx::mma_f8(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           } else {
@@ -502,7 +523,10 @@ __device__ void gemm_gather(const GemmParams& p, GemmSmem& s, uint8_t* tiles, in
     uint32_t soff[kRowsPerLane];
     const uint8_t* src[kRowsPerLane];
     const int* rows = s.rows[q_task];
-    const uint8_t* hblock = reinterpret_cast<const uint8_t*>(p.h + (size_t)(task.b % p.ring_blocks) * p.BM * p.I);
+    // activation rows: bf16, or FP8 codes (rows of I bytes); x rows: bf16, or FP8 codes
+    const size_t hpitch = p.fp8 ? (size_t)p.I : (size_t)p.I * 2;
+    const int ring_row0 = (task.b % p.ring_blocks) * p.BM;
+    const uint8_t* hblock = (p.fp8 ? p.h8 : reinterpret_cast<const uint8_t*>(p.h)) + (size_t)ring_row0 * hpitch;
     const uint8_t* xrows = p.fp8 ? p.xq : reinterpret_cast<const uint8_t*>(p.x);
     const size_t xpitch = p.fp8 ? (size_t)p.H : (size_t)p.H * 2;
 #pragma unroll
@@ -511,14 +535,15 @@ __device__ void gemm_gather(const GemmParams& p, GemmSmem& s, uint8_t* tiles, in
       soff[j] = r * 128 + ((c ^ (r & 7)) << 4);
       src[j] = xrows + c * 16;
       if (r < p.BM) {
-        src[j] = task.phase == 0 ? xrows + (size_t)rows[r] * xpitch + c * 16 : hblock + (size_t)r * p.I * 2 + c * 16;
+        src[j] = task.phase == 0 ? xrows + (size_t)rows[r] * xpitch + c * 16 : hblock + (size_t)r * hpitch + c * 16;
         nrows = j + 1;
       }
     }
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive(&s.task_empty[q_task]);   // slot (and its rows) free
-    const int nk = task.phase == 0 ? l1_ksteps(p) : p.I / kBK;
+    const int nk = task.phase == 0 ? l1_ksteps(p) : l2_ksteps(p);
     bool ok = true;
+
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait(&s.empty[stage], phase ^ 1, p, s, 9)) {
         ok = false;
@@ -564,6 +589,30 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// h[0..31] = bf16(silu(g) * u) for one row's 32 columns; amax = max(amax, |silu(g) * u|).
+__device__ __forceinline__ void store_swiglu32(bf16* dst, const uint32_t (&g)[32], const uint32_t (&u)[32],
+                                               float& amax) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    float f[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      f[i] = silu_mul(__uint_as_float(g[8 * v + i]), __uint_as_float(u[8 * v + i]));
+      amax = fmaxf(amax, fabsf(f[i]));
+    }
+    d4[v] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                       pack_bf16x2(f[6], f[7]));
+  }
+}
+
+// FP8: raise the row's activation amax (non-negative floats order as their bits) to `amax`,
+// the largest |h| of this task's columns (bf16 rounding is monotonic: the rounded maximum
+// is the maximum of the rounded values).
+__device__ __forceinline__ void publish_act_amax(float* act_amax, int row, float amax) {
+  atomicMax(reinterpret_cast<unsigned int*>(act_amax + row), __float_as_uint(__bfloat162float(__float2bfloat16_rn(amax))));
+}
+
 // Combine of one epilogue warp's 32 accumulator rows (TMEM lanes tbase..+31,
 // columns 0..ncols-1, ncols a multiple of 64): y_acc[tok_r][c] += w_r *
 // acc[r][c] for every row r with tok_r >= 0. Each lane holds row `lane`; per
@@ -576,7 +625,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 // accumulator while the last reductions are still being issued.
 __device__ __forceinline__ void combine_stage_and_reduce(const uint32_t (&v)[32], int c, float w, float* srow,
                                                          float (*stage)[36], float* const (&ybase)[8], int sub,
-                                                         int cc) {
+                                                         int cc, const float* cs) {
+  // per-column scales of the lane's 4 transposed columns (FP8 W2), loaded before the staging
+  const float4 m = cs != nullptr ? __ldg(reinterpret_cast<const float4*>(cs + c * 32 + cc)) : make_float4(1.f, 1.f, 1.f, 1.f);
 #pragma unroll
   for (int i = 0; i < 8; ++i)
     reinterpret_cast<float4*>(srow)[i] =
@@ -585,14 +636,18 @@ __device__ __forceinline__ void combine_stage_and_reduce(const uint32_t (&v)[32]
   __syncwarp();
 #pragma unroll
   for (int i = 0; i < 8; ++i)
-    if (ybase[i] != nullptr)
-      ptx::red_add_v4_f32(ybase[i] + c * 32, *reinterpret_cast<const float4*>(&stage[i * 4 + sub][cc]));
+    if (ybase[i] != nullptr) {
+      float4 a = *reinterpret_cast<const float4*>(&stage[i * 4 + sub][cc]);
+      if (cs != nullptr) a = make_float4(a.x * m.x, a.y * m.y, a.z * m.z, a.w * m.w);
+      ptx::red_add_v4_f32(ybase[i] + c * 32, a);
+    }
   __syncwarp();
 }
 
 template <typename Release>
 __device__ __forceinline__ void combine_rows(uint32_t tbase, int ncols, float w, int tok, float* y_acc, int H,
-                                             int col0, float (*stage)[36], int* stage_tok, Release release) {
+                                             int col0, float (*stage)[36], int* stage_tok, const float* cs,
+                                             Release release) {
   const int lane = ptx::lane_id();
   stage_tok[lane] = tok;
   __syncwarp();
@@ -611,11 +666,11 @@ __device__ __forceinline__ void combine_rows(uint32_t tbase, int ncols, float w,
   for (int c = 0; c < ncols / 32; c += 2) {
     ptx::tmem_ld_wait();                                         // va holds columns 32c ..
     ptx::tmem_ld32(tbase + (c + 1) * 32, vb);
-    combine_stage_and_reduce(va, c, w, srow, stage, ybase, sub, cc);
+    combine_stage_and_reduce(va, c, w, srow, stage, ybase, sub, cc, cs);
     ptx::tmem_ld_wait();                                         // vb holds columns 32(c+1) ..
     if (c + 2 < ncols / 32) ptx::tmem_ld32(tbase + (c + 2) * 32, va);
     else release();                                              // no TMEM reads left
-    combine_stage_and_reduce(vb, c + 1, w, srow, stage, ybase, sub, cc);
+    combine_stage_and_reduce(vb, c + 1, w, srow, stage, ybase, sub, cc, cs);
   }
 }
 
@@ -656,7 +711,8 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
       }
       const int ring_row = (task.b % p.ring_blocks) * p.BM + r;
       bf16* hrow = p.h + (size_t)ring_row * p.I + task.n * kL1TileN;
-      float tscale = 1.f;   // FP8 first GEMM: the token's scale (padding rows: any)
+      float tscale = 0.f;   // FP8: the token's scale (padding rows: 0, so their activation is 0)
+      float amax = 0.f;     // FP8: the row's largest |h| over this task's columns
       if (p.fp8 && valid) {
         const int tok = p.slot_token[slot];
         tscale = (tok >= 0 && tok < p.T) ? p.sx[tok] : 0.f;
@@ -668,23 +724,9 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
         ptx::tmem_ld32(tbase + kL1TileN + c * 32, u);
         ptx::tmem_ld_wait();
         if (p.fp8) fp8_scale_columns(g, u, tscale, p.s1, p.s3, (size_t)task.e * p.I + task.n * kL1TileN + c * 32);
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(hrow + c * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 o;
-            o.x = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 0]), __uint_as_float(u[8 * v + 0])),
-                              silu_mul(__uint_as_float(g[8 * v + 1]), __uint_as_float(u[8 * v + 1])));
-            o.y = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 2]), __uint_as_float(u[8 * v + 2])),
-                              silu_mul(__uint_as_float(g[8 * v + 3]), __uint_as_float(u[8 * v + 3])));
-            o.z = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 4]), __uint_as_float(u[8 * v + 4])),
-                              silu_mul(__uint_as_float(g[8 * v + 5]), __uint_as_float(u[8 * v + 5])));
-            o.w = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 6]), __uint_as_float(u[8 * v + 6])),
-                              silu_mul(__uint_as_float(g[8 * v + 7]), __uint_as_float(u[8 * v + 7])));
-            dst[v] = o;
-          }
-        }
+        if (store) store_swiglu32(hrow + c * 32, g, u, amax);
       }
+      if (p.fp8 && store) publish_act_amax(p.act_amax, ring_row, amax);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&s.acc_empty[acc]);
@@ -717,9 +759,11 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
           }
         }
       }
+      // FP8: o = acc * (activation scale of the row) * (W2 column scale)
+      if (p.fp8 && tok >= 0) w *= __ldcg(p.act_scale + (task.b % p.ring_blocks) * p.BM + r);   // FP8: the row's scale
       // Combine: y_acc[token] += w * o, 128-byte row segments per red.v4 (the L2 does the fp32 adds).
       combine_rows(tbase, p.BN2, w, tok, p.y_acc, p.H, task.n * p.BN2, s.out_stage[quarter], s.out_tok[quarter],
-                   [&]() {
+                   p.fp8 ? p.s2 + (size_t)task.e * p.H + task.n * p.BN2 : nullptr, [&]() {
                      ptx::tc_fence_before();
                      __syncwarp();
                      if (lane == 0) ptx::mbar_arrive(&s.acc_empty[acc]);

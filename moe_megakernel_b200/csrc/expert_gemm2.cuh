@@ -71,6 +71,12 @@ struct Gemm2Params {
   const float* sx;
   const float* s1;
   const float* s3;
+  const uint8_t* w2q;   // FP8: W2 codes K-major [E, H, I] (the A-row warps copy this CTA's half)
+  const float* s2;      // FP8: W2 column scales [E, H]
+  float* act_amax;         // FP8: [h rows] row amax of the bf16 activation (see GemmParams)
+  const float* act_scale;  // FP8: [h rows] row scale written by the activation quantizer
+  const uint8_t* h8;       // FP8: [h rows, I] activation codes
+  int phase_only;          // -1: both phases; 0: first GEMM only; 1: second GEMM only
   int ring_pairs, max_groups;
   unsigned long long timeout_ns;
   int withhold_pair;            // test hook: never publish L1 completion of this pair (-1: off)
@@ -188,6 +194,9 @@ __device__ __forceinline__ Task2 decode_task2(int t, const Gemm2Smem& s, const G
   Task2 task{-1, 0, 0, 0, -1, -1, 0, 0};
   const int G = s.num_groups;
   const int np_total = s.pair_start[p.E + p.S];
+  // one-phase launches (a single block group): the second GEMM's tasks follow the first's
+  if (p.phase_only == 1) t += np_total * p.N1;
+  else if (p.phase_only == 0 && t >= np_total * p.N1) return task;
   if (t < 0 || t >= np_total * (p.N1 + p.N2) || G <= 0) return task;
   int lo = 0, hi = 2 * G;
   while (lo < hi) {
@@ -232,6 +241,8 @@ __device__ __forceinline__ uint8_t* stage2_ptr(uint8_t* tiles, int stage) { retu
 
 // K blocks of an L1 task: 64 bf16 or 128 FP8 elements (one 128-byte swizzle row).
 __device__ __forceinline__ int l1_ksteps2(const Gemm2Params& p) { return p.fp8 ? p.H / 128 : p.H / kBK; }
+
+__device__ __forceinline__ int l2_ksteps2(const Gemm2Params& p) { return p.fp8 ? p.I / 128 : p.I / kBK; }
 
 // ---------------------------------------------------------------- leader scheduler (last warp)
 // Claims tasks, decodes them, stages the token rows of both CTAs' A tiles
@@ -357,7 +368,7 @@ __device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_
       qphase ^= 1;
     }
     if (task.phase < 0) break;
-    const int nk = task.phase == 0 ? l1_ksteps2(p) : p.I / kBK;
+    const int nk = task.phase == 0 ? l1_ksteps2(p) : l2_ksteps2(p);
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait2(&s.empty[stage], phase ^ 1, p, s, 2)) {
         ok = false;
@@ -447,7 +458,7 @@ __device__ void gemm2_follower_producer(const Gemm2Params& p, Gemm2Smem& s, uint
     Task2 task;
     if (!pop_task2(task, q, qphase, nullptr, false, p, s, 3, true)) break;
     if (task.phase < 0) break;
-    const int nk = task.phase == 0 ? l1_ksteps2(p) : p.I / kBK;
+    const int nk = task.phase == 0 ? l1_ksteps2(p) : l2_ksteps2(p);
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait2(&s.empty[stage], phase ^ 1, p, s, 4)) {
@@ -498,7 +509,7 @@ __device__ void gemm2_follower_relay(const Gemm2Params& p, Gemm2Smem& s) {
     Task2 task;
     if (!pop_task2(task, q, qphase, nullptr, false, p, s, 5, true)) break;
     if (task.phase < 0) break;
-    const int nk = task.phase == 0 ? l1_ksteps2(p) : p.I / kBK;
+    const int nk = task.phase == 0 ? l1_ksteps2(p) : l2_ksteps2(p);
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait2(&s.full[stage], phase, p, s, 6)) {
@@ -525,7 +536,7 @@ __device__ void gemm2_mma(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, ui
   const uint32_t idesc_l1 =
       p.fp8 ? ptx::idesc_e4m3_f32(256, 2 * kL1TileN) : ptx::idesc_bf16_f32(256, 2 * kL1TileN, false, true);
   const bool f8 = p.fp8 != 0;
-  const uint32_t idesc_l2 = ptx::idesc_bf16_f32(256, p.BN2, false, true);
+  const uint32_t idesc_l2 = p.fp8 ? ptx::idesc_e4m3_f32(256, p.BN2) : ptx::idesc_bf16_f32(256, p.BN2, false, true);
   int stage = 0;
   uint32_t phase = 0;
   int q = 0;
@@ -541,7 +552,7 @@ __device__ void gemm2_mma(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, ui
     ptx::tc_fence_after();
     const uint32_t d_tmem = tmem_base + acc * 256;
     const uint32_t idesc = task.phase == 0 ? idesc_l1 : idesc_l2;
-    const int nk = task.phase == 0 ? l1_ksteps2(p) : p.I / kBK;
+    const int nk = task.phase == 0 ? l1_ksteps2(p) : l2_ksteps2(p);
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait2(&s.full[stage], phase, p, s, 9)) {
@@ -556,8 +567,8 @@ __device__ void gemm2_mma(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, ui
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t ad = ptx::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
-          if (f8 && task.phase == 0) {
-            // B half: K-major FP8 codes, 128 rows of 128 bytes in each CTA
+          if (f8) {
+            // B half: K-major FP8 codes (W1 | W3, or W2), rows of 128 bytes in each CTA
             const uint64_t bd = ptx::smem_desc_sw128(b_addr + kk * 32, 16, 1024);
             ptx::mma_f8_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           } else {
@@ -625,7 +636,8 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
       }
       const int ring_row = ((task.p % p.ring_pairs) * 2 + (int)rank) * p.BM + r;
       bf16* hrow = p.h + (size_t)ring_row * p.I + task.n * kL1TileN;
-      float tscale = 1.f;   // FP8 first GEMM: the token's scale (padding rows: any)
+      float tscale = 0.f;   // FP8: the token's scale (padding rows: 0, so their activation is 0)
+      float amax = 0.f;     // FP8: the row's largest |h| over this task's columns
       if (p.fp8 && valid) {
         const int tok = p.slot_token[slot];
         tscale = (tok >= 0 && tok < p.T) ? p.sx[tok] : 0.f;
@@ -637,23 +649,9 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
         ptx::tmem_ld32(tbase + kL1TileN + c * 32, u);
         ptx::tmem_ld_wait();
         if (p.fp8) fp8_scale_columns(g, u, tscale, p.s1, p.s3, (size_t)task.e * p.I + task.n * kL1TileN + c * 32);
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(hrow + c * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 o;
-            o.x = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 0]), __uint_as_float(u[8 * v + 0])),
-                              silu_mul(__uint_as_float(g[8 * v + 1]), __uint_as_float(u[8 * v + 1])));
-            o.y = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 2]), __uint_as_float(u[8 * v + 2])),
-                              silu_mul(__uint_as_float(g[8 * v + 3]), __uint_as_float(u[8 * v + 3])));
-            o.z = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 4]), __uint_as_float(u[8 * v + 4])),
-                              silu_mul(__uint_as_float(g[8 * v + 5]), __uint_as_float(u[8 * v + 5])));
-            o.w = pack_bf16x2(silu_mul(__uint_as_float(g[8 * v + 6]), __uint_as_float(u[8 * v + 6])),
-                              silu_mul(__uint_as_float(g[8 * v + 7]), __uint_as_float(u[8 * v + 7])));
-            dst[v] = o;
-          }
-        }
+        if (store) store_swiglu32(hrow + c * 32, g, u, amax);
       }
+      if (p.fp8 && store) publish_act_amax(p.act_amax, ring_row, amax);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -685,8 +683,10 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
           }
         }
       }
+      if (p.fp8 && tok >= 0)   // FP8: the row's scale
+        w *= __ldcg(p.act_scale + ((task.p % p.ring_pairs) * 2 + (int)rank) * p.BM + r);
       combine_rows(tbase, p.BN2, w, tok, p.y_acc, p.H, task.n * p.BN2, s.out_stage[quarter], s.out_tok[quarter],
-                   [&]() {
+                   p.fp8 ? p.s2 + (size_t)task.e * p.H + task.n * p.BN2 : nullptr, [&]() {
                      ptx::tc_fence_before();
                      __syncwarp();
                      if (lane == 0) {
@@ -719,14 +719,16 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
     if (!pop_task2(task, q, qphase, &q_task, is_leader, p, s, 12, false)) break;
     if (task.phase < 0) break;
     const int b_own = rank == 0 ? task.b0 : task.b1;
+    const int ring_row0 = ((task.p % p.ring_pairs) * 2 + (int)rank) * p.BM;
     int nrows = 0;
     uint32_t soff[kRowsPerLane];
     const uint8_t* src[kRowsPerLane];   // byte addresses; a stage takes the next 128 bytes of a row
     if (b_own >= 0) {
       // L1: the routed x rows (bf16, or FP8 codes) of this CTA's block; L2: its h rows in the ring
+      // activation rows: bf16, or FP8 codes (rows of I bytes)
       const int* rows = s.rows[q_task];
-      const uint8_t* hblock =
-          reinterpret_cast<const uint8_t*>(p.h + (size_t)((task.p % p.ring_pairs) * 2 + (int)rank) * p.BM * p.I);
+      const size_t hpitch = p.fp8 ? (size_t)p.I : (size_t)p.I * 2;
+      const uint8_t* hblock = (p.fp8 ? p.h8 : reinterpret_cast<const uint8_t*>(p.h)) + (size_t)ring_row0 * hpitch;
       const uint8_t* xrows = p.fp8 ? p.xq : reinterpret_cast<const uint8_t*>(p.x);
       const size_t xpitch = p.fp8 ? (size_t)p.H : (size_t)p.H * 2;
 #pragma unroll
@@ -735,8 +737,7 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
         soff[j] = rr * 128 + ((c ^ (rr & 7)) << 4);
         src[j] = xrows + c * 16;
         if (rr < p.BM) {
-          src[j] = task.phase == 0 ? xrows + (size_t)rows[rr] * xpitch + c * 16
-                                   : hblock + (size_t)rr * p.I * 2 + c * 16;
+          src[j] = task.phase == 0 ? xrows + (size_t)rows[rr] * xpitch + c * 16 : hblock + (size_t)rr * hpitch + c * 16;
           nrows = j + 1;
         }
       }
@@ -744,11 +745,18 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
     release_task_slot2(q_task, is_leader, s);   // rows read: the slot may be refilled
     // L2: this CTA's half of the W2 tile too (BN2/2 columns: one or two 64x64
     // boxes, each 64 K-rows of 128 bytes in the same 128-byte swizzle as TMA)
-    const int nhalf = task.phase == 1 ? p.BN2 / 128 : 0;
-    const bf16* w2src = (task.e >= p.E ? p.ws2 + (size_t)(task.e - p.E) * p.I * p.H : p.w2 + (size_t)task.e * p.I * p.H) +
-                        task.n * p.BN2 + (int)rank * (p.BN2 / 2) + c * 8;
-    const int nk = task.phase == 0 ? l1_ksteps2(p) : p.I / kBK;
+    const int nhalf = task.phase == 1 && !p.fp8 ? p.BN2 / 128 : 0;
+    const int nchunk8 = task.phase == 1 && p.fp8 ? (p.BN2 / 2) * 8 / (32 * kGatherWarps) : 0;   // 8, or 4 (BN2 = 128)
+    const uint8_t* w2row8 =
+        p.fp8 ? p.w2q + ((size_t)task.e * p.H + task.n * p.BN2 + (int)rank * (p.BN2 / 2)) * p.I : nullptr;
+    const int tl = g * 32 + lane;
+    const bf16* w2src = p.fp8 ? nullptr
+                              : (task.e >= p.E ? p.ws2 + (size_t)(task.e - p.E) * p.I * p.H
+                                               : p.w2 + (size_t)task.e * p.I * p.H) +
+                                    task.n * p.BN2 + (int)rank * (p.BN2 / 2) + c * 8;
+    const int nk = task.phase == 0 ? l1_ksteps2(p) : l2_ksteps2(p);
     bool ok = true;
+
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait2(&s.empty[stage], phase ^ 1, p, s, 13)) {
         ok = false;
@@ -765,6 +773,13 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
           ptx::cp_async_16_hint(a_addr + kTileABytes + j * kBoxBytes + kr * 128 + ((c ^ (kr & 7)) << 4),
                                 w2src + (size_t)(kb * kBK + kr) * p.H + j * 64, wpol);
         }
+      }
+      // FP8 L2: this CTA's W2 codes, BN2/2 rows of 128 bytes (8 chunks per row), K-major
+      for (int i = 0; i < nchunk8; ++i) {
+        const int qc = i * 32 * kGatherWarps + tl;   // chunk: row qc / 8, 16 bytes (qc & 7)
+        const int wr = qc >> 3, wc = qc & 7;
+        ptx::cp_async_16_hint(a_addr + kTileABytes + wr * 128 + ((wc ^ (wr & 7)) << 4),
+                              w2row8 + (size_t)wr * p.I + kb * 128 + wc * 16, wpol);
       }
       ptx::cp_async_mbar_arrive_noinc(&s.full[stage]);
       if (++stage == kStages2) {

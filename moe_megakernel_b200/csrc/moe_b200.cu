@@ -32,7 +32,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 struct Layout {
   size_t err, sched, topk_idx, topk_w, rank, chunk_count, expert_count, expert_offset, block_start, num_padded,
       slot_token, slot_topk, l1_done, l2_done, group_start, pair_start, router_partial, router_counter, h, y_acc,
-      x_stage, y_stage, x_q, s_x, total;
+      x_stage, y_stage, x_q, s_x, h8, act_amax, act_scale, total;
 };
 
 class DeviceGuard {
@@ -113,6 +113,7 @@ struct moe_plan {
   int pair_clusters = 0;                               // co-resident clusters of the pair kernel
   int pgroup_min, pgroup_max, pmax_groups, ring_pairs; // the same in units of block pairs
   int per_expert;                                      // expected blocks per expert + 1
+  int fp8_rows = 0;                                    // FP8 plans: activation rows of all blocks or pairs
   Layout L;
   uint8_t* ws = nullptr;
   size_t ws_bytes = 0;
@@ -164,12 +165,16 @@ static Layout make_layout(const moe_plan& p) {
   // split-H router: per token tile (fewer tiles than SMs) a logits accumulator and an arrival counter
   L.router_partial = take((size_t)p.num_sms * kRouterTokens * 256 * 4, 256);
   L.router_counter = take((size_t)p.num_sms * 4, 256);
-  L.h = take((size_t)std::max(p.ring_blocks, 2 * p.ring_pairs) * p.BM * p.I * 2, 1024);
+  L.h = take((size_t)std::max({p.ring_blocks * p.BM, 2 * p.ring_pairs * p.BM, p.fp8_rows}) * p.I * 2, 1024);
   L.y_acc = take((size_t)p.T_max * p.H * 4, 1024);
   L.x_stage = take((size_t)p.T_max * p.H * 2, 1024);
   L.y_stage = take((size_t)p.T_max * p.H * 2, 1024);
   L.x_q = take((size_t)p.T_max * p.H, 1024);   // FP8 first GEMM: x codes and token scales
   L.s_x = take((size_t)p.T_max * 4, 256);
+  // FP8 plans: the activation of every block (or pair) at once, its codes and row amax / scale
+  L.h8 = take((size_t)p.fp8_rows * p.I, 1024);
+  L.act_amax = take((size_t)p.fp8_rows * 4, 256);
+  L.act_scale = take((size_t)p.fp8_rows * 4, 256);
   L.total = align_up(o, 1024);
   return L;
 }
@@ -213,27 +218,32 @@ struct SharedWeights {
   const void* Ws2;   // [S, I, H]
 };
 
-// FP8 E4M3 first GEMM: K-major codes of W1 / W3 [E, I, H] and their column scales [E, I].
-struct Fp8First {
+// FP8 E4M3 expert GEMMs: K-major codes of W1 / W3 [E, I, H] and W2 [E, H, I]
+// with their column scales [E, I] and [E, H].
+struct Fp8Weights {
   const void* W1q;
   const float* s1;
   const void* W3q;
   const float* s3;
+  const void* W2q;
+  const float* s2;
 };
 
 static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias, const void* W1, const void* W3,
                    const void* W2, const SharedWeights& sw, int T, void* y, cudaStream_t st, bool full,
-                   const Fp8First* f8 = nullptr) {
+                   const Fp8Weights* f8 = nullptr) {
   if (p->ws == nullptr) return MOE_ERR_NO_WORKSPACE;
   if (T < 0 || T > p->T_max) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;   // nothing to do; empty tensors may carry null pointers
   if (x == nullptr || Wg == nullptr || !aligned16(x) || !aligned16(Wg)) return MOE_ERR_INVALID_ARG;
   if (bias != nullptr && (reinterpret_cast<uintptr_t>(bias) & 3u)) return MOE_ERR_INVALID_ARG;
-  if (f8 != nullptr) {   // the FP8 operands stand in for W1 / W3
-    if (p->S > 0 || f8->s1 == nullptr || f8->s3 == nullptr) return MOE_ERR_INVALID_ARG;
-    if (!aligned16(f8->s1) || !aligned16(f8->s3)) return MOE_ERR_INVALID_ARG;
+  if (f8 != nullptr) {   // the FP8 operands stand in for W1 / W3 / W2
+    if (p->fp8_rows == 0) return MOE_ERR_INVALID_ARG;   // the plan's workspace has no FP8 regions
+    if (p->S > 0 || f8->s1 == nullptr || f8->s3 == nullptr || f8->s2 == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(f8->s1) || !aligned16(f8->s3) || !aligned16(f8->s2)) return MOE_ERR_INVALID_ARG;
     W1 = f8->W1q;
     W3 = f8->W3q;
+    W2 = f8->W2q;
   }
   if (full) {
     if (W1 == nullptr || W3 == nullptr || W2 == nullptr || y == nullptr) return MOE_ERR_INVALID_ARG;
@@ -332,6 +342,7 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   dp.pair_start = p->cta_pairs ? reinterpret_cast<int32_t*>(ws + L.pair_start) : nullptr;
   dp.group_min = p->cta_pairs ? p->pgroup_min : p->group_min;
   dp.group_max = p->cta_pairs ? p->pgroup_max : p->group_max;
+  if (f8 != nullptr) dp.group_min = dp.group_max = 1 << 30;   // FP8: one block group (two one-phase launches)
   dp.max_groups = p->cta_pairs ? p->pmax_groups : p->max_groups;
   mark(1);
   moe_dispatch_scan_kernel<<<1, kScanThreads, 0, st>>>(dp);
@@ -349,9 +360,23 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     return MOE_OK;
   }
 
-  // 4. persistent expert GEMM (L1 + SwiGLU, L2 + weighted scatter-add)
+  // 4. persistent expert GEMM (L1 + SwiGLU, L2 + weighted scatter-add). With
+  // FP8 operands the two GEMMs are two launches of the same kernel around the
+  // activation quantizer (each activation row is quantized once, with the
+  // scale of its full amax, which the first launch gathers).
   bf16* h = reinterpret_cast<bf16*>(ws + L.h);
   const int E = p->E, H = p->H, I = p->I;
+  float* act_amax = reinterpret_cast<float*>(ws + L.act_amax);
+  float* act_scale = reinterpret_cast<float*>(ws + L.act_scale);
+  uint8_t* h8 = ws + L.h8;
+  const int h8_rows = p->fp8_rows;
+  if (f8 != nullptr && cudaMemsetAsync(act_amax, 0, (size_t)h8_rows * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+  // between the two FP8 launches: quantize the activation rows, restart the task counter
+  auto quantize_activation = [&](const int32_t* units, int unit_rows) -> bool {
+    const int grid = p->num_sms * 8;
+    moe_quantize_act_kernel<<<grid, 256, 0, st>>>(h, act_amax, h8, act_scale, units, unit_rows, h8_rows, I);
+    return cudaGetLastError() == cudaSuccess && cudaMemsetAsync(dp.sched, 0, 4, st) == cudaSuccess;
+  };
   if (p->cta_pairs) {
     Gemm2Params gp;
     std::memset(&gp, 0, sizeof(gp));
@@ -363,14 +388,21 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
            make_map(&gp.tm_ws3, sw.Ws3, I, (uint64_t)p->S * H, I, 64);
     if (!ok) return MOE_ERR_CUDA;
     gp.x = static_cast<const bf16*>(x);
+    gp.phase_only = -1;
     if (f8 != nullptr) {
       gp.fp8 = 1;
       gp.xq = ws + L.x_q;
       gp.sx = reinterpret_cast<const float*>(ws + L.s_x);
       gp.s1 = f8->s1;
       gp.s3 = f8->s3;
+      gp.w2q = static_cast<const uint8_t*>(f8->W2q);
+      gp.s2 = f8->s2;
+      gp.act_amax = act_amax;
+      gp.act_scale = act_scale;
+      gp.h8 = h8;
+      gp.phase_only = 0;
     }
-    gp.w2 = static_cast<const bf16*>(W2);
+    gp.w2 = f8 != nullptr ? nullptr : static_cast<const bf16*>(W2);
     gp.ws2 = static_cast<const bf16*>(sw.Ws2);
     gp.S = p->S;
     gp.slot_token = dp.slot_token;
@@ -395,7 +427,7 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     gp.BN2 = p->BN2;
     gp.N1 = p->N1;
     gp.N2 = p->N2;
-    gp.ring_pairs = p->ring_pairs;
+    gp.ring_pairs = f8 != nullptr ? p->fp8_rows / (2 * p->BM) : p->ring_pairs;   // FP8: every pair its own rows
     gp.max_groups = p->pmax_groups;
     gp.timeout_ns = p->timeout_ns;
     gp.withhold_pair = p->withhold;
@@ -413,14 +445,20 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, moe_expert_gemm2_kernel, gp) != cudaSuccess) return MOE_ERR_CUDA;
+    if (f8 != nullptr) {
+      if (!quantize_activation(dp.pair_start + E, 2 * p->BM)) return MOE_ERR_CUDA;
+      gp.phase_only = 1;
+      if (cudaLaunchKernelEx(&cfg, moe_expert_gemm2_kernel, gp) != cudaSuccess) return MOE_ERR_CUDA;
+    }
   } else {
     GemmParams gp;
     std::memset(&gp, 0, sizeof(gp));
-    bool ok = (f8 != nullptr ? make_map_u8(&gp.tm_w1, W1, H, (uint64_t)E * I) &&
-                                   make_map_u8(&gp.tm_w3, W3, H, (uint64_t)E * I)
-                             : make_map(&gp.tm_w1, W1, I, (uint64_t)E * H, I, 64) &&
-                                   make_map(&gp.tm_w3, W3, I, (uint64_t)E * H, I, 64)) &&
-              make_map(&gp.tm_w2, W2, H, (uint64_t)E * I, H, 64);
+    bool ok = f8 != nullptr ? make_map_u8(&gp.tm_w1, W1, H, (uint64_t)E * I) &&
+                                  make_map_u8(&gp.tm_w3, W3, H, (uint64_t)E * I) &&
+                                  make_map_u8(&gp.tm_w2, W2, I, (uint64_t)E * H)
+                            : make_map(&gp.tm_w1, W1, I, (uint64_t)E * H, I, 64) &&
+                                  make_map(&gp.tm_w3, W3, I, (uint64_t)E * H, I, 64) &&
+                                  make_map(&gp.tm_w2, W2, H, (uint64_t)E * I, H, 64);
     if (ok && p->S > 0)
       ok = make_map(&gp.tm_ws1, sw.Ws1, I, (uint64_t)p->S * H, I, 64) &&
            make_map(&gp.tm_ws3, sw.Ws3, I, (uint64_t)p->S * H, I, 64) &&
@@ -428,12 +466,18 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     if (!ok) return MOE_ERR_CUDA;
     gp.S = p->S;
     gp.x = static_cast<const bf16*>(x);
+    gp.phase_only = -1;
     if (f8 != nullptr) {
       gp.fp8 = 1;
       gp.xq = ws + L.x_q;
       gp.sx = reinterpret_cast<const float*>(ws + L.s_x);
       gp.s1 = f8->s1;
       gp.s3 = f8->s3;
+      gp.s2 = f8->s2;
+      gp.act_amax = act_amax;
+      gp.act_scale = act_scale;
+      gp.h8 = h8;
+      gp.phase_only = 0;
     }
     gp.slot_token = dp.slot_token;
     gp.slot_topk = dp.slot_topk;
@@ -444,7 +488,7 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     gp.task_counter = dp.sched;
     gp.l1_done = dp.l1_done;
     gp.l2_done = dp.l2_done;
-    gp.ring_blocks = p->ring_blocks;
+    gp.ring_blocks = f8 != nullptr ? p->fp8_rows / p->BM : p->ring_blocks;   // FP8: every block its own rows
     gp.max_groups = p->max_groups;
     gp.err = dp.err;
     gp.h = h;
@@ -461,6 +505,12 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     gp.timeout_ns = p->timeout_ns;
     gp.withhold_block = p->withhold;
     moe_expert_gemm_kernel<<<p->num_sms, kGemm1Threads, kGemmSmemBytes, st>>>(gp);
+    if (f8 != nullptr) {
+      if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+      if (!quantize_activation(dp.sched + 1, p->BM)) return MOE_ERR_CUDA;
+      gp.phase_only = 1;
+      moe_expert_gemm_kernel<<<p->num_sms, kGemm1Threads, kGemmSmemBytes, st>>>(gp);
+    }
   }
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   mark(4);
@@ -801,7 +851,7 @@ int moe_route(moe_plan_t p, const void* x, const void* Wg, const float* bias, in
 
 static int forward_host(moe_plan_t p, const void* x_host, const void* Wg, const float* bias, const void* W1,
                         const void* W3, const void* W2, const SharedWeights& sw, int T, void* y_host, void* stream,
-                        const Fp8First* f8 = nullptr) {
+                        const Fp8Weights* f8 = nullptr) {
   if (p == nullptr || x_host == nullptr || y_host == nullptr) return MOE_ERR_INVALID_ARG;
   if (p->ws == nullptr) return MOE_ERR_NO_WORKSPACE;
   if (T < 0 || T > p->T_max) return MOE_ERR_INVALID_ARG;
@@ -831,18 +881,18 @@ int moe_forward_host_shared(moe_plan_t p, const void* x_host, const void* Wg, co
 }
 
 int moe_forward_fp8(moe_plan_t p, const void* x, const void* Wg, const float* bias, const void* W1q, const float* s1,
-                    const void* W3q, const float* s3, const void* W2, int T, void* y, void* stream) {
+                    const void* W3q, const float* s3, const void* W2q, const float* s2, int T, void* y, void* stream) {
   if (p == nullptr) return MOE_ERR_INVALID_ARG;
-  const Fp8First f8{W1q, s1, W3q, s3};
-  return enqueue(p, x, Wg, bias, nullptr, nullptr, W2, SharedWeights{}, T, y, static_cast<cudaStream_t>(stream), true,
-                 &f8);
+  const Fp8Weights f8{W1q, s1, W3q, s3, W2q, s2};
+  return enqueue(p, x, Wg, bias, nullptr, nullptr, nullptr, SharedWeights{}, T, y, static_cast<cudaStream_t>(stream),
+                 true, &f8);
 }
 
 int moe_forward_host_fp8(moe_plan_t p, const void* x_host, const void* Wg, const float* bias, const void* W1q,
-                         const float* s1, const void* W3q, const float* s3, const void* W2, int T, void* y_host,
-                         void* stream) {
-  const Fp8First f8{W1q, s1, W3q, s3};
-  return forward_host(p, x_host, Wg, bias, nullptr, nullptr, W2, SharedWeights{}, T, y_host, stream, &f8);
+                         const float* s1, const void* W3q, const float* s3, const void* W2q, const float* s2, int T,
+                         void* y_host, void* stream) {
+  const Fp8Weights f8{W1q, s1, W3q, s3, W2q, s2};
+  return forward_host(p, x_host, Wg, bias, nullptr, nullptr, nullptr, SharedWeights{}, T, y_host, stream, &f8);
 }
 
 int moe_quantize_x_fp8(const void* x, void* xq, float* sx, int T, int H, void* stream) {
@@ -926,6 +976,18 @@ int moe_plan_set_debug(moe_plan_t p, int withhold_block, uint64_t timeout_ns) {
   if (p == nullptr) return MOE_ERR_INVALID_ARG;
   p->withhold = withhold_block;
   p->timeout_ns = timeout_ns ? timeout_ns : 2000000000ull;
+  return MOE_OK;
+}
+
+int moe_plan_set_fp8(moe_plan_t p, int enable) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  if (enable && p->S > 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  // every block, or every pair of blocks of one expert (at most one half-empty pair per expert)
+  const int pairs_cap = std::min(p->blocks_max, (p->blocks_max + p->E + 1) / 2);
+  p->fp8_rows = enable ? std::max(p->blocks_max, 2 * pairs_cap) * p->BM : 0;
+  p->L = make_layout(*p);
+  p->ws = nullptr;   // the workspace size changed: bind again
+  p->ws_bytes = 0;
   return MOE_OK;
 }
 

@@ -1,6 +1,7 @@
-// FP8 E4M3 operands of the first expert GEMM: per-token quantization of x and
-// the one-time per-(expert, column) quantization of W1 / W3 into the K-major
-// layout the tcgen05 kind::f8f6f4 MMA reads.
+// FP8 E4M3 operands of the expert GEMMs: per-token quantization of x, the
+// one-time per-(expert, column) quantization of W1 / W3 / W2 into the K-major
+// layout the tcgen05 kind::f8f6f4 MMA reads, and the bf16 -> E4M3 conversion
+// the expert GEMM applies to the activation rows it loads.
 //
 // "MegaMoE 在 MoE 系统谱系中的位置", section 一 (the Mega MoE GEMMs take 8-bit
 // operands with scale factors loaded beside them) and section 2.1 (amax and
@@ -24,6 +25,19 @@ __device__ __forceinline__ int pow2_scale_exp(float amax) {
   int e;
   const float m = frexpf(amax / kE4m3Max, &e);   // amax/448 = m * 2**e, m in [0.5, 1)
   return m == 0.5f ? e - 1 : e;
+}
+
+// Eight bf16 values (one uint4) times `inv` (an exact power of two) -> eight E4M3 codes, in order.
+__device__ __forceinline__ uint2 bf16x8_to_e4m3(const uint4 v, float inv) {
+  const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
+  uint32_t w[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const float2 f0 = __bfloat1622float2(b[2 * j]);
+    const float2 f1 = __bfloat1622float2(b[2 * j + 1]);
+    w[j] = (uint32_t)ptx::cvt_e4m3x2(f0.x * inv, f0.y * inv) | ((uint32_t)ptx::cvt_e4m3x2(f1.x * inv, f1.y * inv) << 16);
+  }
+  return make_uint2(w[0], w[1]);
 }
 
 // One warp per token: amax over the row, then codes xq = e4m3(x * 2**-k) and sx = 2**k.
@@ -50,17 +64,28 @@ __global__ void __launch_bounds__(256) moe_quantize_x_kernel(const bf16* __restr
   const float inv = ldexpf(1.f, -k);
   if (lane == 0) sx[warp] = ldexpf(1.f, k);
   uint2* out = reinterpret_cast<uint2*>(xq + (size_t)warp * H);   // 8 codes per uint2
-  for (int i = lane; i < n8; i += 32) {
-    const uint4 v = __ldg(row + i);
-    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
-    uint32_t w[2];
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const float2 f0 = __bfloat1622float2(b[2 * j]);
-      const float2 f1 = __bfloat1622float2(b[2 * j + 1]);
-      w[j] = (uint32_t)ptx::cvt_e4m3x2(f0.x * inv, f0.y * inv) | ((uint32_t)ptx::cvt_e4m3x2(f1.x * inv, f1.y * inv) << 16);
-    }
-    out[i] = make_uint2(w[0], w[1]);
+  for (int i = lane; i < n8; i += 32) out[i] = bf16x8_to_e4m3(__ldg(row + i), inv);
+}
+
+// Second-GEMM operand of the FP8 layer: every h row (bf16, I columns) to E4M3
+// codes with the row's power-of-two scale, from the row amax the first GEMM's
+// epilogues gathered. Rows: *units * unit_rows (blocks or block pairs of the
+// dispatch); one warp per row, grid-stride. act_scale[row] = the scale 2**k.
+__global__ void __launch_bounds__(256) moe_quantize_act_kernel(const bf16* __restrict__ h,
+                                                               const float* __restrict__ act_amax,
+                                                               uint8_t* __restrict__ h8, float* __restrict__ act_scale,
+                                                               const int32_t* __restrict__ units, int unit_rows,
+                                                               int max_rows, int I) {
+  const int nrows = min(*units * unit_rows, max_rows);
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < nrows; row += warps) {
+    const int k = pow2_scale_exp(__ldcg(act_amax + row));
+    const float inv = ldexpf(1.f, -k);
+    if (lane == 0) act_scale[row] = ldexpf(1.f, k);
+    const uint4* in = reinterpret_cast<const uint4*>(h + (size_t)row * I);
+    uint2* out = reinterpret_cast<uint2*>(h8 + (size_t)row * I);
+    for (int i = lane; i < I / 8; i += 32) out[i] = bf16x8_to_e4m3(__ldcg(in + i), inv);
   }
 }
 

@@ -1,12 +1,12 @@
-"""FP8 E4M3 first GEMM on the GPU against the oracle.
+"""FP8 E4M3 expert GEMMs on the GPU against the oracle.
 
 "MegaMoE 在 MoE 系统谱系中的位置", section 一 (the expert GEMMs take 8-bit
 operands with scale factors beside them) and section 2.1 (activation amax and
-quantization): x is quantized per token, W1 / W3 per (expert, column), with
-power-of-two scales, and x.W1, x.W3 run on tcgen05 kind::f8f6f4; h and W2
-stay bf16. Codes and scales are compared bit-exactly with the oracle's
-(both sides convert the same fp32 / fp64-exact quotient with round to nearest
-even), y with the layer tolerances on the oracle's FP8 layer.
+quantization between the GEMMs): x and the activation are quantized per
+token, W1 / W3 / W2 per (expert, column), with power-of-two scales, and both
+GEMMs run on tcgen05 kind::f8f6f4. Codes and scales are compared bit-exactly
+with the oracle's (both sides convert the same fp32 / fp64-exact quotient with
+round to nearest even), y with the layer tolerances on the oracle's FP8 layer.
 """
 import numpy as np
 import pytest
@@ -94,7 +94,8 @@ def _fp8_weights(inp):
     from moe_megakernel_b200 import quantize_weights_fp8
     W1q, s1 = quantize_weights_fp8(inp["W1"])
     W3q, s3 = quantize_weights_fp8(inp["W3"])
-    return W1q, s1, W3q, s3
+    W2q, s2 = quantize_weights_fp8(inp["W2"])
+    return W1q, s1, W3q, s3, W2q, s2
 
 
 @pytest.mark.parametrize("pairs", [True, False], ids=["pairs", "single"])
@@ -103,17 +104,19 @@ def test_fp8_forward_matches_oracle(T, H, I, E, k, bm, zipf, pairs):
     from moe_megakernel_b200 import MoEPlan
     shape = custom_shape(T, H, I, E, k, zipf)
     inp = make_inputs(shape, device=DEV)
-    plan = MoEPlan(T, H, I, E, k, block_m=bm)
+    plan = MoEPlan(T, H, I, E, k, block_m=bm, fp8=True)
     plan.set_cta_pairs(pairs)
     plan.workspace.fill_(0xFF)   # poison: unwritten reads show up as NaN
     plan.lib.moe_plan_bind_workspace(plan._plan, plan.workspace.data_ptr(), plan.workspace_bytes)
-    W1q, s1, W3q, s3 = _fp8_weights(inp)
-    y = plan.forward_fp8(inp["x"], inp["Wg"], inp["bias"], W1q, s1, W3q, s3, inp["W2"])
+    fw = _fp8_weights(inp)
+    y = plan.forward_fp8(inp["x"], inp["Wg"], inp["bias"], *fw)
     plan.check()
     ref = oracle_forward(inp, block_m=plan.block_m, fp8=True)
     assert_routing_equal(plan.routing(T), ref)
     fro, mx = assert_y_close(y, ref["y"], "y (fp8)")
     # the FP8 layer differs from the bf16 one by the quantization, well above the kernel's own error
+    # (the W2 codes are [E, H, I]: W2 transposed per expert)
+    assert fw[4].shape == (E, H, I) and fw[5].shape == (E, H)
     ref16 = oracle_forward(inp, block_m=plan.block_m)
     q_err = np.linalg.norm(ref["y"] - ref16["y"]) / np.linalg.norm(ref16["y"])
     print(f"fp8 {'pairs' if pairs else 'single'} T={T} H={H} I={I} E={E} k={k} BM={plan.block_m}: "
@@ -124,21 +127,32 @@ def test_fp8_forward_rejects_shared_plan_and_bad_pointers():
     from moe_megakernel_b200 import MoEPlan
     shape = custom_shape(64, 128, 256, 8, 2)
     inp = make_inputs(shape, device=DEV)
-    W1q, s1, W3q, s3 = _fp8_weights(inp)
+    fw = _fp8_weights(inp)
     y = torch.empty_like(inp["x"])
+    W1q, s1, W3q, s3, W2q, s2 = fw
     shared = MoEPlan(64, 128, 256, 8, 2, n_shared=1)
     rc = shared.lib.moe_forward_fp8(shared._plan, inp["x"].data_ptr(), inp["Wg"].data_ptr(), None,
                                     W1q.data_ptr(), s1.data_ptr(), W3q.data_ptr(), s3.data_ptr(),
-                                    inp["W2"].data_ptr(), 64, y.data_ptr(), None)
-    assert rc == 1   # MOE_ERR_INVALID_ARG: FP8 first GEMM without shared experts
-    plan = MoEPlan(64, 128, 256, 8, 2)
-    rc = plan.lib.moe_forward_fp8(plan._plan, inp["x"].data_ptr(), inp["Wg"].data_ptr(), None,
-                                  W1q.data_ptr(), None, W3q.data_ptr(), s3.data_ptr(),
-                                  inp["W2"].data_ptr(), 64, y.data_ptr(), None)
-    assert rc == 1   # missing column scales
+                                    W2q.data_ptr(), s2.data_ptr(), 64, y.data_ptr(), None)
+    assert rc == 1   # MOE_ERR_INVALID_ARG: the FP8 layer has no shared experts
+    assert shared.lib.moe_plan_set_fp8(shared._plan, 1) == 2   # MOE_ERR_UNSUPPORTED_SHAPE: shared experts
+    plain = MoEPlan(64, 128, 256, 8, 2)   # no FP8 workspace regions
+    rc = plain.lib.moe_forward_fp8(plain._plan, inp["x"].data_ptr(), inp["Wg"].data_ptr(), None,
+                                   W1q.data_ptr(), s1.data_ptr(), W3q.data_ptr(), s3.data_ptr(),
+                                   W2q.data_ptr(), s2.data_ptr(), 64, y.data_ptr(), None)
+    assert rc == 1
+    plan = MoEPlan(64, 128, 256, 8, 2, fp8=True)
+    assert plan.workspace_bytes > plain.workspace_bytes
+    for missing in ("s1", "s2"):
+        rc = plan.lib.moe_forward_fp8(plan._plan, inp["x"].data_ptr(), inp["Wg"].data_ptr(), None,
+                                      W1q.data_ptr(), None if missing == "s1" else s1.data_ptr(), W3q.data_ptr(),
+                                      s3.data_ptr(), W2q.data_ptr(), None if missing == "s2" else s2.data_ptr(),
+                                      64, y.data_ptr(), None)
+        assert rc == 1   # missing column scales
     with pytest.raises(ValueError):
-        plan.forward_fp8(inp["x"], inp["Wg"], None, inp["W1"], s1, W3q, s3, inp["W2"])   # bf16 W1: wrong layout
+        plan.forward_fp8(inp["x"], inp["Wg"], None, W1q, s1, W3q, s3, inp["W2"], s2)   # bf16 W2: wrong layout
     shared.check()
+    plain.check()
     plan.check()
 
 
@@ -146,13 +160,13 @@ def test_fp8_host_entry_matches_device_entry():
     from moe_megakernel_b200 import MoEPlan
     shape = custom_shape(300, 256, 384, 16, 4)
     inp = make_inputs(shape, device=DEV)
-    W1q, s1, W3q, s3 = _fp8_weights(inp)
-    plan = MoEPlan(shape.T, shape.H, shape.I, shape.E, shape.k)
-    y = plan.forward_fp8(inp["x"], inp["Wg"], None, W1q, s1, W3q, s3, inp["W2"]).float()
+    fw = _fp8_weights(inp)
+    plan = MoEPlan(shape.T, shape.H, shape.I, shape.E, shape.k, fp8=True)
+    y = plan.forward_fp8(inp["x"], inp["Wg"], None, *fw).float()
     plan.check()
     x_host = inp["x"].cpu().pin_memory()
     y_host = torch.empty((shape.T, shape.H), dtype=torch.bfloat16).pin_memory()
-    plan.forward_host_fp8(x_host, inp["Wg"], None, W1q, s1, W3q, s3, inp["W2"], y_host)
+    plan.forward_host_fp8(x_host, inp["Wg"], None, *fw, y_host)
     plan.check()
     assert (y_host.float() - y.cpu()).abs().max().item() <= 1e-2
 
@@ -164,9 +178,9 @@ def test_fp8_workload_matches_oracle(name):
     from moe_megakernel_b200 import MoEPlan
     shape = WORKLOADS[name]
     inp = make_inputs(shape, device=DEV)
-    W1q, s1, W3q, s3 = _fp8_weights(inp)
-    plan = MoEPlan(shape.T, shape.H, shape.I, shape.E, shape.k)
-    y = plan.forward_fp8(inp["x"], inp["Wg"], inp["bias"], W1q, s1, W3q, s3, inp["W2"])
+    fw = _fp8_weights(inp)
+    plan = MoEPlan(shape.T, shape.H, shape.I, shape.E, shape.k, fp8=True)
+    y = plan.forward_fp8(inp["x"], inp["Wg"], inp["bias"], *fw)
     plan.check()
     rows = sample_tokens(shape.T, {"mixtral": 8, "fine_grained_prefill": 4, "decode": 4}[name])
     # (few tokens: the oracle quantizes every expert a sampled token reaches, in fp64)

@@ -222,8 +222,10 @@ __device__ __forceinline__ Task decode_task(int t, const GemmSmem& s, const Gemm
 __device__ __forceinline__ uint8_t* stage_ptr(uint8_t* tiles, int stage) { return tiles + stage * kStageBytes; }
 
 // K blocks of an L1 task: 64 bf16 or 128 FP8 elements, one 128-byte swizzle row either way.
-__device__ __forceinline__ int l1_ksteps(const GemmParams& p) { return p.fp8 ? p.H / 128 : p.H / kBK; }
-__device__ __forceinline__ int l2_ksteps(const GemmParams& p) { return p.fp8 ? p.I / 128 : p.I / kBK; }
+template <bool F8>
+__device__ __forceinline__ int l1_ksteps(const GemmParams& p) { return F8 ? p.H / 128 : p.H / kBK; }
+template <bool F8>
+__device__ __forceinline__ int l2_ksteps(const GemmParams& p) { return F8 ? p.I / 128 : p.I / kBK; }
 
 // ---------------------------------------------------------------- scheduler (last warp)
 // Claims tasks from the global counter, decodes them, stages the routed row
@@ -258,6 +260,7 @@ __device__ __forceinline__ bool wait_taken(int n, const GemmParams& p, GemmSmem&
   return true;
 }
 
+template <bool F8>
 __device__ void gemm_scheduler(const GemmParams& p, GemmSmem& s) {
   const int lane = ptx::lane_id();
   int q = 0;
@@ -314,6 +317,7 @@ __device__ void gemm_scheduler(const GemmParams& p, GemmSmem& s) {
 
 // ---------------------------------------------------------------- producer (warp 0)
 // Weight-tile TMA (and the h tiles of L2 tasks) for the tasks the scheduler publishes.
+template <bool F8>
 __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) {
   const int lane = ptx::lane_id();
   // Weight tiles are streamed: the few m-blocks sharing a slice read it at
@@ -339,7 +343,7 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
     }
     if (task.phase < 0) break;
 
-    const int nk = task.phase == 0 ? l1_ksteps(p) : l2_ksteps(p);
+    const int nk = task.phase == 0 ? l1_ksteps<F8>(p) : l2_ksteps<F8>(p);
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait(&s.empty[stage], phase ^ 1, p, s, 2)) {
         ok = false;
@@ -352,7 +356,7 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
         if (lane == 0) {
           ptx::mbar_arrive_expect_tx(&s.full[stage], 4 * kBoxBytes);
           const int n0 = task.n * kL1TileN;
-          if (p.fp8) {
+          if (F8) {
             // K-major FP8 codes: 64 rows (columns of I) x 128 bytes (K) per box
 #pragma unroll
             for (int j = 0; j < 4; ++j)
@@ -371,7 +375,7 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
         }
       } else {
         // B: 256 (or 128) columns of W2; A (the block's h rows) comes from the gather warps.
-        if (lane == 0 && p.fp8) {   // K-major E4M3 codes: BN2 rows of 128 bytes, 64 per box
+        if (lane == 0 && F8) {   // K-major E4M3 codes: BN2 rows of 128 bytes, 64 per box
           const int nbox = p.BN2 / 64;
           ptx::mbar_arrive_expect_tx(&s.full[stage], nbox * kBoxBytes);
           for (int j = 0; j < nbox; ++j)
@@ -408,12 +412,13 @@ __device__ void gemm_producer(const GemmParams& p, GemmSmem& s, uint8_t* tiles) 
 }
 
 // ---------------------------------------------------------------- MMA issuer (warp 1)
+template <bool F8>
 __device__ void gemm_mma(const GemmParams& p, GemmSmem& s, uint8_t* tiles, uint32_t tmem_base) {
   const int lane = ptx::lane_id();
   const uint32_t idesc_l1 =
-      p.fp8 ? ptx::idesc_e4m3_f32(128, 2 * kL1TileN) : ptx::idesc_bf16_f32(128, 2 * kL1TileN, false, true);
-  const bool f8 = p.fp8 != 0;
-  const uint32_t idesc_l2 = p.fp8 ? ptx::idesc_e4m3_f32(128, p.BN2) : ptx::idesc_bf16_f32(128, p.BN2, false, true);
+      F8 ? ptx::idesc_e4m3_f32(128, 2 * kL1TileN) : ptx::idesc_bf16_f32(128, 2 * kL1TileN, false, true);
+  constexpr bool f8 = F8;
+  const uint32_t idesc_l2 = F8 ? ptx::idesc_e4m3_f32(128, p.BN2) : ptx::idesc_bf16_f32(128, p.BN2, false, true);
   int stage = 0;
   uint32_t phase = 0;
   int q = 0;
@@ -435,7 +440,7 @@ __device__ void gemm_mma(const GemmParams& p, GemmSmem& s, uint8_t* tiles, uint3
     ptx::tc_fence_after();
     const uint32_t d_tmem = tmem_base + acc * 256;
     const uint32_t idesc = task.phase == 0 ? idesc_l1 : idesc_l2;
-    const int nk = task.phase == 0 ? l1_ksteps(p) : l2_ksteps(p);
+    const int nk = task.phase == 0 ? l1_ksteps<F8>(p) : l2_ksteps<F8>(p);
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait(&s.full[stage], phase, p, s, 5)) {
@@ -499,6 +504,7 @@ __device__ void gemm_mma(const GemmParams& p, GemmSmem& s, uint8_t* tiles, uint3
 // lane arrives on the stage's full barrier when its own copies have landed.
 // L2 tasks: the same for the block's BM rows of h in the ring (a single
 // 128-row TMA box per stage kept the tensor pipe waiting twice as long).
+template <bool F8>
 __device__ void gemm_gather(const GemmParams& p, GemmSmem& s, uint8_t* tiles, int g) {
   constexpr int kRowsPerLane = (kTileM / 4 + kGatherWarps - 1) / kGatherWarps;   // rows >= BM are skipped
   const int lane = ptx::lane_id();
@@ -524,11 +530,11 @@ __device__ void gemm_gather(const GemmParams& p, GemmSmem& s, uint8_t* tiles, in
     const uint8_t* src[kRowsPerLane];
     const int* rows = s.rows[q_task];
     // activation rows: bf16, or FP8 codes (rows of I bytes); x rows: bf16, or FP8 codes
-    const size_t hpitch = p.fp8 ? (size_t)p.I : (size_t)p.I * 2;
+    const size_t hpitch = F8 ? (size_t)p.I : (size_t)p.I * 2;
     const int ring_row0 = (task.b % p.ring_blocks) * p.BM;
-    const uint8_t* hblock = (p.fp8 ? p.h8 : reinterpret_cast<const uint8_t*>(p.h)) + (size_t)ring_row0 * hpitch;
-    const uint8_t* xrows = p.fp8 ? p.xq : reinterpret_cast<const uint8_t*>(p.x);
-    const size_t xpitch = p.fp8 ? (size_t)p.H : (size_t)p.H * 2;
+    const uint8_t* hblock = (F8 ? p.h8 : reinterpret_cast<const uint8_t*>(p.h)) + (size_t)ring_row0 * hpitch;
+    const uint8_t* xrows = F8 ? p.xq : reinterpret_cast<const uint8_t*>(p.x);
+    const size_t xpitch = F8 ? (size_t)p.H : (size_t)p.H * 2;
 #pragma unroll
     for (int j = 0; j < kRowsPerLane; ++j) {
       const int r = (j * kGatherWarps + g) * 4 + (lane >> 3);
@@ -541,7 +547,7 @@ __device__ void gemm_gather(const GemmParams& p, GemmSmem& s, uint8_t* tiles, in
     }
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive(&s.task_empty[q_task]);   // slot (and its rows) free
-    const int nk = task.phase == 0 ? l1_ksteps(p) : l2_ksteps(p);
+    const int nk = task.phase == 0 ? l1_ksteps<F8>(p) : l2_ksteps<F8>(p);
     bool ok = true;
 
     for (int kb = 0; kb < nk; ++kb) {
@@ -675,6 +681,7 @@ __device__ __forceinline__ void combine_rows(uint32_t tbase, int ncols, float w,
 }
 
 // ---------------------------------------------------------------- epilogue (warps 2..5)
+template <bool F8>
 __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_base) {
   const int warp = threadIdx.x >> 5;
   const int lane = ptx::lane_id();
@@ -713,7 +720,7 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
       bf16* hrow = p.h + (size_t)ring_row * p.I + task.n * kL1TileN;
       float tscale = 0.f;   // FP8: the token's scale (padding rows: 0, so their activation is 0)
       float amax = 0.f;     // FP8: the row's largest |h| over this task's columns
-      if (p.fp8 && valid) {
+      if (F8 && valid) {
         const int tok = p.slot_token[slot];
         tscale = (tok >= 0 && tok < p.T) ? p.sx[tok] : 0.f;
       }
@@ -723,10 +730,10 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
         ptx::tmem_ld32(tbase + c * 32, g);
         ptx::tmem_ld32(tbase + kL1TileN + c * 32, u);
         ptx::tmem_ld_wait();
-        if (p.fp8) fp8_scale_columns(g, u, tscale, p.s1, p.s3, (size_t)task.e * p.I + task.n * kL1TileN + c * 32);
+        if (F8) fp8_scale_columns(g, u, tscale, p.s1, p.s3, (size_t)task.e * p.I + task.n * kL1TileN + c * 32);
         if (store) store_swiglu32(hrow + c * 32, g, u, amax);
       }
-      if (p.fp8 && store) publish_act_amax(p.act_amax, ring_row, amax);
+      if (F8 && store) publish_act_amax(p.act_amax, ring_row, amax);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&s.acc_empty[acc]);
@@ -760,10 +767,10 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
         }
       }
       // FP8: o = acc * (activation scale of the row) * (W2 column scale)
-      if (p.fp8 && tok >= 0) w *= __ldcg(p.act_scale + (task.b % p.ring_blocks) * p.BM + r);   // FP8: the row's scale
+      if (F8 && tok >= 0) w *= __ldcg(p.act_scale + (task.b % p.ring_blocks) * p.BM + r);   // FP8: the row's scale
       // Combine: y_acc[token] += w * o, 128-byte row segments per red.v4 (the L2 does the fp32 adds).
       combine_rows(tbase, p.BN2, w, tok, p.y_acc, p.H, task.n * p.BN2, s.out_stage[quarter], s.out_tok[quarter],
-                   p.fp8 ? p.s2 + (size_t)task.e * p.H + task.n * p.BN2 : nullptr, [&]() {
+                   F8 ? p.s2 + (size_t)task.e * p.H + task.n * p.BN2 : nullptr, [&]() {
                      ptx::tc_fence_before();
                      __syncwarp();
                      if (lane == 0) ptx::mbar_arrive(&s.acc_empty[acc]);
@@ -776,6 +783,7 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
   }
 }
 
+template <bool F8>
 __global__ void __launch_bounds__(kGemm1Threads, 1) moe_expert_gemm_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -836,11 +844,11 @@ __global__ void __launch_bounds__(kGemm1Threads, 1) moe_expert_gemm_kernel(const
   ptx::tc_fence_after();
   const uint32_t tmem_base = s.tmem_base;
 
-  if (warp == 0) gemm_producer(p, s, tiles);
-  else if (warp == 1) gemm_mma(p, s, tiles, tmem_base);
-  else if (warp < 6) gemm_epilogue(p, s, tmem_base);
-  else if (warp < 6 + kGatherWarps) gemm_gather(p, s, tiles, warp - 6);
-  else gemm_scheduler(p, s);
+  if (warp == 0) gemm_producer<F8>(p, s, tiles);
+  else if (warp == 1) gemm_mma<F8>(p, s, tiles, tmem_base);
+  else if (warp < 6) gemm_epilogue<F8>(p, s, tmem_base);
+  else if (warp < 6 + kGatherWarps) gemm_gather<F8>(p, s, tiles, warp - 6);
+  else gemm_scheduler<F8>(p, s);
 
   ptx::tc_fence_before();
   __syncthreads();

@@ -240,9 +240,11 @@ __device__ __forceinline__ Task2 decode_task2(int t, const Gemm2Smem& s, const G
 __device__ __forceinline__ uint8_t* stage2_ptr(uint8_t* tiles, int stage) { return tiles + stage * kStage2Bytes; }
 
 // K blocks of an L1 task: 64 bf16 or 128 FP8 elements (one 128-byte swizzle row).
-__device__ __forceinline__ int l1_ksteps2(const Gemm2Params& p) { return p.fp8 ? p.H / 128 : p.H / kBK; }
+template <bool F8>
+__device__ __forceinline__ int l1_ksteps2(const Gemm2Params& p) { return F8 ? p.H / 128 : p.H / kBK; }
 
-__device__ __forceinline__ int l2_ksteps2(const Gemm2Params& p) { return p.fp8 ? p.I / 128 : p.I / kBK; }
+template <bool F8>
+__device__ __forceinline__ int l2_ksteps2(const Gemm2Params& p) { return F8 ? p.I / 128 : p.I / kBK; }
 
 // ---------------------------------------------------------------- leader scheduler (last warp)
 // Claims tasks, decodes them, stages the token rows of both CTAs' A tiles
@@ -320,6 +322,7 @@ __device__ __forceinline__ bool wait_taken2(int n, const Gemm2Params& p, Gemm2Sm
   return true;
 }
 
+template <bool F8>
 __device__ void gemm2_scheduler(const Gemm2Params& p, Gemm2Smem& s) {
   const int lane = ptx::lane_id();
   int q = 0;
@@ -346,6 +349,7 @@ __device__ void gemm2_scheduler(const Gemm2Params& p, Gemm2Smem& s) {
 }
 
 // ---------------------------------------------------------------- leader warp 0: TMA
+template <bool F8>
 __device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles) {
   const int lane = ptx::lane_id();
   const uint64_t pol = ptx::policy_evict_first();
@@ -368,7 +372,7 @@ __device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_
       qphase ^= 1;
     }
     if (task.phase < 0) break;
-    const int nk = task.phase == 0 ? l1_ksteps2(p) : l2_ksteps2(p);
+    const int nk = task.phase == 0 ? l1_ksteps2<F8>(p) : l2_ksteps2<F8>(p);
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait2(&s.empty[stage], phase ^ 1, p, s, 2)) {
         ok = false;
@@ -382,7 +386,7 @@ __device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_
         if (task.phase == 0) {
           ptx::mbar_arrive_expect_tx(&s.full[stage], 2 * kBoxBytes);
           const int n0 = task.n * kL1TileN;
-          if (p.fp8) {   // K-major FP8 codes: 64 rows (columns of I) x 128 bytes per box
+          if (F8) {   // K-major FP8 codes: 64 rows (columns of I) x 128 bytes per box
             ptx::tma_load_2d(b_addr, &p.tm_w1, &s.full[stage], kb * 128, task.e * p.I + n0, pol);
             ptx::tma_load_2d(b_addr + kBoxBytes, &p.tm_w1, &s.full[stage], kb * 128, task.e * p.I + n0 + 64, pol);
           } else {
@@ -447,6 +451,7 @@ __device__ __forceinline__ void release_task_slot2(int q, bool is_leader, Gemm2S
 }
 
 // ---------------------------------------------------------------- follower warp 0: its TMA halves
+template <bool F8>
 __device__ void gemm2_follower_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles) {
   const int lane = ptx::lane_id();
   const uint64_t pol = ptx::policy_evict_first();
@@ -458,7 +463,7 @@ __device__ void gemm2_follower_producer(const Gemm2Params& p, Gemm2Smem& s, uint
     Task2 task;
     if (!pop_task2(task, q, qphase, nullptr, false, p, s, 3, true)) break;
     if (task.phase < 0) break;
-    const int nk = task.phase == 0 ? l1_ksteps2(p) : l2_ksteps2(p);
+    const int nk = task.phase == 0 ? l1_ksteps2<F8>(p) : l2_ksteps2<F8>(p);
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait2(&s.empty[stage], phase ^ 1, p, s, 4)) {
@@ -471,7 +476,7 @@ __device__ void gemm2_follower_producer(const Gemm2Params& p, Gemm2Smem& s, uint
         if (task.phase == 0) {
           ptx::mbar_arrive_expect_tx(&s.full[stage], 2 * kBoxBytes);
           const int n0 = task.n * kL1TileN;
-          if (p.fp8) {
+          if (F8) {
             ptx::tma_load_2d(b_addr, &p.tm_w3, &s.full[stage], kb * 128, task.e * p.I + n0, pol);
             ptx::tma_load_2d(b_addr + kBoxBytes, &p.tm_w3, &s.full[stage], kb * 128, task.e * p.I + n0 + 64, pol);
           } else {
@@ -498,6 +503,7 @@ __device__ void gemm2_follower_producer(const Gemm2Params& p, Gemm2Smem& s, uint
 // ---------------------------------------------------------------- follower warp 1: stage relay
 // The follower's TMA bytes and gather lanes land on its own stage barrier;
 // once a stage is complete, one arrival on the leader's barrier of that stage.
+template <bool F8>
 __device__ void gemm2_follower_relay(const Gemm2Params& p, Gemm2Smem& s) {
   const int lane = ptx::lane_id();
   const uint32_t lead_full0 = ptx::mapa(ptx::smem_u32(&s.full[0]), 0);
@@ -509,7 +515,7 @@ __device__ void gemm2_follower_relay(const Gemm2Params& p, Gemm2Smem& s) {
     Task2 task;
     if (!pop_task2(task, q, qphase, nullptr, false, p, s, 5, true)) break;
     if (task.phase < 0) break;
-    const int nk = task.phase == 0 ? l1_ksteps2(p) : l2_ksteps2(p);
+    const int nk = task.phase == 0 ? l1_ksteps2<F8>(p) : l2_ksteps2<F8>(p);
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait2(&s.full[stage], phase, p, s, 6)) {
@@ -531,12 +537,13 @@ __device__ void gemm2_follower_relay(const Gemm2Params& p, Gemm2Smem& s) {
 }
 
 // ---------------------------------------------------------------- leader warp 1: MMA issuer
+template <bool F8>
 __device__ void gemm2_mma(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, uint32_t tmem_base) {
   const int lane = ptx::lane_id();
   const uint32_t idesc_l1 =
-      p.fp8 ? ptx::idesc_e4m3_f32(256, 2 * kL1TileN) : ptx::idesc_bf16_f32(256, 2 * kL1TileN, false, true);
-  const bool f8 = p.fp8 != 0;
-  const uint32_t idesc_l2 = p.fp8 ? ptx::idesc_e4m3_f32(256, p.BN2) : ptx::idesc_bf16_f32(256, p.BN2, false, true);
+      F8 ? ptx::idesc_e4m3_f32(256, 2 * kL1TileN) : ptx::idesc_bf16_f32(256, 2 * kL1TileN, false, true);
+  constexpr bool f8 = F8;
+  const uint32_t idesc_l2 = F8 ? ptx::idesc_e4m3_f32(256, p.BN2) : ptx::idesc_bf16_f32(256, p.BN2, false, true);
   int stage = 0;
   uint32_t phase = 0;
   int q = 0;
@@ -552,7 +559,7 @@ __device__ void gemm2_mma(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, ui
     ptx::tc_fence_after();
     const uint32_t d_tmem = tmem_base + acc * 256;
     const uint32_t idesc = task.phase == 0 ? idesc_l1 : idesc_l2;
-    const int nk = task.phase == 0 ? l1_ksteps2(p) : l2_ksteps2(p);
+    const int nk = task.phase == 0 ? l1_ksteps2<F8>(p) : l2_ksteps2<F8>(p);
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait2(&s.full[stage], phase, p, s, 9)) {
@@ -605,6 +612,7 @@ __device__ void gemm2_mma(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, ui
 }
 
 // ---------------------------------------------------------------- epilogue (warps 2..5 of both CTAs)
+template <bool F8>
 __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem_base, uint32_t rank) {
   const int warp = threadIdx.x >> 5;
   const int lane = ptx::lane_id();
@@ -638,7 +646,7 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
       bf16* hrow = p.h + (size_t)ring_row * p.I + task.n * kL1TileN;
       float tscale = 0.f;   // FP8: the token's scale (padding rows: 0, so their activation is 0)
       float amax = 0.f;     // FP8: the row's largest |h| over this task's columns
-      if (p.fp8 && valid) {
+      if (F8 && valid) {
         const int tok = p.slot_token[slot];
         tscale = (tok >= 0 && tok < p.T) ? p.sx[tok] : 0.f;
       }
@@ -648,10 +656,10 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
         ptx::tmem_ld32(tbase + c * 32, g);
         ptx::tmem_ld32(tbase + kL1TileN + c * 32, u);
         ptx::tmem_ld_wait();
-        if (p.fp8) fp8_scale_columns(g, u, tscale, p.s1, p.s3, (size_t)task.e * p.I + task.n * kL1TileN + c * 32);
+        if (F8) fp8_scale_columns(g, u, tscale, p.s1, p.s3, (size_t)task.e * p.I + task.n * kL1TileN + c * 32);
         if (store) store_swiglu32(hrow + c * 32, g, u, amax);
       }
-      if (p.fp8 && store) publish_act_amax(p.act_amax, ring_row, amax);
+      if (F8 && store) publish_act_amax(p.act_amax, ring_row, amax);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -683,10 +691,10 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
           }
         }
       }
-      if (p.fp8 && tok >= 0)   // FP8: the row's scale
+      if (F8 && tok >= 0)   // FP8: the row's scale
         w *= __ldcg(p.act_scale + ((task.p % p.ring_pairs) * 2 + (int)rank) * p.BM + r);
       combine_rows(tbase, p.BN2, w, tok, p.y_acc, p.H, task.n * p.BN2, s.out_stage[quarter], s.out_tok[quarter],
-                   p.fp8 ? p.s2 + (size_t)task.e * p.H + task.n * p.BN2 : nullptr, [&]() {
+                   F8 ? p.s2 + (size_t)task.e * p.H + task.n * p.BN2 : nullptr, [&]() {
                      ptx::tc_fence_before();
                      __syncwarp();
                      if (lane == 0) {
@@ -703,6 +711,7 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
 }
 
 // ---------------------------------------------------------------- gather warps (warps 6.. of both CTAs)
+template <bool F8>
 __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, int g, uint32_t rank) {
   constexpr int kRowsPerLane = (kTileM / 4 + kGatherWarps - 1) / kGatherWarps;
   const uint64_t wpol = ptx::policy_evict_first();
@@ -727,10 +736,10 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
       // L1: the routed x rows (bf16, or FP8 codes) of this CTA's block; L2: its h rows in the ring
       // activation rows: bf16, or FP8 codes (rows of I bytes)
       const int* rows = s.rows[q_task];
-      const size_t hpitch = p.fp8 ? (size_t)p.I : (size_t)p.I * 2;
-      const uint8_t* hblock = (p.fp8 ? p.h8 : reinterpret_cast<const uint8_t*>(p.h)) + (size_t)ring_row0 * hpitch;
-      const uint8_t* xrows = p.fp8 ? p.xq : reinterpret_cast<const uint8_t*>(p.x);
-      const size_t xpitch = p.fp8 ? (size_t)p.H : (size_t)p.H * 2;
+      const size_t hpitch = F8 ? (size_t)p.I : (size_t)p.I * 2;
+      const uint8_t* hblock = (F8 ? p.h8 : reinterpret_cast<const uint8_t*>(p.h)) + (size_t)ring_row0 * hpitch;
+      const uint8_t* xrows = F8 ? p.xq : reinterpret_cast<const uint8_t*>(p.x);
+      const size_t xpitch = F8 ? (size_t)p.H : (size_t)p.H * 2;
 #pragma unroll
       for (int j = 0; j < kRowsPerLane; ++j) {
         const int rr = (j * kGatherWarps + g) * 4 + (lane >> 3);
@@ -745,16 +754,16 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
     release_task_slot2(q_task, is_leader, s);   // rows read: the slot may be refilled
     // L2: this CTA's half of the W2 tile too (BN2/2 columns: one or two 64x64
     // boxes, each 64 K-rows of 128 bytes in the same 128-byte swizzle as TMA)
-    const int nhalf = task.phase == 1 && !p.fp8 ? p.BN2 / 128 : 0;
-    const int nchunk8 = task.phase == 1 && p.fp8 ? (p.BN2 / 2) * 8 / (32 * kGatherWarps) : 0;   // 8, or 4 (BN2 = 128)
+    const int nhalf = task.phase == 1 && !F8 ? p.BN2 / 128 : 0;
+    const int nchunk8 = task.phase == 1 && F8 ? (p.BN2 / 2) * 8 / (32 * kGatherWarps) : 0;   // 8, or 4 (BN2 = 128)
     const uint8_t* w2row8 =
-        p.fp8 ? p.w2q + ((size_t)task.e * p.H + task.n * p.BN2 + (int)rank * (p.BN2 / 2)) * p.I : nullptr;
+        F8 ? p.w2q + ((size_t)task.e * p.H + task.n * p.BN2 + (int)rank * (p.BN2 / 2)) * p.I : nullptr;
     const int tl = g * 32 + lane;
-    const bf16* w2src = p.fp8 ? nullptr
+    const bf16* w2src = F8 ? nullptr
                               : (task.e >= p.E ? p.ws2 + (size_t)(task.e - p.E) * p.I * p.H
                                                : p.w2 + (size_t)task.e * p.I * p.H) +
                                     task.n * p.BN2 + (int)rank * (p.BN2 / 2) + c * 8;
-    const int nk = task.phase == 0 ? l1_ksteps2(p) : l2_ksteps2(p);
+    const int nk = task.phase == 0 ? l1_ksteps2<F8>(p) : l2_ksteps2<F8>(p);
     bool ok = true;
 
     for (int kb = 0; kb < nk; ++kb) {
@@ -792,6 +801,7 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
   ptx::cp_async_wait_all();
 }
 
+template <bool F8>
 __global__ void __launch_bounds__(kGemm1Threads, 1) moe_expert_gemm2_kernel(const __grid_constant__ Gemm2Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -859,17 +869,17 @@ __global__ void __launch_bounds__(kGemm1Threads, 1) moe_expert_gemm2_kernel(cons
   const uint32_t tmem_base = s.tmem_base;
 
   if (warp == 0) {
-    if (is_leader) gemm2_leader_producer(p, s, tiles);
-    else gemm2_follower_producer(p, s, tiles);
+    if (is_leader) gemm2_leader_producer<F8>(p, s, tiles);
+    else gemm2_follower_producer<F8>(p, s, tiles);
   } else if (warp == 1) {
-    if (is_leader) gemm2_mma(p, s, tiles, tmem_base);
-    else gemm2_follower_relay(p, s);
+    if (is_leader) gemm2_mma<F8>(p, s, tiles, tmem_base);
+    else gemm2_follower_relay<F8>(p, s);
   } else if (warp < 6) {
-    gemm2_epilogue(p, s, tmem_base, rank);
+    gemm2_epilogue<F8>(p, s, tmem_base, rank);
   } else if (warp < 6 + kGatherWarps) {
-    gemm2_gather(p, s, tiles, warp - 6, rank);
+    gemm2_gather<F8>(p, s, tiles, warp - 6, rank);
   } else if (is_leader) {
-    gemm2_scheduler(p, s);
+    gemm2_scheduler<F8>(p, s);
   }
 
   ptx::tc_fence_before();

@@ -444,11 +444,12 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, moe_expert_gemm2_kernel, gp) != cudaSuccess) return MOE_ERR_CUDA;
+    void (*kfn)(Gemm2Params) = f8 != nullptr ? moe_expert_gemm2_kernel<true> : moe_expert_gemm2_kernel<false>;
+    if (cudaLaunchKernelEx(&cfg, kfn, gp) != cudaSuccess) return MOE_ERR_CUDA;
     if (f8 != nullptr) {
       if (!quantize_activation(dp.pair_start + E, 2 * p->BM)) return MOE_ERR_CUDA;
       gp.phase_only = 1;
-      if (cudaLaunchKernelEx(&cfg, moe_expert_gemm2_kernel, gp) != cudaSuccess) return MOE_ERR_CUDA;
+      if (cudaLaunchKernelEx(&cfg, kfn, gp) != cudaSuccess) return MOE_ERR_CUDA;
     }
   } else {
     GemmParams gp;
@@ -504,12 +505,13 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     gp.N2 = p->N2;
     gp.timeout_ns = p->timeout_ns;
     gp.withhold_block = p->withhold;
-    moe_expert_gemm_kernel<<<p->num_sms, kGemm1Threads, kGemmSmemBytes, st>>>(gp);
+    void (*kfn)(GemmParams) = f8 != nullptr ? moe_expert_gemm_kernel<true> : moe_expert_gemm_kernel<false>;
+    kfn<<<p->num_sms, kGemm1Threads, kGemmSmemBytes, st>>>(gp);
     if (f8 != nullptr) {
       if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
       if (!quantize_activation(dp.sched + 1, p->BM)) return MOE_ERR_CUDA;
       gp.phase_only = 1;
-      moe_expert_gemm_kernel<<<p->num_sms, kGemm1Threads, kGemmSmemBytes, st>>>(gp);
+      kfn<<<p->num_sms, kGemm1Threads, kGemmSmemBytes, st>>>(gp);
     }
   }
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
@@ -731,10 +733,17 @@ int moe_plan_create_shared(moe_plan_t* out, int T_max, int H, int I, int E, int 
   p->L = make_layout(*p);
 
   DeviceGuard guard(device);
-  cudaError_t ce = cudaFuncSetAttribute(moe_expert_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  // both instances of each expert-GEMM kernel: bf16 and FP8 operands
+  cudaError_t ce = cudaFuncSetAttribute(moe_expert_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)kGemmSmemBytes);
   if (ce == cudaSuccess)
-    ce = cudaFuncSetAttribute(moe_expert_gemm2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    ce = cudaFuncSetAttribute(moe_expert_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)kGemmSmemBytes);
+  if (ce == cudaSuccess)
+    ce = cudaFuncSetAttribute(moe_expert_gemm2_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)kGemm2SmemBytes);
+  if (ce == cudaSuccess)
+    ce = cudaFuncSetAttribute(moe_expert_gemm2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)kGemm2SmemBytes);
   if (ce == cudaSuccess)
     ce = cudaFuncSetAttribute(moe_router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRtcSmemBytes);
@@ -763,7 +772,7 @@ int moe_plan_create_shared(moe_plan_t* out, int T_max, int H, int I, int E, int 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, moe_expert_gemm2_kernel, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&clusters, moe_expert_gemm2_kernel<false>, &cfg) != cudaSuccess) {
       cudaGetLastError();
       clusters = 0;
     }

@@ -572,21 +572,14 @@ __device__ void gemm_gather(const GemmParams& p, GemmSmem& s, uint8_t* tiles, in
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
 
-// FP8 first GEMM: g[i] *= sx * s1[col0 + i], u[i] *= sx * s3[col0 + i] for 32 columns
-// (the column scales are the same for every lane: broadcast loads).
-__device__ __forceinline__ void fp8_scale_columns(uint32_t (&g)[32], uint32_t (&u)[32], float tscale,
-                                                  const float* s1, const float* s3, size_t col0) {
-  const float4* a = reinterpret_cast<const float4*>(s1 + col0);
-  const float4* b = reinterpret_cast<const float4*>(s3 + col0);
+// FP8 first GEMM: g[i] *= tscale * (column i's W1 scale), u[i] *= tscale * (W3 scale) for the
+// 32 columns of a chunk; lane j holds column j's scales (sa, sb) and shuffles them to the warp.
+__device__ __forceinline__ void fp8_scale_columns_shfl(uint32_t (&g)[32], uint32_t (&u)[32], float tscale, float sa,
+                                                       float sb) {
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const float4 sa = __ldg(a + q), sb = __ldg(b + q);
-    const float fa[4] = {sa.x, sa.y, sa.z, sa.w}, fb[4] = {sb.x, sb.y, sb.z, sb.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      g[4 * q + i] = __float_as_uint(__uint_as_float(g[4 * q + i]) * (tscale * fa[i]));
-      u[4 * q + i] = __float_as_uint(__uint_as_float(u[4 * q + i]) * (tscale * fb[i]));
-    }
+  for (int i = 0; i < 32; ++i) {
+    g[i] = __float_as_uint(__uint_as_float(g[i]) * (tscale * __shfl_sync(0xffffffffu, sa, i)));
+    u[i] = __float_as_uint(__uint_as_float(u[i]) * (tscale * __shfl_sync(0xffffffffu, sb, i)));
   }
 }
 
@@ -631,9 +624,12 @@ __device__ __forceinline__ void publish_act_amax(float* act_amax, int row, float
 // accumulator while the last reductions are still being issued.
 __device__ __forceinline__ void combine_stage_and_reduce(const uint32_t (&v)[32], int c, float w, float* srow,
                                                          float (*stage)[36], float* const (&ybase)[8], int sub,
-                                                         int cc, const float* cs) {
-  // per-column scales of the lane's 4 transposed columns (FP8 W2), loaded before the staging
-  const float4 m = cs != nullptr ? __ldg(reinterpret_cast<const float4*>(cs + c * 32 + cc)) : make_float4(1.f, 1.f, 1.f, 1.f);
+                                                         int cc, const float* cs, float csl) {
+  // FP8 W2: scales of the lane's 4 transposed columns, from the lanes that hold them (lane j: column j)
+  float4 m = make_float4(1.f, 1.f, 1.f, 1.f);
+  if (cs != nullptr)
+    m = make_float4(__shfl_sync(0xffffffffu, csl, cc), __shfl_sync(0xffffffffu, csl, cc + 1),
+                    __shfl_sync(0xffffffffu, csl, cc + 2), __shfl_sync(0xffffffffu, csl, cc + 3));
 #pragma unroll
   for (int i = 0; i < 8; ++i)
     reinterpret_cast<float4*>(srow)[i] =
@@ -666,17 +662,31 @@ __device__ __forceinline__ void combine_rows(uint32_t tbase, int ncols, float w,
     ybase[i] = t >= 0 ? y_acc + (size_t)t * H + col0 + cc : nullptr;
   }
   float* srow = stage[lane];
+  // FP8 W2: this lane holds the scale of column 32c + lane of the two chunks in hand, and
+  // loads those of the next two while they are reduced
+  float csa = 1.f, csb = 1.f;
+  if (cs != nullptr) {
+    csa = __ldg(cs + lane);
+    csb = __ldg(cs + 32 + lane);
+  }
   uint32_t va[32], vb[32];
   ptx::tmem_ld32(tbase, va);
 #pragma unroll 1
   for (int c = 0; c < ncols / 32; c += 2) {
+    float nca = 1.f, ncb = 1.f;
+    if (cs != nullptr && c + 2 < ncols / 32) {
+      nca = __ldg(cs + (c + 2) * 32 + lane);
+      ncb = __ldg(cs + (c + 3) * 32 + lane);
+    }
     ptx::tmem_ld_wait();                                         // va holds columns 32c ..
     ptx::tmem_ld32(tbase + (c + 1) * 32, vb);
-    combine_stage_and_reduce(va, c, w, srow, stage, ybase, sub, cc, cs);
+    combine_stage_and_reduce(va, c, w, srow, stage, ybase, sub, cc, cs, csa);
     ptx::tmem_ld_wait();                                         // vb holds columns 32(c+1) ..
     if (c + 2 < ncols / 32) ptx::tmem_ld32(tbase + (c + 2) * 32, va);
     else release();                                              // no TMEM reads left
-    combine_stage_and_reduce(vb, c + 1, w, srow, stage, ybase, sub, cc, cs);
+    combine_stage_and_reduce(vb, c + 1, w, srow, stage, ybase, sub, cc, cs, csb);
+    csa = nca;
+    csb = ncb;
   }
 }
 
@@ -701,6 +711,22 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
       qphase ^= 1;
     }
     if (task.phase < 0) break;
+    // FP8: the task's scales, loaded before the accumulator wait (lane j: column 32c + j of chunk c)
+    float tscale = 0.f, rscale = 1.f, sa[4] = {1.f, 1.f, 1.f, 1.f}, sb[4] = {1.f, 1.f, 1.f, 1.f};
+    if (F8 && task.phase == 0) {
+      const size_t col0 = (size_t)task.e * p.I + task.n * kL1TileN;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        sa[c] = __ldg(p.s1 + col0 + c * 32 + lane);
+        sb[c] = __ldg(p.s3 + col0 + c * 32 + lane);
+      }
+      if (r < p.BM) {   // the token's scale (padding rows: 0, so their activation is 0)
+        const int tok = p.slot_token[task.b * p.BM + r];
+        tscale = (tok >= 0 && tok < p.T) ? __ldg(p.sx + tok) : 0.f;
+      }
+    } else if (F8 && r < p.BM) {
+      rscale = __ldcg(p.act_scale + (task.b % p.ring_blocks) * p.BM + r);   // the activation row's scale
+    }
     if (!warp_wait(&s.acc_full[acc], acc_phase, p, s, 7)) break;
     ptx::tc_fence_after();
     const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * 256;
@@ -718,19 +744,16 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
       }
       const int ring_row = (task.b % p.ring_blocks) * p.BM + r;
       bf16* hrow = p.h + (size_t)ring_row * p.I + task.n * kL1TileN;
-      float tscale = 0.f;   // FP8: the token's scale (padding rows: 0, so their activation is 0)
       float amax = 0.f;     // FP8: the row's largest |h| over this task's columns
-      if (F8 && valid) {
-        const int tok = p.slot_token[slot];
-        tscale = (tok >= 0 && tok < p.T) ? p.sx[tok] : 0.f;
-      }
 #pragma unroll 1
       for (int c = 0; c < kL1TileN / 32; ++c) {
         uint32_t g[32], u[32];
         ptx::tmem_ld32(tbase + c * 32, g);
         ptx::tmem_ld32(tbase + kL1TileN + c * 32, u);
         ptx::tmem_ld_wait();
-        if (F8) fp8_scale_columns(g, u, tscale, p.s1, p.s3, (size_t)task.e * p.I + task.n * kL1TileN + c * 32);
+        if (F8)
+          fp8_scale_columns_shfl(g, u, tscale, c == 0 ? sa[0] : c == 1 ? sa[1] : c == 2 ? sa[2] : sa[3],
+                                 c == 0 ? sb[0] : c == 1 ? sb[1] : c == 2 ? sb[2] : sb[3]);
         if (store) store_swiglu32(hrow + c * 32, g, u, amax);
       }
       if (F8 && store) publish_act_amax(p.act_amax, ring_row, amax);
@@ -767,7 +790,7 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
         }
       }
       // FP8: o = acc * (activation scale of the row) * (W2 column scale)
-      if (F8 && tok >= 0) w *= __ldcg(p.act_scale + (task.b % p.ring_blocks) * p.BM + r);   // FP8: the row's scale
+      if (F8 && tok >= 0) w *= rscale;   // FP8: the activation row's scale
       // Combine: y_acc[token] += w * o, 128-byte row segments per red.v4 (the L2 does the fp32 adds).
       combine_rows(tbase, p.BN2, w, tok, p.y_acc, p.H, task.n * p.BN2, s.out_stage[quarter], s.out_tok[quarter],
                    F8 ? p.s2 + (size_t)task.e * p.H + task.n * p.BN2 : nullptr, [&]() {

@@ -628,6 +628,25 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
     Task2 task;
     if (!pop_task2(task, q, qphase, nullptr, is_leader, p, s, 10, true)) break;
     if (task.phase < 0) break;
+    // FP8: the task's scales, loaded before the accumulator wait (lane j: column 32c + j of chunk c)
+    float tscale = 0.f, rscale = 1.f, sa[4] = {1.f, 1.f, 1.f, 1.f}, sb[4] = {1.f, 1.f, 1.f, 1.f};
+    if (F8) {
+      const int bo = rank == 0 ? task.b0 : task.b1;
+      if (task.phase == 0) {
+        const size_t col0 = (size_t)task.e * p.I + task.n * kL1TileN;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          sa[c] = __ldg(p.s1 + col0 + c * 32 + lane);
+          sb[c] = __ldg(p.s3 + col0 + c * 32 + lane);
+        }
+        if (r < p.BM && bo >= 0) {   // the token's scale (padding rows: 0, so their activation is 0)
+          const int tok = p.slot_token[bo * p.BM + r];
+          tscale = (tok >= 0 && tok < p.T) ? __ldg(p.sx + tok) : 0.f;
+        }
+      } else if (r < p.BM && bo >= 0) {   // the activation row's scale
+        rscale = __ldcg(p.act_scale + ((task.p % p.ring_pairs) * 2 + (int)rank) * p.BM + r);
+      }
+    }
     if (!warp_wait2(&s.acc_full[acc], acc_phase, p, s, 11)) break;
     ptx::tc_fence_after();
     const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * 256;
@@ -644,19 +663,16 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
       }
       const int ring_row = ((task.p % p.ring_pairs) * 2 + (int)rank) * p.BM + r;
       bf16* hrow = p.h + (size_t)ring_row * p.I + task.n * kL1TileN;
-      float tscale = 0.f;   // FP8: the token's scale (padding rows: 0, so their activation is 0)
       float amax = 0.f;     // FP8: the row's largest |h| over this task's columns
-      if (F8 && valid) {
-        const int tok = p.slot_token[slot];
-        tscale = (tok >= 0 && tok < p.T) ? p.sx[tok] : 0.f;
-      }
 #pragma unroll 1
       for (int c = 0; c < kL1TileN / 32; ++c) {
         uint32_t g[32], u[32];
         ptx::tmem_ld32(tbase + c * 32, g);
         ptx::tmem_ld32(tbase + kL1TileN + c * 32, u);
         ptx::tmem_ld_wait();
-        if (F8) fp8_scale_columns(g, u, tscale, p.s1, p.s3, (size_t)task.e * p.I + task.n * kL1TileN + c * 32);
+        if (F8)
+          fp8_scale_columns_shfl(g, u, tscale, c == 0 ? sa[0] : c == 1 ? sa[1] : c == 2 ? sa[2] : sa[3],
+                                 c == 0 ? sb[0] : c == 1 ? sb[1] : c == 2 ? sb[2] : sb[3]);
         if (store) store_swiglu32(hrow + c * 32, g, u, amax);
       }
       if (F8 && store) publish_act_amax(p.act_amax, ring_row, amax);
@@ -691,8 +707,7 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
           }
         }
       }
-      if (F8 && tok >= 0)   // FP8: the row's scale
-        w *= __ldcg(p.act_scale + ((task.p % p.ring_pairs) * 2 + (int)rank) * p.BM + r);
+      if (F8 && tok >= 0) w *= rscale;   // FP8: the activation row's scale
       combine_rows(tbase, p.BN2, w, tok, p.y_acc, p.H, task.n * p.BN2, s.out_stage[quarter], s.out_tok[quarter],
                    F8 ? p.s2 + (size_t)task.e * p.H + task.n * p.BN2 : nullptr, [&]() {
                      ptx::tc_fence_before();

@@ -570,7 +570,10 @@ __device__ void gemm_gather(const GemmParams& p, GemmSmem& s, uint8_t* tiles, in
   ptx::cp_async_wait_all();
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+// silu(g) * u = g / (1 + e^-g) * u. The division is the fast one (__fdividef, within 2 ulp; it
+// returns 0 once 1 + e^-g passes 2^126, where silu(g) is 0 to fp32 precision): an IEEE division
+// here made the first GEMM's epilogue the slowest role of the FP8 kernels.
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
 // FP8 first GEMM: g[i] *= tscale * (column i's W1 scale), u[i] *= tscale * (W3 scale) for the
 // 32 columns of a chunk; lane j holds column j's scales (sa, sb) and shuffles them to the warp.

@@ -19,6 +19,10 @@ The JSON line also carries:
   pinned memory, y copied back, every step);
 * cpu_baseline: the fp64 CPU oracle timed on a bounded sample on rank 0;
 * clocks: SM clock samples and throttle reasons taken during the timed steps.
+
+--fp8 runs the same layer with FP8 E4M3 expert GEMMs (weights quantized once before timing);
+its roofline peak is twice the sustained bf16 figure (the nominal dense fp8/bf16 ratio) and its
+byte count takes 1-byte weights plus their fp32 column scales.
 """
 from __future__ import annotations
 

@@ -247,7 +247,9 @@ int moe_route(moe_plan_t plan, const void* x, const void* Wg, const float* gate_
 int moe_check(moe_plan_t plan, void* stream, int32_t* detail);
 
 /* Profiling: when enabled, moe_forward records CUDA events on its stream
- * around each of its five kernels. moe_plan_profile_read() synchronises on
+ * around each of its five kernels (moe_forward_fp8: the router segment also
+ * holds the x quantizer, the expert-GEMM segment both GEMM launches and the
+ * activation quantizer between them). moe_plan_profile_read() synchronises on
  * the last recorded event, writes the summed milliseconds of each kernel
  * (router, scan, scatter, expert GEMM, finalize) over the forwards recorded
  * since the previous read into ms[0..4], the number of such forwards into

@@ -58,14 +58,13 @@ struct GemmParams {
   float* y_acc;                 // [T, H]
   int T, H, I, E, k, BM, BN2, N1, N2;
   int S;                        // shared experts (0 .. kMaxShared)
-  // FP8 E4M3 expert GEMMs (fp8 != 0): x codes [T, H] with per-token scales,
+  // FP8 E4M3 expert GEMMs (the kernel's FP8 instance): x codes [T, H] with per-token scales,
   // W1/W3 codes K-major [E, I, H] with column scales [E, I], W2 codes K-major
   // [E, H, I] with column scales [E, H] (tensor maps above). The two GEMMs run
   // as two launches (phase_only 0, then 1) around the activation quantizer:
   // the first stores the bf16 activation in h and raises act_amax of its row
   // (zero before the launch) to the row's largest |h|; the quantizer writes
   // the row's codes to h8 and its scale to act_scale; the second reads them.
-  int fp8;
   const uint8_t* xq;
   const float* sx;
   const float* s1;

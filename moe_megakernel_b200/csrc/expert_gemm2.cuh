@@ -64,9 +64,8 @@ struct Gemm2Params {
   float* y_acc;                 // [T, H]
   int T, H, I, E, k, BM, BN2, N1, N2;
   int S;                        // shared experts (0 .. kMaxShared)
-  // FP8 E4M3 first GEMM (see GemmParams): x codes, token scales, K-major W1/W3
-  // codes in tm_w1 / tm_w3 (box {128, 64}), column scales
-  int fp8;
+  // FP8 E4M3 expert GEMMs (the kernel's FP8 instance; see GemmParams): x codes, token scales,
+  // K-major W1/W3 codes in tm_w1 / tm_w3 (box {128, 64}), column scales
   const uint8_t* xq;
   const float* sx;
   const float* s1;

@@ -390,7 +390,6 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     gp.x = static_cast<const bf16*>(x);
     gp.phase_only = -1;
     if (f8 != nullptr) {
-      gp.fp8 = 1;
       gp.xq = ws + L.x_q;
       gp.sx = reinterpret_cast<const float*>(ws + L.s_x);
       gp.s1 = f8->s1;
@@ -469,7 +468,6 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     gp.x = static_cast<const bf16*>(x);
     gp.phase_only = -1;
     if (f8 != nullptr) {
-      gp.fp8 = 1;
       gp.xq = ws + L.x_q;
       gp.sx = reinterpret_cast<const float*>(ws + L.s_x);
       gp.s1 = f8->s1;

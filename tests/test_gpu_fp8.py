@@ -156,6 +156,23 @@ def test_fp8_forward_rejects_shared_plan_and_bad_pointers():
     plan.check()
 
 
+def test_fp8_back_to_back_calls_do_not_leak_state():
+    """x1, then a different x2 (larger activations), then x1 again on one plan: the third call
+    matches the first (the per-row activation amax and scales are rebuilt every call)."""
+    from moe_megakernel_b200 import MoEPlan
+    shape = custom_shape(300, 256, 384, 16, 4)
+    inp = make_inputs(shape, device=DEV)
+    fw = _fp8_weights(inp)
+    plan = MoEPlan(shape.T, shape.H, shape.I, shape.E, shape.k, fp8=True)
+    x2 = (inp["x"].float() * 8.0).to(torch.bfloat16)
+    y1 = plan.forward_fp8(inp["x"], inp["Wg"], None, *fw).float().clone()
+    plan.forward_fp8(x2, inp["Wg"], None, *fw)
+    y3 = plan.forward_fp8(inp["x"], inp["Wg"], None, *fw).float()
+    plan.check()
+    # equal up to the order of the fp32 combine reductions
+    assert (y1 - y3).abs().max().item() <= 1e-2 * max(1.0, y1.abs().max().item())
+
+
 def test_fp8_host_entry_matches_device_entry():
     from moe_megakernel_b200 import MoEPlan
     shape = custom_shape(300, 256, 384, 16, 4)

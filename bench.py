@@ -57,11 +57,22 @@ def measured_peaks():
 GEMM_SOURCES = ("common.cuh", "ptx.cuh", "expert_gemm.cuh", "expert_gemm2.cuh")   # what the expert GEMMs are built from
 
 
-def kernel_source_hash() -> str:
+def code_text(src: str) -> str:
+    """C++ source without comments and blank lines (what the compiler sees, for the hash below)."""
+    import re
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
+def kernel_source_hash(read=None) -> str:
+    """sha256 (16 hex) of the expert-GEMM sources' code, comments excluded."""
     import hashlib
+    if read is None:
+        read = lambda f: open(os.path.join(ROOT, "moe_megakernel_b200", "csrc", f)).read()
     h = hashlib.sha256()
     for f in GEMM_SOURCES:
-        h.update(open(os.path.join(ROOT, "moe_megakernel_b200", "csrc", f), "rb").read())
+        h.update(code_text(read(f)).encode())
     return h.hexdigest()[:16]
 
 

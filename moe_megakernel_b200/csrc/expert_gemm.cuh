@@ -24,6 +24,12 @@
 //   128-byte-swizzled K-major tile (a 4-row TMA gather costs far more TMA
 //   time than its 512 bytes are worth at this tile shape, and one warp of
 //   cp.async cannot keep up either); the weight tiles use TMA.
+//
+// The kernel is a template over the operand type: bf16 (kind::f16), or FP8 E4M3
+// (kind::f8f6f4: x, W1/W3, W2 and the activation as K-major codes, 128 K
+// elements per stage in the same 128-byte swizzle; token, column and
+// activation-row scales applied in the epilogues). The FP8 forward launches it
+// twice, first GEMM only and then second GEMM only (see GemmParams).
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>

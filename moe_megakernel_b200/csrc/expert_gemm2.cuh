@@ -25,6 +25,9 @@
 // Prior art: "MegaMoE 在 MoE 系统谱系中的位置", section 2.1 (the MMA warp issues
 // for the leader CTA only; warp roles with their own jobs) and section 2.7
 // (atomic task queue, L2 waits for its L1 tiles). No TMA multicast is used.
+//
+// Like expert_gemm.cuh, a template over bf16 or FP8 E4M3 operands; in the FP8
+// second GEMM the A-row warps copy the CTA's half of the K-major W2 codes.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>

@@ -257,9 +257,15 @@ def run_gpu(args, rank, world, local_rank):
         else:
             plan.forward(*args_fwd, y=y, **shared_kw)
 
+    # host-buffer steps: the pipelined entry (copies on the plan's own streams overlap the
+    # neighbouring steps' kernels); the plain one for shared experts
+    pipelined = S == 0
+
     def fwd_host(x_host, y_host):
-        if args.fp8:
-            plan.forward_host_fp8(x_host, inp["Wg"], inp["bias"], *fp8_w, y_host)
+        if pipelined and args.fp8:
+            plan.forward_host_pipelined_fp8(x_host, inp["Wg"], inp["bias"], *fp8_w, y_host)
+        elif pipelined:
+            plan.forward_host_pipelined(x_host, inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], y_host)
         else:
             plan.forward_host(x_host, inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], y_host, **shared_kw)
 
@@ -296,17 +302,23 @@ def run_gpu(args, rank, world, local_rank):
 
     # end to end through the host-buffer entry point
     x_host = inp["x"].cpu().pin_memory()
-    y_host = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
-    for _ in range(max(1, args.warmup)):
-        fwd_host(x_host, y_host)
+    y_hosts = [torch.empty((T, H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    for i in range(max(1, args.warmup)):
+        fwd_host(x_host, y_hosts[i % 2])
+    if pipelined:
+        plan.host_pipeline_join(stream)
     plan.check()
     e2e_steps = max(3, args.steps)
     barrier()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        fwd_host(x_host, y_host)
+    if pipelined:
+        plan.host_pipeline_after(stream)   # the first copy-in starts after e0
+    for i in range(e2e_steps):
+        fwd_host(x_host, y_hosts[i % 2])
+    if pipelined:
+        plan.host_pipeline_join(stream)    # e1 after the last copy-out
     e1.record(stream)
     torch.cuda.synchronize(dev)
     plan.check()
@@ -382,7 +394,9 @@ def run_gpu(args, rank, world, local_rank):
             "e2e": {"value": job_tokens_per_s(T, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2,
                     "ms_per_step": e2e_ms,
-                    "api": f"moe_forward_host{'_fp8' if args.fp8 else ''} (pinned host x and y)"},
+                    "api": (f"moe_forward_host_pipelined{'_fp8' if args.fp8 else ''} (pinned host x and y; the "
+                            "copies of each step overlap the neighbouring steps' kernels)") if pipelined
+                    else "moe_forward_host_shared (pinned host x and y)"},
             # FP8: + x quantizer, activation quantizer, second expert-GEMM launch
             "gpu_launches": args.steps * (kernels_per_forward() + (3 if args.fp8 else 0)),
             "clocks": clk,

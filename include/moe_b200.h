@@ -236,6 +236,31 @@ int moe_forward_host_fp8(moe_plan_t plan, const void* x_host, const void* Wg, co
                          const void* W1q, const float* s1, const void* W3q, const float* s3, const void* W2q,
                          const float* s2, int T, void* y_host, void* stream);
 
+/* ---- Pipelined host-buffer forward (serving loops). Like moe_forward_host,
+ * but the copies run on two streams of the plan's own, so that the copy of
+ * one call's x in and the previous call's y out overlap the neighbouring
+ * calls' kernels (which run on `stream`, in call order). Calls use the two
+ * halves of the plan's staging buffers in turn: a half is refilled only after
+ * the forward that read it has finished and its y has been copied out. The
+ * caller keeps x_host and y_host untouched until the call's copies are done:
+ * moe_host_pipeline_join(plan, stream) makes `stream` wait for every copy
+ * issued so far (synchronise `stream` after it before reading y_host).
+ * Plans with shared experts: MOE_ERR_INVALID_ARG. Do not interleave with
+ * moe_forward_host* calls on the same plan without a join in between.
+ * Errors as for moe_forward_host (moe_forward_host_fp8 for the FP8 form). */
+int moe_forward_host_pipelined(moe_plan_t plan, const void* x_host, const void* Wg, const float* gate_bias,
+                               const void* W1, const void* W3, const void* W2, int T, void* y_host, void* stream);
+int moe_forward_host_pipelined_fp8(moe_plan_t plan, const void* x_host, const void* Wg, const float* gate_bias,
+                                   const void* W1q, const float* s1, const void* W3q, const float* s3,
+                                   const void* W2q, const float* s2, int T, void* y_host, void* stream);
+
+/* Order the pipeline's later copies after the work already enqueued on `stream`
+ * (for instance a timing event). A no-op before the first pipelined call. */
+int moe_host_pipeline_after(moe_plan_t plan, void* stream);
+
+/* Make `stream` wait for every pipelined copy issued so far (enqueue only). */
+int moe_host_pipeline_join(moe_plan_t plan, void* stream);
+
 /* Gate and dispatch only (router, scan, scatter) for T tokens; fills the
  * routing results exactly as moe_forward does, without the expert FFN. */
 int moe_route(moe_plan_t plan, const void* x, const void* Wg, const float* gate_bias, int T, void* stream);

@@ -58,6 +58,10 @@ SIGNATURES = {
     "moe_forward_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
     "moe_forward_host_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
     "moe_quantize_weights_fp8": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp]),
+    "moe_forward_host_pipelined": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
+    "moe_forward_host_pipelined_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp]),
+    "moe_host_pipeline_after": (_c_int, [_vp, _vp]),
+    "moe_host_pipeline_join": (_c_int, [_vp, _vp]),
     "moe_quantize_x_fp8": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _vp]),
     "moe_route": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _vp]),
     "moe_check": (_c_int, [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]),
@@ -234,6 +238,37 @@ class MoEPlan:
                                           _ptr(W3q), _ptr(s3), _ptr(W2q), _ptr(s2), T, _ptr(y_host),
                                           _stream_handle(stream, self.device)), "moe_forward_host_fp8")
         return y_host
+
+    def forward_host_pipelined(self, x_host, Wg, bias, W1, W3, W2, y_host, stream=None):
+        """Pipelined host-buffer forward (copies on the plan's own streams, see the C header);
+        call host_pipeline_join(stream) before synchronising and reading y_host."""
+        T = x_host.shape[0]
+        _check(x_host, "x_host", (T, self.H), torch.bfloat16, torch.device("cpu"))
+        _check(y_host, "y_host", (T, self.H), torch.bfloat16, torch.device("cpu"))
+        _check(Wg, "Wg", (self.H, self.E), torch.bfloat16, self.device)
+        _ok(self.lib.moe_forward_host_pipelined(self._plan, _ptr(x_host), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3),
+                                                _ptr(W2), T, _ptr(y_host), _stream_handle(stream, self.device)),
+            "moe_forward_host_pipelined")
+        return y_host
+
+    def forward_host_pipelined_fp8(self, x_host, Wg, bias, W1q, s1, W3q, s3, W2q, s2, y_host, stream=None):
+        """forward_host_pipelined with FP8 expert GEMMs."""
+        T = x_host.shape[0]
+        _check(x_host, "x_host", (T, self.H), torch.bfloat16, torch.device("cpu"))
+        _check(y_host, "y_host", (T, self.H), torch.bfloat16, torch.device("cpu"))
+        _check(Wg, "Wg", (self.H, self.E), torch.bfloat16, self.device)
+        self._check_fp8(W1q, s1, W3q, s3, W2q, s2)
+        _ok(self.lib.moe_forward_host_pipelined_fp8(self._plan, _ptr(x_host), _ptr(Wg), _ptr(bias), _ptr(W1q),
+                                                    _ptr(s1), _ptr(W3q), _ptr(s3), _ptr(W2q), _ptr(s2), T,
+                                                    _ptr(y_host), _stream_handle(stream, self.device)),
+            "moe_forward_host_pipelined_fp8")
+        return y_host
+
+    def host_pipeline_after(self, stream=None):
+        _ok(self.lib.moe_host_pipeline_after(self._plan, _stream_handle(stream, self.device)), "moe_host_pipeline_after")
+
+    def host_pipeline_join(self, stream=None):
+        _ok(self.lib.moe_host_pipeline_join(self._plan, _stream_handle(stream, self.device)), "moe_host_pipeline_join")
 
     def route(self, x, Wg, bias, stream=None):
         T = self._check_inputs(x, Wg, bias)

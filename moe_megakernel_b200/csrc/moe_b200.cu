@@ -114,6 +114,12 @@ struct moe_plan {
   int pgroup_min, pgroup_max, pmax_groups, ring_pairs; // the same in units of block pairs
   int per_expert;                                      // expected blocks per expert + 1
   int fp8_rows = 0;                                    // FP8 plans: activation rows of all blocks or pairs
+  // pipelined host entry: its own copy streams, two staging buffers used in turn, and the events
+  // that order each buffer's copy-in, forward and copy-out
+  cudaStream_t cp_in = nullptr, cp_out = nullptr;
+  cudaEvent_t ev_in[2] = {}, ev_done[2] = {}, ev_out[2] = {}, ev_mark = nullptr;
+  int pipe_next = 0;
+  bool pipe_used[2] = {false, false};
   Layout L;
   uint8_t* ws = nullptr;
   size_t ws_bytes = 0;
@@ -167,8 +173,8 @@ static Layout make_layout(const moe_plan& p) {
   L.router_counter = take((size_t)p.num_sms * 4, 256);
   L.h = take((size_t)std::max({p.ring_blocks * p.BM, 2 * p.ring_pairs * p.BM, p.fp8_rows}) * p.I * 2, 1024);
   L.y_acc = take((size_t)p.T_max * p.H * 4, 1024);
-  L.x_stage = take((size_t)p.T_max * p.H * 2, 1024);
-  L.y_stage = take((size_t)p.T_max * p.H * 2, 1024);
+  L.x_stage = take(2 * (size_t)p.T_max * p.H * 2, 1024);   // two buffers each (the pipelined entry alternates)
+  L.y_stage = take(2 * (size_t)p.T_max * p.H * 2, 1024);
   L.x_q = take((size_t)p.T_max * p.H, 1024);   // FP8 first GEMM: x codes and token scales
   L.s_x = take((size_t)p.T_max * 4, 256);
   // FP8 plans: the activation of every block (or pair) at once, its codes and row amax / scale
@@ -801,6 +807,8 @@ int moe_plan_bind_workspace(moe_plan_t p, void* ws, size_t bytes) {
   if (cudaMemset(p->ws + p->L.router_partial, 0, (size_t)p->num_sms * kRouterTokens * 256 * 4) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  p->pipe_used[0] = p->pipe_used[1] = false;   // a new workspace: no staging buffer is in flight
+  p->pipe_next = 0;
   return MOE_OK;
 }
 
@@ -872,6 +880,85 @@ static int forward_host(moe_plan_t p, const void* x_host, const void* Wg, const 
   const int rc = enqueue(p, xd, Wg, bias, W1, W3, W2, sw, T, yd, st, true, f8);
   if (rc != MOE_OK) return rc;
   if (cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+// The pipelined host entry: x is copied in on the plan's copy-in stream, the forward runs on
+// `stream`, y is copied out on the copy-out stream, each call using the other of two staging
+// buffers, so one call's copies overlap the neighbouring calls' kernels. A buffer is refilled
+// only after the forward that read it has finished, and reused for y only after its previous
+// y has been copied out.
+static int forward_host_pipelined(moe_plan_t p, const void* x_host, const void* Wg, const float* bias,
+                                  const void* W1, const void* W3, const void* W2, int T, void* y_host, void* stream,
+                                  const Fp8Weights* f8) {
+  if (p == nullptr || x_host == nullptr || y_host == nullptr) return MOE_ERR_INVALID_ARG;
+  if (p->ws == nullptr) return MOE_ERR_NO_WORKSPACE;
+  if (p->S > 0) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || T > p->T_max) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  DeviceGuard guard(p->device);
+  if (p->cp_in == nullptr) {
+    if (cudaStreamCreateWithFlags(&p->cp_in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&p->cp_out, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&p->ev_mark, cudaEventDisableTiming) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    for (int b = 0; b < 2; ++b)
+      if (cudaEventCreateWithFlags(&p->ev_in[b], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&p->ev_done[b], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&p->ev_out[b], cudaEventDisableTiming) != cudaSuccess)
+        return MOE_ERR_CUDA;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int b = p->pipe_next;
+  const size_t stage = (size_t)p->T_max * p->H * 2;
+  const size_t bytes = (size_t)T * p->H * 2;
+  void* xd = p->ws + p->L.x_stage + b * stage;
+  void* yd = p->ws + p->L.y_stage + b * stage;
+  if (p->pipe_used[b] && cudaStreamWaitEvent(p->cp_in, p->ev_done[b], 0) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, p->cp_in) != cudaSuccess ||
+      cudaEventRecord(p->ev_in[b], p->cp_in) != cudaSuccess || cudaStreamWaitEvent(st, p->ev_in[b], 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (p->pipe_used[b] && cudaStreamWaitEvent(st, p->ev_out[b], 0) != cudaSuccess) return MOE_ERR_CUDA;
+  const int rc = enqueue(p, xd, Wg, bias, W1, W3, W2, SharedWeights{}, T, yd, st, true, f8);
+  if (rc != MOE_OK) return rc;
+  if (cudaEventRecord(p->ev_done[b], st) != cudaSuccess || cudaStreamWaitEvent(p->cp_out, p->ev_done[b], 0) != cudaSuccess ||
+      cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, p->cp_out) != cudaSuccess ||
+      cudaEventRecord(p->ev_out[b], p->cp_out) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  p->pipe_used[b] = true;
+  p->pipe_next = b ^ 1;
+  return MOE_OK;
+}
+
+int moe_forward_host_pipelined(moe_plan_t p, const void* x_host, const void* Wg, const float* bias, const void* W1,
+                               const void* W3, const void* W2, int T, void* y_host, void* stream) {
+  return forward_host_pipelined(p, x_host, Wg, bias, W1, W3, W2, T, y_host, stream, nullptr);
+}
+
+int moe_forward_host_pipelined_fp8(moe_plan_t p, const void* x_host, const void* Wg, const float* bias,
+                                   const void* W1q, const float* s1, const void* W3q, const float* s3,
+                                   const void* W2q, const float* s2, int T, void* y_host, void* stream) {
+  const Fp8Weights f8{W1q, s1, W3q, s3, W2q, s2};
+  return forward_host_pipelined(p, x_host, Wg, bias, nullptr, nullptr, nullptr, T, y_host, stream, &f8);
+}
+
+int moe_host_pipeline_after(moe_plan_t p, void* stream) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  if (p->cp_in == nullptr) return MOE_OK;   // nothing pipelined yet: the first call creates the streams
+  DeviceGuard guard(p->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaEventRecord(p->ev_mark, st) != cudaSuccess || cudaStreamWaitEvent(p->cp_in, p->ev_mark, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(p->cp_out, p->ev_mark, 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+int moe_host_pipeline_join(moe_plan_t p, void* stream) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(p->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int b = 0; b < 2; ++b)
+    if (p->pipe_used[b] && cudaStreamWaitEvent(st, p->ev_out[b], 0) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 
@@ -1012,6 +1099,18 @@ void moe_plan_destroy(moe_plan_t p) {
   {
     DeviceGuard guard(p->device);
     for (auto& e : p->ev) cudaEventDestroy(e);
+    if (p->cp_in != nullptr) {
+      cudaStreamSynchronize(p->cp_in);
+      cudaStreamSynchronize(p->cp_out);
+      for (int b = 0; b < 2; ++b) {
+        cudaEventDestroy(p->ev_in[b]);
+        cudaEventDestroy(p->ev_done[b]);
+        cudaEventDestroy(p->ev_out[b]);
+      }
+      cudaEventDestroy(p->ev_mark);
+      cudaStreamDestroy(p->cp_in);
+      cudaStreamDestroy(p->cp_out);
+    }
   }
   delete p;
 }

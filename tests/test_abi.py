@@ -81,3 +81,48 @@ def test_null_plan_arguments(lib):
 
 def test_kernel_count(lib):
     assert lib.moe_forward_kernel_count() == 5
+
+
+def test_null_plan_arguments_of_the_newer_entries(lib):
+    """The FP8, pipelined and shared-expert entries reject a null plan before touching a device."""
+    assert lib.moe_plan_set_fp8(None, 1) == 1
+    assert lib.moe_forward_fp8(None, None, None, None, None, None, None, None, None, None, 0, None, None) == 1
+    assert lib.moe_forward_host_pipelined(None, None, None, None, None, None, None, 0, None, None) == 1
+    assert lib.moe_host_pipeline_after(None, None) == 1
+    assert lib.moe_host_pipeline_join(None, None) == 1
+    assert lib.moe_plan_set_cta_pairs(None, 1) == 1
+
+
+@pytest.mark.parametrize("args", [
+    (1, 100, 128),    # K % 64
+    (1, 128, 100),    # N % 64
+    (0, 128, 128),    # E < 1
+])
+def test_weight_quantizer_rejects_bad_sizes_without_device(lib, args):
+    E, K, N = args
+    assert lib.moe_quantize_weights_fp8(None, None, None, E, K, N, None) == 1
+
+
+def test_quantizer_bindings_check_shapes_before_calling(lib):
+    import torch
+
+    from moe_megakernel_b200 import quantize_weights_fp8, quantize_x_fp8
+    with pytest.raises(TypeError):
+        quantize_weights_fp8(torch.zeros(4, 4, dtype=torch.bfloat16))     # not [E, K, N]
+    with pytest.raises(TypeError):
+        quantize_x_fp8(torch.zeros(2, 2, 2, dtype=torch.bfloat16))        # not [T, H]
+    with pytest.raises(ValueError):
+        quantize_weights_fp8(torch.zeros(1, 64, 64, dtype=torch.float32))  # not bf16
+
+
+def test_bench_source_hash_ignores_comments():
+    """bench.py's check that measured counters belong to the current expert-GEMM code: comment
+    and blank-line edits do not change the hash, code edits do."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    a = "int f(int x) {\n  return x + 1;  // add one\n}\n"
+    b = "/* header\n   text */\nint f(int x) {\n\n  return x + 1;\n}  // end\n"
+    c = "int f(int x) {\n  return x + 2;\n}\n"
+    assert bench.code_text(a) == bench.code_text(b)
+    assert bench.code_text(a) != bench.code_text(c)

@@ -236,11 +236,16 @@ def silu(g: np.ndarray) -> np.ndarray:
     return g / (1.0 + np.exp(-g))
 
 
-def expert_ffn(xr: np.ndarray, W1e: np.ndarray, W3e: np.ndarray, W2e: np.ndarray) -> np.ndarray:
-    """o = bf16(silu(xr W1e) * (xr W3e)) W2e for rows xr [n,H]; W1e,W3e [H,I]; W2e [I,H]."""
+def expert_ffn(xr: np.ndarray, W1e: np.ndarray, W3e: np.ndarray, W2e: np.ndarray,
+               round_activation: bool = True) -> np.ndarray:
+    """o = bf16(silu(xr W1e) * (xr W3e)) W2e for rows xr [n,H]; W1e,W3e [H,I]; W2e [I,H].
+    round_activation=False leaves the activation unrounded (the smooth function whose
+    derivative the backward computes)."""
     g = xr @ W1e
     u = xr @ W3e
-    a = bf16_round(silu(g) * u)
+    a = silu(g) * u
+    if round_activation:
+        a = bf16_round(a)
     return a @ W2e
 
 
@@ -267,7 +272,7 @@ def stacked_expert_weights(W1, W3, W2) -> Callable[[int], tuple]:
 def moe_forward(x, Wg, bias, expert_weights: Callable[[int], tuple], k: int,
                 block_m: Optional[int] = None, tokens: Optional[Sequence[int]] = None,
                 shared_weights: Optional[Callable[[int], tuple]] = None, n_shared: int = 0,
-                fp8: bool = False) -> dict:
+                fp8: bool = False, round_activation: bool = True) -> dict:
     """The whole layer: gate, dispatch, expert FFN, gate-weighted combine.
 
     x [T,H] fp64; Wg [H,E] fp64; bias [E] or None; ``expert_weights(e)``
@@ -303,7 +308,7 @@ def moe_forward(x, Wg, bias, expert_weights: Callable[[int], tuple], k: int,
             W2q, s2 = quantize_fp8(W2e, axis=0)
             o = expert_ffn_fp8(xq[rows[hit[0]]], sx[rows[hit[0]]], W1q, s1, W3q, s3, W2q, s2)
         else:
-            o = expert_ffn(x[rows[hit[0]]], W1e, W3e, W2e)
+            o = expert_ffn(x[rows[hit[0]]], W1e, W3e, W2e, round_activation)
         wt = w[rows[hit[0]], hit[1]]
         np.add.at(y, hit[0], wt[:, None] * o)
     if n_shared:

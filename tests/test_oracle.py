@@ -371,9 +371,9 @@ def test_fp8_forward_matches_textbook_dequantized_ffn():
 # ----------------------------------------------------------------- planted mistakes
 
 _MUTANTS = {
-    "no_activation_rounding": ("expert_ffn", lambda xr, W1e, W3e, W2e:
+    "no_activation_rounding": ("expert_ffn", lambda xr, W1e, W3e, W2e, round_activation=True:
                                (O.silu(xr @ W1e) * (xr @ W3e)) @ W2e),
-    "swapped_gate_and_up": ("expert_ffn", lambda xr, W1e, W3e, W2e:
+    "swapped_gate_and_up": ("expert_ffn", lambda xr, W1e, W3e, W2e, round_activation=True:
                             O.bf16_round(O.silu(xr @ W3e) * (xr @ W1e)) @ W2e),
     "silu_sign": ("silu", lambda g: g / (1.0 + np.exp(g))),
     "no_renormalisation": ("renormalised_softmax", lambda l, idx:

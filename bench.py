@@ -42,7 +42,10 @@ sys.path.insert(0, ROOT)
 BASELINE_METRIC = "MoE-layer fwd tokens/s on 1 B200 (device-timed); % of max(TC, HBM) roofline"
 DEFAULT_WORKLOAD = "mixtral"
 FLUSH_BYTES = 256 << 20
-ORACLE_SAMPLE = {"tiny": 64, "mixtral": 128, "fine_grained_prefill": 24, "decode": 8, "skewed": 512}
+# tokens of the fp64 oracle per reference-arm step (about a second each on 16 host cores, so that a
+# --steps 100 run ends in minutes) and for the cpu_baseline of the native arm (about 10 s of work)
+ORACLE_SAMPLE = {"tiny": 64, "mixtral": 128, "fine_grained_prefill": 4, "decode": 4, "skewed": 512}
+CPU_BASELINE_SAMPLE = {"tiny": 64, "mixtral": 1024, "fine_grained_prefill": 32, "decode": 32, "skewed": 4096}
 
 
 def measured_peaks():
@@ -332,7 +335,7 @@ def run_gpu(args, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
-        n = min(T, ORACLE_SAMPLE.get(args.workload, 64))
+        n = min(T, CPU_BASELINE_SAMPLE.get(args.workload, 64))
         v, dt, cores = time_oracle(inp, n, fp8=args.fp8)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"fp64 oracle (gate, dispatch, expert FFN, combine{', FP8 expert GEMMs' if args.fp8 else ''}) "

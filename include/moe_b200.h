@@ -32,7 +32,15 @@
  *  - Device-side failures (a bounded wait that ran out, a routing index out of
  *    range) are sticky in the workspace and are reported by moe_check().
  *  - The caller owns all device memory: inputs, weights, outputs and the
- *    workspace. A plan owns only host state.
+ *    workspace. A plan owns only host state (and, once a pipelined host-buffer
+ *    call has run, its two copy streams and their events).
+ *
+ * Order of use: moe_plan_create (or _shared) -> [moe_plan_set_fp8] ->
+ * moe_plan_workspace_bytes -> allocate -> moe_plan_bind_workspace ->
+ * any number of moe_forward / moe_forward_shared / moe_forward_fp8 /
+ * moe_forward_host* / moe_route calls -> moe_check -> moe_plan_destroy.
+ * moe_route_static routes without a plan or workspace. FP8 weights come from
+ * moe_quantize_weights_fp8, once per set of weights.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H

@@ -14,6 +14,10 @@ enum DeviceError : int {
   kDevBounds = 2,    // an index read from routing metadata was out of range
 };
 
+// Expert id a router writes for a token whose selection it gave up on (a
+// bounded wait ran out); the dispatch scatter skips it and records a timeout.
+constexpr int kAbortedExpert = -1;
+
 // Router tile: tokens per CTA (one 16-row mma.sync tile per warp) and K chunk.
 constexpr int kRouterTokens = 64;
 constexpr int kRouterThreads = 128;

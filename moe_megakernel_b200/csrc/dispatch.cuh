@@ -219,6 +219,10 @@ __global__ void __launch_bounds__(256) moe_dispatch_scatter_kernel(const Dispatc
   if (i >= p.T * p.k) return;
   const int t = i / p.k, j = i - t * p.k;
   const int e = p.topk_idx[i];
+  if (e == kAbortedExpert) {   // the router gave up on this token (and recorded the timeout)
+    atomicCAS(p.err, 0, kDevTimeout);
+    return;
+  }
   if (e < 0 || e >= p.E) {
     atomicCAS(p.err, 0, kDevBounds);
     return;

@@ -93,6 +93,13 @@ bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Entry points that launch kernels first drop whatever error an earlier runtime
+// call on this thread left pending (cudaGetLastError returns and clears it), so
+// that the cudaGetLastError() after each launch below reports that launch only.
+// A sticky error (a lost context) is not cleared by this and still fails the
+// launches that follow.
+void drop_stale_error() { (void)cudaGetLastError(); }
+
 int block_m_rule(int T, int k, int E) {
   // n = T*k/E compared against 16, 32, 64 without rounding
   const long long tk = (long long)T * k;
@@ -260,6 +267,7 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     }
   }
   DeviceGuard guard(p->device);
+  drop_stale_error();
   uint8_t* ws = p->ws;
   const Layout& L = p->L;
   const bool prof = p->profile && p->ev_used < kMaxProfiled;
@@ -589,9 +597,11 @@ extern "C" int moe_route_static(const void* x, const void* Wg, const float* gate
     return MOE_ERR_UNSUPPORTED_SHAPE;
   if (block_m != 0 && block_m != 16 && block_m != 32 && block_m != 64 && block_m != 128)
     return MOE_ERR_UNSUPPORTED_SHAPE;
+  // far beyond the scratch limit below; refused here so that no size arithmetic can overflow
+  if (T > kStaticScratchInts) return MOE_ERR_STATIC_SCRATCH_LIMIT;
   const int BM = block_m ? block_m : block_m_rule(T > 0 ? T : 1, k, E);
   const long long pool = ((long long)T * k + (long long)E * (BM - 1) + BM - 1) / BM * BM;
-  const long long chunks = (T + kRouterTokens - 1) / kRouterTokens;
+  const long long chunks = ((long long)T + kRouterTokens - 1) / kRouterTokens;
   // scratch regions, each rounded up to 64 ints (256 bytes)
   auto r64 = [](long long v) { return (v + 63) / 64 * 64; };
   const long long o_err = 0, o_sched = 64, o_rank = 128;
@@ -607,6 +617,7 @@ extern "C" int moe_route_static(const void* x, const void* Wg, const float* gate
       slot_token == nullptr || slot_topk == nullptr || num_padded == nullptr)
     return MOE_ERR_INVALID_ARG;
   if (pool_capacity < pool) return MOE_ERR_INVALID_ARG;
+  drop_stale_error();
   int32_t* scratch = nullptr;
   int rc = static_scratch_for_current_device(&scratch);
   if (rc != MOE_OK) return rc;
@@ -995,6 +1006,7 @@ int moe_quantize_x_fp8(const void* x, void* xq, float* sx, int T, int H, void* s
   if (x == nullptr || xq == nullptr || sx == nullptr || !aligned16(x) || (reinterpret_cast<uintptr_t>(xq) & 7u) ||
       (reinterpret_cast<uintptr_t>(sx) & 3u))
     return MOE_ERR_INVALID_ARG;
+  drop_stale_error();
   moe_quantize_x_kernel<<<(T + 7) / 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const bf16*>(x), static_cast<uint8_t*>(xq), sx, T, H);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -1007,6 +1019,7 @@ int moe_quantize_weights_fp8(const void* W, void* Wq, float* scale, int E, int H
     return MOE_ERR_INVALID_ARG;
   if (E > 65535 || (long long)E * H * I > (1LL << 40)) return MOE_ERR_UNSUPPORTED_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  drop_stale_error();
   moe_weight_scales_kernel<<<dim3((unsigned)(I / 32), (unsigned)E), 256, 0, st>>>(static_cast<const bf16*>(W), scale,
                                                                                  H, I);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
@@ -1019,12 +1032,17 @@ int moe_check(moe_plan_t p, void* stream, int32_t* detail) {
   if (p == nullptr) return MOE_ERR_INVALID_ARG;
   if (p->ws == nullptr) return MOE_ERR_NO_WORKSPACE;
   DeviceGuard guard(p->device);
+  drop_stale_error();
+  // Everything on `stream` only: the read and the clearing of the error word are
+  // ordered after the plan's kernels there, and no other stream of the device waits.
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
   int32_t e[2] = {0, 0};
-  if (cudaMemcpy(e, p->ws + p->L.err, sizeof(e), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
-  if (e[0] != 0 && cudaMemset(p->ws + p->L.err, 0, sizeof(e)) != cudaSuccess) return MOE_ERR_CUDA;
-  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpyAsync(e, p->ws + p->L.err, sizeof(e), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (e[0] != 0 && (cudaMemsetAsync(p->ws + p->L.err, 0, sizeof(e), st) != cudaSuccess ||
+                    cudaStreamSynchronize(st) != cudaSuccess))
+    return MOE_ERR_CUDA;
   if (detail) *detail = e[1];
   switch (e[0]) {
     case kDevOk: return MOE_OK;

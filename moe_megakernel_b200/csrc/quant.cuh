@@ -19,12 +19,16 @@ namespace moe {
 
 constexpr float kE4m3Max = 448.f;
 
-// Exponent k of the scale 2**k for a row with largest magnitude amax.
+// Exponent k of the scale 2**k for a row with largest magnitude amax: the
+// smallest k with amax <= 448 * 2**k. Decided on amax itself, with no rounded
+// quotient: amax = m * 2**e exactly (m in [0.5, 1)) and 448 = 0.875 * 2**9,
+// so amax <= 0.875 * 2**(k+9) holds from k = e - 9 when m <= 0.875 and from
+// k = e - 8 otherwise.
 __device__ __forceinline__ int pow2_scale_exp(float amax) {
   if (!(amax > 0.f)) return 0;
   int e;
-  const float m = frexpf(amax / kE4m3Max, &e);   // amax/448 = m * 2**e, m in [0.5, 1)
-  return m == 0.5f ? e - 1 : e;
+  const float m = frexpf(amax, &e);
+  return m <= 0.875f ? e - 9 : e - 8;
 }
 
 // Eight bf16 values (one uint4) times `inv` (an exact power of two) -> eight E4M3 codes, in order.

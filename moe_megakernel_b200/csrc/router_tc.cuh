@@ -168,7 +168,10 @@ __global__ void __launch_bounds__(kRtcThreads, 1) moe_router_tc_kernel(const __g
     // ------------------------------------------------ epilogue: one token per thread
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const bool ok = rtc_wait(&s.acc_full, 0, p, s, 3);
+    // the MMA warp commits acc_full even after giving up on a stage, so the
+    // accumulator is complete only if no role of this CTA aborted
+    bool ok = rtc_wait(&s.acc_full, 0, p, s, 3);
+    ok = ok && !*reinterpret_cast<volatile int*>(&s.abort);
     ptx::tc_fence_after();
     // best[0..k-1]: the k largest logits so far, descending; equal values keep
     // arrival order, and candidates arrive in ascending expert id, so a tie
@@ -213,7 +216,14 @@ __global__ void __launch_bounds__(kRtcThreads, 1) moe_router_tc_kernel(const __g
       }
     }
     if (!ok && r < ntok) {
-      // aborted (bounded wait ran out): no selection; mark the rows invalid
+      // aborted (a bounded wait ran out): no selection. The token's rows get the
+      // sentinel expert id -1 (weight 0), which the dispatch scatter skips as a
+      // timeout instead of reading whatever the workspace held before.
+      const size_t o = (size_t)(t0 + r) * p.k;
+      for (int j = 0; j < p.k; ++j) {
+        p.topk_idx[o + j] = kAbortedExpert;
+        p.topk_w[o + j] = 0.f;
+      }
 #pragma unroll
       for (int j = 0; j < 8; ++j) s.sel[r][j] = -1;
       if (r == 0) atomicCAS(p.err, 0, kDevTimeout);

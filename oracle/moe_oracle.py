@@ -272,7 +272,7 @@ def stacked_expert_weights(W1, W3, W2) -> Callable[[int], tuple]:
 def moe_forward(x, Wg, bias, expert_weights: Callable[[int], tuple], k: int,
                 block_m: Optional[int] = None, tokens: Optional[Sequence[int]] = None,
                 shared_weights: Optional[Callable[[int], tuple]] = None, n_shared: int = 0,
-                fp8: bool = False, round_activation: bool = True) -> dict:
+                fp8: bool = False, round_activation: bool = True, workers: int = 1) -> dict:
     """The whole layer: gate, dispatch, expert FFN, gate-weighted combine.
 
     x [T,H] fp64; Wg [H,E] fp64; bias [E] or None; ``expert_weights(e)``
@@ -283,6 +283,11 @@ def moe_forward(x, Wg, bias, expert_weights: Callable[[int], tuple], k: int,
     with ``shared_weights(s)`` returning the shared expert's (W1, W3, W2).
     fp8=True runs both expert GEMMs on FP8 E4M3 operands (see the module notes):
     x and the activation per token, W1/W3/W2 per (expert, column); no shared experts.
+
+    workers > 1 computes the experts' FFN outputs in that many threads (the
+    matrix and rounding routines release the interpreter lock); they are still
+    added into y one expert at a time in ascending expert order, so y is the
+    same for any number of workers.
     """
     x = np.asarray(x, np.float64)
     T, H = x.shape
@@ -296,11 +301,13 @@ def moe_forward(x, Wg, bias, expert_weights: Callable[[int], tuple], k: int,
         if n_shared:
             raise ValueError("the FP8 layer is defined without shared experts")
         xq, sx = quantize_fp8(x, axis=1)
-    for e in range(E):
-        # (row position in `rows`, top-k position) of every selected pair routed to e
+
+    def expert_part(e):
+        # (row position in `rows`, top-k position) of every selected pair routed to e,
+        # and the expert's FFN output for those rows
         hit = np.nonzero(idx[rows] == e)
         if hit[0].size == 0:
-            continue
+            return hit, None
         W1e, W3e, W2e = expert_weights(e)
         if fp8:
             W1q, s1 = quantize_fp8(W1e, axis=0)
@@ -309,8 +316,23 @@ def moe_forward(x, Wg, bias, expert_weights: Callable[[int], tuple], k: int,
             o = expert_ffn_fp8(xq[rows[hit[0]]], sx[rows[hit[0]]], W1q, s1, W3q, s3, W2q, s2)
         else:
             o = expert_ffn(x[rows[hit[0]]], W1e, W3e, W2e, round_activation)
+        return hit, o
+
+    if workers > 1:
+        from concurrent.futures import ThreadPoolExecutor
+        pool = ThreadPoolExecutor(max_workers=workers)
+        parts = pool.map(expert_part, range(E))
+    else:
+        pool = None
+        parts = map(expert_part, range(E))
+    for hit, o in parts:
+        if o is None:
+            continue
         wt = w[rows[hit[0]], hit[1]]
-        np.add.at(y, hit[0], wt[:, None] * o)
+        # a token selects an expert at most once, so the rows hit[0] are distinct
+        y[hit[0]] += wt[:, None] * o
+    if pool is not None:
+        pool.shutdown()
     if n_shared:
         y += shared_ffn_sum(x[rows], shared_weights, n_shared)
     return dict(topk_idx=idx, topk_w=w, logits=logits, y=y, tokens=rows, **disp)

@@ -103,12 +103,15 @@ def _ambiguous_tokens(x, Wg, bias, k: int) -> torch.Tensor:
 
 
 def make_router_inputs(shape: MoEShape, device="cpu", seed: int = 0,
-                       T: Optional[int] = None, wg_zero: bool = False):
-    """x [T,H] bf16, Wg [H,E] bf16, bias [E] fp32 or None, with the gap screen applied."""
+                       T: Optional[int] = None, wg_zero: bool = False, x_seed: Optional[int] = None):
+    """x [T,H] bf16, Wg [H,E] bf16, bias [E] fp32 or None, with the gap screen applied.
+    ``x_seed`` (default ``seed``) seeds the tokens and their redraws only, so that replicas
+    with the same weights can draw different tokens."""
     device = torch.device(device)
     T = shape.T if T is None else T
     H, E, k = shape.H, shape.E, shape.k
-    x = _normal_bf16((T, H), 1.0, _gen(device, seed, _STREAM_X), device)
+    xs = seed if x_seed is None else x_seed
+    x = _normal_bf16((T, H), 1.0, _gen(device, xs, _STREAM_X), device)
     if wg_zero:
         Wg = torch.zeros((H, E), dtype=torch.bfloat16, device=device)
     else:
@@ -123,7 +126,7 @@ def make_router_inputs(shape: MoEShape, device="cpu", seed: int = 0,
             if attempt == MAX_REDRAWS:
                 raise RuntimeError(f"{shape.name}: {bad.numel()} tokens still ambiguous "
                                    f"after {MAX_REDRAWS} redraws")
-            g = _gen(device, seed, _STREAM_REDRAW + attempt)
+            g = _gen(device, xs, _STREAM_REDRAW + attempt)
             x[bad] = _normal_bf16((bad.numel(), H), 1.0, g, device)
             if attempt == 0:
                 redrawn = bad.numel()
@@ -167,12 +170,14 @@ def make_shared_weights(shape: MoEShape, n_shared: int, device="cpu", seed: int 
     return Ws1, Ws3, Ws2
 
 
-def make_inputs(shape, device="cpu", seed: int = 0, T: Optional[int] = None, n_shared: int = 0):
+def make_inputs(shape, device="cpu", seed: int = 0, T: Optional[int] = None, n_shared: int = 0,
+                x_seed: Optional[int] = None):
     """All inputs of one workload as a dict of tensors on ``device`` (plus
-    ``n_shared`` shared experts Ws1/Ws3/Ws2 when asked for)."""
+    ``n_shared`` shared experts Ws1/Ws3/Ws2 when asked for). ``x_seed`` (default
+    ``seed``) draws the tokens from another seed with the same weights."""
     if isinstance(shape, str):
         shape = WORKLOADS[shape]
-    x, Wg, bias, redrawn = make_router_inputs(shape, device, seed, T)
+    x, Wg, bias, redrawn = make_router_inputs(shape, device, seed, T, x_seed=x_seed)
     W1, W3, W2 = make_expert_weights(shape, device, seed)
     out = dict(shape=shape, x=x, Wg=Wg, bias=bias, W1=W1, W3=W3, W2=W2,
                k=shape.k, redrawn=redrawn, n_shared=n_shared)

@@ -14,7 +14,7 @@ import torch
 
 import oracle.moe_oracle as O
 from synth.moe_inputs import WORKLOADS, custom_shape, make_inputs
-from tests.parity_util import assert_routing_equal, assert_y_close, oracle_forward, sample_tokens, to_f64
+from tests.parity_util import assert_routing_equal, assert_y_close, full_oracle, oracle_forward, sample_tokens, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -191,7 +191,7 @@ def test_fp8_host_entry_matches_device_entry():
 @pytest.mark.slow
 @pytest.mark.parametrize("name", ["mixtral", "fine_grained_prefill", "decode"])
 def test_fp8_workload_matches_oracle(name):
-    """Full-size layers with the FP8 first GEMM, y on sampled tokens."""
+    """Full-size layers with FP8 expert GEMMs, y on every token row."""
     from moe_megakernel_b200 import MoEPlan
     shape = WORKLOADS[name]
     inp = make_inputs(shape, device=DEV)
@@ -199,9 +199,7 @@ def test_fp8_workload_matches_oracle(name):
     plan = MoEPlan(shape.T, shape.H, shape.I, shape.E, shape.k, fp8=True)
     y = plan.forward_fp8(inp["x"], inp["Wg"], inp["bias"], *fw)
     plan.check()
-    rows = sample_tokens(shape.T, {"mixtral": 8, "fine_grained_prefill": 4, "decode": 4}[name])
-    # (few tokens: the oracle quantizes every expert a sampled token reaches, in fp64)
-    ref = oracle_forward(inp, tokens=rows, block_m=plan.block_m, fp8=True)
+    ref = full_oracle(name, inp, plan.block_m, fp8=True)
     assert_routing_equal(plan.routing(shape.T), ref)
-    fro, mx = assert_y_close(y[torch.from_numpy(rows).to(y.device)], ref["y"], "y (fp8)")
-    print(f"fp8 {name}: rel_fro={fro:.2e} max_abs={mx:.2e}")
+    fro, mx = assert_y_close(y, ref["y"], "y (fp8)")
+    print(f"fp8 {name}: all {shape.T} rows rel_fro={fro:.2e} max_abs={mx:.2e}")

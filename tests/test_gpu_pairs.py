@@ -13,7 +13,7 @@ import pytest
 import torch
 
 from synth.moe_inputs import WORKLOADS, custom_shape, make_inputs
-from tests.parity_util import assert_routing_equal, assert_y_close, oracle_forward, sample_tokens
+from tests.parity_util import assert_routing_equal, assert_y_close, full_oracle, oracle_forward, sample_tokens
 
 pytestmark = pytest.mark.gpu
 
@@ -97,8 +97,8 @@ def test_pairs_workload_matches_oracle(name):
     plan.set_cta_pairs(plan.block_m != 128)
     y = plan.forward(inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"])
     plan.check()
-    rows = sample_tokens(shape.T, {"mixtral": 32, "fine_grained_prefill": 12, "decode": 32, "skewed": 96}[name])
-    ref = oracle_forward(inp, tokens=rows, block_m=plan.block_m)
+    ref = full_oracle(name, inp, plan.block_m)   # every token row
     assert_routing_equal(plan.routing(shape.T), ref)
-    fro, mx = assert_y_close(y[torch.from_numpy(rows).to(y.device)], ref["y"])
-    print(f"{'pairs' if plan.block_m != 128 else 'single'} {name}: rel_fro={fro:.2e} max_abs={mx:.2e}")
+    fro, mx = assert_y_close(y, ref["y"])
+    print(f"{'pairs' if plan.block_m != 128 else 'single'} {name}: all {shape.T} rows rel_fro={fro:.2e} "
+          f"max_abs={mx:.2e}")

@@ -11,7 +11,9 @@ import pytest
 import torch
 
 from synth.moe_inputs import WORKLOADS, custom_shape, make_inputs
-from tests.parity_util import assert_routing_equal, assert_y_close, oracle_forward, sample_tokens
+import oracle.moe_oracle as O
+from tests.parity_util import (assert_routing_equal, assert_y_close, expert_loader, full_oracle, oracle_forward,
+                                sample_tokens, to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -120,8 +122,10 @@ def test_shared_workload_matches_oracle(name):
     plan = _plan(shape, 1)
     y = _fwd(plan, inp)
     plan.check()
-    rows = sample_tokens(shape.T, {"fine_grained_prefill": 12, "decode": 32}[name])
-    ref = oracle_forward(inp, tokens=rows, block_m=plan.block_m)
+    # every token row: the routed layer (shared with the other full-size tests) plus the
+    # oracle's sum of the shared experts' FFNs, as the oracle's layer adds them
+    ref = full_oracle(name, inp, plan.block_m)
     assert_routing_equal(plan.routing(shape.T), ref)
-    fro, mx = assert_y_close(y[torch.from_numpy(rows).to(y.device)], ref["y"])
-    print(f"shared {name}: rel_fro={fro:.2e} max_abs={mx:.2e}")
+    y_ref = ref["y"] + O.shared_ffn_sum(to_f64(inp["x"]), expert_loader(inp["Ws1"], inp["Ws3"], inp["Ws2"]), 1)
+    fro, mx = assert_y_close(y, y_ref)
+    print(f"shared {name}: all {shape.T} rows rel_fro={fro:.2e} max_abs={mx:.2e}")

@@ -421,3 +421,16 @@ def test_planted_mistake_is_caught(name, monkeypatch):
     attr, fn = _MUTANTS[name]
     monkeypatch.setattr(O, attr, fn)
     assert not _pins_pass(), f"mutant {name} slipped past every pin"
+
+
+def test_moe_forward_threaded_experts_give_the_same_y():
+    """The worker threads only compute the experts' outputs; y is added in expert order."""
+    rng = _rng(7)
+    T, H, I, E, k = 97, 128, 256, 16, 4
+    x, Wg = _bf16_vals(rng, (T, H)), _bf16_vals(rng, (H, E), H ** -0.5)
+    W1, W3 = _bf16_vals(rng, (E, H, I), H ** -0.5), _bf16_vals(rng, (E, H, I), H ** -0.5)
+    W2 = _bf16_vals(rng, (E, I, H), I ** -0.5)
+    load = O.stacked_expert_weights(W1, W3, W2)
+    a = O.moe_forward(x, Wg, None, load, k)
+    b = O.moe_forward(x, Wg, None, load, k, workers=4)
+    assert np.array_equal(a["y"], b["y"])

@@ -265,6 +265,10 @@ def run_gpu(args, rank, world, local_rank):
     shared_kw = dict(Ws1=inp["Ws1"], Ws3=inp["Ws3"], Ws2=inp["Ws2"]) if S else {}
     if args.cta_pairs is not None:
         plan.set_cta_pairs(bool(args.cta_pairs))
+    if args.task_order is not None:
+        plan.set_task_order(args.task_order)
+    if args.half_tails is not None:
+        plan.set_half_tails(bool(args.half_tails))
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
@@ -420,7 +424,8 @@ def run_gpu(args, rank, world, local_rank):
             "dtype": "e4m3 (expert GEMMs) + bf16" if args.fp8 else "bf16",
             "data": "synthetic (seeded N(0,1) x, N(0,1/H) Wg/W1/W3, N(0,1/I) W2, bf16; random-init weights)",
             "config": {"workload": workload_label(shape, S, args.fp8), "T_per_gpu": T, "H": H, "I": I, "E": E, "k": k,
-                       "block_m": plan.block_m, "cta_pairs": plan.cta_pairs, "active_experts": active, "padded_slots": num_padded,
+                       "block_m": plan.block_m, "cta_pairs": plan.cta_pairs, "task_order": plan.task_order,
+                       "half_tails": plan.half_tails, "active_experts": active, "padded_slots": num_padded,
                        "l2": "flushed between steps (256 MB write, outside per-step events)",
                        "parallelism": "replicas" if world > 1 else "single"},
             "roofline": roof,
@@ -439,6 +444,67 @@ def run_gpu(args, rank, world, local_rank):
     if dist is not None:
         dist.barrier(device_ids=[local_rank])
         dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ backward (--backward)
+BACKWARD_METRIC = "MoE-layer bwd tokens/s on 1 B200 (device-timed); % of TC roofline"
+
+
+def run_backward(args):
+    """Device-timed moe_backward steps (routing, dgrad, gate, weight gradients) on one GPU.
+
+    FLOP per step: 16*T*k*H*I (dgrad: g, u and dy W2^T 6, dx 4; weight gradients 6) plus the
+    gate's 2*T*H*E for dWg; roofline against the dense bf16 peak chosen from the sampled clocks.
+    """
+    import torch
+
+    from moe_megakernel_b200 import MoEPlan
+    from synth.moe_inputs import WORKLOADS, make_dy, make_inputs
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    shape = WORKLOADS[args.workload]
+    inp = make_inputs(shape, device=dev, seed=args.seed)
+    dy = make_dy(shape, device=dev, seed=args.seed)
+    T, H, I, E, k = shape.T, shape.H, shape.I, shape.E, shape.k
+    plan = MoEPlan(T, H, I, E, k, device=dev, backward=True)
+    out = plan.backward(inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], dy)
+    for _ in range(args.warmup):
+        plan.backward(inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], dy, out=out)
+    plan.check()
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(0)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    clocks.begin()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        plan.backward(inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], dy, out=out)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.end()
+    clk = clocks.stop()
+    plan.check()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    flop = 16.0 * T * k * H * I + 2.0 * T * H * E
+    peaks = measured_peaks()
+    peak, peak_name = choose_tc_peak(peaks, clk)
+    achieved = flop / (ms * 1e-3) / 1e12
+    print(json.dumps({
+        "metric": BACKWARD_METRIC, "value": T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded x, weights and dy ~ N(0,1) dy; random-init weights)",
+        "config": {"workload": workload_label(shape) + " backward", "T": T, "H": H, "I": I, "E": E, "k": k,
+                   "block_m": plan.block_m, "l2": "flushed between steps (256 MB write, outside per-step events)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peaks['source']} ({peak_name})", "flop_per_step": flop,
+                     "frac_vs_burst": achieved / peaks["bf16_tflops"],
+                     "frac_vs_sustained": achieved / peaks["bf16_tflops_sustained"]},
+        "gpu_launches": args.steps * 10,
+        "clocks": clk,
+    }), flush=True)
 
 
 # ------------------------------------------------------------------ reference arm (the oracle)
@@ -488,6 +554,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cta-pairs", type=int, default=None, choices=[0, 1],
                     help="expert GEMM on CTA pairs (1) or one CTA per block (0); default: the plan's")
+    ap.add_argument("--task-order", type=int, default=None, choices=[-1, 0, 1],
+                    help="expert-GEMM task order: -1 automatic, 0 staggered, 1 interleaved; default: the plan's")
+    ap.add_argument("--half-tails", type=int, default=None, choices=[0, 1],
+                    help="an expert's lone last block as M = 128 pair MMAs (1) or a full pair (0); default: the plan's")
+    ap.add_argument("--backward", action="store_true",
+                    help="time moe_backward (routing, dgrad, gate, weight gradients) instead of the forward")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -507,6 +579,10 @@ def main():
         world = max(world, 1)
     if args.impl == "reference":
         run_reference(args, rank, world)
+    elif args.backward:
+        if world > 1:
+            ap.error("--backward runs on one GPU")
+        run_backward(args)
     else:
         run_gpu(args, rank, world, local_rank)
 

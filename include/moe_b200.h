@@ -105,6 +105,10 @@ typedef struct {
   int32_t cta_pairs;       /* 1: the expert GEMM runs on CTA pairs (see moe_plan_set_cta_pairs) */
   int32_t n_shared;        /* shared experts (moe_plan_create_shared) */
   size_t workspace_bytes;
+  int32_t task_order;      /* expert-GEMM task order in use: 0 staggered, 1 interleaved
+                              (see moe_plan_set_task_order) */
+  int32_t half_tails;      /* 1: bf16 forwards on CTA pairs run an expert's lone last block
+                              as M = 128 pair MMAs (see moe_plan_set_half_tails) */
 } moe_plan_desc;
 
 /* Create a plan for up to T_max tokens of a layer with hidden size H, expert
@@ -342,6 +346,77 @@ int moe_route_static(const void* x, const void* Wg, const float* gate_bias, int 
  * does not depend on it. Errors: MOE_ERR_INVALID_ARG (null plan),
  * MOE_ERR_UNSUPPORTED_SHAPE (pairs requested where no 2-CTA cluster fits). */
 int moe_plan_set_cta_pairs(moe_plan_t plan, int enable);
+
+/* Order in which the persistent expert GEMM hands out its tasks (the same
+ * tasks and results either way; "MegaMoE 在 MoE 系统谱系中的位置", section 2.7:
+ * one queue holds the tasks of both GEMMs and an L2 task runs once the L1
+ * tasks of its rows are done). Blocks (or block pairs) are cut into groups;
+ *   0  staggered: L1 of group 0, L1 of group 1, L2 of group 0, L1 of group 2,
+ *      L2 of group 1, ...;
+ *   1  interleaved: after the L1 tasks of group 0, each segment hands out a
+ *      lag of L1 tasks of group m and then mixes the rest of them evenly with
+ *      the L2 tasks of group m-1, so that a CTA alternates the two kinds and
+ *      a second-GEMM combine epilogue overlaps a first-GEMM MMA;
+ *  -1  automatic (the default): staggered, which measured 1-2 % faster than
+ *      interleaved on the fine-grained and skewed layers and as fast on the
+ *      others.
+ * FP8 forwards (one launch per GEMM) ignore it. Errors: MOE_ERR_INVALID_ARG
+ * (null plan or another mode). */
+int moe_plan_set_task_order(moe_plan_t plan, int mode);
+
+/* Tile size of an expert's last block on CTA pairs, chosen from the expert's
+ * load ("MegaFlux: Skew-Resilient MoE Megakernels via Pipelined Expert
+ * Replication", abstract: the planner cuts each expert's tokens into
+ * tile-aligned blocks; here on one GPU, without replication). A pair task
+ * covers two 128-row blocks of one expert with M = 256 MMAs. When an expert
+ * has an odd number of blocks (every cold expert with at most 128 tokens has
+ * one), its last block alone would leave the second CTA of the pair without
+ * rows while the M = 256 MMA still costs two blocks. With enable = 1 (the
+ * default) that block runs as M = 128 pair MMAs, 64 of its rows in each CTA,
+ * at half the tensor time; with 0 it runs as before. Applies to bf16
+ * forwards with BLOCK_M = 128 on CTA pairs; results are the same either way
+ * (up to the order of the fp32 combine additions). Errors: MOE_ERR_INVALID_ARG
+ * (null plan). */
+int moe_plan_set_half_tails(moe_plan_t plan, int enable);
+
+/* Give the plan the workspace regions of moe_backward (enable = 1) or drop them
+ * (0). The workspace size changes: query moe_plan_workspace_bytes and bind a
+ * workspace again. Plans with shared experts have no backward.
+ * Errors: MOE_ERR_INVALID_ARG (null plan), MOE_ERR_UNSUPPORTED_SHAPE (shared experts). */
+int moe_plan_set_backward(moe_plan_t plan, int enable);
+
+/* Backward of the layer for the upstream gradient dy: the chain-rule gradients
+ * of y = sum_j w[t,j] FFN_{e_j}(x[t]) with respect to x, Wg, the gate bias and
+ * the expert weights ("MegaFlux: Skew-Resilient MoE Megakernels via Pipelined
+ * Expert Replication", abstract: a backward MoE megakernel that reduces the
+ * experts' weight gradients; the pages do not define it further). Readings:
+ * the choice of the k experts is piecewise constant (no gradient through it);
+ * the softmax over the k kept logits is differentiated; the bf16 rounding of
+ * the SwiGLU activation passes the gradient unchanged, while dW2 and the
+ * gradient of the combine weights use the rounded activation the forward
+ * multiplied. The routing is recomputed from x on the device (router and
+ * dispatch, as in moe_forward), then: dgrad (x and dy rows gathered through
+ * the slot records; g, u and dy W2^T on tcgen05; dg, du in the epilogue; dx
+ * added through the slot records), the gate backward, and the weight
+ * gradients as reductions over each expert's slots on tcgen05.
+ *   x, Wg, gate_bias, W1, W3, W2: as for moe_forward (device)
+ *   dy   bf16 [T, H]  device, the upstream gradient of y
+ *   dx   bf16 [T, H]  device, out
+ *   dWg  fp32 [H, E]  device, out
+ *   dbias fp32 [E]    device, out, or NULL (not computed)
+ *   dW1, dW3 bf16 [E, H, I], dW2 bf16 [E, I, H]  device, out (experts no token
+ *        chose get zeros)
+ * Outputs are overwritten, not accumulated into. The plan needs
+ * moe_plan_set_backward(plan, 1) and a bound workspace; every pointer but
+ * dbias non-NULL and 16-byte aligned (dWg and dbias 4-byte). Enqueued on
+ * `stream` only. Intermediates: dg, du and w * activation per slot
+ * ([pool, I] bf16 each) and the dense gate-logit gradient live in the
+ * workspace. Errors: MOE_ERR_INVALID_ARG (no backward regions, shared
+ * experts, bad pointers, T out of range), MOE_ERR_NO_WORKSPACE,
+ * MOE_ERR_CUDA; device-side errors through moe_check. */
+int moe_backward(moe_plan_t plan, const void* x, const void* Wg, const float* gate_bias, const void* W1,
+                 const void* W3, const void* W2, const void* dy, int T, void* dx, float* dWg, float* dbias,
+                 void* dW1, void* dW3, void* dW2, void* stream);
 
 /* Number of kernels one moe_forward launches (for launch accounting). */
 int moe_forward_kernel_count(void);

@@ -39,7 +39,8 @@ class MoEPlanDesc(ctypes.Structure):
                 ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("block_m", ctypes.c_int32),
                 ("pool_capacity", ctypes.c_int32), ("num_sms", ctypes.c_int32),
                 ("pair_clusters", ctypes.c_int32), ("cta_pairs", ctypes.c_int32),
-                ("n_shared", ctypes.c_int32), ("workspace_bytes", ctypes.c_size_t)]
+                ("n_shared", ctypes.c_int32), ("workspace_bytes", ctypes.c_size_t),
+                ("task_order", ctypes.c_int32), ("half_tails", ctypes.c_int32)]
 
 
 # exported symbol -> (restype, argtypes); the same list as include/moe_b200.h
@@ -71,6 +72,10 @@ SIGNATURES = {
     "moe_route_static": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp,
                                   _vp, _vp, _c_int, _vp, _vp, _vp]),
     "moe_plan_set_cta_pairs": (_c_int, [_vp, _c_int]),
+    "moe_plan_set_backward": (_c_int, [_vp, _c_int]),
+    "moe_backward": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_plan_set_task_order": (_c_int, [_vp, _c_int]),
+    "moe_plan_set_half_tails": (_c_int, [_vp, _c_int]),
     "moe_plan_set_fp8": (_c_int, [_vp, _c_int]),
     "moe_forward_kernel_count": (_c_int, []),
     "moe_plan_destroy": (None, [_vp]),
@@ -143,7 +148,7 @@ class MoEPlan:
     """
 
     def __init__(self, T_max: int, H: int, I: int, E: int, k: int, block_m: int = 0, device=None,
-                 n_shared: int = 0, fp8: bool = False):
+                 n_shared: int = 0, fp8: bool = False, backward: bool = False):
         self.lib = load_library()
         self.device = torch.device("cuda", torch.cuda.current_device() if device is None
                                    else torch.device(device).index or 0)
@@ -154,6 +159,9 @@ class MoEPlan:
         self.fp8 = bool(fp8)
         if fp8:   # workspace regions of forward_fp8
             _ok(self.lib.moe_plan_set_fp8(self._plan, 1), "moe_plan_set_fp8")
+        self.has_backward = bool(backward)
+        if backward:   # workspace regions of backward
+            _ok(self.lib.moe_plan_set_backward(self._plan, 1), "moe_plan_set_backward")
         d = MoEPlanDesc()
         _ok(self.lib.moe_plan_describe(self._plan, ctypes.byref(d)), "moe_plan_describe")
         self.block_m, self.pool_capacity, self.num_sms = d.block_m, d.pool_capacity, d.num_sms
@@ -270,6 +278,33 @@ class MoEPlan:
     def host_pipeline_join(self, stream=None):
         _ok(self.lib.moe_host_pipeline_join(self._plan, _stream_handle(stream, self.device)), "moe_host_pipeline_join")
 
+    def backward(self, x, Wg, bias, W1, W3, W2, dy, stream=None, out=None) -> dict:
+        """Gradients of the layer for the upstream dy [T,H] bf16 (plan made with backward=True):
+        dict of dx [T,H] bf16, dWg [H,E] fp32, dbias [E] fp32 (None when bias is None),
+        dW1/dW3 [E,H,I] bf16, dW2 [E,I,H] bf16. ``out`` may supply these tensors."""
+        T = self._check_inputs(x, Wg, bias, (W1, W3, W2))
+        _check(dy, "dy", (T, self.H), torch.bfloat16, self.device)
+        o = dict(out) if out is not None else {}
+        dev = self.device
+        E, H, I = self.E, self.H, self.I
+        o.setdefault("dx", torch.empty((T, H), dtype=torch.bfloat16, device=dev))
+        o.setdefault("dWg", torch.empty((H, E), dtype=torch.float32, device=dev))
+        o.setdefault("dbias", None if bias is None else torch.empty((E,), dtype=torch.float32, device=dev))
+        o.setdefault("dW1", torch.empty((E, H, I), dtype=torch.bfloat16, device=dev))
+        o.setdefault("dW3", torch.empty((E, H, I), dtype=torch.bfloat16, device=dev))
+        o.setdefault("dW2", torch.empty((E, I, H), dtype=torch.bfloat16, device=dev))
+        _check(o["dx"], "dx", (T, H), torch.bfloat16, dev)
+        _check(o["dWg"], "dWg", (H, E), torch.float32, dev)
+        if o["dbias"] is not None:
+            _check(o["dbias"], "dbias", (E,), torch.float32, dev)
+        _check(o["dW1"], "dW1", (E, H, I), torch.bfloat16, dev)
+        _check(o["dW3"], "dW3", (E, H, I), torch.bfloat16, dev)
+        _check(o["dW2"], "dW2", (E, I, H), torch.bfloat16, dev)
+        _ok(self.lib.moe_backward(self._plan, _ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(dy),
+                                  T, _ptr(o["dx"]), _ptr(o["dWg"]), _ptr(o["dbias"]), _ptr(o["dW1"]), _ptr(o["dW3"]),
+                                  _ptr(o["dW2"]), _stream_handle(stream, dev)), "moe_backward")
+        return o
+
     def route(self, x, Wg, bias, stream=None):
         T = self._check_inputs(x, Wg, bias)
         _ok(self.lib.moe_route(self._plan, _ptr(x), _ptr(Wg), _ptr(bias), T,
@@ -318,6 +353,27 @@ class MoEPlan:
 
     def set_cta_pairs(self, enable: bool):
         _ok(self.lib.moe_plan_set_cta_pairs(self._plan, 1 if enable else 0), "moe_plan_set_cta_pairs")
+
+    def set_task_order(self, mode: int):
+        """-1 automatic, 0 staggered, 1 interleaved (see moe_plan_set_task_order)."""
+        _ok(self.lib.moe_plan_set_task_order(self._plan, int(mode)), "moe_plan_set_task_order")
+
+    def set_half_tails(self, enable: bool):
+        """Run an expert's lone last block as M = 128 pair MMAs (see moe_plan_set_half_tails)."""
+        _ok(self.lib.moe_plan_set_half_tails(self._plan, 1 if enable else 0), "moe_plan_set_half_tails")
+
+    @property
+    def half_tails(self) -> bool:
+        d = MoEPlanDesc()
+        _ok(self.lib.moe_plan_describe(self._plan, ctypes.byref(d)), "moe_plan_describe")
+        return bool(d.half_tails)
+
+    @property
+    def task_order(self) -> int:
+        """The expert-GEMM task order in use: 0 staggered, 1 interleaved."""
+        d = MoEPlanDesc()
+        _ok(self.lib.moe_plan_describe(self._plan, ctypes.byref(d)), "moe_plan_describe")
+        return int(d.task_order)
 
     @property
     def cta_pairs(self) -> bool:

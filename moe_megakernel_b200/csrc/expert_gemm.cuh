@@ -82,6 +82,8 @@ struct GemmParams {
   int phase_only;            // -1: both phases in one launch; 0: first GEMM only; 1: second GEMM only
   int ring_blocks;              // block b uses ring slot b % ring_blocks
   int max_groups;
+  int order_lag;                // task order (see locate_task): -1 staggered, >= 0 interleaved after this lag
+  const uint8_t* zero_row;      // 2*H zero bytes: the A row of a padding slot
   unsigned long long timeout_ns;
   int withhold_block;           // test hook: never publish L1 completion of this block (-1: off)
 };
@@ -169,12 +171,64 @@ __device__ __forceinline__ bool wait_counter(const int* ctr, int need, const Gem
   return true;
 }
 
-__device__ __forceinline__ int segment_start(const GemmSmem& s, const GemmParams& p, int seg) {
-  const int G = s.num_groups;
-  if (seg == 0) return 0;
-  const int g = (seg + 1) >> 1;
-  if (seg & 1) return s.group_start[g] * p.N1 + s.group_start[g - 1] * p.N2;           // L1(g)
-  return s.group_start[min(g + 1, G)] * p.N1 + s.group_start[g - 1] * p.N2;            // L2(g-1)
+// Where task t falls in the task order: its phase (0 = L1, 1 = L2), its group
+// g and its index tl among that phase's tasks of group g. Group g holds the
+// units (blocks, or block pairs) gs[g] .. gs[g+1]-1 and has (gs[g+1]-gs[g])*N1
+// L1 tasks and (..)*N2 L2 tasks. The L2 tasks of a group always come after
+// every L1 task of that group and before the L1 tasks of the group two later
+// (whose h rows reuse its ring slots). Two orders:
+//
+// * staggered (lag < 0): L1(0), L1(1), L2(0), L1(2), L2(1), ..., L2(G-1);
+// * interleaved (lag >= 0): L1(0), then for m = 1..G-1 one segment that
+//   starts with `lag` L1 tasks of group m (so that the last L1 tasks of group
+//   m-1 have finished) and then mixes the rest of L1(m) with L2(m-1) evenly
+//   (Bresenham: L2 task c is the v-th of the mixed part when
+//   floor(v*n2/R) = c < floor((v+1)*n2/R)), then L2(G-1). A CTA then
+//   alternates long-K first-GEMM tasks with second-GEMM tasks whose
+//   combine epilogue would otherwise outlast their short MMAs.
+struct TaskPos {
+  int phase, g, tl;
+};
+
+__device__ __forceinline__ TaskPos locate_task(int t, const int* gs, int G, int N1, int N2, int lag) {
+  if (lag < 0) {
+    // segment 0 = L1(0); odd 2g-1 = L1(g); even 2g = L2(g-1)
+    auto start = [&](int seg) {
+      if (seg == 0) return 0;
+      const int g = (seg + 1) >> 1;
+      if (seg & 1) return gs[g] * N1 + gs[g - 1] * N2;
+      return gs[min(g + 1, G)] * N1 + gs[g - 1] * N2;
+    };
+    int lo = 0, hi = 2 * G;   // last segment whose start is <= t (empty segments share the next start)
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (start(mid) <= t) lo = mid;
+      else hi = mid - 1;
+    }
+    const int seg = lo;
+    if (seg == 0 || (seg & 1)) return TaskPos{0, (seg + 1) >> 1, t - start(seg)};
+    return TaskPos{1, (seg >> 1) - 1, t - start(seg)};
+  }
+  // segment m >= 1 starts after every L1 task of groups < m and every L2 task of groups < m-1
+  auto start = [&](int m) { return m == 0 ? 0 : gs[m] * N1 + gs[m - 1] * N2; };
+  int lo = 0, hi = G;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (start(mid) <= t) lo = mid;
+    else hi = mid - 1;
+  }
+  const int m = lo;
+  const int u = t - start(m);
+  if (m == 0) return TaskPos{0, 0, u};
+  const int n1 = m < G ? (gs[m + 1] - gs[m]) * N1 : 0;
+  const int n2 = (gs[m] - gs[m - 1]) * N2;
+  const int l = min(lag, n1);
+  if (u < l) return TaskPos{0, m, u};
+  const long long v = u - l, R = (long long)(n1 - l) + n2;
+  const int c2 = (int)(v * n2 / R);
+  const int c2_next = (int)((v + 1) * n2 / R);
+  if (c2_next > c2) return TaskPos{1, m - 1, c2};
+  return TaskPos{0, m, l + (int)v - c2};
 }
 
 __device__ __forceinline__ Task decode_task(int t, const GemmSmem& s, const GemmParams& p) {
@@ -185,26 +239,11 @@ __device__ __forceinline__ Task decode_task(int t, const GemmSmem& s, const Gemm
   if (p.phase_only == 1) t += nb_total * p.N1;
   else if (p.phase_only == 0 && t >= nb_total * p.N1) return task;
   if (t < 0 || t >= nb_total * (p.N1 + p.N2) || G <= 0) return task;
-  // last segment whose start is <= t (empty segments share the next start)
-  int lo = 0, hi = 2 * G;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (segment_start(s, p, mid) <= t) lo = mid;
-    else hi = mid - 1;
-  }
-  const int seg = lo;
-  int g, NT;
-  if (seg == 0 || (seg & 1)) {
-    task.phase = 0;
-    g = (seg + 1) >> 1;
-    NT = p.N1;
-  } else {
-    task.phase = 1;
-    g = (seg >> 1) - 1;
-    NT = p.N2;
-  }
+  const TaskPos pos = locate_task(t, s.group_start, G, p.N1, p.N2, p.phase_only >= 0 ? -1 : p.order_lag);
+  task.phase = pos.phase;
+  const int g = pos.g, NT = pos.phase == 0 ? p.N1 : p.N2;
   const int gb0 = s.group_start[g], gb1 = s.group_start[g + 1];
-  const int tl = t - segment_start(s, p, seg);
+  const int tl = pos.tl;
   // expert of the tl-th task: its blocks inside the group occupy consecutive NT-task runs
   const int vb = gb0 + tl / NT;
   int elo = 0, ehi = p.E + p.S - 1;
@@ -295,7 +334,7 @@ __device__ void gemm_scheduler(const GemmParams& p, GemmSmem& s) {
             set_error(p, s, kDevBounds, task.b);
             tok[i] = 0;
           }
-          s.rows[q][r] = tok[i] < 0 ? 0 : tok[i];   // padding slot: any valid row, the epilogue drops it
+          s.rows[q][r] = tok[i] < 0 ? -1 : tok[i];   // padding slot: the gather fills the row with zeros
         }
       }
     } else if (task.phase == 1) {
@@ -546,7 +585,12 @@ __device__ void gemm_gather(const GemmParams& p, GemmSmem& s, uint8_t* tiles, in
       soff[j] = r * 128 + ((c ^ (r & 7)) << 4);
       src[j] = xrows + c * 16;
       if (r < p.BM) {
-        src[j] = task.phase == 0 ? xrows + (size_t)rows[r] * xpitch + c * 16 : hblock + (size_t)r * hpitch + c * 16;
+        // L1 padding slots (row index -1) read the all-zero row: the tensor core
+        // multiplies zeros and their h rows come out 0 for the L2 tasks
+        const int xr = rows[r];
+        src[j] = task.phase == 1 ? hblock + (size_t)r * hpitch + c * 16
+                 : xr < 0        ? p.zero_row + c * 16
+                                 : xrows + (size_t)xr * xpitch + c * 16;
         nrows = j + 1;
       }
     }

@@ -28,6 +28,20 @@
 //
 // Like expert_gemm.cuh, a template over bf16 or FP8 E4M3 operands; in the FP8
 // second GEMM the A-row warps copy the CTA's half of the K-major W2 codes.
+//
+// Half tasks (bf16, BLOCK_M = 128): when an expert has an odd number of
+// blocks, its last block would leave the second CTA of its pair without
+// rows, and an M = 256 MMA would still spend the time of two blocks on it.
+// Instead that block runs as M = 128 pair MMAs (64 rows in each CTA: rows
+// 0-63 of the block in CTA 0, rows 64-127 in CTA 1), which take half the
+// tensor time. Their accumulator layout differs from M = 256: each CTA's D
+// (64 rows x N) puts columns 0 .. N/2-1 (the CTA-0 half of the B tile) in
+// TMEM lanes 0-63 and columns N/2 .. N-1 (the CTA-1 half) in lanes 64-127,
+// both at TMEM columns 0 .. N/2-1. So in a half L1 task each CTA loads one
+// 64-column box of W1 and the matching box of W3 (CTA 0 the first 64 of the
+// task's 128 columns of I, CTA 1 the next 64), and epilogue warp q finds g
+// and u of row 32*(q%2) + lane, columns 64*(q/2) + c, at TMEM columns c and
+// 64 + c; in a half L2 task warp q combines columns 128*(q/2) .. +127.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -80,6 +94,9 @@ struct Gemm2Params {
   const uint8_t* h8;       // FP8: [h rows, I] activation codes
   int phase_only;          // -1: both phases; 0: first GEMM only; 1: second GEMM only
   int ring_pairs, max_groups;
+  int order_lag;                // task order (locate_task in expert_gemm.cuh): -1 staggered, >= 0 interleaved
+  int half_tails;               // 1: an expert's lone last block runs as an M = 128 pair MMA (bf16, BM = 128)
+  const uint8_t* zero_row;      // 2*H zero bytes: the A row of a padding slot
   unsigned long long timeout_ns;
   int withhold_pair;            // test hook: never publish L1 completion of this pair (-1: off)
 };
@@ -88,7 +105,8 @@ struct Task2 {
   int phase;    // 0 = L1, 1 = L2, -1 = no more work
   int e, p, n;  // expert, pair, n-tile
   int b0, b1;   // blocks of CTA 0 and CTA 1 (b1 = -1: the expert has an odd block count)
-  int pad0, pad1;
+  int half;     // 1: the lone block b0 split over the pair, rows 0-63 in CTA 0 and 64-127 in CTA 1
+  int pad1;
 };
 
 struct Gemm2Smem {
@@ -183,15 +201,7 @@ __device__ __forceinline__ int claim_task_any(int32_t* counter, const int32_t* e
   return t;   // valid in lane 0 only
 }
 
-// Task order as in expert_gemm.cuh, in units of block pairs.
-__device__ __forceinline__ int segment_start2(const Gemm2Smem& s, const Gemm2Params& p, int seg) {
-  const int G = s.num_groups;
-  if (seg == 0) return 0;
-  const int g = (seg + 1) >> 1;
-  if (seg & 1) return s.group_start[g] * p.N1 + s.group_start[g - 1] * p.N2;
-  return s.group_start[min(g + 1, G)] * p.N1 + s.group_start[g - 1] * p.N2;
-}
-
+// Task order as in expert_gemm.cuh (locate_task), in units of block pairs.
 __device__ __forceinline__ Task2 decode_task2(int t, const Gemm2Smem& s, const Gemm2Params& p) {
   Task2 task{-1, 0, 0, 0, -1, -1, 0, 0};
   const int G = s.num_groups;
@@ -200,25 +210,11 @@ __device__ __forceinline__ Task2 decode_task2(int t, const Gemm2Smem& s, const G
   if (p.phase_only == 1) t += np_total * p.N1;
   else if (p.phase_only == 0 && t >= np_total * p.N1) return task;
   if (t < 0 || t >= np_total * (p.N1 + p.N2) || G <= 0) return task;
-  int lo = 0, hi = 2 * G;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (segment_start2(s, p, mid) <= t) lo = mid;
-    else hi = mid - 1;
-  }
-  const int seg = lo;
-  int g, NT;
-  if (seg == 0 || (seg & 1)) {
-    task.phase = 0;
-    g = (seg + 1) >> 1;
-    NT = p.N1;
-  } else {
-    task.phase = 1;
-    g = (seg >> 1) - 1;
-    NT = p.N2;
-  }
+  const TaskPos pos = locate_task(t, s.group_start, G, p.N1, p.N2, p.phase_only >= 0 ? -1 : p.order_lag);
+  task.phase = pos.phase;
+  const int g = pos.g, NT = pos.phase == 0 ? p.N1 : p.N2;
   const int gp0 = s.group_start[g], gp1 = s.group_start[g + 1];
-  const int tl = t - segment_start2(s, p, seg);
+  const int tl = pos.tl;
   const int vp = gp0 + tl / NT;
   int elo = 0, ehi = p.E + p.S - 1;
   while (elo < ehi) {
@@ -236,6 +232,7 @@ __device__ __forceinline__ Task2 decode_task2(int t, const Gemm2Smem& s, const G
   task.p = ep0 + (local - task.n * np);
   task.b0 = s.block_start[e] + 2 * (task.p - s.pair_start[e]);
   task.b1 = task.b0 + 1 < s.block_start[e + 1] ? task.b0 + 1 : -1;
+  task.half = (task.b1 < 0 && p.half_tails) ? 1 : 0;
   return task;
 }
 
@@ -264,8 +261,13 @@ __device__ __forceinline__ bool prepare_task2(Task2& task, int q, uint32_t qpari
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
       const int r = lane + 32 * i;
-      tok0[i] = r < p.BM ? p.slot_token[task.b0 * p.BM + r] : 0;
-      tok1[i] = r < p.BM && task.b1 >= 0 ? p.slot_token[task.b1 * p.BM + r] : 0;
+      if (task.half) {   // rows 0-63 of block b0 in CTA 0, rows 64-127 in CTA 1
+        tok0[i] = r < 64 ? p.slot_token[task.b0 * p.BM + r] : -1;
+        tok1[i] = r < 64 ? p.slot_token[task.b0 * p.BM + 64 + r] : -1;
+      } else {
+        tok0[i] = r < p.BM ? p.slot_token[task.b0 * p.BM + r] : 0;
+        tok1[i] = r < p.BM && task.b1 >= 0 ? p.slot_token[task.b1 * p.BM + r] : 0;
+      }
     }
     const uint32_t peer_rows = ptx::mapa(ptx::smem_u32(&s.rows[q][0]), 1);
 #pragma unroll
@@ -277,8 +279,10 @@ __device__ __forceinline__ bool prepare_task2(Task2& task, int q, uint32_t qpari
           tok0[i] = tok0[i] >= p.T ? 0 : tok0[i];
           tok1[i] = tok1[i] >= p.T ? 0 : tok1[i];
         }
-        s.rows[q][r] = tok0[i] < 0 ? 0 : tok0[i];   // padding slot: any valid row, the epilogue drops it
-        ptx::st_cluster_u32(peer_rows + 4 * r, tok1[i] < 0 ? 0 : tok1[i]);
+        // padding slot (or no block): -1, the gather fills the row with zeros
+        s.rows[q][r] = tok0[i] < 0 ? -1 : tok0[i];
+        ptx::st_cluster_u32(peer_rows + 4 * r,
+                            (tok1[i] < 0 || (task.b1 < 0 && !task.half)) ? 0xffffffffu : (uint32_t)tok1[i]);
       }
     }
   } else if (task.phase == 1) {
@@ -395,8 +399,13 @@ __device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_
             const bool sh = task.e >= p.E;   // shared expert: its own weight tensors
             const int wrow = (sh ? task.e - p.E : task.e) * p.H + kb * kBK;
             const CUtensorMap* m1 = sh ? &p.tm_ws1 : &p.tm_w1;
-            ptx::tma_load_2d(b_addr, m1, &s.full[stage], n0, wrow, pol);
-            ptx::tma_load_2d(b_addr + kBoxBytes, m1, &s.full[stage], n0 + 64, wrow, pol);
+            if (task.half) {   // columns n0 .. n0+63 of W1 and of W3 (the follower takes the next 64)
+              ptx::tma_load_2d(b_addr, m1, &s.full[stage], n0, wrow, pol);
+              ptx::tma_load_2d(b_addr + kBoxBytes, sh ? &p.tm_ws3 : &p.tm_w3, &s.full[stage], n0, wrow, pol);
+            } else {
+              ptx::tma_load_2d(b_addr, m1, &s.full[stage], n0, wrow, pol);
+              ptx::tma_load_2d(b_addr + kBoxBytes, m1, &s.full[stage], n0 + 64, wrow, pol);
+            }
           }
         } else {
           // L2: both operands come from the A-row warps' cp.async (a TMA box of
@@ -485,8 +494,13 @@ __device__ void gemm2_follower_producer(const Gemm2Params& p, Gemm2Smem& s, uint
             const bool sh = task.e >= p.E;
             const int wrow = (sh ? task.e - p.E : task.e) * p.H + kb * kBK;
             const CUtensorMap* m3 = sh ? &p.tm_ws3 : &p.tm_w3;
-            ptx::tma_load_2d(b_addr, m3, &s.full[stage], n0, wrow, pol);
-            ptx::tma_load_2d(b_addr + kBoxBytes, m3, &s.full[stage], n0 + 64, wrow, pol);
+            if (task.half) {   // columns n0+64 .. n0+127 of W1 and of W3
+              ptx::tma_load_2d(b_addr, sh ? &p.tm_ws1 : &p.tm_w1, &s.full[stage], n0 + 64, wrow, pol);
+              ptx::tma_load_2d(b_addr + kBoxBytes, m3, &s.full[stage], n0 + 64, wrow, pol);
+            } else {
+              ptx::tma_load_2d(b_addr, m3, &s.full[stage], n0, wrow, pol);
+              ptx::tma_load_2d(b_addr + kBoxBytes, m3, &s.full[stage], n0 + 64, wrow, pol);
+            }
           }
         } else {
           ptx::mbar_arrive(&s.full[stage]);   // L2: operands by the A-row warps (see the leader)
@@ -546,6 +560,9 @@ __device__ void gemm2_mma(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, ui
       F8 ? ptx::idesc_e4m3_f32(256, 2 * kL1TileN) : ptx::idesc_bf16_f32(256, 2 * kL1TileN, false, true);
   constexpr bool f8 = F8;
   const uint32_t idesc_l2 = F8 ? ptx::idesc_e4m3_f32(256, p.BN2) : ptx::idesc_bf16_f32(256, p.BN2, false, true);
+  // half tasks (bf16 only): 64 rows per CTA
+  const uint32_t idesc_l1_half = ptx::idesc_bf16_f32(128, 2 * kL1TileN, false, true);
+  const uint32_t idesc_l2_half = ptx::idesc_bf16_f32(128, p.BN2, false, true);
   int stage = 0;
   uint32_t phase = 0;
   int q = 0;
@@ -560,7 +577,8 @@ __device__ void gemm2_mma(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, ui
     if (!warp_wait2(&s.acc_empty[acc], acc_phase ^ 1, p, s, 8)) break;
     ptx::tc_fence_after();
     const uint32_t d_tmem = tmem_base + acc * 256;
-    const uint32_t idesc = task.phase == 0 ? idesc_l1 : idesc_l2;
+    const uint32_t idesc = task.half ? (task.phase == 0 ? idesc_l1_half : idesc_l2_half)
+                                     : (task.phase == 0 ? idesc_l1 : idesc_l2);
     const int nk = task.phase == 0 ? l1_ksteps2<F8>(p) : l2_ksteps2<F8>(p);
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
@@ -652,6 +670,74 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
     if (!warp_wait2(&s.acc_full[acc], acc_phase, p, s, 11)) break;
     ptx::tc_fence_after();
     const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * 256;
+    if (!F8 && task.half) {
+      // M = 128 pair accumulator: this warp's lanes hold row hr of this CTA's 64
+      // rows (block row 64*rank + hr) and the column half hc of the tile
+      const int hr = (quarter & 1) * 32 + lane, hc = quarter >> 1;
+      const int brow = (int)rank * 64 + hr;
+      if (task.phase == 0) {
+        bool store = true;
+        if (task.p >= p.ring_pairs) {
+          bool ok = true;
+          if (lane == 0) ok = wait_counter2(p.l2_done + (task.p - p.ring_pairs), p.N2, p, s, 0x40000 | task.p);
+          store = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        }
+        // g at TMEM columns 0..63, u at 64..127: columns 64*hc .. +63 of the task's 128 of I
+        bf16* hrow = p.h + ((size_t)(task.p % p.ring_pairs) * 2 * p.BM + brow) * p.I + task.n * kL1TileN + hc * 64;
+        float amax = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t g[32], u[32];
+          ptx::tmem_ld32(tbase + c * 32, g);
+          ptx::tmem_ld32(tbase + 64 + c * 32, u);
+          ptx::tmem_ld_wait();
+          if (store) store_swiglu32(hrow + c * 32, g, u, amax);
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (is_leader) ptx::mbar_arrive(&s.acc_empty[acc]);
+          else ptx::mbar_arrive_peer(lead_acc_empty0 + 8 * acc);
+        }
+        __threadfence();
+        __syncwarp();
+        if (lane == 0 && task.p != p.withhold_pair) ptx::red_release_gpu_add(p.l1_done + task.p, 1);
+      } else {
+        if (is_leader && quarter == 0 && lane == 0) ptx::red_release_gpu_add(p.l2_done + task.p, 1);
+        const int slot = task.b0 * p.BM + brow;
+        int tok = p.slot_token[slot];
+        float w = 0.f;
+        if (tok >= p.T) {
+          set_error2(p, s, kDevBounds, 0x20000 | task.p);
+          tok = -1;
+        }
+        if (tok >= 0) {
+          const int j = p.slot_topk[slot];
+          if (task.e >= p.E) {
+            w = 1.f;
+          } else if (j < 0 || j >= p.k) {
+            set_error2(p, s, kDevBounds, 0x30000 | task.p);
+            tok = -1;
+          } else {
+            w = p.topk_w[(size_t)tok * p.k + j];
+          }
+        }
+        combine_rows(tbase, p.BN2 / 2, w, tok, p.y_acc, p.H, task.n * p.BN2 + hc * (p.BN2 / 2), s.out_stage[quarter],
+                     s.out_tok[quarter], nullptr, [&]() {
+                       ptx::tc_fence_before();
+                       __syncwarp();
+                       if (lane == 0) {
+                         if (is_leader) ptx::mbar_arrive(&s.acc_empty[acc]);
+                         else ptx::mbar_arrive_peer(lead_acc_empty0 + 8 * acc);
+                       }
+                     });
+      }
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+      continue;
+    }
     const int b_own = rank == 0 ? task.b0 : task.b1;
     const bool valid = r < p.BM && b_own >= 0;
     const int slot = (b_own < 0 ? 0 : b_own) * p.BM + r;
@@ -744,8 +830,11 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
     int q_task = 0;
     if (!pop_task2(task, q, qphase, &q_task, is_leader, p, s, 12, false)) break;
     if (task.phase < 0) break;
-    const int b_own = rank == 0 ? task.b0 : task.b1;
-    const int ring_row0 = ((task.p % p.ring_pairs) * 2 + (int)rank) * p.BM;
+    // half task: both CTAs take block b0, 64 rows each (CTA 1 its rows 64-127)
+    const int b_own = task.half ? task.b0 : (rank == 0 ? task.b0 : task.b1);
+    const int rows_own = task.half ? 64 : p.BM;
+    const int ring_row0 = task.half ? (task.p % p.ring_pairs) * 2 * p.BM + (int)rank * 64
+                                    : ((task.p % p.ring_pairs) * 2 + (int)rank) * p.BM;
     int nrows = 0;
     uint32_t soff[kRowsPerLane];
     const uint8_t* src[kRowsPerLane];   // byte addresses; a stage takes the next 128 bytes of a row
@@ -762,8 +851,13 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
         const int rr = (j * kGatherWarps + g) * 4 + (lane >> 3);
         soff[j] = rr * 128 + ((c ^ (rr & 7)) << 4);
         src[j] = xrows + c * 16;
-        if (rr < p.BM) {
-          src[j] = task.phase == 0 ? xrows + (size_t)rows[rr] * xpitch + c * 16 : hblock + (size_t)rr * hpitch + c * 16;
+        if (rr < rows_own) {
+          // L1 padding slot (-1): the all-zero row, so the tensor core multiplies zeros and
+          // the slot's h row comes out 0
+          const int xr = rows[rr];
+          src[j] = task.phase == 1 ? hblock + (size_t)rr * hpitch + c * 16
+                   : xr < 0        ? p.zero_row + c * 16
+                                   : xrows + (size_t)xr * xpitch + c * 16;
           nrows = j + 1;
         }
       }

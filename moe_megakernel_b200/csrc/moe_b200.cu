@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "dispatch.cuh"
 #include "expert_gemm.cuh"
+#include "backward.cuh"
 #include "expert_gemm2.cuh"
 #include "quant.cuh"
 #include "router.cuh"
@@ -32,7 +33,8 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 struct Layout {
   size_t err, sched, topk_idx, topk_w, rank, chunk_count, expert_count, expert_offset, block_start, num_padded,
       slot_token, slot_topk, l1_done, l2_done, group_start, pair_start, router_partial, router_counter, h, y_acc,
-      x_stage, y_stage, x_q, s_x, h8, act_amax, act_scale, total;
+      x_stage, y_stage, x_q, s_x, h8, act_amax, act_scale, bwd_dg, bwd_du, bwd_aw, bwd_dw, bwd_dl, bwd_wgt,
+      zero_row, total;
 };
 
 class DeviceGuard {
@@ -117,10 +119,13 @@ struct moe_plan {
   int BN2, N1, N2, pool, chunks_max, blocks_max;
   int group_min, group_max, max_groups, ring_blocks;   // expert-GEMM task groups and h ring
   bool cta_pairs = false;                              // run the expert GEMM on CTA pairs
+  int task_order = -1;                                 // -1 automatic, 0 staggered, 1 interleaved
+  bool half_tails = true;                              // pair kernel: lone last blocks as M = 128 pair MMAs
   int pair_clusters = 0;                               // co-resident clusters of the pair kernel
   int pgroup_min, pgroup_max, pmax_groups, ring_pairs; // the same in units of block pairs
   int per_expert;                                      // expected blocks per expert + 1
   int fp8_rows = 0;                                    // FP8 plans: activation rows of all blocks or pairs
+  bool backward = false;                               // workspace holds the backward's regions
   // pipelined host entry: its own copy streams, two staging buffers used in turn, and the events
   // that order each buffer's copy-in, forward and copy-out
   cudaStream_t cp_in = nullptr, cp_out = nullptr;
@@ -149,6 +154,17 @@ static void size_pair_groups(moe_plan* p) {
   p->ring_pairs = std::min(3 * p->pgroup_max, pairs_max);
 }
 
+// order_lag of the expert GEMM's parameters: -1 for the staggered task order;
+// for the interleaved one, two waves of concurrent tasks (pairs run
+// pair_clusters tasks at once, the single-CTA kernel num_sms), which is the
+// head start the last L1 tasks of the previous group get before its L2 tasks
+// are handed out.
+static int order_lag(const moe_plan& p) {
+  const bool inter = p.task_order == 1;   // automatic: staggered (measured 1-2 % faster on every workload)
+  if (!inter) return -1;
+  return 2 * (p.cta_pairs ? std::max(1, p.pair_clusters) : p.num_sms);
+}
+
 static Layout make_layout(const moe_plan& p) {
   Layout L{};
   size_t o = 0;
@@ -160,6 +176,7 @@ static Layout make_layout(const moe_plan& p) {
   };
   const size_t tk = (size_t)p.T_max * p.k;
   L.err = take(16 * 4, 256);
+  L.zero_row = take((size_t)p.H * 2, 256);   // zeroed when bound, never written: padding slots' A rows
   L.sched = take(16 * 4, 256);
   L.topk_idx = take(tk * 4, 256);
   L.topk_w = take(tk * 4, 256);
@@ -188,6 +205,16 @@ static Layout make_layout(const moe_plan& p) {
   L.h8 = take((size_t)p.fp8_rows * p.I, 1024);
   L.act_amax = take((size_t)p.fp8_rows * 4, 256);
   L.act_scale = take((size_t)p.fp8_rows * 4, 256);
+  // backward plans: dg, du and w * activation per slot [pool, I] bf16, dw [T_max, k] fp32, the dense
+  // gate-logit gradient [T_max, E rounded up to 64] bf16, Wg transposed [E, H] bf16 (the fp32 dx
+  // accumulator is the forward's y accumulator)
+  const size_t bp = p.backward ? (size_t)p.pool : 0;
+  L.bwd_dg = take(bp * p.I * 2, 1024);
+  L.bwd_du = take(bp * p.I * 2, 1024);
+  L.bwd_aw = take(bp * p.I * 2, 1024);
+  L.bwd_dw = take(p.backward ? (size_t)p.T_max * p.k * 4 : 0, 256);
+  L.bwd_dl = take(p.backward ? (size_t)p.T_max * ((p.E + 63) / 64 * 64) * 2 : 0, 1024);
+  L.bwd_wgt = take(p.backward ? (size_t)p.E * p.H * 2 : 0, 1024);
   L.total = align_up(o, 1024);
   return L;
 }
@@ -442,6 +469,9 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     gp.N2 = p->N2;
     gp.ring_pairs = f8 != nullptr ? p->fp8_rows / (2 * p->BM) : p->ring_pairs;   // FP8: every pair its own rows
     gp.max_groups = p->pmax_groups;
+    gp.order_lag = order_lag(*p);
+    gp.half_tails = (p->half_tails && f8 == nullptr && p->BM == kTileM) ? 1 : 0;   // bf16, 128-row blocks
+    gp.zero_row = ws + L.zero_row;
     gp.timeout_ns = p->timeout_ns;
     gp.withhold_pair = p->withhold;
     cudaLaunchConfig_t cfg;
@@ -503,6 +533,8 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     gp.l2_done = dp.l2_done;
     gp.ring_blocks = f8 != nullptr ? p->fp8_rows / p->BM : p->ring_blocks;   // FP8: every block its own rows
     gp.max_groups = p->max_groups;
+    gp.order_lag = order_lag(*p);
+    gp.zero_row = ws + L.zero_row;
     gp.err = dp.err;
     gp.h = h;
     gp.y_acc = rp.y_acc;
@@ -537,6 +569,13 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   mark(5);
   if (prof) ++p->ev_used;
   return MOE_OK;
+}
+
+// One launch of the backward GEMM kernel of kind K on the plan's persistent grid.
+template <int K>
+static cudaError_t launch_bwd(const BwdParams& bp, int grid, cudaStream_t st) {
+  moe_backward_gemm_kernel<K><<<grid, kBwdThreads, kBwdSmemBytes, st>>>(bp);
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- routing with no allocation
@@ -762,6 +801,21 @@ int moe_plan_create_shared(moe_plan_t* out, int T_max, int H, int I, int E, int 
                               (int)kGemm2SmemBytes);
   if (ce == cudaSuccess)
     ce = cudaFuncSetAttribute(moe_router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRtcSmemBytes);
+  if (ce == cudaSuccess)
+    ce = cudaFuncSetAttribute(moe_backward_gemm_kernel<kBwdDgrad1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)kBwdSmemBytes);
+  if (ce == cudaSuccess)
+    ce = cudaFuncSetAttribute(moe_backward_gemm_kernel<kBwdDgrad2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)kBwdSmemBytes);
+  if (ce == cudaSuccess)
+    ce = cudaFuncSetAttribute(moe_backward_gemm_kernel<kBwdWgrad13>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)kBwdSmemBytes);
+  if (ce == cudaSuccess)
+    ce = cudaFuncSetAttribute(moe_backward_gemm_kernel<kBwdWgrad2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)kBwdSmemBytes);
+  if (ce == cudaSuccess)
+    ce = cudaFuncSetAttribute(moe_backward_gemm_kernel<kBwdDwg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)kBwdSmemBytes);
   if (ce == cudaSuccess) ce = set_router_smem<16>();
   if (ce == cudaSuccess) ce = set_router_smem<32>();
   if (ce == cudaSuccess) ce = set_router_smem<64>();
@@ -810,8 +864,9 @@ int moe_plan_bind_workspace(moe_plan_t p, void* ws, size_t bytes) {
   p->ws = static_cast<uint8_t*>(ws);
   p->ws_bytes = bytes;
   DeviceGuard guard(p->device);
-  // error word and scheduler counters start at zero
+  // error word and scheduler counters start at zero, and the zero row is zero
   if (cudaMemset(p->ws + p->L.err, 0, 16 * 4) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemset(p->ws + p->L.zero_row, 0, (size_t)p->H * 2) != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaMemset(p->ws + p->L.sched, 0, 16 * 4) != cudaSuccess) return MOE_ERR_CUDA;
   // split-H router state: accumulators and counters are zero between calls
   if (cudaMemset(p->ws + p->L.router_counter, 0, (size_t)p->num_sms * 4) != cudaSuccess) return MOE_ERR_CUDA;
@@ -837,6 +892,8 @@ int moe_plan_describe(moe_plan_t p, moe_plan_desc* d) {
   d->n_shared = p->S;
   d->cta_pairs = p->cta_pairs ? 1 : 0;
   d->workspace_bytes = p->L.total;
+  d->task_order = order_lag(*p) >= 0 ? 1 : 0;
+  d->half_tails = (p->cta_pairs && p->half_tails && p->BM == kTileM) ? 1 : 0;
   return MOE_OK;
 }
 
@@ -1103,10 +1160,129 @@ int moe_plan_set_fp8(moe_plan_t p, int enable) {
   return MOE_OK;
 }
 
+int moe_plan_set_backward(moe_plan_t p, int enable) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  if (enable && p->S > 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  p->backward = enable != 0;
+  p->L = make_layout(*p);
+  p->ws = nullptr;   // the workspace size changed: bind again
+  p->ws_bytes = 0;
+  return MOE_OK;
+}
+
+int moe_backward(moe_plan_t p, const void* x, const void* Wg, const float* bias, const void* W1, const void* W3,
+                 const void* W2, const void* dy, int T, void* dx, float* dWg, float* dbias, void* dW1, void* dW3,
+                 void* dW2, void* stream) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!p->backward || p->S > 0) return MOE_ERR_INVALID_ARG;
+  if (p->ws == nullptr) return MOE_ERR_NO_WORKSPACE;
+  if (T < 0 || T > p->T_max) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  const void* need16[] = {W1, W3, W2, dy, dx, dW1, dW3, dW2};
+  for (const void* q : need16)
+    if (q == nullptr || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  if (dWg == nullptr || (reinterpret_cast<uintptr_t>(dWg) & 3u)) return MOE_ERR_INVALID_ARG;
+  if (dbias != nullptr && (reinterpret_cast<uintptr_t>(dbias) & 3u)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // routing of x (router, dispatch scan, scatter), as the forward computes it; the
+  // router also zeroes the fp32 accumulator rows that collect dx
+  int rc = enqueue(p, x, Wg, bias, nullptr, nullptr, nullptr, SharedWeights{}, T, nullptr, st, false);
+  if (rc != MOE_OK) return rc;
+  DeviceGuard guard(p->device);
+  uint8_t* ws = p->ws;
+  const Layout& L = p->L;
+  const int E = p->E, H = p->H, I = p->I, k = p->k;
+  const int NE = (E + 63) / 64 * 64;
+  bf16* dg = reinterpret_cast<bf16*>(ws + L.bwd_dg);
+  bf16* du = reinterpret_cast<bf16*>(ws + L.bwd_du);
+  bf16* aw = reinterpret_cast<bf16*>(ws + L.bwd_aw);
+  float* dw = reinterpret_cast<float*>(ws + L.bwd_dw);
+  bf16* dl = reinterpret_cast<bf16*>(ws + L.bwd_dl);
+  bf16* wgt = reinterpret_cast<bf16*>(ws + L.bwd_wgt);
+  if (cudaMemsetAsync(dw, 0, (size_t)T * k * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dbias != nullptr && cudaMemsetAsync(dbias, 0, (size_t)E * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  BwdParams bp;
+  std::memset(&bp, 0, sizeof(bp));
+  bp.slot_token = reinterpret_cast<const int32_t*>(ws + L.slot_token);
+  bp.slot_topk = reinterpret_cast<const int32_t*>(ws + L.slot_topk);
+  bp.topk_w = reinterpret_cast<const float*>(ws + L.topk_w);
+  bp.block_start = reinterpret_cast<const int32_t*>(ws + L.block_start);
+  bp.sched = reinterpret_cast<const int32_t*>(ws + L.sched) + 1;   // blocks in use (the scan writes it)
+  bp.x = static_cast<const bf16*>(x);
+  bp.dy = static_cast<const bf16*>(dy);
+  bp.zero_row = reinterpret_cast<const bf16*>(ws + L.zero_row);
+  bp.dg = dg;
+  bp.du = du;
+  bp.aw = aw;
+  bp.dw = dw;
+  bp.dx_acc = reinterpret_cast<float*>(ws + L.y_acc);
+  bp.dW1 = static_cast<bf16*>(dW1);
+  bp.dW3 = static_cast<bf16*>(dW3);
+  bp.dW2 = static_cast<bf16*>(dW2);
+  bp.dWg = dWg;
+  bp.err = reinterpret_cast<int32_t*>(ws + L.err);
+  bp.T = T;
+  bp.H = H;
+  bp.I = I;
+  bp.E = E;
+  bp.k = k;
+  bp.BM = p->BM;
+  bp.pool = p->pool;
+  bp.BN = (H % 256 == 0) ? 256 : 128;
+  bp.NE = NE;
+  bp.timeout_ns = p->timeout_ns;
+  const int grid = p->num_sms;
+
+  // 1. dgrad-1: g|u recomputed, da = dy W2^T; dg, du, w*a per slot; dw
+  BwdParams b1 = bp;
+  if (!make_map(&b1.tm_w1, W1, I, (uint64_t)E * H, I, 64) || !make_map(&b1.tm_w3, W3, I, (uint64_t)E * H, I, 64) ||
+      !make_map(&b1.tm_w2, W2, H, (uint64_t)E * I, H, 128))
+    return MOE_ERR_CUDA;
+  if (launch_bwd<kBwdDgrad1>(b1, grid, st) != cudaSuccess) return MOE_ERR_CUDA;
+  // 2. dgrad-2: dx += [dg|du] [W1|W3]^T through the slot records
+  BwdParams b2 = bp;
+  if (!make_map(&b2.tm_a, dg, I, p->pool, I, 128) || !make_map(&b2.tm_a2, du, I, p->pool, I, 128) ||
+      !make_map(&b2.tm_w1, W1, I, (uint64_t)E * H, I, bp.BN) || !make_map(&b2.tm_w3, W3, I, (uint64_t)E * H, I, bp.BN))
+    return MOE_ERR_CUDA;
+  if (launch_bwd<kBwdDgrad2>(b2, grid, st) != cudaSuccess) return MOE_ERR_CUDA;
+  // 3. gate: dl from dw, dbias, dx = bf16(dx_acc + dl Wg^T), the dense dl for dWg
+  moe_transpose_wg_kernel<<<dim3((unsigned)((H + 31) / 32), (unsigned)((E + 31) / 32)), 256, 0, st>>>(
+      static_cast<const bf16*>(Wg), wgt, H, E);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  moe_gate_backward_kernel<<<(T * 32 + kGateThreads - 1) / kGateThreads, kGateThreads, 0, st>>>(
+      reinterpret_cast<const int32_t*>(ws + L.topk_idx), bp.topk_w, dw, wgt, bp.dx_acc, static_cast<bf16*>(dx), dl,
+      dbias, bp.err, T, H, E, k, NE);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  // 4. weight gradients: dW1 = x^T dg, dW3 = x^T du; dW2 = (w a)^T dy; dWg = x^T dl
+  BwdParams b3 = bp;
+  if (!make_map(&b3.tm_b, dg, I, p->pool, I, 64) || !make_map(&b3.tm_b2, du, I, p->pool, I, 64)) return MOE_ERR_CUDA;
+  if (launch_bwd<kBwdWgrad13>(b3, grid, st) != cudaSuccess) return MOE_ERR_CUDA;
+  BwdParams b4 = bp;
+  if (!make_map(&b4.tm_a, aw, I, p->pool, I, 64)) return MOE_ERR_CUDA;
+  if (launch_bwd<kBwdWgrad2>(b4, grid, st) != cudaSuccess) return MOE_ERR_CUDA;
+  BwdParams b5 = bp;
+  if (!make_map(&b5.tm_a, x, H, T, H, 64) || !make_map(&b5.tm_b, dl, NE, T, NE, 64)) return MOE_ERR_CUDA;
+  if (launch_bwd<kBwdDwg>(b5, grid, st) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
 int moe_plan_set_cta_pairs(moe_plan_t p, int enable) {
   if (p == nullptr) return MOE_ERR_INVALID_ARG;
   if (enable && p->pair_clusters < 1) return MOE_ERR_UNSUPPORTED_SHAPE;
   p->cta_pairs = enable != 0;
+  return MOE_OK;
+}
+
+int moe_plan_set_task_order(moe_plan_t p, int mode) {
+  if (p == nullptr || mode < -1 || mode > 1) return MOE_ERR_INVALID_ARG;
+  p->task_order = mode;
+  return MOE_OK;
+}
+
+int moe_plan_set_half_tails(moe_plan_t p, int enable) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  p->half_tails = enable != 0;
   return MOE_OK;
 }
 

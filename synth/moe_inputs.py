@@ -40,6 +40,7 @@ MAX_REDRAWS = 64        # redraw rounds before giving up
 
 _STREAM_X, _STREAM_WG, _STREAM_W1, _STREAM_W3, _STREAM_W2 = 1, 2, 3, 4, 5
 _STREAM_WS1, _STREAM_WS3, _STREAM_WS2 = 6, 7, 8   # shared experts
+_STREAM_DY = 9          # upstream gradient of the backward
 _STREAM_REDRAW = 100    # + attempt number
 
 
@@ -188,3 +189,10 @@ def make_inputs(shape, device="cpu", seed: int = 0, T: Optional[int] = None, n_s
 
 def custom_shape(T, H, I, E, k, zipf=False, name="custom") -> MoEShape:
     return MoEShape(name, T, H, I, E, k, zipf)
+
+
+def make_dy(shape: MoEShape, device="cpu", seed: int = 0, T: Optional[int] = None) -> torch.Tensor:
+    """Upstream gradient dy [T,H] ~ N(0,1), bf16, for the backward."""
+    device = torch.device(device)
+    T = shape.T if T is None else T
+    return _normal_bf16((T, shape.H), 1.0, _gen(device, seed, _STREAM_DY), device)

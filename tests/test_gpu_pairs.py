@@ -49,10 +49,9 @@ def test_pairs_forward_matches_oracle(T, H, I, E, k, bm, zipf, pairs):
     plan.lib.moe_plan_bind_workspace(plan._plan, plan.workspace.data_ptr(), plan.workspace_bytes)
     y = plan.forward(inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"])
     plan.check()
-    rows = sample_tokens(T, 256)
-    ref = oracle_forward(inp, tokens=rows, block_m=plan.block_m)
+    ref = oracle_forward(inp, block_m=plan.block_m)   # every token row
     assert_routing_equal(plan.routing(T), ref)
-    fro, mx = assert_y_close(y[torch.from_numpy(rows).to(y.device)], ref["y"])
+    fro, mx = assert_y_close(y, ref["y"])
     print(f"{'pairs' if pairs else 'single'} T={T} H={H} I={I} E={E} k={k}: rel_fro={fro:.2e} max_abs={mx:.2e}")
 
 
@@ -102,3 +101,37 @@ def test_pairs_workload_matches_oracle(name):
     fro, mx = assert_y_close(y, ref["y"])
     print(f"{'pairs' if plan.block_m != 128 else 'single'} {name}: all {shape.T} rows rel_fro={fro:.2e} "
           f"max_abs={mx:.2e}")
+
+
+HALF_SHAPES = [
+    # T,    H,   I,   E,  k, zipf   odd block counts; with Zipf many cold experts of one block
+    (1000, 256, 512, 8, 2, False),
+    (3000, 512, 768, 64, 8, True),
+    (700, 384, 256, 32, 4, True),     # H % 256 != 0: L2 tile of 128 columns, 64 per warp in half tasks
+    (2600, 128, 1024, 16, 2, False),
+]
+
+
+@pytest.mark.parametrize("T,H,I,E,k,zipf", HALF_SHAPES)
+def test_half_tail_tasks_match_oracle(T, H, I, E, k, zipf):
+    """An expert's lone last block as M = 128 pair MMAs (64 rows per CTA) against full pairs and the oracle."""
+    shape = custom_shape(T, H, I, E, k, zipf)
+    inp = make_inputs(shape, device=DEV)
+    ref = oracle_forward(inp, block_m=128)
+    nb = (ref["count"] + 127) // 128
+    assert (nb % 2 == 1).any(), "the shape must have experts with an odd block count"
+    ys = []
+    for half in (True, False):
+        plan = _plan(shape, 128, True)
+        plan.set_half_tails(half)
+        assert plan.half_tails == half
+        plan.workspace.fill_(0xFF)   # poison: rows the half tasks miss would show up as NaN
+        plan.lib.moe_plan_bind_workspace(plan._plan, plan.workspace.data_ptr(), plan.workspace_bytes)
+        y = plan.forward(inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"])
+        plan.check()
+        assert_routing_equal(plan.routing(T), ref)
+        fro, mx = assert_y_close(y, ref["y"], f"y (half tails {half})")
+        print(f"half={half} T={T} H={H} I={I} E={E} k={k}: odd-block experts {int((nb % 2 == 1).sum())} "
+              f"rel_fro={fro:.2e} max_abs={mx:.2e}")
+        ys.append(y.float())
+    assert (ys[0] - ys[1]).abs().max().item() <= 2e-2

@@ -261,7 +261,7 @@ def run_gpu(args, rank, world, local_rank):
     # replicated weights, each rank its own tokens (rank 0 draws the single-GPU tokens)
     inp = make_inputs(shape, device=dev, seed=args.seed, n_shared=S, x_seed=args.seed + rank)
     T, H, I, E, k = shape.T, shape.H, shape.I, shape.E, shape.k
-    plan = MoEPlan(T, H, I, E, k, device=dev, n_shared=S, fp8=args.fp8)
+    plan = MoEPlan(T, H, I, E, k, device=dev, n_shared=S, fp8=args.fp8, task_log=args.task_log)
     shared_kw = dict(Ws1=inp["Ws1"], Ws3=inp["Ws3"], Ws2=inp["Ws2"]) if S else {}
     if args.cta_pairs is not None:
         plan.set_cta_pairs(bool(args.cta_pairs))
@@ -269,6 +269,8 @@ def run_gpu(args, rank, world, local_rank):
         plan.set_task_order(args.task_order)
     if args.half_tails is not None:
         plan.set_half_tails(bool(args.half_tails))
+    if args.wide_l1 is not None:
+        plan.set_wide_l1(bool(args.wide_l1))
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
@@ -353,6 +355,20 @@ def run_gpu(args, rank, world, local_rank):
     plan.check()
     e2e_ms = reduce_max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dist, dev)
 
+    # task log of the last forward: how busy each SM's MMA issue was over the expert GEMM
+    tlog = None
+    if args.task_log:
+        lg = plan.task_log()
+        span = float(lg["t_done"].max() - lg["t_first_mma"].min())
+        busy = torch.zeros(int(lg["cta"].max()) + 1, dtype=torch.float64)
+        busy.scatter_add_(0, lg["cta"], (lg["t_last_mma"] - lg["t_first_mma"]).double())
+        issuing = busy[busy > 0] / span
+        tlog = {"tasks": int(lg["task"].numel()), "ctas_issuing_mma": int(issuing.numel()), "span_us": span / 1e3,
+                "mma_issue_occupancy": {"mean": float(issuing.mean()), "min": float(issuing.min()),
+                                        "max": float(issuing.max())},
+                "note": "per MMA-issuing CTA (the leader of a pair): sum over its tasks of first-to-last MMA "
+                        "issue time, over the launch's span (first MMA to last epilogue)"}
+
     # routing statistics for the roofline's byte count
     r = plan.routing(T)
     counts = r["expert_count"].cpu()
@@ -425,7 +441,8 @@ def run_gpu(args, rank, world, local_rank):
             "data": "synthetic (seeded N(0,1) x, N(0,1/H) Wg/W1/W3, N(0,1/I) W2, bf16; random-init weights)",
             "config": {"workload": workload_label(shape, S, args.fp8), "T_per_gpu": T, "H": H, "I": I, "E": E, "k": k,
                        "block_m": plan.block_m, "cta_pairs": plan.cta_pairs, "task_order": plan.task_order,
-                       "half_tails": plan.half_tails, "active_experts": active, "padded_slots": num_padded,
+                       "half_tails": plan.half_tails, "wide_l1": plan.wide_l1, "active_experts": active,
+                       "padded_slots": num_padded,
                        "l2": "flushed between steps (256 MB write, outside per-step events)",
                        "parallelism": "replicas" if world > 1 else "single"},
             "roofline": roof,
@@ -440,6 +457,8 @@ def run_gpu(args, rank, world, local_rank):
             "gpu_launches": args.steps * (kernels_per_forward() + (3 if args.fp8 else 0)),
             "clocks": clk,
         }
+        if tlog is not None:
+            line["task_log"] = tlog
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier(device_ids=[local_rank])
@@ -558,6 +577,10 @@ def main():
                     help="expert-GEMM task order: -1 automatic, 0 staggered, 1 interleaved; default: the plan's")
     ap.add_argument("--half-tails", type=int, default=None, choices=[0, 1],
                     help="an expert's lone last block as M = 128 pair MMAs (1) or a full pair (0); default: the plan's")
+    ap.add_argument("--wide-l1", type=int, default=None, choices=[0, 1],
+                    help="256-column (1) or 128-column (0) first-GEMM tasks on CTA pairs; default: the plan's")
+    ap.add_argument("--task-log", action="store_true",
+                    help="record the expert GEMM's task log and report each SM's MMA-issue occupancy")
     ap.add_argument("--backward", action="store_true",
                     help="time moe_backward (routing, dgrad, gate, weight gradients) instead of the forward")
     args = ap.parse_args()

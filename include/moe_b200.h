@@ -94,6 +94,29 @@ typedef struct {
   int32_t pool_capacity;
 } moe_routing;
 
+/* One record of the expert GEMM's task log (moe_plan_set_task_log). Every
+ * task of the persistent kernel (one column tile of one GEMM for one block,
+ * or pair of blocks) is written by the CTA that ran it: its number in the
+ * task order, its block (or pair), expert, phase (0: x W1 / x W3 + SwiGLU,
+ * 1: h W2 + combine) and column tile, the SM and CTA that issued its MMAs,
+ * and three %globaltimer stamps in nanoseconds: the issue of its first MMA,
+ * of its last one, and the end of its epilogue. A record whose task is
+ * 0xFFFFFFFF belongs to no task of the last launch. (Tracing of the task
+ * queue; "MegaMoE 在 MoE 系统谱系中的位置", section 2.7, describes the queue,
+ * and "FlashMoE Kernel", section 实测摘要, reports SM utilisation, which these
+ * records measure.) */
+typedef struct {
+  uint32_t task;
+  uint32_t unit;
+  uint32_t expert;
+  uint32_t phase_n;   /* phase << 16 | column tile */
+  uint32_t smid;
+  uint32_t cta;
+  uint64_t t_first_mma;
+  uint64_t t_last_mma;
+  uint64_t t_done;
+} moe_task_record;
+
 /* Static description of a plan. */
 typedef struct {
   int32_t T_max, H, I, E, k;
@@ -109,6 +132,8 @@ typedef struct {
                               (see moe_plan_set_task_order) */
   int32_t half_tails;      /* 1: bf16 forwards on CTA pairs run an expert's lone last block
                               as M = 128 pair MMAs (see moe_plan_set_half_tails) */
+  int32_t wide_l1;         /* 1: bf16 forwards on CTA pairs run 256-column first-GEMM tasks
+                              (see moe_plan_set_wide_l1) */
 } moe_plan_desc;
 
 /* Create a plan for up to T_max tokens of a layer with hidden size H, expert
@@ -379,6 +404,16 @@ int moe_plan_set_task_order(moe_plan_t plan, int mode);
  * (null plan). */
 int moe_plan_set_half_tails(moe_plan_t plan, int enable);
 
+/* Width of the first GEMM's tasks on CTA pairs (bf16, I % 256 == 0). With
+ * mode = 1 an L1 task computes 256 columns of I (W1 and W3 both) for its 256
+ * routed rows as two N = 256 MMAs per K block on the same gathered x tile,
+ * filling both TMEM accumulators (four 48 KB pipeline stages instead of six
+ * of 32 KB); with 0 it computes 128 columns; -1 (the default) picks 1 when
+ * I <= 1024, where the first-GEMM tasks are short (measured: 2.5 % faster on
+ * I = 768, 1.5-3 % slower on I = 2048 and 14336). Results are the same
+ * either way. Errors: MOE_ERR_INVALID_ARG (null plan or another mode). */
+int moe_plan_set_wide_l1(moe_plan_t plan, int mode);
+
 /* Give the plan the workspace regions of moe_backward (enable = 1) or drop them
  * (0). The workspace size changes: query moe_plan_workspace_bytes and bind a
  * workspace again. Plans with shared experts have no backward.
@@ -417,6 +452,21 @@ int moe_plan_set_backward(moe_plan_t plan, int enable);
 int moe_backward(moe_plan_t plan, const void* x, const void* Wg, const float* gate_bias, const void* W1,
                  const void* W3, const void* W2, const void* dy, int T, void* dx, float* dWg, float* dbias,
                  void* dW1, void* dW3, void* dW2, void* stream);
+
+/* Give the plan a task log (enable = 1) or drop it (0): every expert-GEMM
+ * launch then writes one moe_task_record per task into the workspace (48
+ * bytes x every block, or pair, x the GEMMs' column tiles; the region is
+ * reset before each launch, on the stream). The workspace size changes:
+ * bind a workspace again. Costs one store per task. Errors:
+ * MOE_ERR_INVALID_ARG (null plan). */
+int moe_plan_set_task_log(moe_plan_t plan, int enable);
+
+/* Device pointer to the task log of the last launch and its number of
+ * records (read it after the forward's stream work has finished, e.g. after
+ * moe_check). With FP8 forwards (two launches) it holds the second launch.
+ * Errors: MOE_ERR_INVALID_ARG (null arguments, no task log),
+ * MOE_ERR_NO_WORKSPACE. */
+int moe_plan_get_task_log(moe_plan_t plan, const moe_task_record** records, int* capacity);
 
 /* Number of kernels one moe_forward launches (for launch accounting). */
 int moe_forward_kernel_count(void);

@@ -40,7 +40,7 @@ class MoEPlanDesc(ctypes.Structure):
                 ("pool_capacity", ctypes.c_int32), ("num_sms", ctypes.c_int32),
                 ("pair_clusters", ctypes.c_int32), ("cta_pairs", ctypes.c_int32),
                 ("n_shared", ctypes.c_int32), ("workspace_bytes", ctypes.c_size_t),
-                ("task_order", ctypes.c_int32), ("half_tails", ctypes.c_int32)]
+                ("task_order", ctypes.c_int32), ("half_tails", ctypes.c_int32), ("wide_l1", ctypes.c_int32)]
 
 
 # exported symbol -> (restype, argtypes); the same list as include/moe_b200.h
@@ -76,6 +76,9 @@ SIGNATURES = {
     "moe_backward": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_plan_set_task_order": (_c_int, [_vp, _c_int]),
     "moe_plan_set_half_tails": (_c_int, [_vp, _c_int]),
+    "moe_plan_set_wide_l1": (_c_int, [_vp, _c_int]),
+    "moe_plan_set_task_log": (_c_int, [_vp, _c_int]),
+    "moe_plan_get_task_log": (_c_int, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_c_int)]),
     "moe_plan_set_fp8": (_c_int, [_vp, _c_int]),
     "moe_forward_kernel_count": (_c_int, []),
     "moe_plan_destroy": (None, [_vp]),
@@ -148,7 +151,7 @@ class MoEPlan:
     """
 
     def __init__(self, T_max: int, H: int, I: int, E: int, k: int, block_m: int = 0, device=None,
-                 n_shared: int = 0, fp8: bool = False, backward: bool = False):
+                 n_shared: int = 0, fp8: bool = False, backward: bool = False, task_log: bool = False):
         self.lib = load_library()
         self.device = torch.device("cuda", torch.cuda.current_device() if device is None
                                    else torch.device(device).index or 0)
@@ -162,6 +165,8 @@ class MoEPlan:
         self.has_backward = bool(backward)
         if backward:   # workspace regions of backward
             _ok(self.lib.moe_plan_set_backward(self._plan, 1), "moe_plan_set_backward")
+        if task_log:   # workspace region of the expert GEMM's task log
+            _ok(self.lib.moe_plan_set_task_log(self._plan, 1), "moe_plan_set_task_log")
         d = MoEPlanDesc()
         _ok(self.lib.moe_plan_describe(self._plan, ctypes.byref(d)), "moe_plan_describe")
         self.block_m, self.pool_capacity, self.num_sms = d.block_m, d.pool_capacity, d.num_sms
@@ -341,6 +346,21 @@ class MoEPlan:
             block_m=r.block_m,
         )
 
+    def task_log(self) -> dict:
+        """The expert GEMM's task records of the last launch (plan made with task_log=True), as
+        int64 tensors on the host: task, unit, expert, phase, n, smid, cta, t_first_mma,
+        t_last_mma, t_done (ns); only the records of tasks that ran."""
+        ptr, cap = ctypes.c_void_p(), ctypes.c_int(0)
+        _ok(self.lib.moe_plan_get_task_log(self._plan, ctypes.byref(ptr), ctypes.byref(cap)), "moe_plan_get_task_log")
+        off = ptr.value - self.workspace.data_ptr()
+        raw = self.workspace[off:off + cap.value * 48].cpu()
+        u32 = raw.view(torch.int32).view(cap.value, 12).to(torch.int64) & 0xFFFFFFFF
+        u64 = raw.view(torch.int64).view(cap.value, 6)
+        keep = u32[:, 0] != 0xFFFFFFFF
+        return dict(task=u32[keep, 0], unit=u32[keep, 1], expert=u32[keep, 2], phase=u32[keep, 3] >> 16,
+                    n=u32[keep, 3] & 0xFFFF, smid=u32[keep, 4], cta=u32[keep, 5], t_first_mma=u64[keep, 3],
+                    t_last_mma=u64[keep, 4], t_done=u64[keep, 5])
+
     def set_profiling(self, enable: bool):
         _ok(self.lib.moe_plan_set_profiling(self._plan, 1 if enable else 0), "moe_plan_set_profiling")
 
@@ -361,6 +381,18 @@ class MoEPlan:
     def set_half_tails(self, enable: bool):
         """Run an expert's lone last block as M = 128 pair MMAs (see moe_plan_set_half_tails)."""
         _ok(self.lib.moe_plan_set_half_tails(self._plan, 1 if enable else 0), "moe_plan_set_half_tails")
+
+    def set_wide_l1(self, mode):
+        """256-column first-GEMM tasks on CTA pairs: True / 1, False / 0, or -1 automatic
+        (see moe_plan_set_wide_l1)."""
+        m = int(mode) if not isinstance(mode, bool) else (1 if mode else 0)
+        _ok(self.lib.moe_plan_set_wide_l1(self._plan, m), "moe_plan_set_wide_l1")
+
+    @property
+    def wide_l1(self) -> bool:
+        d = MoEPlanDesc()
+        _ok(self.lib.moe_plan_describe(self._plan, ctypes.byref(d)), "moe_plan_describe")
+        return bool(d.wide_l1)
 
     @property
     def half_tails(self) -> bool:

@@ -27,8 +27,10 @@
 //            record like the forward's combine (weight 1);
 //   kWgrad13 (expert, 128 rows of H, 128 columns of I): dW1[e] = x^T dg,
 //            dW3[e] = x^T du over the expert's slots (K = its padded slots);
-//   kWgrad2  (expert, 128 rows of I, 256 or 128 columns of H):
-//            dW2[e] = aw^T dy over the expert's slots;
+//   kWgrad2  (expert, 128 rows of H, 256 or 128 columns of I):
+//            dW2[e]^T = dy^T aw over the expert's slots (the transpose keeps
+//            the gathered operand at 128 columns of dy and loads the wider
+//            aw tile by TMA), stored transposed into dW2[e] [I, H];
 //   kDwg     (128 rows of H): dWg = x^T dl over all tokens (dl dense [T, E],
 //            written by the gate kernel).
 //
@@ -77,9 +79,9 @@ struct BwdParams {
   CUtensorMap tm_w1;   // dgrad1: W1 as [E*H, I], box {64, 64} (MN-major B); dgrad2: box {64, BNd} (K-major B)
   CUtensorMap tm_w3;   // the same for W3
   CUtensorMap tm_w2;   // dgrad1: W2 as [E*I, H], box {64, 128} (K-major B: rows i, K = h)
-  CUtensorMap tm_a;    // dgrad2: dg as [pool, I] box {64, 128}; wgrad2: aw [pool, I] box {64, 64}; dwg: x [T, H] box {64, 64}
+  CUtensorMap tm_a;    // dgrad2: dg as [pool, I] box {64, 128}; dwg: x [T, H] box {64, 64}
   CUtensorMap tm_a2;   // dgrad2: du as [pool, I], box {64, 128}
-  CUtensorMap tm_b;    // wgrad13: dg as [pool, I] box {64, 64}; dwg: dl as [T, E] box {64, 64}
+  CUtensorMap tm_b;    // wgrad13: dg as [pool, I] box {64, 64}; wgrad2: aw [pool, I] box {64, 64}; dwg: dl [T, NE]
   CUtensorMap tm_b2;   // wgrad13: du as [pool, I] box {64, 64}
   bf16* dg;            // [pool, I]
   bf16* du;            // [pool, I]
@@ -93,7 +95,8 @@ struct BwdParams {
   int32_t* err;
   int T, H, I, E, k, BM;
   int pool;            // rows of dg / du / aw
-  int BN;              // dgrad2 / wgrad2: columns of H per task (256, or 128 when H % 256 != 0)
+  int BN;              // dgrad2: columns of H per task (256, or 128 when H % 256 != 0)
+  int BNi;             // wgrad2: columns of I per task (256, or 128 when I % 256 != 0)
   int NE;              // dwg: columns of the dl tile, E rounded up to 64
   unsigned long long timeout_ns;
 };
@@ -157,7 +160,7 @@ __device__ __forceinline__ int bwd_num_tasks(const BwdParams& p, const BwdSmem& 
   if (Kind == kBwdDgrad1) return s.nblocks * (p.I / 128);
   if (Kind == kBwdDgrad2) return s.nblocks * (p.H / p.BN);
   if (Kind == kBwdWgrad13) return p.E * (p.H / 128) * (p.I / 128);
-  if (Kind == kBwdWgrad2) return p.E * (p.I / 128) * (p.H / p.BN);
+  if (Kind == kBwdWgrad2) return p.E * (p.H / 128) * (p.I / p.BNi);
   return p.H / 128;
 }
 
@@ -187,8 +190,8 @@ __device__ __forceinline__ BwdTask bwd_decode(int t, const BwdParams& p, const B
     task.b = s.block_start[e] + local % nb;
     task.nk = Kind == kBwdDgrad1 ? 2 * (p.H / 64) : 2 * (p.I / 64);
   } else if (Kind == kBwdWgrad13 || Kind == kBwdWgrad2) {
-    const int MT = Kind == kBwdWgrad13 ? p.H / 128 : p.I / 128;
-    const int NT = Kind == kBwdWgrad13 ? p.I / 128 : p.H / p.BN;
+    const int MT = p.H / 128;
+    const int NT = Kind == kBwdWgrad13 ? p.I / 128 : p.I / p.BNi;
     task.e = t / (MT * NT);
     const int local = t - task.e * MT * NT;
     task.m = local / NT;
@@ -250,11 +253,10 @@ __device__ void bwd_producer(const BwdParams& p, BwdSmem& s, uint8_t* tiles) {
           ptx::tma_load_2d(b + kBoxBytes, &p.tm_b, bar, n0 + 64, s0, pol_n);
           ptx::tma_load_2d(b + 2 * kBoxBytes, &p.tm_b2, bar, n0, s0, pol_n);
           ptx::tma_load_2d(b + 3 * kBoxBytes, &p.tm_b2, bar, n0 + 64, s0, pol_n);
-        } else if (Kind == kBwdWgrad2) {
-          const int s0 = s.block_start[task.e] * p.BM + kb * 64, m0 = task.m * 128;
-          ptx::mbar_arrive_expect_tx(bar, 2 * kBoxBytes);
-          ptx::tma_load_2d(a, &p.tm_a, bar, m0, s0, pol_n);
-          ptx::tma_load_2d(a + kBoxBytes, &p.tm_a, bar, m0 + 64, s0, pol_n);
+        } else if (Kind == kBwdWgrad2) {   // aw columns n0 .. n0+BNi-1 of the slots (MN-major B)
+          const int s0 = s.block_start[task.e] * p.BM + kb * 64, n0 = task.n * p.BNi;
+          ptx::mbar_arrive_expect_tx(bar, (p.BNi / 64) * kBoxBytes);
+          for (int j = 0; j < p.BNi / 64; ++j) ptx::tma_load_2d(b + j * kBoxBytes, &p.tm_b, bar, n0 + j * 64, s0, pol_n);
         } else {   // dwg: x^T (rows h) and dl (columns e), K = tokens
           const int m0 = task.m * 128;
           ptx::mbar_arrive_expect_tx(bar, 2 * kBoxBytes + (p.NE / 64) * kBoxBytes);
@@ -334,34 +336,50 @@ __device__ void bwd_gather(const BwdParams& p, BwdSmem& s, uint8_t* tiles, int g
     } else if (Kind == kBwdWgrad13 || Kind == kBwdWgrad2) {
       const int s_begin = s.block_start[task.e] * p.BM;
       const int s_end = s.block_start[task.e + 1] * p.BM;
-      // wgrad13: 64 rows x 16 chunks (A, 128 columns of x); wgrad2: 64 rows x BN/8 chunks (B, dy)
-      const int cpr = Kind == kBwdWgrad13 ? 16 : p.BN / 8;   // 16-byte chunks per row
-      const int col0 = Kind == kBwdWgrad13 ? task.m * 128 : task.n * p.BN;
+      // the A operand, 64 slot rows x 16 chunks (128 columns of H) of x (wgrad13) or dy (wgrad2).
+      // A thread's chunks of a stage lie on rows kr0 + rstep * i (i < per) at one chunk column:
+      // thread tid takes chunk q = 128 i + tid, i.e. row q / cpr, column q % cpr.
+      const int cpr = 16;   // 16-byte chunks per row
+      const int col0 = task.m * 128;
       const bf16* base = Kind == kBwdWgrad13 ? p.x : p.dy;
-      const int per = 64 * cpr / 128;   // chunks per thread per stage: 8 or 16 (or 8 when BN = 128)
+      const int per = 64 * cpr / 128;   // chunks per thread per stage: 8
+      const int kr0 = tid / cpr, rstep = 128 / cpr, cc = tid % cpr;
+      const int box = cc >> 3, c = cc & 7;
+      // the tokens of a stage's rows are loaded one stage ahead, so that their round trip
+      // overlaps the wait for a free stage and the previous stage's copies
+      auto load_tokens = [&](int kb, int (&tk)[16]) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          tk[i] = -1;
+          const int slot = s_begin + kb * 64 + kr0 + rstep * i;
+          if (i < per && kb < task.nk && slot < s_end) tk[i] = __ldg(p.slot_token + slot);
+        }
+      };
+      int tk_cur[16], tk_next[16];
+      load_tokens(0, tk_cur);
       for (int kb = 0; kb < task.nk; ++kb) {
+        load_tokens(kb + 1, tk_next);
         if (!bwd_wait(&s.empty[stage], phase ^ 1, p, s, 3)) {
           ok = false;
           break;
         }
-        const uint32_t dst0 = ptx::smem_u32(tiles + stage * kBwdStageBytes) + (Kind == kBwdWgrad13 ? 0 : kBwdABytes);
-        for (int i = 0; i < per; ++i) {
-          const int q = i * 128 + tid;
-          const int kr = q / cpr, cc = q % cpr;   // K row (slot) and 16-byte chunk of the row
-          const int slot = s_begin + kb * 64 + kr;
-          int tk = -1;
-          if (slot < s_end) {
-            tk = p.slot_token[slot];
+        const uint32_t dst0 = ptx::smem_u32(tiles + stage * kBwdStageBytes);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (i < per) {
+            const int kr = kr0 + rstep * i;
+            int tk = tk_cur[i];
             if (tk >= p.T) {
               bwd_error(p, s, kDevBounds, 0x2000 | task.e);
               tk = -1;
             }
+            const bf16* src = (tk < 0 ? p.zero_row : base + (size_t)tk * p.H) + col0 + cc * 8;
+            ptx::cp_async_16(dst0 + box * kBoxBytes + kr * 128 + ((c ^ (kr & 7)) << 4), src);
           }
-          const int box = cc >> 3, c = cc & 7;
-          const bf16* src = (tk < 0 ? p.zero_row : base + (size_t)tk * p.H) + col0 + cc * 8;
-          ptx::cp_async_16(dst0 + box * kBoxBytes + kr * 128 + ((c ^ (kr & 7)) << 4), src);
         }
         ptx::cp_async_mbar_arrive_noinc(&s.full[stage]);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) tk_cur[i] = tk_next[i];
         if (++stage == kBwdStages) {
           stage = 0;
           phase ^= 1;
@@ -397,7 +415,7 @@ __device__ void bwd_mma(const BwdParams& p, BwdSmem& s, uint8_t* tiles, uint32_t
       Kind == kBwdDgrad1 ? ptx::idesc_bf16_f32(128, 256, false, true)
       : Kind == kBwdDgrad2 ? ptx::idesc_bf16_f32(128, p.BN, false, false)
       : Kind == kBwdWgrad13 ? ptx::idesc_bf16_f32(128, 256, true, true)
-      : Kind == kBwdWgrad2 ? ptx::idesc_bf16_f32(128, p.BN, true, true)
+      : Kind == kBwdWgrad2 ? ptx::idesc_bf16_f32(128, p.BNi, true, true)
                            : ptx::idesc_bf16_f32(128, p.NE, true, true);
   const uint32_t id_da = ptx::idesc_bf16_f32(128, 128, false, false);   // dgrad1: dy W2^T, W2 rows K-major
   int stage = 0;
@@ -562,7 +580,7 @@ __device__ void bwd_epilogue(const BwdParams& p, BwdSmem& s, uint32_t tmem_base)
                    nullptr, release);
     } else {
       // weight-gradient tiles: row r of the tile, ncols columns, bf16 (fp32 for dWg)
-      const int ncols = Kind == kBwdWgrad13 ? 256 : Kind == kBwdWgrad2 ? p.BN : p.NE;
+      const int ncols = Kind == kBwdWgrad13 ? 256 : Kind == kBwdWgrad2 ? p.BNi : p.NE;
 #pragma unroll 1
       for (int c = 0; c < ncols / 32; ++c) {
         float f[32];
@@ -581,8 +599,19 @@ __device__ void bwd_epilogue(const BwdParams& p, BwdSmem& s, uint32_t tmem_base)
           const size_t o = ((size_t)task.e * p.H + task.m * 128 + r) * p.I + task.n * 128 + (c & 3) * 32;
           store_bf16x32(out + o, f);
         } else if (Kind == kBwdWgrad2) {
-          const size_t o = ((size_t)task.e * p.I + task.m * 128 + r) * p.H + task.n * p.BN + c * 32;
-          store_bf16x32(p.dW2 + o, f);
+          // the tile is dW2[e]^T (rows h, columns i): transpose each 32 x 32 block through the
+          // warp's staging rows, so that lane l writes 32 consecutive h of row i = i0 + 32c + l
+          float* srow = s.out_stage[quarter][lane];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            reinterpret_cast<float4*>(srow)[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+          __syncwarp();
+          float t[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) t[i] = s.out_stage[quarter][i][lane];
+          __syncwarp();
+          const size_t o = ((size_t)task.e * p.I + task.n * p.BNi + c * 32 + lane) * p.H + task.m * 128 + quarter * 32;
+          store_bf16x32(p.dW2 + o, t);
         } else {
           float* out = p.dWg + (size_t)(task.m * 128 + r) * p.E;
 #pragma unroll

@@ -48,4 +48,27 @@ constexpr int kMaxExperts = 256;                   // routed experts per plan
 constexpr int kMaxShared = 8;                      // shared experts per plan
 constexpr int kMaxExpertsAll = kMaxExperts + kMaxShared;
 
+// One record of the expert GEMM's task log (a plan option): written by the
+// CTA (or CTA pair) that ran task number `task` of the launch. Timestamps are
+// %globaltimer nanoseconds: the issue of the task's first MMA, the issue of
+// its last one (the accumulator commit), and the end of its epilogue.
+struct TaskRecord {
+  uint32_t task;      // task number in the launch's task order
+  uint32_t unit;      // block (single-CTA kernel) or block pair (CTA pairs)
+  uint32_t expert;
+  uint32_t phase_n;   // phase (0 = first GEMM, 1 = second GEMM) << 16 | n-tile
+  uint32_t smid;      // SM of the CTA that issued the MMAs
+  uint32_t cta;       // its blockIdx.x
+  uint64_t t_first_mma;
+  uint64_t t_last_mma;
+  uint64_t t_done;
+};
+static_assert(sizeof(TaskRecord) == 48, "task records are 48 bytes");
+
+__device__ __forceinline__ uint32_t smid_u32() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
+  return r;
+}
+
 }  // namespace moe

@@ -83,6 +83,8 @@ struct GemmParams {
   int ring_blocks;              // block b uses ring slot b % ring_blocks
   int max_groups;
   int order_lag;                // task order (see locate_task): -1 staggered, >= 0 interleaved after this lag
+  TaskRecord* task_log;         // one record per task of the launch, or null (no log)
+  int task_log_cap;
   const uint8_t* zero_row;      // 2*H zero bytes: the A row of a padding slot
   unsigned long long timeout_ns;
   int withhold_block;           // test hook: never publish L1 completion of this block (-1: off)
@@ -91,6 +93,7 @@ struct GemmParams {
 struct Task {
   int phase;   // 0 = L1, 1 = L2, -1 = no more work
   int e, b, n;
+  int id;      // task number (the claimed counter value)
 };
 
 struct GemmSmem {
@@ -232,7 +235,7 @@ __device__ __forceinline__ TaskPos locate_task(int t, const int* gs, int G, int 
 }
 
 __device__ __forceinline__ Task decode_task(int t, const GemmSmem& s, const GemmParams& p) {
-  Task task{-1, 0, 0, 0};
+  Task task{-1, 0, 0, 0, 0};
   const int G = s.num_groups;
   const int nb_total = s.block_start[p.E + p.S];
   // one-phase launches (a single block group): the second GEMM's tasks follow the first's
@@ -260,6 +263,7 @@ __device__ __forceinline__ Task decode_task(int t, const GemmSmem& s, const Gemm
   task.e = e;
   task.n = local / nb;
   task.b = eb0 + (local - task.n * nb);
+  task.id = t;
   return task;
 }
 
@@ -314,7 +318,7 @@ __device__ void gemm_scheduler(const GemmParams& p, GemmSmem& s) {
     bool ok = true;
     if (lane == 0) ok = wait_taken(pushed, p, s);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    Task task{-1, 0, 0, 0};
+    Task task{-1, 0, 0, 0, 0};
     if (ok) task = decode_task(claim_task(p, s, lane), s, p);
     if (!warp_wait(&s.task_empty[q], qphase ^ 1, p, s, 1)) break;
     if (task.phase == 0) {
@@ -486,6 +490,7 @@ __device__ void gemm_mma(const GemmParams& p, GemmSmem& s, uint8_t* tiles, uint3
     const uint32_t idesc = task.phase == 0 ? idesc_l1 : idesc_l2;
     const int nk = task.phase == 0 ? l1_ksteps<F8>(p) : l2_ksteps<F8>(p);
     bool ok = true;
+    uint64_t t_first = 0;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait(&s.full[stage], phase, p, s, 5)) {
         ok = false;
@@ -493,6 +498,7 @@ __device__ void gemm_mma(const GemmParams& p, GemmSmem& s, uint8_t* tiles, uint3
       }
       ptx::tc_fence_after();
       ptx::fence_proxy_async_shared();   // cp.async-written A rows -> tensor-core reads
+      if (kb == 0) t_first = ptx::globaltimer();
       if (lane == 0) {
         const uint32_t a_addr = ptx::smem_u32(stage_ptr(tiles, stage));
         const uint32_t b_addr = a_addr + kTileABytes;
@@ -522,6 +528,17 @@ __device__ void gemm_mma(const GemmParams& p, GemmSmem& s, uint8_t* tiles, uint3
     }
     if (!ok) break;
     if (lane == 0) ptx::mma_commit(&s.acc_full[acc]);
+    if (lane == 0 && p.task_log != nullptr && task.id < p.task_log_cap) {
+      TaskRecord* r = p.task_log + task.id;
+      r->task = task.id;
+      r->unit = task.b;
+      r->expert = task.e;
+      r->phase_n = ((uint32_t)task.phase << 16) | (uint32_t)task.n;
+      r->smid = smid_u32();
+      r->cta = blockIdx.x;
+      r->t_first_mma = t_first;
+      r->t_last_mma = ptx::globaltimer();
+    }
     __syncwarp();
     if (++acc == 2) {
       acc = 0;
@@ -851,6 +868,8 @@ __device__ void gemm_epilogue(const GemmParams& p, GemmSmem& s, uint32_t tmem_ba
                      if (lane == 0) ptx::mbar_arrive(&s.acc_empty[acc]);
                    });
     }
+    if (p.task_log != nullptr && quarter == 0 && lane == 0 && task.id < p.task_log_cap)
+      p.task_log[task.id].t_done = ptx::globaltimer();
     if (++acc == 2) {
       acc = 0;
       acc_phase ^= 1;

@@ -97,6 +97,8 @@ struct Gemm2Params {
   int order_lag;                // task order (locate_task in expert_gemm.cuh): -1 staggered, >= 0 interleaved
   int half_tails;               // 1: an expert's lone last block runs as an M = 128 pair MMA (bf16, BM = 128)
   const uint8_t* zero_row;      // 2*H zero bytes: the A row of a padding slot
+  TaskRecord* task_log;         // one record per task of the launch (written by the leader), or null
+  int task_log_cap;
   unsigned long long timeout_ns;
   int withhold_pair;            // test hook: never publish L1 completion of this pair (-1: off)
 };
@@ -106,7 +108,7 @@ struct Task2 {
   int e, p, n;  // expert, pair, n-tile
   int b0, b1;   // blocks of CTA 0 and CTA 1 (b1 = -1: the expert has an odd block count)
   int half;     // 1: the lone block b0 split over the pair, rows 0-63 in CTA 0 and 64-127 in CTA 1
-  int pad1;
+  int id;       // task number (the claimed counter value)
 };
 
 struct Gemm2Smem {
@@ -134,6 +136,19 @@ static_assert(offsetof(Gemm2Smem, out_stage) % 16 == 0, "staging rows are read a
 static_assert(sizeof(Task2) == 32, "tasks are copied to the peer as 8 words");
 
 constexpr size_t kGemm2SmemBytes = 1024 + (size_t)kStages2 * kStage2Bytes + sizeof(Gemm2Smem);
+
+// Wide variant (bf16, I % 256 == 0): an L1 task covers 256 columns of I (two
+// N = 256 MMAs per K block on the same A tile, into both TMEM accumulators),
+// so the routed x rows are gathered once per 256 columns instead of per 128;
+// a stage then holds 128 B-tile columns per CTA (48 KB), four stages.
+constexpr int kStages2W = 4;
+constexpr int kStage2BytesW = kTileABytes + 2 * kTileB2Bytes;   // 48 KB
+constexpr size_t kGemm2SmemBytesW = 1024 + (size_t)kStages2W * kStage2BytesW + sizeof(Gemm2Smem);
+static_assert(kGemm2SmemBytesW <= 232448, "wide pair kernel exceeds the shared memory of a CTA");
+template <bool W>
+__host__ __device__ constexpr int stages2() { return W ? kStages2W : kStages2; }
+template <bool W>
+__host__ __device__ constexpr int stage2_bytes() { return W ? kStage2BytesW : kStage2Bytes; }
 
 __device__ __forceinline__ void set_error2(const Gemm2Params& p, Gemm2Smem& s, int code, int detail) {
   if (atomicCAS(p.err, 0, code) == 0) p.err[1] = detail;
@@ -233,10 +248,12 @@ __device__ __forceinline__ Task2 decode_task2(int t, const Gemm2Smem& s, const G
   task.b0 = s.block_start[e] + 2 * (task.p - s.pair_start[e]);
   task.b1 = task.b0 + 1 < s.block_start[e + 1] ? task.b0 + 1 : -1;
   task.half = (task.b1 < 0 && p.half_tails) ? 1 : 0;
+  task.id = t;
   return task;
 }
 
-__device__ __forceinline__ uint8_t* stage2_ptr(uint8_t* tiles, int stage) { return tiles + stage * kStage2Bytes; }
+template <bool W>
+__device__ __forceinline__ uint8_t* stage2_ptr(uint8_t* tiles, int stage) { return tiles + stage * stage2_bytes<W>(); }
 
 // K blocks of an L1 task: 64 bf16 or 128 FP8 elements (one 128-byte swizzle row).
 template <bool F8>
@@ -328,7 +345,7 @@ __device__ __forceinline__ bool wait_taken2(int n, const Gemm2Params& p, Gemm2Sm
   return true;
 }
 
-template <bool F8>
+template <bool F8, bool W>
 __device__ void gemm2_scheduler(const Gemm2Params& p, Gemm2Smem& s) {
   const int lane = ptx::lane_id();
   int q = 0;
@@ -355,7 +372,7 @@ __device__ void gemm2_scheduler(const Gemm2Params& p, Gemm2Smem& s) {
 }
 
 // ---------------------------------------------------------------- leader warp 0: TMA
-template <bool F8>
+template <bool F8, bool W>
 __device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles) {
   const int lane = ptx::lane_id();
   const uint64_t pol = ptx::policy_evict_first();
@@ -384,12 +401,27 @@ __device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_
         ok = false;
         break;
       }
-      const uint32_t a_addr = ptx::smem_u32(stage2_ptr(tiles, stage));
+      const uint32_t a_addr = ptx::smem_u32(stage2_ptr<W>(tiles, stage));
       const uint32_t b_addr = a_addr + kTileABytes;
       if (lane == 0) {
         // this CTA's half only; the follower's half lands on the follower's own
         // barrier and reaches this one through its relay arrival
-        if (task.phase == 0) {
+        if (W && task.phase == 0) {
+          // 256 columns of I: W1 columns n0 .. n0+255 (the follower: W3), or in a half task
+          // W1 and W3 columns n0 .. n0+63 and n0+128 .. n0+191 (the follower: the other 64s)
+          ptx::mbar_arrive_expect_tx(&s.full[stage], 4 * kBoxBytes);
+          const int n0 = task.n * 2 * kL1TileN;
+          const bool sh = task.e >= p.E;
+          const int wrow = (sh ? task.e - p.E : task.e) * p.H + kb * kBK;
+          const CUtensorMap* m1 = sh ? &p.tm_ws1 : &p.tm_w1;
+          const CUtensorMap* m3 = sh ? &p.tm_ws3 : &p.tm_w3;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const CUtensorMap* m = task.half ? ((j & 1) ? m3 : m1) : m1;
+            const int col = task.half ? n0 + (j >> 1) * kL1TileN : n0 + j * 64;
+            ptx::tma_load_2d(b_addr + j * kBoxBytes, m, &s.full[stage], col, wrow, pol);
+          }
+        } else if (task.phase == 0) {
           ptx::mbar_arrive_expect_tx(&s.full[stage], 2 * kBoxBytes);
           const int n0 = task.n * kL1TileN;
           if (F8) {   // K-major FP8 codes: 64 rows (columns of I) x 128 bytes per box
@@ -416,13 +448,13 @@ __device__ void gemm2_leader_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_
       __syncwarp();
       issued |= 1u << stage;
       issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-      if (++stage == kStages2) {
+      if (++stage == stages2<W>()) {
         stage = 0;
         phase ^= 1;
       }
     }
   }
-  for (int st = 0; st < kStages2; ++st)
+  for (int st = 0; st < stages2<W>(); ++st)
     if (issued & (1u << st)) {
       const uint64_t t0 = ptx::globaltimer();
       while (!ptx::mbar_try_wait(&s.full[st], (issued_parity >> st) & 1u))
@@ -462,7 +494,7 @@ __device__ __forceinline__ void release_task_slot2(int q, bool is_leader, Gemm2S
 }
 
 // ---------------------------------------------------------------- follower warp 0: its TMA halves
-template <bool F8>
+template <bool F8, bool W>
 __device__ void gemm2_follower_producer(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles) {
   const int lane = ptx::lane_id();
   const uint64_t pol = ptx::policy_evict_first();
@@ -482,9 +514,22 @@ __device__ void gemm2_follower_producer(const Gemm2Params& p, Gemm2Smem& s, uint
         break;
       }
       if (lane == 0) {
-        const uint32_t a_addr = ptx::smem_u32(stage2_ptr(tiles, stage));
+        const uint32_t a_addr = ptx::smem_u32(stage2_ptr<W>(tiles, stage));
         const uint32_t b_addr = a_addr + kTileABytes;
-        if (task.phase == 0) {
+        if (W && task.phase == 0) {   // the leader's layout, with W3 (or the other 64 columns)
+          ptx::mbar_arrive_expect_tx(&s.full[stage], 4 * kBoxBytes);
+          const int n0 = task.n * 2 * kL1TileN;
+          const bool sh = task.e >= p.E;
+          const int wrow = (sh ? task.e - p.E : task.e) * p.H + kb * kBK;
+          const CUtensorMap* m1 = sh ? &p.tm_ws1 : &p.tm_w1;
+          const CUtensorMap* m3 = sh ? &p.tm_ws3 : &p.tm_w3;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const CUtensorMap* m = task.half ? ((j & 1) ? m3 : m1) : m3;
+            const int col = task.half ? n0 + (j >> 1) * kL1TileN + 64 : n0 + j * 64;
+            ptx::tma_load_2d(b_addr + j * kBoxBytes, m, &s.full[stage], col, wrow, pol);
+          }
+        } else if (task.phase == 0) {
           ptx::mbar_arrive_expect_tx(&s.full[stage], 2 * kBoxBytes);
           const int n0 = task.n * kL1TileN;
           if (F8) {
@@ -507,7 +552,7 @@ __device__ void gemm2_follower_producer(const Gemm2Params& p, Gemm2Smem& s, uint
         }
       }
       __syncwarp();
-      if (++stage == kStages2) {
+      if (++stage == stages2<W>()) {
         stage = 0;
         phase ^= 1;
       }
@@ -519,7 +564,7 @@ __device__ void gemm2_follower_producer(const Gemm2Params& p, Gemm2Smem& s, uint
 // ---------------------------------------------------------------- follower warp 1: stage relay
 // The follower's TMA bytes and gather lanes land on its own stage barrier;
 // once a stage is complete, one arrival on the leader's barrier of that stage.
-template <bool F8>
+template <bool F8, bool W>
 __device__ void gemm2_follower_relay(const Gemm2Params& p, Gemm2Smem& s) {
   const int lane = ptx::lane_id();
   const uint32_t lead_full0 = ptx::mapa(ptx::smem_u32(&s.full[0]), 0);
@@ -543,7 +588,7 @@ __device__ void gemm2_follower_relay(const Gemm2Params& p, Gemm2Smem& s) {
         ptx::mbar_arrive_peer(lead_full0 + 8 * stage);
       }
       __syncwarp();
-      if (++stage == kStages2) {
+      if (++stage == stages2<W>()) {
         stage = 0;
         phase ^= 1;
       }
@@ -553,7 +598,7 @@ __device__ void gemm2_follower_relay(const Gemm2Params& p, Gemm2Smem& s) {
 }
 
 // ---------------------------------------------------------------- leader warp 1: MMA issuer
-template <bool F8>
+template <bool F8, bool W>
 __device__ void gemm2_mma(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, uint32_t tmem_base) {
   const int lane = ptx::lane_id();
   const uint32_t idesc_l1 =
@@ -575,12 +620,19 @@ __device__ void gemm2_mma(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, ui
     if (!pop_task2(task, q, qphase, nullptr, true, p, s, 7, true)) break;
     if (task.phase < 0) break;
     if (!warp_wait2(&s.acc_empty[acc], acc_phase ^ 1, p, s, 8)) break;
+    // wide L1 task: both accumulators, this slot and the next one in turn
+    const bool two = W && task.phase == 0;
+    const int acc2 = acc ^ 1;
+    const uint32_t acc2_phase = acc == 1 ? acc_phase ^ 1 : acc_phase;
+    if (two && !warp_wait2(&s.acc_empty[acc2], acc2_phase ^ 1, p, s, 8)) break;
     ptx::tc_fence_after();
     const uint32_t d_tmem = tmem_base + acc * 256;
+    const uint32_t d_tmem2 = tmem_base + acc2 * 256;
     const uint32_t idesc = task.half ? (task.phase == 0 ? idesc_l1_half : idesc_l2_half)
                                      : (task.phase == 0 ? idesc_l1 : idesc_l2);
     const int nk = task.phase == 0 ? l1_ksteps2<F8>(p) : l2_ksteps2<F8>(p);
     bool ok = true;
+    uint64_t t_first = 0;
     for (int kb = 0; kb < nk; ++kb) {
       if (!warp_wait2(&s.full[stage], phase, p, s, 9)) {
         ok = false;
@@ -588,8 +640,9 @@ __device__ void gemm2_mma(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, ui
       }
       ptx::tc_fence_after();
       ptx::fence_proxy_async_shared();
+      if (kb == 0) t_first = ptx::globaltimer();
       if (lane == 0) {
-        const uint32_t a_addr = ptx::smem_u32(stage2_ptr(tiles, stage));
+        const uint32_t a_addr = ptx::smem_u32(stage2_ptr<W>(tiles, stage));
         const uint32_t b_addr = a_addr + kTileABytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
@@ -601,24 +654,43 @@ __device__ void gemm2_mma(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, ui
           } else {
             const uint64_t bd = ptx::smem_desc_sw128(b_addr + kk * 2048, kBoxBytes, 1024);
             ptx::mma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            if (two) {   // the next 128 columns of I: B boxes 2 and 3, the same A tile
+              const uint64_t bd2 = ptx::smem_desc_sw128(b_addr + 2 * kBoxBytes + kk * 2048, kBoxBytes, 1024);
+              ptx::mma_bf16_pair(d_tmem2, ad, bd2, idesc, (kb | kk) != 0 ? 1u : 0u);
+            }
           }
         }
         ptx::mma_commit_pair_multicast(&s.empty[stage], 0x3);
         issued_any = true;
       }
       __syncwarp();
-      if (++stage == kStages2) {
+      if (++stage == stages2<W>()) {
         stage = 0;
         phase ^= 1;
       }
     }
     if (!ok) break;
-    if (lane == 0) ptx::mma_commit_pair_multicast(&s.acc_full[acc], 0x3);
-    __syncwarp();
-    if (++acc == 2) {
-      acc = 0;
-      acc_phase ^= 1;
+    if (lane == 0) {
+      ptx::mma_commit_pair_multicast(&s.acc_full[acc], 0x3);
+      if (two) ptx::mma_commit_pair_multicast(&s.acc_full[acc2], 0x3);
     }
+    if (lane == 0 && p.task_log != nullptr && task.id < p.task_log_cap) {
+      TaskRecord* r = p.task_log + task.id;
+      r->task = task.id;
+      r->unit = task.p;
+      r->expert = task.e;
+      r->phase_n = ((uint32_t)task.phase << 16) | (uint32_t)task.n;
+      r->smid = smid_u32();
+      r->cta = blockIdx.x;
+      r->t_first_mma = t_first;
+      r->t_last_mma = ptx::globaltimer();
+    }
+    __syncwarp();
+    for (int used = two ? 2 : 1; used > 0; --used)
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
   }
   issued_any = __any_sync(0xffffffffu, issued_any);
   if (issued_any) {
@@ -632,7 +704,7 @@ __device__ void gemm2_mma(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, ui
 }
 
 // ---------------------------------------------------------------- epilogue (warps 2..5 of both CTAs)
-template <bool F8>
+template <bool F8, bool W>
 __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem_base, uint32_t rank) {
   const int warp = threadIdx.x >> 5;
   const int lane = ptx::lane_id();
@@ -666,6 +738,76 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
       } else if (r < p.BM && bo >= 0) {   // the activation row's scale
         rscale = __ldcg(p.act_scale + ((task.p % p.ring_pairs) * 2 + (int)rank) * p.BM + r);
       }
+    }
+    auto next_acc = [&]() {
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    };
+    auto release_acc = [&]() {
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (is_leader) ptx::mbar_arrive(&s.acc_empty[acc]);
+        else ptx::mbar_arrive_peer(lead_acc_empty0 + 8 * acc);
+      }
+    };
+    if (W && !F8 && task.phase == 0) {
+      // wide L1 task: 256 columns of I in two accumulators (this slot, then the next), each
+      // released as soon as it is read, so the next task's MMAs start on the first one
+      const bool hf = task.half != 0;
+      const int hr = (quarter & 1) * 32 + lane, hc = quarter >> 1;   // half task: row and column half
+      const int b_own = hf ? task.b0 : (rank == 0 ? task.b0 : task.b1);
+      bool store = hf || (r < p.BM && b_own >= 0);
+      if (task.p >= p.ring_pairs) {
+        bool ok = true;
+        if (lane == 0) ok = wait_counter2(p.l2_done + (task.p - p.ring_pairs), p.N2, p, s, 0x40000 | task.p);
+        store = store && __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      }
+      const int ring_row = hf ? (task.p % p.ring_pairs) * 2 * p.BM + (int)rank * 64 + hr
+                              : ((task.p % p.ring_pairs) * 2 + (int)rank) * p.BM + r;
+      bool fine = true;
+      for (int sub = 0; sub < 2; ++sub) {
+        if (!warp_wait2(&s.acc_full[acc], acc_phase, p, s, 11)) {
+          fine = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t tb = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * 256;
+        const int n0 = task.n * 2 * kL1TileN + sub * kL1TileN;
+        float amax = 0.f;
+        if (hf) {   // g at TMEM columns 0..63, u at 64..127: columns 64*hc .. +63 of these 128
+          bf16* hrow = p.h + (size_t)ring_row * p.I + n0 + hc * 64;
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            uint32_t g[32], u[32];
+            ptx::tmem_ld32(tb + c * 32, g);
+            ptx::tmem_ld32(tb + 64 + c * 32, u);
+            ptx::tmem_ld_wait();
+            if (store) store_swiglu32(hrow + c * 32, g, u, amax);
+          }
+        } else {
+          bf16* hrow = p.h + (size_t)ring_row * p.I + n0;
+#pragma unroll 1
+          for (int c = 0; c < kL1TileN / 32; ++c) {
+            uint32_t g[32], u[32];
+            ptx::tmem_ld32(tb + c * 32, g);
+            ptx::tmem_ld32(tb + kL1TileN + c * 32, u);
+            ptx::tmem_ld_wait();
+            if (store) store_swiglu32(hrow + c * 32, g, u, amax);
+          }
+        }
+        release_acc();
+        next_acc();
+      }
+      if (!fine) break;
+      __threadfence();
+      __syncwarp();
+      if (lane == 0 && task.p != p.withhold_pair) ptx::red_release_gpu_add(p.l1_done + task.p, 1);
+      if (p.task_log != nullptr && is_leader && quarter == 0 && lane == 0 && task.id < p.task_log_cap)
+        p.task_log[task.id].t_done = ptx::globaltimer();
+      continue;
     }
     if (!warp_wait2(&s.acc_full[acc], acc_phase, p, s, 11)) break;
     ptx::tc_fence_after();
@@ -732,6 +874,8 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
                        }
                      });
       }
+      if (p.task_log != nullptr && is_leader && quarter == 0 && lane == 0 && task.id < p.task_log_cap)
+        p.task_log[task.id].t_done = ptx::globaltimer();
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
@@ -806,6 +950,8 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
                      }
                    });
     }
+    if (p.task_log != nullptr && is_leader && quarter == 0 && lane == 0 && task.id < p.task_log_cap)
+      p.task_log[task.id].t_done = ptx::globaltimer();
     if (++acc == 2) {
       acc = 0;
       acc_phase ^= 1;
@@ -814,7 +960,7 @@ __device__ void gemm2_epilogue(const Gemm2Params& p, Gemm2Smem& s, uint32_t tmem
 }
 
 // ---------------------------------------------------------------- gather warps (warps 6.. of both CTAs)
-template <bool F8>
+template <bool F8, bool W>
 __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles, int g, uint32_t rank) {
   constexpr int kRowsPerLane = (kTileM / 4 + kGatherWarps - 1) / kGatherWarps;
   const uint64_t wpol = ptx::policy_evict_first();
@@ -882,7 +1028,7 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
         ok = false;
         break;
       }
-      const uint32_t a_addr = ptx::smem_u32(stage2_ptr(tiles, stage));
+      const uint32_t a_addr = ptx::smem_u32(stage2_ptr<W>(tiles, stage));
 #pragma unroll
       for (int j = 0; j < kRowsPerLane; ++j)
         if (j < nrows) ptx::cp_async_16(a_addr + soff[j], src[j] + (size_t)kb * 128);
@@ -902,7 +1048,7 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
                               w2row8 + (size_t)wr * p.I + kb * 128 + wc * 16, wpol);
       }
       ptx::cp_async_mbar_arrive_noinc(&s.full[stage]);
-      if (++stage == kStages2) {
+      if (++stage == stages2<W>()) {
         stage = 0;
         phase ^= 1;
       }
@@ -912,18 +1058,18 @@ __device__ void gemm2_gather(const Gemm2Params& p, Gemm2Smem& s, uint8_t* tiles,
   ptx::cp_async_wait_all();
 }
 
-template <bool F8>
+template <bool F8, bool W>
 __global__ void __launch_bounds__(kGemm1Threads, 1) moe_expert_gemm2_kernel(const __grid_constant__ Gemm2Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Gemm2Smem& s = *reinterpret_cast<Gemm2Smem*>(tiles + (size_t)kStages2 * kStage2Bytes);
+  Gemm2Smem& s = *reinterpret_cast<Gemm2Smem*>(tiles + (size_t)stages2<W>() * stage2_bytes<W>());
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = ptx::cluster_ctarank();
   const bool is_leader = rank == 0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages2; ++i) {
+    for (int i = 0; i < stages2<W>(); ++i) {
       // leader: its producer, its gather lanes and the follower's relay; follower: its producer
       // (with its TMA bytes) and its gather lanes
       ptx::mbar_init(&s.full[i], is_leader ? 1 + 32 * kGatherWarps + 1 : 1 + 32 * kGatherWarps);
@@ -966,8 +1112,8 @@ __global__ void __launch_bounds__(kGemm1Threads, 1) moe_expert_gemm2_kernel(cons
     ptx::tmem_relinquish_pair();
   }
   if (p.BM < kTileM) {
-    for (int st = 0; st < kStages2; ++st) {
-      uint4* a = reinterpret_cast<uint4*>(stage2_ptr(tiles, st) + p.BM * 128);
+    for (int st = 0; st < stages2<W>(); ++st) {
+      uint4* a = reinterpret_cast<uint4*>(stage2_ptr<W>(tiles, st) + p.BM * 128);
       const int n = (kTileM - p.BM) * 128 / 16;
       for (int i = threadIdx.x; i < n; i += kGemm1Threads) a[i] = make_uint4(0, 0, 0, 0);
     }
@@ -980,17 +1126,17 @@ __global__ void __launch_bounds__(kGemm1Threads, 1) moe_expert_gemm2_kernel(cons
   const uint32_t tmem_base = s.tmem_base;
 
   if (warp == 0) {
-    if (is_leader) gemm2_leader_producer<F8>(p, s, tiles);
-    else gemm2_follower_producer<F8>(p, s, tiles);
+    if (is_leader) gemm2_leader_producer<F8, W>(p, s, tiles);
+    else gemm2_follower_producer<F8, W>(p, s, tiles);
   } else if (warp == 1) {
-    if (is_leader) gemm2_mma<F8>(p, s, tiles, tmem_base);
-    else gemm2_follower_relay<F8>(p, s);
+    if (is_leader) gemm2_mma<F8, W>(p, s, tiles, tmem_base);
+    else gemm2_follower_relay<F8, W>(p, s);
   } else if (warp < 6) {
-    gemm2_epilogue<F8>(p, s, tmem_base, rank);
+    gemm2_epilogue<F8, W>(p, s, tmem_base, rank);
   } else if (warp < 6 + kGatherWarps) {
-    gemm2_gather<F8>(p, s, tiles, warp - 6, rank);
+    gemm2_gather<F8, W>(p, s, tiles, warp - 6, rank);
   } else if (is_leader) {
-    gemm2_scheduler<F8>(p, s);
+    gemm2_scheduler<F8, W>(p, s);
   }
 
   ptx::tc_fence_before();

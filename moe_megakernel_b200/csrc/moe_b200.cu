@@ -34,7 +34,7 @@ struct Layout {
   size_t err, sched, topk_idx, topk_w, rank, chunk_count, expert_count, expert_offset, block_start, num_padded,
       slot_token, slot_topk, l1_done, l2_done, group_start, pair_start, router_partial, router_counter, h, y_acc,
       x_stage, y_stage, x_q, s_x, h8, act_amax, act_scale, bwd_dg, bwd_du, bwd_aw, bwd_dw, bwd_dl, bwd_wgt,
-      zero_row, total;
+      zero_row, task_log, total;
 };
 
 class DeviceGuard {
@@ -113,6 +113,8 @@ int block_m_rule(int T, int k, int E) {
 
 }  // namespace
 
+static_assert(sizeof(moe_task_record) == sizeof(TaskRecord), "the public task record is the kernels' record");
+
 struct moe_plan {
   int T_max, H, I, E, k, BM, device, num_sms;
   int S = 0;                                           // shared experts
@@ -121,11 +123,14 @@ struct moe_plan {
   bool cta_pairs = false;                              // run the expert GEMM on CTA pairs
   int task_order = -1;                                 // -1 automatic, 0 staggered, 1 interleaved
   bool half_tails = true;                              // pair kernel: lone last blocks as M = 128 pair MMAs
+  int wide_l1 = -1;                                    // pair kernel, bf16, I % 256 == 0: 256-column L1 tasks
+                                                       // (-1 automatic: when I <= 1024)
   int pair_clusters = 0;                               // co-resident clusters of the pair kernel
   int pgroup_min, pgroup_max, pmax_groups, ring_pairs; // the same in units of block pairs
   int per_expert;                                      // expected blocks per expert + 1
   int fp8_rows = 0;                                    // FP8 plans: activation rows of all blocks or pairs
   bool backward = false;                               // workspace holds the backward's regions
+  bool task_log = false;                               // workspace holds the expert GEMM's task log
   // pipelined host entry: its own copy streams, two staging buffers used in turn, and the events
   // that order each buffer's copy-in, forward and copy-out
   cudaStream_t cp_in = nullptr, cp_out = nullptr;
@@ -144,10 +149,21 @@ struct moe_plan {
 
 // CTA-pair mode: a task is a pair of consecutive blocks run by one cluster of
 // two CTAs, so there are pair_clusters concurrent tasks (groups and ring in pairs).
+// Wide L1 tasks measured 2.5 % faster on the skewed layer (I = 768: short first-GEMM tasks, whose
+// per-task costs halve) and 1.5-3 % slower where I is large (fine-grained, mixtral: the wide
+// variant's four 48 KB stages instead of six), so the automatic choice is I <= 1024.
+static bool wide_l1_active(const moe_plan& p) {
+  const bool want = p.wide_l1 > 0 || (p.wide_l1 < 0 && p.I <= 1024);
+  return want && p.I % (2 * kL1TileN) == 0;
+}
+
 static void size_pair_groups(moe_plan* p) {
   const int pairs_max = p->blocks_max;   // each pair holds at least one block
   const int clusters = std::max(1, p->pair_clusters > 0 ? p->pair_clusters : p->num_sms / 2);
-  p->pgroup_min = (2 * clusters + p->N1 - 1) / p->N1;
+  // L1 tasks per pair: I/256 with the wide L1 tasks (sized for them also when they are switched
+  // off later, which changes only the performance)
+  const int n1 = wide_l1_active(*p) ? p->I / (2 * kL1TileN) : p->N1;
+  p->pgroup_min = (2 * clusters + n1 - 1) / n1;
   p->pgroup_min = std::max(p->pgroup_min, (pairs_max + kMaxGroups - 3) / (kMaxGroups - 2));
   p->pgroup_max = std::max(2 * p->pgroup_min, (p->per_expert + 1) / 2);
   p->pmax_groups = pairs_max / p->pgroup_min + 2;
@@ -164,6 +180,9 @@ static int order_lag(const moe_plan& p) {
   if (!inter) return -1;
   return 2 * (p.cta_pairs ? std::max(1, p.pair_clusters) : p.num_sms);
 }
+
+// Records of the task log: every task of a launch (at most every block, or pair, times N1 + N2).
+static int task_log_capacity(const moe_plan& p) { return p.blocks_max * (p.N1 + p.N2); }
 
 static Layout make_layout(const moe_plan& p) {
   Layout L{};
@@ -215,6 +234,7 @@ static Layout make_layout(const moe_plan& p) {
   L.bwd_dw = take(p.backward ? (size_t)p.T_max * p.k * 4 : 0, 256);
   L.bwd_dl = take(p.backward ? (size_t)p.T_max * ((p.E + 63) / 64 * 64) * 2 : 0, 1024);
   L.bwd_wgt = take(p.backward ? (size_t)p.E * p.H * 2 : 0, 1024);
+  L.task_log = take(p.task_log ? (size_t)task_log_capacity(p) * sizeof(TaskRecord) : 0, 256);
   L.total = align_up(o, 1024);
   return L;
 }
@@ -465,20 +485,27 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     gp.k = p->k;
     gp.BM = p->BM;
     gp.BN2 = p->BN2;
-    gp.N1 = p->N1;
+    const bool wide = f8 == nullptr && wide_l1_active(*p);   // 256 columns of I per L1 task
+    gp.N1 = wide ? I / (2 * kL1TileN) : p->N1;
     gp.N2 = p->N2;
     gp.ring_pairs = f8 != nullptr ? p->fp8_rows / (2 * p->BM) : p->ring_pairs;   // FP8: every pair its own rows
     gp.max_groups = p->pmax_groups;
     gp.order_lag = order_lag(*p);
     gp.half_tails = (p->half_tails && f8 == nullptr && p->BM == kTileM) ? 1 : 0;   // bf16, 128-row blocks
     gp.zero_row = ws + L.zero_row;
+    if (p->task_log) {
+      gp.task_log = reinterpret_cast<TaskRecord*>(ws + L.task_log);
+      gp.task_log_cap = task_log_capacity(*p);
+      if (cudaMemsetAsync(gp.task_log, 0xFF, (size_t)gp.task_log_cap * sizeof(TaskRecord), st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
     gp.timeout_ns = p->timeout_ns;
     gp.withhold_pair = p->withhold;
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3((unsigned)(2 * p->pair_clusters));
     cfg.blockDim = dim3(kGemm1Threads);
-    cfg.dynamicSmemBytes = kGemm2SmemBytes;
+    cfg.dynamicSmemBytes = wide ? kGemm2SmemBytesW : kGemm2SmemBytes;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -487,7 +514,9 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    void (*kfn)(Gemm2Params) = f8 != nullptr ? moe_expert_gemm2_kernel<true> : moe_expert_gemm2_kernel<false>;
+    void (*kfn)(Gemm2Params) = f8 != nullptr ? moe_expert_gemm2_kernel<true, false>
+                               : wide       ? moe_expert_gemm2_kernel<false, true>
+                                            : moe_expert_gemm2_kernel<false, false>;
     if (cudaLaunchKernelEx(&cfg, kfn, gp) != cudaSuccess) return MOE_ERR_CUDA;
     if (f8 != nullptr) {
       if (!quantize_activation(dp.pair_start + E, 2 * p->BM)) return MOE_ERR_CUDA;
@@ -535,6 +564,12 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     gp.max_groups = p->max_groups;
     gp.order_lag = order_lag(*p);
     gp.zero_row = ws + L.zero_row;
+    if (p->task_log) {
+      gp.task_log = reinterpret_cast<TaskRecord*>(ws + L.task_log);
+      gp.task_log_cap = task_log_capacity(*p);
+      if (cudaMemsetAsync(gp.task_log, 0xFF, (size_t)gp.task_log_cap * sizeof(TaskRecord), st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
     gp.err = dp.err;
     gp.h = h;
     gp.y_acc = rp.y_acc;
@@ -794,10 +829,13 @@ int moe_plan_create_shared(moe_plan_t* out, int T_max, int H, int I, int E, int 
     ce = cudaFuncSetAttribute(moe_expert_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)kGemmSmemBytes);
   if (ce == cudaSuccess)
-    ce = cudaFuncSetAttribute(moe_expert_gemm2_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    ce = cudaFuncSetAttribute(moe_expert_gemm2_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)kGemm2SmemBytesW);
+  if (ce == cudaSuccess)
+    ce = cudaFuncSetAttribute(moe_expert_gemm2_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)kGemm2SmemBytes);
   if (ce == cudaSuccess)
-    ce = cudaFuncSetAttribute(moe_expert_gemm2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    ce = cudaFuncSetAttribute(moe_expert_gemm2_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)kGemm2SmemBytes);
   if (ce == cudaSuccess)
     ce = cudaFuncSetAttribute(moe_router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRtcSmemBytes);
@@ -841,7 +879,7 @@ int moe_plan_create_shared(moe_plan_t* out, int T_max, int H, int I, int E, int 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, moe_expert_gemm2_kernel<false>, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&clusters, moe_expert_gemm2_kernel<false, false>, &cfg) != cudaSuccess) {
       cudaGetLastError();
       clusters = 0;
     }
@@ -894,6 +932,7 @@ int moe_plan_describe(moe_plan_t p, moe_plan_desc* d) {
   d->workspace_bytes = p->L.total;
   d->task_order = order_lag(*p) >= 0 ? 1 : 0;
   d->half_tails = (p->cta_pairs && p->half_tails && p->BM == kTileM) ? 1 : 0;
+  d->wide_l1 = (p->cta_pairs && wide_l1_active(*p)) ? 1 : 0;
   return MOE_OK;
 }
 
@@ -1230,6 +1269,7 @@ int moe_backward(moe_plan_t p, const void* x, const void* Wg, const float* bias,
   bp.BM = p->BM;
   bp.pool = p->pool;
   bp.BN = (H % 256 == 0) ? 256 : 128;
+  bp.BNi = (I % 256 == 0) ? 256 : 128;
   bp.NE = NE;
   bp.timeout_ns = p->timeout_ns;
   const int grid = p->num_sms;
@@ -1259,7 +1299,7 @@ int moe_backward(moe_plan_t p, const void* x, const void* Wg, const float* bias,
   if (!make_map(&b3.tm_b, dg, I, p->pool, I, 64) || !make_map(&b3.tm_b2, du, I, p->pool, I, 64)) return MOE_ERR_CUDA;
   if (launch_bwd<kBwdWgrad13>(b3, grid, st) != cudaSuccess) return MOE_ERR_CUDA;
   BwdParams b4 = bp;
-  if (!make_map(&b4.tm_a, aw, I, p->pool, I, 64)) return MOE_ERR_CUDA;
+  if (!make_map(&b4.tm_b, aw, I, p->pool, I, 64)) return MOE_ERR_CUDA;
   if (launch_bwd<kBwdWgrad2>(b4, grid, st) != cudaSuccess) return MOE_ERR_CUDA;
   BwdParams b5 = bp;
   if (!make_map(&b5.tm_a, x, H, T, H, 64) || !make_map(&b5.tm_b, dl, NE, T, NE, 64)) return MOE_ERR_CUDA;
@@ -1277,6 +1317,30 @@ int moe_plan_set_cta_pairs(moe_plan_t p, int enable) {
 int moe_plan_set_task_order(moe_plan_t p, int mode) {
   if (p == nullptr || mode < -1 || mode > 1) return MOE_ERR_INVALID_ARG;
   p->task_order = mode;
+  return MOE_OK;
+}
+
+int moe_plan_set_task_log(moe_plan_t p, int enable) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  p->task_log = enable != 0;
+  p->L = make_layout(*p);
+  p->ws = nullptr;   // the workspace size changed: bind again
+  p->ws_bytes = 0;
+  return MOE_OK;
+}
+
+int moe_plan_get_task_log(moe_plan_t p, const moe_task_record** records, int* capacity) {
+  if (p == nullptr || records == nullptr || capacity == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!p->task_log) return MOE_ERR_INVALID_ARG;
+  if (p->ws == nullptr) return MOE_ERR_NO_WORKSPACE;
+  *records = reinterpret_cast<const moe_task_record*>(p->ws + p->L.task_log);
+  *capacity = task_log_capacity(*p);
+  return MOE_OK;
+}
+
+int moe_plan_set_wide_l1(moe_plan_t p, int mode) {
+  if (p == nullptr || mode < -1 || mode > 1) return MOE_ERR_INVALID_ARG;
+  p->wide_l1 = mode;
   return MOE_OK;
 }
 

@@ -135,3 +135,39 @@ def test_half_tail_tasks_match_oracle(T, H, I, E, k, zipf):
               f"rel_fro={fro:.2e} max_abs={mx:.2e}")
         ys.append(y.float())
     assert (ys[0] - ys[1]).abs().max().item() <= 2e-2
+
+
+WIDE_SHAPES = [
+    # T,    H,   I,   E,  k, zipf   (I % 256 == 0: wide first-GEMM tasks apply)
+    (1000, 256, 512, 8, 2, False),
+    (3000, 512, 768, 64, 8, True),
+    (4096, 128, 2048, 16, 2, False),   # H % 256 != 0 (L2 tile of 128 columns)
+    (2600, 384, 256, 16, 2, False),    # one wide task per pair (I = 256)
+]
+
+
+@pytest.mark.parametrize("T,H,I,E,k,zipf", WIDE_SHAPES)
+def test_wide_l1_tasks_match_oracle(T, H, I, E, k, zipf):
+    """256-column first-GEMM tasks (two N = 256 MMAs on one gathered x tile), with and without
+    half tail tasks, against 128-column tasks and the oracle."""
+    shape = custom_shape(T, H, I, E, k, zipf)
+    inp = make_inputs(shape, device=DEV)
+    ref = oracle_forward(inp, block_m=128)
+    ys = {}
+    for wide in (True, False):
+        for half in (True, False):
+            plan = _plan(shape, 128, True)
+            plan.set_wide_l1(wide)
+            plan.set_half_tails(half)
+            assert plan.wide_l1 == wide
+            plan.workspace.fill_(0xFF)
+            plan.lib.moe_plan_bind_workspace(plan._plan, plan.workspace.data_ptr(), plan.workspace_bytes)
+            y = plan.forward(inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"])
+            plan.check()
+            assert_routing_equal(plan.routing(T), ref)
+            fro, mx = assert_y_close(y, ref["y"], f"y (wide {wide}, half {half})")
+            print(f"wide={wide} half={half} T={T} H={H} I={I} E={E} k={k}: rel_fro={fro:.2e} max_abs={mx:.2e}")
+            ys[(wide, half)] = y.float()
+    base = ys[(False, False)]
+    for key, y in ys.items():
+        assert (y - base).abs().max().item() <= 2e-2, key

@@ -75,6 +75,9 @@ struct BwdParams {
   const bf16* x;                 // [T, H]
   const bf16* dy;                // [T, H]
   const bf16* zero_row;          // [H] zeros: the gathered row of a padding slot or a slot past the expert
+  int permuted;                  // 1: x and dy rows in slot order (tm_xp, tm_dyp) replace the gathers
+  CUtensorMap tm_xp;             // x rows in slot order [pool, H]: dgrad1 box {64, 128} (K-major A),
+  CUtensorMap tm_dyp;            // wgrad box {64, 64} (MN-major A); dy rows likewise
   // tensor maps (128-byte swizzle), per kind
   CUtensorMap tm_w1;   // dgrad1: W1 as [E*H, I], box {64, 64} (MN-major B); dgrad2: box {64, BNd} (K-major B)
   CUtensorMap tm_w3;   // the same for W3
@@ -229,15 +232,19 @@ __device__ void bwd_producer(const BwdParams& p, BwdSmem& s, uint8_t* tiles) {
         uint64_t* bar = &s.full[stage];
         if (Kind == kBwdDgrad1) {
           const int n0 = task.n * 128;
-          if (kb < p.H / 64) {   // W1 | W3 columns n0 .. n0+127, rows h of this K block (MN-major)
+          const bool second = kb >= p.H / 64;
+          // one arrival with every byte of the stage: B, and A when it comes by TMA
+          ptx::mbar_arrive_expect_tx(bar, (second ? 2 : 4) * kBoxBytes + (p.permuted ? kTileABytes : 0));
+          if (p.permuted)   // the block's x rows (first half of K) or dy rows (second half)
+            ptx::tma_load_2d(a, second ? &p.tm_dyp : &p.tm_xp, bar, (second ? kb - p.H / 64 : kb) * 64, task.b * p.BM,
+                             pol_n);
+          if (!second) {   // W1 | W3 columns n0 .. n0+127, rows h of this K block (MN-major)
             const int row = task.e * p.H + kb * 64;
-            ptx::mbar_arrive_expect_tx(bar, 4 * kBoxBytes);
             ptx::tma_load_2d(b, &p.tm_w1, bar, n0, row, pol_w);
             ptx::tma_load_2d(b + kBoxBytes, &p.tm_w1, bar, n0 + 64, row, pol_w);
             ptx::tma_load_2d(b + 2 * kBoxBytes, &p.tm_w3, bar, n0, row, pol_w);
             ptx::tma_load_2d(b + 3 * kBoxBytes, &p.tm_w3, bar, n0 + 64, row, pol_w);
-          } else {               // W2 rows i = n0 .. n0+127, K = h (K-major)
-            ptx::mbar_arrive_expect_tx(bar, 2 * kBoxBytes);
+          } else {         // W2 rows i = n0 .. n0+127, K = h (K-major)
             ptx::tma_load_2d(b, &p.tm_w2, bar, (kb - p.H / 64) * 64, task.e * p.I + n0, pol_w);
           }
         } else if (Kind == kBwdDgrad2) {
@@ -248,14 +255,22 @@ __device__ void bwd_producer(const BwdParams& p, BwdSmem& s, uint8_t* tiles) {
           ptx::tma_load_2d(b, second ? &p.tm_w3 : &p.tm_w1, bar, ki * 64, task.e * p.H + task.n * p.BN, pol_w);
         } else if (Kind == kBwdWgrad13) {
           const int s0 = s.block_start[task.e] * p.BM + kb * 64, n0 = task.n * 128;
-          ptx::mbar_arrive_expect_tx(bar, 4 * kBoxBytes);
+          ptx::mbar_arrive_expect_tx(bar, 4 * kBoxBytes + (p.permuted ? 2 * kBoxBytes : 0));
+          if (p.permuted) {   // x^T: 128 columns of x (2 MN-major boxes) of the slots
+            ptx::tma_load_2d(a, &p.tm_xp, bar, task.m * 128, s0, pol_n);
+            ptx::tma_load_2d(a + kBoxBytes, &p.tm_xp, bar, task.m * 128 + 64, s0, pol_n);
+          }
           ptx::tma_load_2d(b, &p.tm_b, bar, n0, s0, pol_n);
           ptx::tma_load_2d(b + kBoxBytes, &p.tm_b, bar, n0 + 64, s0, pol_n);
           ptx::tma_load_2d(b + 2 * kBoxBytes, &p.tm_b2, bar, n0, s0, pol_n);
           ptx::tma_load_2d(b + 3 * kBoxBytes, &p.tm_b2, bar, n0 + 64, s0, pol_n);
         } else if (Kind == kBwdWgrad2) {   // aw columns n0 .. n0+BNi-1 of the slots (MN-major B)
           const int s0 = s.block_start[task.e] * p.BM + kb * 64, n0 = task.n * p.BNi;
-          ptx::mbar_arrive_expect_tx(bar, (p.BNi / 64) * kBoxBytes);
+          ptx::mbar_arrive_expect_tx(bar, (p.BNi / 64) * kBoxBytes + (p.permuted ? 2 * kBoxBytes : 0));
+          if (p.permuted) {   // dy^T: 128 columns of dy (2 MN-major boxes) of the slots
+            ptx::tma_load_2d(a, &p.tm_dyp, bar, task.m * 128, s0, pol_n);
+            ptx::tma_load_2d(a + kBoxBytes, &p.tm_dyp, bar, task.m * 128 + 64, s0, pol_n);
+          }
           for (int j = 0; j < p.BNi / 64; ++j) ptx::tma_load_2d(b + j * kBoxBytes, &p.tm_b, bar, n0 + j * 64, s0, pol_n);
         } else {   // dwg: x^T (rows h) and dl (columns e), K = tokens
           const int m0 = task.m * 128;
@@ -299,7 +314,7 @@ __device__ void bwd_gather(const BwdParams& p, BwdSmem& s, uint8_t* tiles, int g
   bool ok = true;
   for (int t = blockIdx.x; t < ntasks && ok; t += gridDim.x) {
     const BwdTask task = bwd_decode<Kind>(t, p, s);
-    if (Kind == kBwdDgrad1) {
+    if (Kind == kBwdDgrad1 && !p.permuted) {
       // this lane's 8 rows of the block and its 16-byte column c (as in the forward's gather)
       const int c = lane & 7;
       int tok[8];
@@ -333,7 +348,7 @@ __device__ void bwd_gather(const BwdParams& p, BwdSmem& s, uint8_t* tiles, int g
           phase ^= 1;
         }
       }
-    } else if (Kind == kBwdWgrad13 || Kind == kBwdWgrad2) {
+    } else if ((Kind == kBwdWgrad13 || Kind == kBwdWgrad2) && !p.permuted) {
       const int s_begin = s.block_start[task.e] * p.BM;
       const int s_end = s.block_start[task.e + 1] * p.BM;
       // the A operand, 64 slot rows x 16 chunks (128 columns of H) of x (wgrad13) or dy (wgrad2).
@@ -768,6 +783,36 @@ __global__ void __launch_bounds__(kGateThreads) moe_gate_backward_kernel(
   if (dbias != nullptr)
     for (int e = threadIdx.x; e < E; e += kGateThreads)
       if (s_bias[e] != 0.f) atomicAdd(dbias + e, s_bias[e]);
+}
+
+// Rows of x and dy in slot order for the backward's TMA operands: xp[s] = x[t], dyp[s] = dy[t]
+// for slot s with token t, zeros for padding slots and for the 64 rows after the last used
+// slot (a weight-gradient K block of 64 slots may reach past the pool's last expert). One
+// warp per row, 16 bytes per lane per step.
+__global__ void __launch_bounds__(256) moe_permute_rows_kernel(const bf16* __restrict__ x, const bf16* __restrict__ dy,
+                                                               const int32_t* __restrict__ slot_token,
+                                                               const int32_t* __restrict__ nblocks, bf16* __restrict__ xp,
+                                                               bf16* __restrict__ dyp, int32_t* err, int T, int H, int BM,
+                                                               int pool) {
+  const int rows = min(*nblocks * BM + 64, pool);
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  for (int sl = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; sl < rows; sl += warps) {
+    int t = sl < *nblocks * BM ? slot_token[sl] : -1;
+    if (t >= T) {
+      atomicCAS(err, 0, kDevBounds);
+      t = -1;
+    }
+    const uint4* xs = reinterpret_cast<const uint4*>(x + (size_t)(t < 0 ? 0 : t) * H);
+    const uint4* ds = reinterpret_cast<const uint4*>(dy + (size_t)(t < 0 ? 0 : t) * H);
+    uint4* xo = reinterpret_cast<uint4*>(xp + (size_t)sl * H);
+    uint4* dout = reinterpret_cast<uint4*>(dyp + (size_t)sl * H);
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    for (int i = lane; i < H / 8; i += 32) {
+      xo[i] = t < 0 ? z : __ldg(xs + i);
+      dout[i] = t < 0 ? z : __ldg(ds + i);
+    }
+  }
 }
 
 // WgT[e][h] = Wg[h][e] (32 x 32 tiles through shared memory).

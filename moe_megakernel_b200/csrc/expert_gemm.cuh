@@ -67,7 +67,7 @@ struct GemmParams {
   // FP8 E4M3 expert GEMMs (the kernel's FP8 instance): x codes [T, H] with per-token scales,
   // W1/W3 codes K-major [E, I, H] with column scales [E, I], W2 codes K-major
   // [E, H, I] with column scales [E, H] (tensor maps above). The two GEMMs run
-  // as two launches (phase_only 0, then 1) around the activation quantizer:
+  // as two launches per block group (phase_only 0, then 1) around the activation quantizer:
   // the first stores the bf16 activation in h and raises act_amax of its row
   // (zero before the launch) to the row's largest |h|; the quantizer writes
   // the row's codes to h8 and its scale to act_scale; the second reads them.
@@ -80,6 +80,7 @@ struct GemmParams {
   const float* act_scale;    // [h rows]
   const uint8_t* h8;         // [h rows, I]
   int phase_only;            // -1: both phases in one launch; 0: first GEMM only; 1: second GEMM only
+  int only_group;            // with phase_only >= 0: the block group whose tasks this launch runs
   int ring_blocks;              // block b uses ring slot b % ring_blocks
   int max_groups;
   int order_lag;                // task order (see locate_task): -1 staggered, >= 0 interleaved after this lag
@@ -239,10 +240,18 @@ __device__ __forceinline__ Task decode_task(int t, const GemmSmem& s, const Gemm
   const int G = s.num_groups;
   const int nb_total = s.block_start[p.E + p.S];
   // one-phase launches (a single block group): the second GEMM's tasks follow the first's
-  if (p.phase_only == 1) t += nb_total * p.N1;
-  else if (p.phase_only == 0 && t >= nb_total * p.N1) return task;
-  if (t < 0 || t >= nb_total * (p.N1 + p.N2) || G <= 0) return task;
-  const TaskPos pos = locate_task(t, s.group_start, G, p.N1, p.N2, p.phase_only >= 0 ? -1 : p.order_lag);
+  TaskPos pos;
+  if (p.phase_only >= 0) {
+    // one GEMM of one block group (the FP8 forward's launches): its tasks in order
+    const int g = p.only_group;
+    if (g < 0 || g >= G) return task;
+    const int NT = p.phase_only == 0 ? p.N1 : p.N2;
+    if (t < 0 || t >= (s.group_start[g + 1] - s.group_start[g]) * NT) return task;
+    pos = TaskPos{p.phase_only, g, t};
+  } else {
+    if (t < 0 || t >= nb_total * (p.N1 + p.N2) || G <= 0) return task;
+    pos = locate_task(t, s.group_start, G, p.N1, p.N2, p.order_lag);
+  }
   task.phase = pos.phase;
   const int g = pos.g, NT = pos.phase == 0 ? p.N1 : p.N2;
   const int gb0 = s.group_start[g], gb1 = s.group_start[g + 1];

@@ -93,6 +93,7 @@ struct Gemm2Params {
   const float* act_scale;  // FP8: [h rows] row scale written by the activation quantizer
   const uint8_t* h8;       // FP8: [h rows, I] activation codes
   int phase_only;          // -1: both phases; 0: first GEMM only; 1: second GEMM only
+  int only_group;          // with phase_only >= 0: the block group whose tasks this launch runs
   int ring_pairs, max_groups;
   int order_lag;                // task order (locate_task in expert_gemm.cuh): -1 staggered, >= 0 interleaved
   int half_tails;               // 1: an expert's lone last block runs as an M = 128 pair MMA (bf16, BM = 128)
@@ -222,10 +223,18 @@ __device__ __forceinline__ Task2 decode_task2(int t, const Gemm2Smem& s, const G
   const int G = s.num_groups;
   const int np_total = s.pair_start[p.E + p.S];
   // one-phase launches (a single block group): the second GEMM's tasks follow the first's
-  if (p.phase_only == 1) t += np_total * p.N1;
-  else if (p.phase_only == 0 && t >= np_total * p.N1) return task;
-  if (t < 0 || t >= np_total * (p.N1 + p.N2) || G <= 0) return task;
-  const TaskPos pos = locate_task(t, s.group_start, G, p.N1, p.N2, p.phase_only >= 0 ? -1 : p.order_lag);
+  TaskPos pos;
+  if (p.phase_only >= 0) {
+    // one GEMM of one block group (the FP8 forward's launches): its tasks in order
+    const int g = p.only_group;
+    if (g < 0 || g >= G) return task;
+    const int NT = p.phase_only == 0 ? p.N1 : p.N2;
+    if (t < 0 || t >= (s.group_start[g + 1] - s.group_start[g]) * NT) return task;
+    pos = TaskPos{p.phase_only, g, t};
+  } else {
+    if (t < 0 || t >= np_total * (p.N1 + p.N2) || G <= 0) return task;
+    pos = locate_task(t, s.group_start, G, p.N1, p.N2, p.order_lag);
+  }
   task.phase = pos.phase;
   const int g = pos.g, NT = pos.phase == 0 ? p.N1 : p.N2;
   const int gp0 = s.group_start[g], gp1 = s.group_start[g + 1];

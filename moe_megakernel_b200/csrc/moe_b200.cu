@@ -34,7 +34,7 @@ struct Layout {
   size_t err, sched, topk_idx, topk_w, rank, chunk_count, expert_count, expert_offset, block_start, num_padded,
       slot_token, slot_topk, l1_done, l2_done, group_start, pair_start, router_partial, router_counter, h, y_acc,
       x_stage, y_stage, x_q, s_x, h8, act_amax, act_scale, bwd_dg, bwd_du, bwd_aw, bwd_dw, bwd_dl, bwd_wgt,
-      zero_row, task_log, total;
+      zero_row, task_log, bwd_xp, bwd_dyp, total;
 };
 
 class DeviceGuard {
@@ -128,7 +128,7 @@ struct moe_plan {
   int pair_clusters = 0;                               // co-resident clusters of the pair kernel
   int pgroup_min, pgroup_max, pmax_groups, ring_pairs; // the same in units of block pairs
   int per_expert;                                      // expected blocks per expert + 1
-  int fp8_rows = 0;                                    // FP8 plans: activation rows of all blocks or pairs
+  int fp8_rows = 0;                                    // FP8 plans: activation rows of one block group
   bool backward = false;                               // workspace holds the backward's regions
   bool task_log = false;                               // workspace holds the expert GEMM's task log
   // pipelined host entry: its own copy streams, two staging buffers used in turn, and the events
@@ -180,6 +180,8 @@ static int order_lag(const moe_plan& p) {
   if (!inter) return -1;
   return 2 * (p.cta_pairs ? std::max(1, p.pair_clusters) : p.num_sms);
 }
+
+static bool backward_permuted(const moe_plan& p) { return p.backward && p.BM >= 64; }
 
 // Records of the task log: every task of a launch (at most every block, or pair, times N1 + N2).
 static int task_log_capacity(const moe_plan& p) { return p.blocks_max * (p.N1 + p.N2); }
@@ -234,6 +236,11 @@ static Layout make_layout(const moe_plan& p) {
   L.bwd_dw = take(p.backward ? (size_t)p.T_max * p.k * 4 : 0, 256);
   L.bwd_dl = take(p.backward ? (size_t)p.T_max * ((p.E + 63) / 64 * 64) * 2 : 0, 1024);
   L.bwd_wgt = take(p.backward ? (size_t)p.E * p.H * 2 : 0, 1024);
+  // x and dy rows in slot order [pool, H] bf16 each, when BLOCK_M >= 64 (no 64-slot K block of the
+  // weight gradients crosses an expert, so the rows can come by TMA); else the kernels gather them
+  const size_t bperm = backward_permuted(p) ? (size_t)p.pool * p.H * 2 : 0;
+  L.bwd_xp = take(bperm, 1024);
+  L.bwd_dyp = take(bperm, 1024);
   L.task_log = take(p.task_log ? (size_t)task_log_capacity(p) * sizeof(TaskRecord) : 0, 256);
   L.total = align_up(o, 1024);
   return L;
@@ -403,8 +410,13 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   dp.pair_start = p->cta_pairs ? reinterpret_cast<int32_t*>(ws + L.pair_start) : nullptr;
   dp.group_min = p->cta_pairs ? p->pgroup_min : p->group_min;
   dp.group_max = p->cta_pairs ? p->pgroup_max : p->group_max;
-  if (f8 != nullptr) dp.group_min = dp.group_max = 1 << 30;   // FP8: one block group (two one-phase launches)
   dp.max_groups = p->cta_pairs ? p->pmax_groups : p->max_groups;
+  if (f8 != nullptr) {
+    // FP8: groups of exactly the units whose activation the buffer holds, run one after another
+    const int units = std::max(1, p->fp8_rows / (p->cta_pairs ? 2 * p->BM : p->BM));
+    dp.group_min = dp.group_max = units;
+    dp.max_groups = std::min(kMaxGroups, p->blocks_max / units + 2);
+  }
   mark(1);
   moe_dispatch_scan_kernel<<<1, kScanThreads, 0, st>>>(dp);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
@@ -431,12 +443,18 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
   float* act_scale = reinterpret_cast<float*>(ws + L.act_scale);
   uint8_t* h8 = ws + L.h8;
   const int h8_rows = p->fp8_rows;
-  if (f8 != nullptr && cudaMemsetAsync(act_amax, 0, (size_t)h8_rows * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
-  // between the two FP8 launches: quantize the activation rows, restart the task counter
-  auto quantize_activation = [&](const int32_t* units, int unit_rows) -> bool {
+  // FP8: per block group (groups of fp8_units units, each the rows the buffer holds), the
+  // first GEMM alone, the activation quantizer over the group's rows, the second GEMM alone;
+  // the task counter restarts before each launch, the row amaxes before each group
+  const int unit_rows = p->cta_pairs ? 2 * p->BM : p->BM;
+  const int fp8_units = std::max(1, h8_rows / unit_rows);
+  const int fp8_groups = (p->blocks_max + fp8_units - 1) / fp8_units;   // enough for any routing
+  auto restart_counter = [&]() { return cudaMemsetAsync(dp.sched, 0, 4, st) == cudaSuccess; };
+  auto quantize_group = [&](int g) -> bool {
     const int grid = p->num_sms * 8;
-    moe_quantize_act_kernel<<<grid, 256, 0, st>>>(h, act_amax, h8, act_scale, units, unit_rows, h8_rows, I);
-    return cudaGetLastError() == cudaSuccess && cudaMemsetAsync(dp.sched, 0, 4, st) == cudaSuccess;
+    moe_quantize_act_kernel<<<grid, 256, 0, st>>>(h, act_amax, h8, act_scale, dp.group_start, dp.sched + 3, g,
+                                                  fp8_units, unit_rows, I);
+    return cudaGetLastError() == cudaSuccess && restart_counter();
   };
   if (p->cta_pairs) {
     Gemm2Params gp;
@@ -488,7 +506,7 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     const bool wide = f8 == nullptr && wide_l1_active(*p);   // 256 columns of I per L1 task
     gp.N1 = wide ? I / (2 * kL1TileN) : p->N1;
     gp.N2 = p->N2;
-    gp.ring_pairs = f8 != nullptr ? p->fp8_rows / (2 * p->BM) : p->ring_pairs;   // FP8: every pair its own rows
+    gp.ring_pairs = f8 != nullptr ? fp8_units : p->ring_pairs;   // FP8: a group's pairs, each its own rows
     gp.max_groups = p->pmax_groups;
     gp.order_lag = order_lag(*p);
     gp.half_tails = (p->half_tails && f8 == nullptr && p->BM == kTileM) ? 1 : 0;   // bf16, 128-row blocks
@@ -517,11 +535,18 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     void (*kfn)(Gemm2Params) = f8 != nullptr ? moe_expert_gemm2_kernel<true, false>
                                : wide       ? moe_expert_gemm2_kernel<false, true>
                                             : moe_expert_gemm2_kernel<false, false>;
-    if (cudaLaunchKernelEx(&cfg, kfn, gp) != cudaSuccess) return MOE_ERR_CUDA;
-    if (f8 != nullptr) {
-      if (!quantize_activation(dp.pair_start + E, 2 * p->BM)) return MOE_ERR_CUDA;
-      gp.phase_only = 1;
+    if (f8 == nullptr) {
       if (cudaLaunchKernelEx(&cfg, kfn, gp) != cudaSuccess) return MOE_ERR_CUDA;
+    } else {
+      for (int g = 0; g < fp8_groups; ++g) {   // groups past the routing's last exit at once
+        gp.only_group = g;
+        gp.phase_only = 0;
+        if (cudaMemsetAsync(act_amax, 0, (size_t)h8_rows * 4, st) != cudaSuccess ||
+            cudaLaunchKernelEx(&cfg, kfn, gp) != cudaSuccess || !restart_counter() || !quantize_group(g))
+          return MOE_ERR_CUDA;
+        gp.phase_only = 1;
+        if (cudaLaunchKernelEx(&cfg, kfn, gp) != cudaSuccess || !restart_counter()) return MOE_ERR_CUDA;
+      }
     }
   } else {
     GemmParams gp;
@@ -560,7 +585,7 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     gp.task_counter = dp.sched;
     gp.l1_done = dp.l1_done;
     gp.l2_done = dp.l2_done;
-    gp.ring_blocks = f8 != nullptr ? p->fp8_rows / p->BM : p->ring_blocks;   // FP8: every block its own rows
+    gp.ring_blocks = f8 != nullptr ? fp8_units : p->ring_blocks;   // FP8: a group's blocks, each its own rows
     gp.max_groups = p->max_groups;
     gp.order_lag = order_lag(*p);
     gp.zero_row = ws + L.zero_row;
@@ -585,12 +610,19 @@ static int enqueue(moe_plan* p, const void* x, const void* Wg, const float* bias
     gp.timeout_ns = p->timeout_ns;
     gp.withhold_block = p->withhold;
     void (*kfn)(GemmParams) = f8 != nullptr ? moe_expert_gemm_kernel<true> : moe_expert_gemm_kernel<false>;
-    kfn<<<p->num_sms, kGemm1Threads, kGemmSmemBytes, st>>>(gp);
-    if (f8 != nullptr) {
-      if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
-      if (!quantize_activation(dp.sched + 1, p->BM)) return MOE_ERR_CUDA;
-      gp.phase_only = 1;
+    if (f8 == nullptr) {
       kfn<<<p->num_sms, kGemm1Threads, kGemmSmemBytes, st>>>(gp);
+    } else {
+      for (int g = 0; g < fp8_groups; ++g) {
+        gp.only_group = g;
+        gp.phase_only = 0;
+        if (cudaMemsetAsync(act_amax, 0, (size_t)h8_rows * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+        kfn<<<p->num_sms, kGemm1Threads, kGemmSmemBytes, st>>>(gp);
+        if (cudaGetLastError() != cudaSuccess || !restart_counter() || !quantize_group(g)) return MOE_ERR_CUDA;
+        gp.phase_only = 1;
+        kfn<<<p->num_sms, kGemm1Threads, kGemmSmemBytes, st>>>(gp);
+        if (cudaGetLastError() != cudaSuccess || !restart_counter()) return MOE_ERR_CUDA;
+      }
     }
   }
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
@@ -1190,9 +1222,16 @@ int moe_plan_set_debug(moe_plan_t p, int withhold_block, uint64_t timeout_ns) {
 int moe_plan_set_fp8(moe_plan_t p, int enable) {
   if (p == nullptr) return MOE_ERR_INVALID_ARG;
   if (enable && p->S > 0) return MOE_ERR_UNSUPPORTED_SHAPE;
-  // every block, or every pair of blocks of one expert (at most one half-empty pair per expert)
+  // The activation rows of one block group (bf16 and codes, I * 3 + 8 bytes a row): up to
+  // 256 MB, at least two rows per concurrent task slot of either kernel (a pair: 2 * BLOCK_M
+  // rows per cluster; one CTA: BLOCK_M), at most every block's (or pair's) rows, in whole pairs.
   const int pairs_cap = std::min(p->blocks_max, (p->blocks_max + p->E + 1) / 2);
-  p->fp8_rows = enable ? std::max(p->blocks_max, 2 * pairs_cap) * p->BM : 0;
+  const long long all_rows = (long long)std::max(p->blocks_max, 2 * pairs_cap) * p->BM;
+  const long long budget = (256LL << 20) / ((long long)p->I * 3 + 8);
+  const long long floor_rows = 2LL * std::max(2 * std::max(p->pair_clusters, 1), p->num_sms) * p->BM;
+  long long rows = std::min(all_rows, std::max(budget, floor_rows));
+  rows = std::max(2LL * p->BM, rows / (2 * p->BM) * (2 * p->BM));
+  p->fp8_rows = enable ? (int)rows : 0;
   p->L = make_layout(*p);
   p->ws = nullptr;   // the workspace size changed: bind again
   p->ws_bytes = 0;
@@ -1273,11 +1312,22 @@ int moe_backward(moe_plan_t p, const void* x, const void* Wg, const float* bias,
   bp.NE = NE;
   bp.timeout_ns = p->timeout_ns;
   const int grid = p->num_sms;
+  bf16* xp = reinterpret_cast<bf16*>(ws + L.bwd_xp);
+  bf16* dyp = reinterpret_cast<bf16*>(ws + L.bwd_dyp);
+  bp.permuted = backward_permuted(*p) ? 1 : 0;
+  if (bp.permuted) {
+    // x and dy rows in slot order (their operands then come by TMA)
+    moe_permute_rows_kernel<<<p->num_sms * 8, 256, 0, st>>>(static_cast<const bf16*>(x), static_cast<const bf16*>(dy),
+                                                         bp.slot_token, bp.sched, xp, dyp, bp.err, T, H, p->BM, p->pool);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  }
 
   // 1. dgrad-1: g|u recomputed, da = dy W2^T; dg, du, w*a per slot; dw
   BwdParams b1 = bp;
   if (!make_map(&b1.tm_w1, W1, I, (uint64_t)E * H, I, 64) || !make_map(&b1.tm_w3, W3, I, (uint64_t)E * H, I, 64) ||
       !make_map(&b1.tm_w2, W2, H, (uint64_t)E * I, H, 128))
+    return MOE_ERR_CUDA;
+  if (bp.permuted && (!make_map(&b1.tm_xp, xp, H, p->pool, H, 128) || !make_map(&b1.tm_dyp, dyp, H, p->pool, H, 128)))
     return MOE_ERR_CUDA;
   if (launch_bwd<kBwdDgrad1>(b1, grid, st) != cudaSuccess) return MOE_ERR_CUDA;
   // 2. dgrad-2: dx += [dg|du] [W1|W3]^T through the slot records
@@ -1297,9 +1347,11 @@ int moe_backward(moe_plan_t p, const void* x, const void* Wg, const float* bias,
   // 4. weight gradients: dW1 = x^T dg, dW3 = x^T du; dW2 = (w a)^T dy; dWg = x^T dl
   BwdParams b3 = bp;
   if (!make_map(&b3.tm_b, dg, I, p->pool, I, 64) || !make_map(&b3.tm_b2, du, I, p->pool, I, 64)) return MOE_ERR_CUDA;
+  if (bp.permuted && !make_map(&b3.tm_xp, xp, H, p->pool, H, 64)) return MOE_ERR_CUDA;
   if (launch_bwd<kBwdWgrad13>(b3, grid, st) != cudaSuccess) return MOE_ERR_CUDA;
   BwdParams b4 = bp;
   if (!make_map(&b4.tm_b, aw, I, p->pool, I, 64)) return MOE_ERR_CUDA;
+  if (bp.permuted && !make_map(&b4.tm_dyp, dyp, H, p->pool, H, 64)) return MOE_ERR_CUDA;
   if (launch_bwd<kBwdWgrad2>(b4, grid, st) != cudaSuccess) return MOE_ERR_CUDA;
   BwdParams b5 = bp;
   if (!make_map(&b5.tm_a, x, H, T, H, 64) || !make_map(&b5.tm_b, dl, NE, T, NE, 64)) return MOE_ERR_CUDA;

@@ -78,12 +78,18 @@ __global__ void __launch_bounds__(256) moe_quantize_x_kernel(const bf16* __restr
 __global__ void __launch_bounds__(256) moe_quantize_act_kernel(const bf16* __restrict__ h,
                                                                const float* __restrict__ act_amax,
                                                                uint8_t* __restrict__ h8, float* __restrict__ act_scale,
-                                                               const int32_t* __restrict__ units, int unit_rows,
-                                                               int max_rows, int I) {
-  const int nrows = min(*units * unit_rows, max_rows);
+                                                               const int32_t* __restrict__ group_start,
+                                                               const int32_t* __restrict__ num_groups, int group,
+                                                               int ring_units, int unit_rows, int I) {
+  // the rows of block group `group`: its units (blocks, or block pairs) u map to buffer slot u % ring_units
+  if (group >= *num_groups) return;
+  const int u0 = group_start[group], u1 = group_start[group + 1];
+  if (u1 - u0 > ring_units) return;   // never: the host sizes the groups to the buffer
+  const int nrows = (u1 - u0) * unit_rows;
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (blockDim.x >> 5);
-  for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < nrows; row += warps) {
+  for (int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < nrows; i += warps) {
+    const int row = ((u0 + i / unit_rows) % ring_units) * unit_rows + i % unit_rows;
     const int k = pow2_scale_exp(__ldcg(act_amax + row));
     const float inv = ldexpf(1.f, -k);
     if (lane == 0) act_scale[row] = ldexpf(1.f, k);

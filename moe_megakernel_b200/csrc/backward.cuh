@@ -505,12 +505,22 @@ __device__ __forceinline__ void store_bf16x32(bf16* dst, const float (&v)[32]) {
 }
 
 // ---------------------------------------------------------------- warps 2..5: epilogue
+// With the operands by TMA (p.permuted), the four gather warps have nothing to copy; for
+// dgrad-1 and dW1/dW3 they become a second set of epilogue warps: the warp of each TMEM lane
+// quarter in warps 2-5 takes the first half of the accumulator's columns, the one in 6-9 the
+// second half.
 template <int Kind>
-__device__ void bwd_epilogue(const BwdParams& p, BwdSmem& s, uint32_t tmem_base) {
+__device__ __forceinline__ bool bwd_helpers(const BwdParams& p) {
+  return p.permuted && (Kind == kBwdDgrad1 || Kind == kBwdWgrad13);
+}
+
+template <int Kind>
+__device__ void bwd_epilogue(const BwdParams& p, BwdSmem& s, uint32_t tmem_base, int half) {
   const int warp = threadIdx.x >> 5;
   const int lane = ptx::lane_id();
   const int quarter = warp & 3;
   const int r = quarter * 32 + lane;   // accumulator row (TMEM lane) of this thread
+  const bool split = bwd_helpers<Kind>(p);   // columns split between this warp and its helper
   const int ntasks = bwd_num_tasks<Kind>(p, s);
   constexpr int kAccs = Kind == kBwdDgrad1 ? 1 : 2;
   int acc = 0;
@@ -547,9 +557,10 @@ __device__ void bwd_epilogue(const BwdParams& p, BwdSmem& s, uint32_t tmem_base)
         }
       }
       const int n0 = task.n * 128;
-      float dwp = 0.f;   // sum over this tile's columns of a_i * da~_i
+      float dwp = 0.f;   // sum over this warp's columns of a_i * da~_i
+      const int c0 = split ? 2 * half : 0, c1 = split ? c0 + 2 : 4;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = c0; c < c1; ++c) {
         uint32_t g[32], u[32], v[32];
         ptx::tmem_ld32(tb + c * 32, g);
         ptx::tmem_ld32(tb + 128 + c * 32, u);
@@ -596,8 +607,9 @@ __device__ void bwd_epilogue(const BwdParams& p, BwdSmem& s, uint32_t tmem_base)
     } else {
       // weight-gradient tiles: row r of the tile, ncols columns, bf16 (fp32 for dWg)
       const int ncols = Kind == kBwdWgrad13 ? 256 : Kind == kBwdWgrad2 ? p.BNi : p.NE;
+      const int c0 = split ? half * (ncols / 64) : 0, c1 = split ? c0 + ncols / 64 : ncols / 32;
 #pragma unroll 1
-      for (int c = 0; c < ncols / 32; ++c) {
+      for (int c = c0; c < c1; ++c) {
         float f[32];
         if (has_acc) {
           uint32_t v[32];
@@ -649,14 +661,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) moe_backward_gemm_kernel(const
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   BwdSmem& s = *reinterpret_cast<BwdSmem*>(tiles + (size_t)kBwdStages * kBwdStageBytes);
   const int warp = threadIdx.x >> 5;
+  const bool helpers = bwd_helpers<Kind>(p);
   if (threadIdx.x == 0) {
     for (int i = 0; i < kBwdStages; ++i) {
-      ptx::mbar_init(&s.full[i], 1 + 32 * kBwdGatherWarps);   // producer + every gather lane
+      // producer + every gather lane (with helper epilogue warps: the producer alone)
+      ptx::mbar_init(&s.full[i], helpers ? 1 : 1 + 32 * kBwdGatherWarps);
       ptx::mbar_init(&s.empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&s.acc_full[i], 1);
-      ptx::mbar_init(&s.acc_empty[i], 4);
+      ptx::mbar_init(&s.acc_empty[i], helpers ? 8 : 4);   // every epilogue warp releases the accumulator
     }
     ptx::mbar_init(&s.mma_done, 1);
     s.abort = 0;
@@ -697,7 +711,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) moe_backward_gemm_kernel(const
   if (!*reinterpret_cast<volatile int*>(&s.abort)) {
     if (warp == 0) bwd_producer<Kind>(p, s, tiles);
     else if (warp == 1) bwd_mma<Kind>(p, s, tiles, tmem_base);
-    else if (warp < 6) bwd_epilogue<Kind>(p, s, tmem_base);
+    else if (warp < 6) bwd_epilogue<Kind>(p, s, tmem_base, 0);
+    else if (helpers) bwd_epilogue<Kind>(p, s, tmem_base, 1);
     else bwd_gather<Kind>(p, s, tiles, warp - 6);
   }
   ptx::tc_fence_before();

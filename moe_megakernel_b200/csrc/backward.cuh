@@ -17,8 +17,11 @@
 // TMEM accumulator; per slot s of expert e with token t, top-k position j
 // and weight w = topk_w[t,j]:
 //
-//   kDgrad1  (block, 128 columns n of I): g|u = x_t [W1|W3][e] (K = H, as the
-//            forward's first GEMM) and da~ = dy_t W2[e]^T (K = H); epilogue:
+//   kDgrad1  (block, 128 columns n of I): da~ = dy_t W2[e]^T (K = H, first, into
+//            one of two 128-column TMEM slots used in turn) and g|u =
+//            x_t [W1|W3][e] (K = H, as the forward's first GEMM, into columns
+//            0-255), so that a task's da~ loop overlaps the previous task's
+//            epilogue; epilogue:
 //            a = bf16(silu(g) u), da = w da~, dg = da u silu'(g),
 //            du = da silu(g); stores dg, du and aw = bf16(w a) per slot, and
 //            adds sum_i a_i da~_i (= dy_t . o) into dw[t,j];
@@ -111,6 +114,7 @@ struct BwdSmem {
   uint64_t empty[kBwdStages];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
+  uint64_t da_empty[2];         // dgrad1: the two da slots (TMEM columns 256.., 384..) are free
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
@@ -232,20 +236,20 @@ __device__ void bwd_producer(const BwdParams& p, BwdSmem& s, uint8_t* tiles) {
         uint64_t* bar = &s.full[stage];
         if (Kind == kBwdDgrad1) {
           const int n0 = task.n * 128;
-          const bool second = kb >= p.H / 64;
+          const bool da_part = kb < p.H / 64;   // dy W2^T first, then x [W1 | W3]
+          const int kh = (da_part ? kb : kb - p.H / 64) * 64;
           // one arrival with every byte of the stage: B, and A when it comes by TMA
-          ptx::mbar_arrive_expect_tx(bar, (second ? 2 : 4) * kBoxBytes + (p.permuted ? kTileABytes : 0));
-          if (p.permuted)   // the block's x rows (first half of K) or dy rows (second half)
-            ptx::tma_load_2d(a, second ? &p.tm_dyp : &p.tm_xp, bar, (second ? kb - p.H / 64 : kb) * 64, task.b * p.BM,
-                             pol_n);
-          if (!second) {   // W1 | W3 columns n0 .. n0+127, rows h of this K block (MN-major)
-            const int row = task.e * p.H + kb * 64;
+          ptx::mbar_arrive_expect_tx(bar, (da_part ? 2 : 4) * kBoxBytes + (p.permuted ? kTileABytes : 0));
+          if (p.permuted)   // the block's dy rows (first half of K) or x rows (second half)
+            ptx::tma_load_2d(a, da_part ? &p.tm_dyp : &p.tm_xp, bar, kh, task.b * p.BM, pol_n);
+          if (da_part) {   // W2 rows i = n0 .. n0+127, K = h (K-major)
+            ptx::tma_load_2d(b, &p.tm_w2, bar, kh, task.e * p.I + n0, pol_w);
+          } else {         // W1 | W3 columns n0 .. n0+127, rows h of this K block (MN-major)
+            const int row = task.e * p.H + kh;
             ptx::tma_load_2d(b, &p.tm_w1, bar, n0, row, pol_w);
             ptx::tma_load_2d(b + kBoxBytes, &p.tm_w1, bar, n0 + 64, row, pol_w);
             ptx::tma_load_2d(b + 2 * kBoxBytes, &p.tm_w3, bar, n0, row, pol_w);
             ptx::tma_load_2d(b + 3 * kBoxBytes, &p.tm_w3, bar, n0 + 64, row, pol_w);
-          } else {         // W2 rows i = n0 .. n0+127, K = h (K-major)
-            ptx::tma_load_2d(b, &p.tm_w2, bar, (kb - p.H / 64) * 64, task.e * p.I + n0, pol_w);
           }
         } else if (Kind == kBwdDgrad2) {
           const int ki = kb < p.I / 64 ? kb : kb - p.I / 64;
@@ -333,9 +337,9 @@ __device__ void bwd_gather(const BwdParams& p, BwdSmem& s, uint8_t* tiles, int g
           break;
         }
         const uint32_t a = ptx::smem_u32(tiles + stage * kBwdStageBytes);
-        const bool second = kb >= p.H / 64;
-        const bf16* base = second ? p.dy : p.x;
-        const int kc = (second ? kb - p.H / 64 : kb) * 64 + c * 8;
+        const bool da_part = kb < p.H / 64;   // dy rows first, then x rows
+        const bf16* base = da_part ? p.dy : p.x;
+        const int kc = (da_part ? kb : kb - p.H / 64) * 64 + c * 8;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int r = (j * kBwdGatherWarps + g) * 4 + (lane >> 3);
@@ -439,13 +443,30 @@ __device__ void bwd_mma(const BwdParams& p, BwdSmem& s, uint8_t* tiles, uint32_t
   uint32_t acc_phase = 0;
   bool issued_any = false;
   bool ok = true;
+  int nt = 0;   // dgrad1: tasks of this CTA so far (da slot nt & 1; g|u columns shared)
   for (int t = blockIdx.x; t < ntasks && ok; t += gridDim.x) {
     const BwdTask task = bwd_decode<Kind>(t, p, s);
     if (task.nk == 0) continue;   // no K: the epilogue writes zeros without the accumulator
-    if (!bwd_wait(&s.acc_empty[acc], acc_phase ^ 1, p, s, 5)) break;
+    uint32_t d = tmem_base + acc * 256, d_da = 0;
+    if (Kind == kBwdDgrad1) {
+      // da slot nt & 1 was last read by the epilogue of task nt - 2 (use (nt >> 1) of the slot)
+      const int slot = nt & 1;
+      if (!bwd_wait(&s.da_empty[slot], ((nt >> 1) & 1) ^ 1, p, s, 5)) break;
+      d = tmem_base;
+      d_da = tmem_base + 256 + 128 * slot;
+    } else if (!bwd_wait(&s.acc_empty[acc], acc_phase ^ 1, p, s, 5)) {
+      break;
+    }
     ptx::tc_fence_after();
-    const uint32_t d = tmem_base + acc * 256;
     for (int kb = 0; kb < task.nk; ++kb) {
+      // dgrad1: the g|u columns were last read by the epilogue of task nt - 1
+      if (Kind == kBwdDgrad1 && kb == p.H / 64) {
+        if (!bwd_wait(&s.acc_empty[0], (nt & 1) ^ 1, p, s, 5)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+      }
       if (!bwd_wait(&s.full[stage], phase, p, s, 6)) {
         ok = false;
         break;
@@ -455,8 +476,8 @@ __device__ void bwd_mma(const BwdParams& p, BwdSmem& s, uint8_t* tiles, uint32_t
       if (lane == 0) {
         const uint32_t a = ptx::smem_u32(tiles + stage * kBwdStageBytes);
         const uint32_t b = a + kBwdABytes;
-        const bool da_part = Kind == kBwdDgrad1 && kb >= p.H / 64;
-        const int kfirst = Kind == kBwdDgrad1 ? (da_part ? p.H / 64 : 0) : 0;
+        const bool da_part = Kind == kBwdDgrad1 && kb < p.H / 64;
+        const int kfirst = Kind == kBwdDgrad1 && !da_part ? p.H / 64 : 0;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t ad = a_mn ? ptx::smem_desc_sw128(a + kk * 2048, kBoxBytes, 1024)
@@ -466,7 +487,7 @@ __device__ void bwd_mma(const BwdParams& p, BwdSmem& s, uint8_t* tiles, uint32_t
           const uint64_t bd = b_kmajor ? ptx::smem_desc_sw128(b + kk * 32, 16, 1024)
                                        : ptx::smem_desc_sw128(b + kk * 2048, kBoxBytes, 1024);
           const uint32_t acc_flag = (kb != kfirst || kk != 0) ? 1u : 0u;
-          ptx::mma_bf16(da_part ? d + 256 : d, ad, bd, da_part ? id_da : id_main, acc_flag);
+          ptx::mma_bf16(da_part ? d_da : d, ad, bd, da_part ? id_da : id_main, acc_flag);
         }
         ptx::mma_commit(&s.empty[stage]);
         issued_any = true;
@@ -480,6 +501,7 @@ __device__ void bwd_mma(const BwdParams& p, BwdSmem& s, uint8_t* tiles, uint32_t
     if (!ok) break;
     if (lane == 0) ptx::mma_commit(&s.acc_full[acc]);
     __syncwarp();
+    ++nt;
     if (++acc == kAccs) {
       acc = 0;
       acc_phase ^= 1;
@@ -525,6 +547,7 @@ __device__ void bwd_epilogue(const BwdParams& p, BwdSmem& s, uint32_t tmem_base,
   constexpr int kAccs = Kind == kBwdDgrad1 ? 1 : 2;
   int acc = 0;
   uint32_t acc_phase = 0;
+  int nt_epi = 0;   // dgrad1: tasks of this CTA so far (their da slots alternate)
   for (int t = blockIdx.x; t < ntasks; t += gridDim.x) {
     const BwdTask task = bwd_decode<Kind>(t, p, s);
     const bool has_acc = task.nk > 0;
@@ -539,6 +562,7 @@ __device__ void bwd_epilogue(const BwdParams& p, BwdSmem& s, uint32_t tmem_base,
       if (lane == 0) ptx::mbar_arrive(&s.acc_empty[acc]);
     };
     if (Kind == kBwdDgrad1) {
+      const int dslot = nt_epi & 1;   // this task's da slot (TMEM columns 256 + 128 * dslot)
       const int slot = task.b * p.BM + r;
       int tok = r < p.BM ? p.slot_token[slot] : -1;
       int j = 0;
@@ -564,7 +588,7 @@ __device__ void bwd_epilogue(const BwdParams& p, BwdSmem& s, uint32_t tmem_base,
         uint32_t g[32], u[32], v[32];
         ptx::tmem_ld32(tb + c * 32, g);
         ptx::tmem_ld32(tb + 128 + c * 32, u);
-        ptx::tmem_ld32(tb + 256 + c * 32, v);
+        ptx::tmem_ld32(tb + 256 + 128 * dslot + c * 32, v);
         ptx::tmem_ld_wait();
         float dg[32], du[32], aw[32];
 #pragma unroll
@@ -594,7 +618,9 @@ __device__ void bwd_epilogue(const BwdParams& p, BwdSmem& s, uint32_t tmem_base,
           store_bf16x32(p.aw + o, z);
         }
       }
-      release();
+      release();   // the g|u columns
+      if (lane == 0) ptx::mbar_arrive(&s.da_empty[dslot]);
+      ++nt_epi;
       if (tok >= 0) atomicAdd(p.dw + (size_t)tok * p.k + j, dwp);
     } else if (Kind == kBwdDgrad2) {
       int tok = r < p.BM ? p.slot_token[task.b * p.BM + r] : -1;
@@ -671,6 +697,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) moe_backward_gemm_kernel(const
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&s.acc_full[i], 1);
       ptx::mbar_init(&s.acc_empty[i], helpers ? 8 : 4);   // every epilogue warp releases the accumulator
+      ptx::mbar_init(&s.da_empty[i], helpers ? 8 : 4);
     }
     ptx::mbar_init(&s.mma_done, 1);
     s.abort = 0;

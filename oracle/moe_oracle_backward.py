@@ -63,12 +63,18 @@ def expert_ffn_backward(xr: np.ndarray, W1e: np.ndarray, W3e: np.ndarray, W2e: n
 
 
 def moe_backward(x, Wg, bias, expert_weights: Callable[[int], tuple], k: int, dy,
-                 round_activation: bool = True) -> dict:
+                 round_activation: bool = True, workers: int = 1,
+                 on_expert: Optional[Callable[..., None]] = None) -> dict:
     """Gradients of the layer for the upstream dy [T,H] (see the module notes).
 
     x [T,H], Wg [H,E], bias [E] or None, expert_weights(e) -> (W1[e] [H,I], W3[e] [H,I], W2[e] [I,H]).
     Returns dx [T,H], dWg [H,E], dbias [E] (zeros when bias is None), dW1/dW3 [E,H,I],
     dW2 [E,I,H], and the routing (topk_idx, topk_w) and dw [T,k] for inspection.
+
+    workers > 1 runs the experts' backward in that many threads; their contributions are
+    still added in ascending expert order. With on_expert, each expert's weight gradients are
+    handed to on_expert(e, dW1e, dW3e, dW2e) (None for an expert no token chose) instead of
+    being kept (dW1, dW3, dW2 are then returned as None).
     """
     x = np.asarray(x, np.float64)
     Wg = np.asarray(Wg, np.float64)
@@ -79,26 +85,46 @@ def moe_backward(x, Wg, bias, expert_weights: Callable[[int], tuple], k: int, dy
     dx = np.zeros_like(x)
     dw = np.zeros((T, k))
     dW1 = dW3 = dW2 = None
-    for e in range(E):
-        W1e, W3e, W2e = expert_weights(e)
-        if dW1 is None:
-            I = W1e.shape[1]
-            dW1 = np.zeros((E, H, I))
-            dW3 = np.zeros((E, H, I))
-            dW2 = np.zeros((E, I, H))
+
+    def expert_part(e):
         t, j = np.nonzero(idx == e)
         if t.size == 0:
-            continue
+            return e, t, j, None
+        W1e, W3e, W2e = expert_weights(e)
         do = w[t, j][:, None] * dy[t]
-        o, dxr, dW1[e], dW3[e], dW2[e] = expert_ffn_backward(x[t], W1e, W3e, W2e, do, round_activation)
-        np.add.at(dx, t, dxr)
+        return e, t, j, (W1e.shape[1],) + expert_ffn_backward(x[t], W1e, W3e, W2e, do, round_activation)
+
+    if workers > 1:
+        from concurrent.futures import ThreadPoolExecutor
+        pool = ThreadPoolExecutor(max_workers=workers)
+        parts = pool.map(expert_part, range(E))
+    else:
+        pool = None
+        parts = map(expert_part, range(E))
+    for e, t, j, res in parts:
+        if res is None:
+            if on_expert is not None:
+                on_expert(e, None, None, None)
+            continue
+        I, o, dxr, dW1e, dW3e, dW2e = res
+        if on_expert is not None:
+            on_expert(e, dW1e, dW3e, dW2e)
+        else:
+            if dW1 is None:
+                dW1 = np.zeros((E, H, I))
+                dW3 = np.zeros((E, H, I))
+                dW2 = np.zeros((E, I, H))
+            dW1[e], dW3[e], dW2[e] = dW1e, dW3e, dW2e
+        dx[t] += dxr                      # a token chooses an expert at most once: rows t are distinct
         dw[t, j] = np.sum(dy[t] * o, axis=1)
+    if pool is not None:
+        pool.shutdown()
     dl = selected_softmax_grad(w, dw)
-    dWg = np.zeros_like(Wg)
-    dbias = np.zeros(E)
-    for j in range(k):
-        e = idx[:, j]
-        np.add.at(dWg.T, e, x * dl[:, j:j + 1])
-        np.add.at(dbias, e, dl[:, j])
-        dx += Wg[:, e].T * dl[:, j:j + 1]
+    # the gate gradients with the selected logits' gradients as a dense [T, E] matrix (zero where
+    # an expert was not chosen): dWg = x^T dl, dbias = column sums of dl, dx += dl Wg^T
+    dl_dense = np.zeros((T, E))
+    np.put_along_axis(dl_dense, idx, dl, axis=1)
+    dWg = x.T @ dl_dense
+    dbias = dl_dense.sum(axis=0)
+    dx += dl_dense @ Wg.T
     return dict(dx=dx, dWg=dWg, dbias=dbias, dW1=dW1, dW3=dW3, dW2=dW2, topk_idx=idx, topk_w=w, dw=dw)

@@ -107,3 +107,52 @@ def test_backward_twice_gives_the_same_gradients():
     for n in a:
         d = (a[n].float() - b[n].float()).abs().max().item()
         assert d <= 2e-2 * max(a[n].float().abs().max().item(), 1e-30), n
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["tiny", "mixtral", "decode", "skewed", "fine_grained_prefill"])
+def test_backward_workload_matches_oracle(name):
+    """moe_backward at the five workloads' full sizes, every gradient compared in full: dx on every
+    row, dWg and dbias, and each expert's dW1 / dW3 / dW2 (the oracle hands them over one expert
+    at a time; the tolerances apply to each whole gradient tensor)."""
+    from threadpoolctl import threadpool_limits
+
+    from moe_megakernel_b200 import MoEPlan
+    from synth.moe_inputs import WORKLOADS
+    from tests.parity_util import expert_loader, oracle_workers
+    shape = WORKLOADS[name]
+    inp = make_inputs(shape, device="cuda")
+    dy = make_dy(shape, device="cuda")
+    plan = MoEPlan(shape.T, shape.H, shape.I, shape.E, shape.k, backward=True)
+    g = plan.backward(inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], dy)
+    plan.check()
+    acc = {n: [0.0, 0.0, 0.0, 0.0] for n in ("dW1", "dW3", "dW2")}   # |d|^2, |ref|^2, max|d|, max|ref|
+    idle = []
+
+    def on_expert(e, dW1e, dW3e, dW2e):
+        if dW1e is None:
+            idle.append(e)
+            return
+        for n, ref in (("dW1", dW1e), ("dW3", dW3e), ("dW2", dW2e)):
+            got = g[n][e].to(torch.float64).cpu().numpy()
+            d = got - ref
+            a = acc[n]
+            a[0] += float(np.sum(d * d))
+            a[1] += float(np.sum(ref * ref))
+            a[2] = max(a[2], float(np.abs(d).max()))
+            a[3] = max(a[3], float(np.abs(ref).max()))
+
+    with threadpool_limits(limits=1):
+        ref = B.moe_backward(to_f64(inp["x"]), to_f64(inp["Wg"]), None if inp["bias"] is None else to_f64(inp["bias"]),
+                             expert_loader(inp["W1"], inp["W3"], inp["W2"]), shape.k, to_f64(dy),
+                             workers=oracle_workers(), on_expert=on_expert)
+    errs = {n: _compare(n, g[n], ref[n]) for n in ("dx", "dWg")}
+    if inp["bias"] is not None:
+        errs["dbias"] = _compare("dbias", g["dbias"], ref["dbias"])
+    for n, (d2, r2, mx, rmax) in acc.items():
+        fro = (d2 / max(r2, 1e-300)) ** 0.5
+        assert fro <= REL_FRO and mx <= MAX_REL * max(rmax, 1e-30), f"{n}: rel Frobenius {fro:.3e}, max abs {mx:.3e}"
+        errs[n] = fro
+    for e in idle:
+        assert g["dW1"][e].abs().max().item() == 0 and g["dW2"][e].abs().max().item() == 0
+    print(f"backward {name}: idle experts {len(idle)} " + " ".join(f"{n}={v:.2e}" for n, v in errs.items()))

@@ -830,7 +830,7 @@ __global__ void __launch_bounds__(kGateThreads) moe_gate_backward_kernel(
 // Rows of x and dy in slot order for the backward's TMA operands: xp[s] = x[t], dyp[s] = dy[t]
 // for slot s with token t, zeros for padding slots and for the 64 rows after the last used
 // slot (a weight-gradient K block of 64 slots may reach past the pool's last expert). One
-// warp per row, 16 bytes per lane per step.
+// warp per row, up to four 16-byte loads of x and four of dy per lane in flight.
 __global__ void __launch_bounds__(256) moe_permute_rows_kernel(const bf16* __restrict__ x, const bf16* __restrict__ dy,
                                                                const int32_t* __restrict__ slot_token,
                                                                const int32_t* __restrict__ nblocks, bf16* __restrict__ xp,
@@ -850,9 +850,24 @@ __global__ void __launch_bounds__(256) moe_permute_rows_kernel(const bf16* __res
     uint4* xo = reinterpret_cast<uint4*>(xp + (size_t)sl * H);
     uint4* dout = reinterpret_cast<uint4*>(dyp + (size_t)sl * H);
     const uint4 z = make_uint4(0, 0, 0, 0);
-    for (int i = lane; i < H / 8; i += 32) {
-      xo[i] = t < 0 ? z : __ldg(xs + i);
-      dout[i] = t < 0 ? z : __ldg(ds + i);
+    const int n = H / 8;
+    // four 16-byte pieces of each row in flight per lane before the stores
+    for (int i0 = lane; i0 < n; i0 += 32 * 4) {
+      uint4 a[4], b[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + 32 * u;
+        a[u] = (t < 0 || i >= n) ? z : __ldg(xs + i);
+        b[u] = (t < 0 || i >= n) ? z : __ldg(ds + i);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + 32 * u;
+        if (i < n) {
+          xo[i] = a[u];
+          dout[i] = b[u];
+        }
+      }
     }
   }
 }

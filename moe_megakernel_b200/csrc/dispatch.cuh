@@ -60,16 +60,19 @@ __global__ void __launch_bounds__(kScanThreads) moe_dispatch_scan_kernel(const D
   __shared__ int32_t s_cnt[kMaxExperts];
   __shared__ int32_t s_part[kScanThreads];
   const int tid = threadIdx.x;
-  // (1) per-expert scan over chunks: threads per expert tpe (a power of two)
+  // (1) per-expert scan over chunks: threads per expert tpe (a power of two), each a run of
+  // chunks; neighbouring threads take neighbouring experts, so a warp's loads are contiguous
   int tpe = 1;
   while (tpe * 2 * p.E <= kScanThreads) tpe *= 2;
-  const int e = tid / tpe, sub = tid % tpe;
+  const bool act = tid < tpe * p.E;
+  const int e = act ? tid % p.E : p.E, sub = act ? tid / p.E : 0;
   const int per = (p.num_chunks + tpe - 1) / tpe;
   const int c0 = min(sub * per, p.num_chunks), c1 = min(c0 + per, p.num_chunks);
   int local = 0;
-  if (e < p.E)
+  if (e < p.E) {
     for (int c = c0; c < c1; ++c) local += p.chunk_count[(size_t)c * p.E + e];
-  s_part[tid] = local;
+    s_part[e * tpe + sub] = local;
+  }
   __syncthreads();
   if (e < p.E) {
     int base = 0;

@@ -2,7 +2,8 @@
 // of 64 (E <= 256): logits = x Wg (+ b) for 128 tokens per CTA with tcgen05
 // MMAs (TMA-fed, fp32 accumulator in TMEM), then top-k and the softmax over
 // the k kept logits, then the same per-64-token histogram and stable ranks as
-// the warp-MMA router, and zeroing of the tokens' output-accumulator rows.
+// the warp-MMA router; the epilogue warps zero the tokens' output-accumulator
+// rows while the MMAs run.
 //
 // Gate definition: "FlashMoE Kernel", opening paragraph (gate is the first step
 // of the fused layer); softmax top-k renormalised over the k selected experts;
@@ -168,6 +169,13 @@ __global__ void __launch_bounds__(kRtcThreads, 1) moe_router_tc_kernel(const __g
     // ------------------------------------------------ epilogue: one token per thread
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
+    {
+      // while the MMAs run: zero these tokens' rows of the fp32 output accumulator
+      float4* dst = reinterpret_cast<float4*>(p.y_acc + (size_t)t0 * p.H);
+      const size_t n4 = (size_t)ntok * p.H / 4;
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (size_t i = r; i < n4; i += 128) dst[i] = z;
+    }
     // the MMA warp commits acc_full even after giving up on a stage, so the
     // accumulator is complete only if no role of this CTA aborted
     bool ok = rtc_wait(&s.acc_full, 0, p, s, 3);
@@ -257,13 +265,6 @@ __global__ void __launch_bounds__(kRtcThreads, 1) moe_router_tc_kernel(const __g
   // Per 64-token chunk: histogram and stable ranks (tokens ascending).
   chunk_histogram(&s.sel[0][0], s.mask, ntok, 2, blockIdx.x * 2, t0, p.E, p.k, p.rank, p.chunk_count,
                   kRtcThreads);
-  // Zero these tokens' rows of the fp32 output accumulator.
-  {
-    float4* dst = reinterpret_cast<float4*>(p.y_acc + (size_t)t0 * p.H);
-    const size_t n4 = (size_t)ntok * p.H / 4;
-    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (size_t i = threadIdx.x; i < n4; i += kRtcThreads) dst[i] = z;
-  }
 }
 
 }  // namespace moe

@@ -283,11 +283,11 @@ __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(const Router
         }
         chosen[r] = bi;
         chosen_l[r] = best;
-        if ((bi & 31) == lane) {
+        // the chosen logit leaves the race (selects, not a store at the runtime index bi >> 5,
+        // which would put v in local memory)
+        const bool mine = (bi & 31) == lane;
 #pragma unroll
-          for (int i = 0; i < VPL; ++i)
-            if (i == (bi >> 5)) v[i] = -INFINITY;
-        }
+        for (int i = 0; i < VPL; ++i) v[i] = (mine && i == (bi >> 5)) ? -INFINITY : v[i];
       }
     }
     // Softmax over the k selected; chosen_l[0] is their maximum.
@@ -298,11 +298,10 @@ __global__ void __launch_bounds__(kRouterThreads) moe_router_kernel(const Router
     int me = 0x7fffffff;
     float ml = 0.f;
 #pragma unroll
-    for (int r = 0; r < 8; ++r)
-      if (r == lane) {
-        me = chosen[r];
-        ml = chosen_l[r];
-      }
+    for (int r = 0; r < 8; ++r) {
+      me = r == lane ? chosen[r] : me;
+      ml = r == lane ? chosen_l[r] : ml;
+    }
     if (lane < p.k) {
       int pos = 0;   // position in ascending expert order
 #pragma unroll

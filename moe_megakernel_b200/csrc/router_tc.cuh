@@ -50,6 +50,7 @@ struct RouterTcSmem {
   uint32_t tmem_base;
   int abort;
   int sel[kRtcTokens][8];   // selected experts per token, ascending id
+  float bias[256];          // the gate bias (when given)
   unsigned long long mask[2 * 256];   // per 64-token chunk and expert: token bitmask
 };
 
@@ -169,6 +170,9 @@ __global__ void __launch_bounds__(kRtcThreads, 1) moe_router_tc_kernel(const __g
     // ------------------------------------------------ epilogue: one token per thread
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
+    if (p.bias != nullptr)
+      for (int e = r; e < p.E; e += 128) s.bias[e] = p.bias[e];
+    asm volatile("bar.sync 1, 128;" ::: "memory");   // the four epilogue warps: bias staged
     {
       // while the MMAs run: zero these tokens' rows of the fp32 output accumulator
       float4* dst = reinterpret_cast<float4*>(p.y_acc + (size_t)t0 * p.H);
@@ -193,6 +197,7 @@ __global__ void __launch_bounds__(kRtcThreads, 1) moe_router_tc_kernel(const __g
     }
     float kth = -INFINITY;   // best[k-1]
     const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const float* bias = p.bias != nullptr ? s.bias : nullptr;
     for (int c = 0; c < p.E / 32; ++c) {
       uint32_t v[32];
       ptx::tmem_ld32(tbase + c * 32, v);
@@ -200,26 +205,31 @@ __global__ void __launch_bounds__(kRtcThreads, 1) moe_router_tc_kernel(const __g
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const int e = c * 32 + i;
-        const float l = __uint_as_float(v[i]) + (p.bias != nullptr ? p.bias[e] : 0.f);
+        const float l = __uint_as_float(v[i]) + (bias != nullptr ? bias[e] : 0.f);
         if (l > kth) {
-          int pos = 0;
+          // insert by one pass of compare-and-exchange down the list: the new
+          // value moves past only strictly smaller ones (a tie keeps the earlier,
+          // lower id), and the list stays in registers
+          float x = l;
+          int xi = e;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) pos += (j < p.k && best[j] >= l) ? 1 : 0;
-#pragma unroll
-          for (int j = 7; j > 0; --j)
-            if (j > pos && j < p.k) {
-              best[j] = best[j - 1];
-              bidx[j] = bidx[j - 1];
+          for (int j = 0; j < 8; ++j) {
+            if (j < p.k) {
+              const bool sw = x > best[j];
+              const float tb = best[j];
+              const int ti = bidx[j];
+              best[j] = sw ? x : tb;
+              bidx[j] = sw ? xi : ti;
+              x = sw ? tb : x;
+              xi = sw ? ti : xi;
             }
+          }
+          // the k-th largest is the smallest of the k kept (a select by the runtime index k - 1
+          // would become an indexed load and put the list in local memory)
+          kth = best[0];
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (j == pos) {
-              best[j] = l;
-              bidx[j] = e;
-            }
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (j == p.k - 1) kth = best[j];
+          for (int j = 1; j < 8; ++j)
+            if (j < p.k) kth = fminf(kth, best[j]);
         }
       }
     }

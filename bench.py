@@ -245,7 +245,7 @@ def time_oracle(inp, n_tokens: int, fp8: bool = False):
 def run_gpu(args, rank, world, local_rank):
     import torch
 
-    from moe_megakernel_b200 import MoEPlan, kernels_per_forward, quantize_weights_fp8
+    from moe_megakernel_b200 import MoEPlan, quantize_weights_fp8
     from synth.moe_inputs import WORKLOADS, make_inputs
 
     dist = None
@@ -453,8 +453,9 @@ def run_gpu(args, rank, world, local_rank):
                     "api": (f"moe_forward_host_pipelined{'_fp8' if args.fp8 else ''} (pinned host x and y; the "
                             "copies of each step overlap the neighbouring steps' kernels)") if pipelined
                     else "moe_forward_host_shared (pinned host x and y)"},
-            # FP8: + x quantizer, activation quantizer, second expert-GEMM launch
-            "gpu_launches": args.steps * (kernels_per_forward() + (3 if args.fp8 else 0)),
+            # FP8: + the x quantizer and, per block group, a first-GEMM launch, the activation
+            # quantizer and a second-GEMM launch (the library counts them)
+            "gpu_launches": args.steps * plan.forward_launches(args.fp8),
             "clocks": clk,
         }
         if tlog is not None:
@@ -521,7 +522,9 @@ def run_backward(args):
                      "peak_source": f"{peaks['source']} ({peak_name})", "flop_per_step": flop,
                      "frac_vs_burst": achieved / peaks["bf16_tflops"],
                      "frac_vs_sustained": achieved / peaks["bf16_tflops_sustained"]},
-        "gpu_launches": args.steps * 10,
+        # router, scan, scatter, dgrad-1, dgrad-2, Wg transpose, gate, dW1/dW3, dW2, dWg, and with
+        # BLOCK_M >= 64 the permutation of x and dy rows into slot order
+        "gpu_launches": args.steps * (10 + (1 if plan.block_m >= 64 else 0)),
         "clocks": clk,
     }), flush=True)
 

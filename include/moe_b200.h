@@ -471,6 +471,14 @@ int moe_plan_get_task_log(moe_plan_t plan, const moe_task_record** records, int*
 /* Number of kernels one moe_forward launches (for launch accounting). */
 int moe_forward_kernel_count(void);
 
+/* Number of kernels one forward of this plan launches: moe_forward_kernel_count()
+ * for bf16 (fp8 = 0); for moe_forward_fp8 (fp8 = 1) the router, dispatch scan
+ * and scatter and the finalize, the x quantizer, and per block group of the FP8
+ * schedule the first GEMM, the activation quantizer and the second GEMM (groups
+ * past the routing's last block exit at once but are still launched).
+ * -1: null plan, or fp8 = 1 on a plan without FP8 regions. */
+int moe_plan_forward_launches(moe_plan_t plan, int fp8);
+
 void moe_plan_destroy(moe_plan_t plan);
 const char* moe_status_string(int status);
 

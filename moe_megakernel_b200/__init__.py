@@ -81,6 +81,7 @@ SIGNATURES = {
     "moe_plan_get_task_log": (_c_int, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_c_int)]),
     "moe_plan_set_fp8": (_c_int, [_vp, _c_int]),
     "moe_forward_kernel_count": (_c_int, []),
+    "moe_plan_forward_launches": (_c_int, [_vp, _c_int]),
     "moe_plan_destroy": (None, [_vp]),
     "moe_status_string": (ctypes.c_char_p, [_c_int]),
 }
@@ -387,6 +388,13 @@ class MoEPlan:
         (see moe_plan_set_wide_l1)."""
         m = int(mode) if not isinstance(mode, bool) else (1 if mode else 0)
         _ok(self.lib.moe_plan_set_wide_l1(self._plan, m), "moe_plan_set_wide_l1")
+
+    def forward_launches(self, fp8: bool = False) -> int:
+        """Kernels one forward of this plan launches (see moe_plan_forward_launches)."""
+        n = self.lib.moe_plan_forward_launches(self._plan, 1 if fp8 else 0)
+        if n < 0:
+            raise RuntimeError("moe_plan_forward_launches: no FP8 regions in this plan")
+        return n
 
     @property
     def wide_l1(self) -> bool:

@@ -1404,6 +1404,16 @@ int moe_plan_set_half_tails(moe_plan_t p, int enable) {
 
 int moe_forward_kernel_count(void) { return kNumKernels; }
 
+int moe_plan_forward_launches(moe_plan_t p, int fp8) {
+  if (p == nullptr) return -1;
+  if (fp8 == 0) return kNumKernels;
+  if (p->fp8_rows == 0) return -1;
+  // the x quantizer, then per block group the first GEMM, the activation quantizer and the second
+  const int fp8_units = std::max(1, p->fp8_rows / (p->cta_pairs ? 2 * p->BM : p->BM));
+  const int fp8_groups = (p->blocks_max + fp8_units - 1) / fp8_units;
+  return kNumKernels - 1 + 1 + 3 * fp8_groups;
+}
+
 void moe_plan_destroy(moe_plan_t p) {
   if (p == nullptr) return;
   {

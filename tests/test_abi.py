@@ -91,6 +91,8 @@ def test_null_plan_arguments_of_the_newer_entries(lib):
     assert lib.moe_host_pipeline_after(None, None) == 1
     assert lib.moe_host_pipeline_join(None, None) == 1
     assert lib.moe_plan_set_cta_pairs(None, 1) == 1
+    assert lib.moe_plan_forward_launches(None, 0) == -1
+    assert lib.moe_plan_forward_launches(None, 1) == -1
 
 
 @pytest.mark.parametrize("args", [

@@ -409,7 +409,8 @@ def run_gpu(args, rank, world, local_rank):
             roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": gbs / peaks["hbm_gbs"]}
         roof.update({"kernel": "moe_expert_gemm2_kernel" if plan.cta_pairs else "moe_expert_gemm_kernel",
-                     "traffic": measured_traffic(args.workload + ("+fp8" if args.fp8 else "")),
+                     "traffic": measured_traffic(args.workload + ("+fp8" if args.fp8 else "")
+                                                 + (f"+shared{S}" if S else "")),
                      "traffic_unit": "bytes per launch (ncu dram read+write)",
                      "peak_source": f"{peaks['source']} ({tc_peak_name if bound == 'tensor' else 'hbm_gbs'})"
                                     + (" x 2: FP8 at the nominal fp8/bf16 ratio" if args.fp8 and bound == "tensor"

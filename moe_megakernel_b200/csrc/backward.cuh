@@ -526,6 +526,29 @@ __device__ __forceinline__ void store_bf16x32(bf16* dst, const float (&v)[32]) {
                        pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
 }
 
+// A warp's 32 rows x 32 columns of a bf16 output (lane = row, f = its 32 columns, base = row 0,
+// column 0, pitch in elements), staged in shared memory (rows padded to 36 floats) so that each
+// store instruction writes 8 rows x 64 contiguous bytes (4 lanes a row) instead of 32 rows x 16
+// bytes: a quarter of the store transactions.
+__device__ __forceinline__ void store_rows_bf16_staged(float (*stage)[36], const float (&f)[32], bf16* base,
+                                                       size_t pitch) {
+  const int lane = ptx::lane_id();
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    reinterpret_cast<float4*>(stage[lane])[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+  __syncwarp();
+  const int cq = (lane & 3) * 8;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int rr = (lane >> 2) + 8 * j;
+    const float4 a = *reinterpret_cast<const float4*>(&stage[rr][cq]);
+    const float4 b = *reinterpret_cast<const float4*>(&stage[rr][cq + 4]);
+    *reinterpret_cast<uint4*>(base + (size_t)rr * pitch + cq) =
+        make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+  }
+  __syncwarp();
+}
+
 // ---------------------------------------------------------------- warps 2..5: epilogue
 // With the operands by TMA (p.permuted), the four gather warps have nothing to copy; for
 // dgrad-1 and dW1/dW3 they become a second set of epilogue warps: the warp of each TMEM lane
@@ -649,22 +672,32 @@ __device__ void bwd_epilogue(const BwdParams& p, BwdSmem& s, uint32_t tmem_base,
         }
         if (Kind == kBwdWgrad13) {   // columns 0..127: dW1, 128..255: dW3, of I columns n*128 ..
           bf16* out = c < 4 ? p.dW1 : p.dW3;
-          const size_t o = ((size_t)task.e * p.H + task.m * 128 + r) * p.I + task.n * 128 + (c & 3) * 32;
-          store_bf16x32(out + o, f);
+          if (split) {   // helper epilogue warps share the staging rows: one row per lane
+            const size_t o = ((size_t)task.e * p.H + task.m * 128 + r) * p.I + task.n * 128 + (c & 3) * 32;
+            store_bf16x32(out + o, f);
+          } else {
+            const size_t o = ((size_t)task.e * p.H + task.m * 128 + quarter * 32) * p.I + task.n * 128 + (c & 3) * 32;
+            store_rows_bf16_staged(s.out_stage[quarter], f, out + o, p.I);
+          }
         } else if (Kind == kBwdWgrad2) {
-          // the tile is dW2[e]^T (rows h, columns i): transpose each 32 x 32 block through the
-          // warp's staging rows, so that lane l writes 32 consecutive h of row i = i0 + 32c + l
-          float* srow = s.out_stage[quarter][lane];
+          // the tile is dW2[e]^T (rows h, columns i): each 32 x 32 block goes through the warp's
+          // staging rows transposed (row ii = column i0 + 32c + ii of the tile), then 4 lanes write
+          // 32 consecutive h (64 bytes) of each of 8 rows of dW2 per instruction
+          float (*stg)[36] = s.out_stage[quarter];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            reinterpret_cast<float4*>(srow)[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+          for (int i = 0; i < 32; ++i) stg[i][lane] = f[i];
           __syncwarp();
-          float t[32];
+          const int hq = (lane & 3) * 8;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) t[i] = s.out_stage[quarter][i][lane];
+          for (int j = 0; j < 4; ++j) {
+            const int ii = (lane >> 2) + 8 * j;
+            const float4 a = *reinterpret_cast<const float4*>(&stg[ii][hq]);
+            const float4 b = *reinterpret_cast<const float4*>(&stg[ii][hq + 4]);
+            const size_t o = ((size_t)task.e * p.I + task.n * p.BNi + c * 32 + ii) * p.H + task.m * 128 + quarter * 32 + hq;
+            *reinterpret_cast<uint4*>(p.dW2 + o) = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w),
+                                                             pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+          }
           __syncwarp();
-          const size_t o = ((size_t)task.e * p.I + task.n * p.BNi + c * 32 + lane) * p.H + task.m * 128 + quarter * 32;
-          store_bf16x32(p.dW2 + o, t);
         } else {
           float* out = p.dWg + (size_t)(task.m * 128 + r) * p.E;
 #pragma unroll

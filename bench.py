@@ -100,12 +100,16 @@ def kernel_source_hash(read=None) -> str:
     return h.hexdigest()[:16]
 
 
-def measured_traffic(workload: str):
-    """ncu DRAM bytes per expert-GEMM launch, if captured on the current kernel sources."""
-    p = os.path.join(ROOT, "profiles", "traffic.txt")
+def measured_traffic(workload: str, table=None, source_hash=None):
+    """ncu DRAM bytes per expert-GEMM launch, if captured on the current kernel sources.
+
+    `workload` is the table's key (the workload name, + "+fp8" / "+shared<S>" for those forwards);
+    a row counts only if its source hash is the current one (the counters of a changed kernel are
+    not reported)."""
+    p = table if table is not None else os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
-    cur = kernel_source_hash()
+    cur = source_hash if source_hash is not None else kernel_source_hash()
     for line in open(p):
         f = line.split()
         if len(f) >= 3 and not f[0].startswith("#") and f[0] == workload and f[1] == cur:

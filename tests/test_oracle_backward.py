@@ -145,3 +145,25 @@ def test_planted_mistake_is_caught(name, monkeypatch):
     fn, repl = _MUTANTS[name]
     monkeypatch.setattr(B, fn, repl)
     assert not _pins_pass(), f"mutant {name} was not caught"
+
+
+def test_threaded_experts_and_per_expert_callback_give_the_same_gradients():
+    """The full-size parity tests run the backward oracle with experts on host threads and take
+    each expert's weight gradients through a callback; both give the plain run's values."""
+    x, Wg, bias, W1, W3, W2, dy = _layer(51, T=20, E=6)
+    bias[-1] = -1e3                      # one expert no token picks: the callback gets None for it
+    plain = _grads(x, Wg, bias, W1, W3, W2, dy, 2, round_activation=True)
+    got = {}
+
+    def on_expert(e, dW1e, dW3e, dW2e):
+        got[e] = (dW1e, dW3e, dW2e)
+
+    t = B.moe_backward(x, Wg, bias, O.stacked_expert_weights(W1, W3, W2), 2, dy, True, workers=3,
+                       on_expert=on_expert)
+    assert t["dW1"] is None and sorted(got) == list(range(6))
+    assert got[5] == (None, None, None)
+    for e in range(5):
+        for i, key in enumerate(("dW1", "dW3", "dW2")):
+            np.testing.assert_allclose(got[e][i], plain[key][e], rtol=1e-12, atol=1e-14, err_msg=f"{key}[{e}]")
+    for key in ("dx", "dWg", "dbias", "dw"):
+        np.testing.assert_allclose(t[key], plain[key], rtol=1e-12, atol=1e-14, err_msg=key)

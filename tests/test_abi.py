@@ -128,3 +128,24 @@ def test_bench_source_hash_ignores_comments():
     c = "int f(int x) {\n  return x + 2;\n}\n"
     assert bench.code_text(a) == bench.code_text(b)
     assert bench.code_text(a) != bench.code_text(c)
+
+
+def test_readme_c_example_compiles_against_the_header(tmp_path):
+    """The C usage example in the README stays in step with include/moe_b200.h (syntax and types)."""
+    import re
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    cuda_inc = "/usr/local/cuda/include"
+    if cc is None or not os.path.exists(os.path.join(cuda_inc, "cuda_runtime.h")):
+        pytest.skip("no C compiler or CUDA headers")
+    readme = open(os.path.join(ROOT, "README.md")).read()
+    code = re.search(r"```c\n(.*?)```", readme, re.S).group(1).replace('#include "moe_b200.h"', "")
+    src = tmp_path / "example.c"
+    src.write_text("#include <stdio.h>\n#include <cuda_runtime.h>\n#include \"moe_b200.h\"\n"
+                   "int example(int T_max, int H, int I, int E, int k, int T, const void* x, const void* Wg,\n"
+                   "            const void* W1, const void* W3, const void* W2, void* y, void* stream) {\n"
+                   + code + "\n  return st;\n}\n")
+    r = subprocess.run([cc, "-fsyntax-only", "-Wall", "-I", os.path.join(ROOT, "include"), "-I", cuda_inc, str(src)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
